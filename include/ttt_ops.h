@@ -1,0 +1,71 @@
+/*
+ * ttt_ops.h — op-level C ABI of the kernels behind ttt.h, for testing each
+ * stage of the prefill loop on its own.  Every call is asynchronous on
+ * `stream` (a cudaStream_t, NULL = legacy default stream); pointers are
+ * device pointers owned by the caller; the return value is TTT_OK or a
+ * TTT_ERR_* code from ttt.h (message: ttt_last_error(NULL)).  Kernel-side
+ * failures (bounded waits that gave up) are reported by ttt_op_sync().
+ */
+#ifndef TTT_OPS_H_
+#define TTT_OPS_H_
+
+#include <stdint.h>
+
+#include "ttt.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues of ttt_op_gemm (acc = the fp32 accumulator of one output element). */
+#define TTT_EPI_STORE_F32 0  /* c (fp32) = acc */
+#define TTT_EPI_STORE_BF16 1 /* c (bf16) = acc */
+#define TTT_EPI_ADD_F32 2    /* c (fp32) += acc (residual update, x += o W^T) */
+#define TTT_EPI_SWIGLU 3     /* columns in (gate 64 | up 64) pairs: c[:, 64*pair + i] = silu(g) * u;
+                                c2 (optional) = raw acc.  Output dtype = the GEMM's dtype. */
+#define TTT_EPI_CE_FWD 4     /* softmax-CE partials per row and N tile (see below) */
+#define TTT_EPI_CE_BWD 5     /* c = (exp(acc - row_f[m]) - [n + col_offset == row_i[m]]) * row_g[m] */
+#define TTT_EPI_SGD 6        /* c (fp32) -= alpha * acc;  c2 (optional, bf16) = new c */
+
+typedef struct ttt_epilogue_args {
+  void* c;
+  int64_t ldc;
+  void* c2;
+  int64_t ldc2;
+  const float* row_f;      /* CE_BWD: log-sum-exp per row */
+  const float* row_g;      /* CE_BWD: scale per row (1/n_c, or 0 for rows without a target) */
+  const int32_t* row_i;    /* CE_FWD / CE_BWD: target id per row */
+  float* part_max;         /* CE_FWD: [n_tiles, part_ld] running max per tile and row */
+  float* part_sum;         /* CE_FWD: [n_tiles, part_ld] sum of exp(acc - max) */
+  float* target_logit;     /* CE_FWD: acc at the target column (written by the tile holding it) */
+  int64_t part_ld;
+  float alpha;             /* SGD: learning rate */
+  int64_t col_offset;      /* global column index of output column 0 (vocab chunks) */
+} ttt_epilogue_args;
+
+/*
+ * acc[m][n] = sum_k A(m,k) B(n,k) for m < M, n < N, then the epilogue.
+ * dtype TTT_BF16 runs the tcgen05 tensor-core kernel (bf16 operands, fp32
+ * accumulation); TTT_F32 the fp32 SIMT kernel (all operands fp32).
+ * a_mn = 0: A stored [M, K] with row pitch lda;  a_mn = 1: stored [K, M].
+ * b_mn = 0: B stored [N, K] with row pitch ldb;  b_mn = 1: stored [K, N].
+ * bf16 operands: 16-byte aligned base and row pitch.  (a_mn, b_mn) = (1, 0)
+ * is not supported with TTT_BF16.  bn_hint: 0 (auto), 128 or 256 (tile
+ * width; TTT_BF16 only).  CE_FWD writes ceil(N / tile) partial tiles:
+ * query the tile count with ttt_op_gemm_ce_tiles.
+ */
+int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A,
+                int64_t lda, const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args,
+                int32_t bn_hint, void* stream);
+
+/* Number of N tiles a CE_FWD ttt_op_gemm of width N writes partials for. */
+int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint);
+
+/* Wait for `stream`; return TTT_ERR_TIMEOUT if a kernel launched through this
+ * header recorded a bounded-wait timeout since the last call (then clears it). */
+int ttt_op_sync(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_OPS_H_ */

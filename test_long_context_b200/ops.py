@@ -1,0 +1,50 @@
+"""torch-tensor wrappers of the op-level entry points (include/ttt_ops.h).
+Argument marshalling only."""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib as L
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t):
+    if t.dtype == torch.bfloat16:
+        return L.TTT_BF16
+    if t.dtype == torch.float32:
+        return L.TTT_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def gemm(A, B, a_mn, b_mn, epi, c=None, c2=None, row_f=None, row_g=None, row_i=None, part_max=None,
+         part_sum=None, target_logit=None, part_ld=0, alpha=0.0, col_offset=0, bn=0, M=None, N=None, K=None,
+         stream=None):
+    """ttt_op_gemm on 2-D tensors in storage order (see ttt_ops.h)."""
+    dt = _dtype(A)
+    M = (A.shape[1] if a_mn else A.shape[0]) if M is None else M
+    K = (A.shape[0] if a_mn else A.shape[1]) if K is None else K
+    N = (B.shape[1] if b_mn else B.shape[0]) if N is None else N
+    args = L.ttt_epilogue_args(
+        _p(c), c.stride(0) if c is not None else 0, _p(c2), c2.stride(0) if c2 is not None else 0,
+        _p(row_f), _p(row_g), _p(row_i), _p(part_max), _p(part_sum), _p(target_logit), part_ld, alpha, col_offset)
+    rc = L.lib().ttt_op_gemm(dt, int(a_mn), int(b_mn), M, N, K, _p(A), A.stride(0), _p(B), B.stride(0), epi,
+                             ctypes.byref(args), bn, _stream(stream))
+    L.check(rc)
+
+
+def gemm_ce_tiles(dtype_is_bf16, M, N, bn=0):
+    return int(L.lib().ttt_op_gemm_ce_tiles(L.TTT_BF16 if dtype_is_bf16 else L.TTT_F32, M, N, bn))
+
+
+def sync(stream=None):
+    L.check(L.lib().ttt_op_sync(_stream(stream)))

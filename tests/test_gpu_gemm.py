@@ -1,0 +1,112 @@
+"""GEMM kernels through the op-level C ABI vs torch (fp64 reference of the
+same rounded operands).  tcgen05 path for bf16, SIMT path for fp32."""
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [(256, 512, 256), (200, 392, 136), (128, 128, 64), (1000, 1280, 520)]
+COMBOS = [(0, 0), (0, 1), (1, 1)]
+
+
+def _operands(M, N, K, a_mn, b_mn, dtype, seed=0):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    A = torch.randn((K, M) if a_mn else (M, K), device="cuda", generator=g).to(dtype)
+    B = torch.randn((K, N) if b_mn else (N, K), device="cuda", generator=g).to(dtype)
+    Am = A.double().T if a_mn else A.double()
+    Bm = B.double() if b_mn else B.double().T
+    return A, B, Am @ Bm  # [M, N]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("combo", COMBOS)
+@pytest.mark.parametrize("bn", [128, 256])
+def test_tc_gemm_store(shape, combo, bn):
+    from test_long_context_b200 import ops
+    M, N, K = shape
+    A, B, ref = _operands(M, N, K, *combo, torch.bfloat16)
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, *combo, ops.L.EPI_STORE_F32, c=c, bn=bn)
+    ops.sync()
+    err = (c.double() - ref).abs().max().item()
+    assert err <= 1e-4 * ref.abs().max().item() + 1e-4, err
+
+
+@pytest.mark.parametrize("combo", COMBOS)
+def test_simt_gemm_store(combo):
+    from test_long_context_b200 import ops
+    M, N, K = 200, 392, 136
+    A, B, ref = _operands(M, N, K, *combo, torch.float32)
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, *combo, ops.L.EPI_STORE_F32, c=c)
+    ops.sync()
+    assert (c.double() - ref).abs().max().item() <= 1e-4
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gemm_add_swiglu_sgd(dtype):
+    from test_long_context_b200 import ops
+    M, N, K = 300, 512, 192
+    A, B, ref = _operands(M, N, K, 0, 0, dtype, seed=1)
+    tol = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    # residual add
+    x0 = torch.randn(M, N, device="cuda")
+    x = x0.clone()
+    ops.gemm(A, B, 0, 0, ops.L.EPI_ADD_F32, c=x)
+    ops.sync()
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
+    # SwiGLU over (gate 64 | up 64) column pairs
+    a = torch.empty(M, N // 2, device="cuda", dtype=dtype)
+    raw = torch.empty(M, N, device="cuda", dtype=dtype)
+    ops.gemm(A, B, 0, 0, ops.L.EPI_SWIGLU, c=a, c2=raw)
+    ops.sync()
+    r = ref.view(M, N // 128, 2, 64)
+    g, u = r[:, :, 0], r[:, :, 1]
+    want = (torch.nn.functional.silu(g) * u).reshape(M, N // 2)
+    assert (a.double() - want).abs().max().item() <= tol * want.abs().max().item()
+    assert (raw.double() - ref).abs().max().item() <= tol * ref.abs().max().item()
+    # SGD epilogue on a weight-gradient-shaped product
+    Aw, Bw, G = _operands(160, 384, 256, 1, 1, dtype, seed=2) if dtype == torch.bfloat16 else _operands(160, 384, 256, 1, 1, dtype, seed=2)
+    W = torch.randn(160, 384, device="cuda")
+    W0 = W.clone()
+    W16 = torch.empty(160, 384, device="cuda", dtype=torch.bfloat16) if dtype == torch.bfloat16 else None
+    ops.gemm(Aw, Bw, 1, 1, ops.L.EPI_SGD, c=W, c2=W16, alpha=0.01)
+    ops.sync()
+    want = W0.double() - 0.01 * G
+    assert (W.double() - want).abs().max().item() <= 1e-5
+    if W16 is not None:
+        assert torch.equal(W16, W.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_gemm_cross_entropy_epilogues(dtype):
+    from test_long_context_b200 import ops
+    M, V, K = 260, 1000, 128  # ragged rows and vocab
+    h = (torch.randn(M, K, device="cuda") * 0.5).to(dtype)
+    W = (torch.randn(V, K, device="cuda") * 0.5).to(dtype)
+    z = h.double() @ W.double().T
+    tgt = torch.randint(0, V, (M,), device="cuda", dtype=torch.int32)
+    bf = dtype == torch.bfloat16
+    nt = ops.gemm_ce_tiles(bf, M, V)
+    pm = torch.empty(nt, M, device="cuda")
+    ps = torch.empty(nt, M, device="cuda")
+    zt = torch.full((M,), float("nan"), device="cuda")
+    ops.gemm(h, W, 0, 0, ops.L.EPI_CE_FWD, row_i=tgt, part_max=pm, part_sum=ps, target_logit=zt, part_ld=M)
+    ops.sync()
+    gm = pm.max(0).values
+    lse = gm + torch.log((ps * torch.exp(pm - gm)).sum(0))
+    want_lse = torch.logsumexp(z, 1)
+    assert (lse.double() - want_lse).abs().max().item() <= 1e-4
+    assert (zt.double() - z.gather(1, tgt.long()[:, None])[:, 0]).abs().max().item() <= 1e-4
+    # backward: dz = (softmax - onehot) * scale, columns offset by a vocab chunk start
+    scale = torch.full((M,), 1.0 / M, device="cuda")
+    scale[-3:] = 0
+    off = 300
+    dz = torch.empty(M, V - off, device="cuda", dtype=dtype)
+    ops.gemm(h, W[off:], 0, 0, ops.L.EPI_CE_BWD, c=dz, row_f=want_lse.float(), row_g=scale, row_i=tgt,
+             col_offset=off)
+    ops.sync()
+    p = torch.softmax(z, 1)
+    oh = torch.nn.functional.one_hot(tgt.long(), V).double()
+    want = ((p - oh) * scale.double()[:, None])[:, off:]
+    assert (dz.double() - want).abs().max().item() <= (1e-2 if bf else 2e-5) * want.abs().max().item()
