@@ -49,7 +49,7 @@ extern "C" {
  * QK-norm (the recipe in the jdon.com write-up names QK norm and the Llama3
  * tokenizer), RoPE, SwiGLU MLPs and an untied LM head.
  *   d_model == n_heads * head_dim; head_dim in {32, 64, 80, 96, 128};
- *   d_model and d_ff multiples of 64.
+ *   d_model a multiple of 8; d_ff a multiple of 64.
  *   norm_eps: RMSNorm epsilon (y = x / sqrt(mean(x^2) + eps) * g).
  *   rope_theta: RoPE base; element i is paired with i + head_dim/2.
  */

@@ -20,7 +20,8 @@ extern "C" {
 /* Epilogues of ttt_op_gemm (acc = the fp32 accumulator of one output element). */
 #define TTT_EPI_STORE_F32 0  /* c (fp32) = acc */
 #define TTT_EPI_STORE_BF16 1 /* c (bf16) = acc */
-#define TTT_EPI_ADD_F32 2    /* c (fp32) += acc (residual update, x += o W^T) */
+#define TTT_EPI_ADD_F32 2    /* c (fp32) = r + acc with r = c2 (fp32) if given, else c itself
+                                (residual update, x_out = x_in + o W^T) */
 #define TTT_EPI_SWIGLU 3     /* columns in (gate 64 | up 64) pairs: c[:, 64*pair + i] = silu(g) * u;
                                 c2 (optional) = raw acc.  Output dtype = the GEMM's dtype. */
 #define TTT_EPI_CE_FWD 4     /* softmax-CE partials per row and N tile (see below) */
@@ -60,6 +61,33 @@ int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N,
 
 /* Number of N tiles a CE_FWD ttt_op_gemm of width N writes partials for. */
 int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint);
+
+/*
+ * Sliding-window causal attention, eq. (1) of the reading notes: query at
+ * absolute position p = q_pos0 + i attends to keys p-window+1 .. p.
+ *   q, o: [n_q, ldq] / [n_q, ldo] rows, head h in columns h*head_dim ...
+ *   k_ring, v_ring: [ring_slots, n_heads*head_dim]; the key at position j is
+ *   in slot j % ring_slots, so ring_slots >= window + n_q - 1 is required
+ *   when the ring holds earlier positions as well.
+ *   lse: [n_heads, n_q] fp32 natural-log log-sum-exp of the scaled scores.
+ * dtype TTT_F32 (all fp32) or TTT_BF16 (bf16 tensors, fp32 math).
+ * Scores are scaled by 1/sqrt(head_dim).
+ */
+int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
+                       const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
+                       void* o, int64_t ldo, float* lse, void* stream);
+
+/*
+ * Backward of ttt_op_swa_forward given dout = dL/do: dq for every query (over
+ * the full band, cached keys included) and dk, dv for the keys at positions
+ * q_pos0 .. q_pos0+n_q-1 only (row i = position q_pos0 + i); keys of earlier
+ * positions are treated as constants.  dq: [n_q, lddq]; dk, dv: [n_q, lddkv].
+ * D_scratch: fp32 [n_heads * n_q] work space.
+ */
+int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
+                        const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
+                        const void* o, int64_t ldo, const float* lse, const void* dout, int64_t lddo, void* dq,
+                        int64_t lddq, void* dk, void* dv, int64_t lddkv, float* D_scratch, void* stream);
 
 /* Wait for `stream`; return TTT_ERR_TIMEOUT if a kernel launched through this
  * header recorded a bounded-wait timeout since the last call (then clears it). */

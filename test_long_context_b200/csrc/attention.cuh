@@ -1,0 +1,40 @@
+// Sliding-window attention launch interface.
+#pragma once
+#include "common.cuh"
+
+namespace ttt {
+
+// All row pitches in elements.  q/o/dout/dq: [n, heads*head_dim] chunk-local
+// rows (row i is absolute position p0 + i).  k/v: ring [ring, heads*head_dim],
+// slot = position % ring.  lse, D: [heads, ld_lse] fp32.  dk/dv: [n, ...]
+// gradients of the keys/values at positions p0 .. p0+n-1 (this chunk's own).
+struct SwaArgs {
+  int heads = 0, head_dim = 0;
+  int64_t n = 0, p0 = 0;
+  int64_t window = 1;
+  float scale = 1.f;
+  const void* q = nullptr;
+  int64_t ldq = 0;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int64_t ldkv = 0, ring = 1;
+  void* o = nullptr;
+  int64_t ldo = 0;
+  float* lse = nullptr;
+  int64_t ld_lse = 0;
+  // backward
+  const void* dout = nullptr;
+  int64_t lddo = 0;
+  void* dq = nullptr;
+  int64_t lddq = 0;
+  void* dk = nullptr;
+  void* dv = nullptr;
+  int64_t lddkv = 0;
+  float* D = nullptr;
+};
+
+int swa_forward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
+// Needs a.o, a.lse from the forward; writes D, dq, dk, dv.
+int swa_backward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
+
+}  // namespace ttt

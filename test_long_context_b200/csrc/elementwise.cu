@@ -1,0 +1,389 @@
+// Memory-bound kernels of the prefill loop (see elementwise.cuh).  Row
+// reductions use one warp per row and warp shuffles; everything else is one
+// thread per element.
+#include "elementwise.cuh"
+
+namespace ttt {
+namespace {
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+constexpr int ROW_WARPS = 8;  // rows per 256-thread block
+
+template <typename T>
+__global__ void embed_kernel(const int32_t* tok, const T* E, int64_t n, int d, int V, float* x, int* err) {
+  const int64_t row = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= n) return;
+  int t = tok[row];
+  if (t < 0 || t >= V) {
+    if (lane == 0) atomicOr(err, DEV_ERR_BAD_TOKEN);
+    t = 0;
+  }
+  const T* src = E + (int64_t)t * d;
+  float* dst = x + row * d;
+  for (int c = lane; c < d; c += 32) dst[c] = to_f32(src[c]);
+}
+
+template <typename T>
+__global__ void rmsnorm_fwd_kernel(const float* x, int64_t ldx, const float* g, float eps, int64_t n, int d, T* y,
+                                   int64_t ldy, float* rstd) {
+  const int64_t row = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= n) return;
+  const float* xr = x + row * ldx;
+  float ss = 0.f;
+  for (int c = lane; c < d; c += 32) ss = fmaf(xr[c], xr[c], ss);
+  ss = warp_sum(ss);
+  const float r = 1.f / sqrtf(ss / (float)d + eps);
+  T* yr = y + row * ldy;
+  for (int c = lane; c < d; c += 32) yr[c] = from_f32<T>(xr[c] * r * g[c]);
+  if (lane == 0 && rstd) rstd[row] = r;
+}
+
+template <typename T>
+__global__ void rmsnorm_bwd_kernel(const float* x, int64_t ldx, const float* rstd, const float* g, const float* dy,
+                                   int64_t lddy, const float* dres, int64_t ldres, int64_t n, int d, float* dx,
+                                   int64_t lddx, T* dx16, int64_t ld16) {
+  const int64_t row = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= n) return;
+  const float r = rstd[row];
+  const float* xr = x + row * ldx;
+  const float* dyr = dy + row * lddy;
+  float dot = 0.f;
+  for (int c = lane; c < d; c += 32) dot = fmaf(xr[c] * r, dyr[c] * g[c], dot);
+  dot = warp_sum(dot) / (float)d;
+  for (int c = lane; c < d; c += 32) {
+    const float u = dyr[c] * g[c];
+    float v = r * (u - xr[c] * r * dot);
+    if (dres) v += dres[row * ldres + c];
+    dx[row * lddx + c] = v;
+    if (dx16) dx16[row * ld16 + c] = from_f32<T>(v);
+  }
+}
+
+// One warp per (token, head); lane t handles rotation pairs t and t + 32.
+constexpr int MAXP = 2;  // pairs per lane (head_dim <= 128)
+
+__device__ __forceinline__ void rope_cs(int64_t pos, int t, int HD, double theta, float& c, float& s) {
+  const double inv = pow(theta, -2.0 * (double)t / (double)HD);
+  double sd, cd;
+  sincos((double)pos * inv, &sd, &cd);
+  c = (float)cd;
+  s = (float)sd;
+}
+
+template <typename T>
+__global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n,
+                                       int64_t p0, int H, int HD, float eps, double theta, T* qout, int64_t ldq,
+                                       T* kring, T* vring, int64_t ldkv, int64_t R, float* rq, float* rk) {
+  const int64_t w = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (w >= n * H) return;
+  const int64_t i = w / H;
+  const int h = (int)(w % H);
+  const int h2 = HD / 2;
+  const int D = H * HD;
+  const T* q = qkv + i * ldqkv + h * HD;
+  const T* k = q + D;
+  const T* v = q + 2 * D;
+  float q1[MAXP], q2[MAXP], k1[MAXP], k2[MAXP];
+  float sq = 0.f, sk = 0.f;
+#pragma unroll
+  for (int u = 0; u < MAXP; ++u) {
+    const int t = lane + 32 * u;
+    q1[u] = q2[u] = k1[u] = k2[u] = 0.f;
+    if (t < h2) {
+      q1[u] = to_f32(q[t]);
+      q2[u] = to_f32(q[t + h2]);
+      k1[u] = to_f32(k[t]);
+      k2[u] = to_f32(k[t + h2]);
+      sq += q1[u] * q1[u] + q2[u] * q2[u];
+      sk += k1[u] * k1[u] + k2[u] * k2[u];
+    }
+  }
+  sq = warp_sum(sq);
+  sk = warp_sum(sk);
+  const float rqv = 1.f / sqrtf(sq / (float)HD + eps);
+  const float rkv = 1.f / sqrtf(sk / (float)HD + eps);
+  const int64_t pos = p0 + i;
+  const int64_t slot = pos % R;
+  T* qo = qout + i * ldq + h * HD;
+  T* ko = kring + slot * ldkv + h * HD;
+  T* vo = vring + slot * ldkv + h * HD;
+#pragma unroll
+  for (int u = 0; u < MAXP; ++u) {
+    const int t = lane + 32 * u;
+    if (t < h2) {
+      float c, s;
+      rope_cs(pos, t, HD, theta, c, s);
+      const float a1 = q1[u] * rqv * gq[t], a2 = q2[u] * rqv * gq[t + h2];
+      const float b1 = k1[u] * rkv * gk[t], b2 = k2[u] * rkv * gk[t + h2];
+      qo[t] = from_f32<T>(a1 * c - a2 * s);
+      qo[t + h2] = from_f32<T>(a2 * c + a1 * s);
+      ko[t] = from_f32<T>(b1 * c - b2 * s);
+      ko[t + h2] = from_f32<T>(b2 * c + b1 * s);
+    }
+  }
+  for (int c = lane; c < HD; c += 32) vo[c] = v[c];
+  if (lane == 0) {
+    rq[i * H + h] = rqv;
+    rk[i * H + h] = rkv;
+  }
+}
+
+template <typename T>
+__global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq,
+                                       const float* gk, const float* rq, const float* rk, int64_t n, int64_t p0,
+                                       int H, int HD, double theta) {
+  const int64_t w = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (w >= n * H * 2) return;
+  const int which = (int)(w % 2);  // 0: q, 1: k
+  const int64_t ih = w / 2;
+  const int64_t i = ih / H;
+  const int h = (int)(ih % H);
+  const int h2 = HD / 2;
+  const int D = H * HD;
+  T* dv = dqkv + i * ld + which * D + h * HD;
+  const T* xv = qkv + i * ldqkv + which * D + h * HD;
+  const float* g = which ? gk : gq;
+  const float r = (which ? rk : rq)[i * H + h];
+  const int64_t pos = p0 + i;
+  float u1[MAXP], u2[MAXP], x1[MAXP], x2[MAXP];
+  float dot = 0.f;
+#pragma unroll
+  for (int u = 0; u < MAXP; ++u) {
+    const int t = lane + 32 * u;
+    u1[u] = u2[u] = x1[u] = x2[u] = 0.f;
+    if (t < h2) {
+      float c, s;
+      rope_cs(pos, t, HD, theta, c, s);
+      const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
+      // transpose of the rotation, then the gain
+      u1[u] = (d1 * c + d2 * s) * g[t];
+      u2[u] = (d2 * c - d1 * s) * g[t + h2];
+      x1[u] = to_f32(xv[t]) * r;
+      x2[u] = to_f32(xv[t + h2]) * r;
+      dot += x1[u] * u1[u] + x2[u] * u2[u];
+    }
+  }
+  dot = warp_sum(dot) / (float)HD;
+#pragma unroll
+  for (int u = 0; u < MAXP; ++u) {
+    const int t = lane + 32 * u;
+    if (t < h2) {
+      dv[t] = from_f32<T>(r * (u1[u] - x1[u] * dot));
+      dv[t + h2] = from_f32<T>(r * (u2[u] - x2[u] * dot));
+    }
+  }
+}
+
+template <typename T>
+__global__ void swiglu_bwd_kernel(const T* da, int64_t ldda, const T* gu, int64_t ldgu, int64_t n, int64_t nfeat,
+                                  T* dgu, int64_t lddgu) {
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t row = blockIdx.y;
+  if (j >= nfeat || row >= n) return;
+  const int64_t gc = 128 * (j / 64) + (j % 64), uc = gc + 64;
+  const float g = to_f32(gu[row * ldgu + gc]), u = to_f32(gu[row * ldgu + uc]);
+  const float a = to_f32(da[row * ldda + j]);
+  const float sg = 1.f / (1.f + expf(-g));
+  dgu[row * lddgu + gc] = from_f32<T>(a * u * sg * (1.f + g * (1.f - sg)));
+  dgu[row * lddgu + uc] = from_f32<T>(a * g * sg);
+}
+
+__global__ void ce_finalize_kernel(const float* pmax, const float* psum, int64_t part_ld, int tiles, const float* zt,
+                                   int64_t n, int64_t n_valid, float inv_nc, float* loss_out, float* lse_out,
+                                   float* scale) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float M = -INFINITY;
+  for (int t = 0; t < tiles; ++t) M = fmaxf(M, pmax[(int64_t)t * part_ld + i]);
+  float S = 0.f;
+  for (int t = 0; t < tiles; ++t) {
+    const float m = pmax[(int64_t)t * part_ld + i];
+    if (m > -INFINITY) S += psum[(int64_t)t * part_ld + i] * expf(m - M);
+  }
+  const float lse = M + logf(S);
+  lse_out[i] = lse;
+  const bool ok = i < n_valid;
+  loss_out[i] = ok ? lse - zt[i] : __int_as_float(0x7fc00000);
+  scale[i] = ok ? inv_nc : 0.f;
+}
+
+__global__ void check_tokens_kernel(const int32_t* tok, int64_t T, int V, int* err) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T) return;
+  const int32_t t = tok[i];
+  if (t < 0 || t >= V) atomicOr(err, DEV_ERR_BAD_TOKEN);
+}
+
+__global__ void chunk_targets_kernel(const int32_t* tok, int64_t T, int64_t p0, int64_t n, int32_t* targets) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  targets[i] = (p0 + i + 1 < T) ? tok[p0 + i + 1] : -1;
+}
+
+template <typename TS, typename TD>
+__global__ void interleave_kernel(const TS* gate, const TS* up, int f, int d, TD* out) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)2 * f * d) return;
+  const int64_t r = idx / d, c = idx % d;
+  const int64_t pair = r / 128, l = r % 128;
+  const TS v = l < 64 ? gate[(64 * pair + l) * d + c] : up[(64 * pair + l - 64) * d + c];
+  out[idx] = from_f32<TD>(to_f32(v));
+}
+
+__global__ void deinterleave_kernel(const float* in, int f, int d, float* gate, float* up) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)2 * f * d) return;
+  const int64_t r = idx / d, c = idx % d;
+  const int64_t pair = r / 128, l = r % 128;
+  if (l < 64) gate[(64 * pair + l) * d + c] = in[idx];
+  else up[(64 * pair + l - 64) * d + c] = in[idx];
+}
+
+template <typename TS, typename TD>
+__global__ void copy2d_kernel(const TS* src, int64_t lds, TD* dst, int64_t ldd, int64_t rows, int64_t cols) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * cols) return;
+  const int64_t r = idx / cols, c = idx % cols;
+  dst[r * ldd + c] = from_f32<TD>(to_f32(src[r * lds + c]));
+}
+
+inline unsigned row_blocks(int64_t rows) { return ceil_div(rows, ROW_WARPS); }
+
+}  // namespace
+
+template <typename T>
+int embed_gather(const int32_t* tok, const T* E, int64_t n, int d, int V, float* x, int* err, cudaStream_t s) {
+  embed_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(tok, E, n, d, V, x, err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int rmsnorm_fwd(const float* x, int64_t ldx, const float* g, float eps, int64_t n, int d, T* y, int64_t ldy,
+                float* rstd, cudaStream_t s) {
+  rmsnorm_fwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, g, eps, n, d, y, ldy, rstd);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int rmsnorm_bwd(const float* x, int64_t ldx, const float* rstd, const float* g, const float* dy, int64_t lddy,
+                const float* dres, int64_t ldres, int64_t n, int d, float* dx, int64_t lddx, T* dx16, int64_t ld16,
+                cudaStream_t s) {
+  rmsnorm_bwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, rstd, g, dy, lddy, dres, ldres, n, d, dx,
+                                                                  lddx, dx16, ld16);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n, int64_t p0, int H,
+                    int HD, float eps, double theta, T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv,
+                    int64_t R, float* rq, float* rk, cudaStream_t s) {
+  if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
+  qknorm_rope_fwd_kernel<T><<<row_blocks(n * H), 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, theta,
+                                                                          qout, ldq, kring, vring, ldkv, R, rq, rk);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int qknorm_rope_bwd(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq, const float* gk,
+                    const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, double theta,
+                    cudaStream_t s) {
+  if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
+  qknorm_rope_bwd_kernel<T><<<row_blocks(n * H * 2), 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n,
+                                                                              p0, H, HD, theta);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int swiglu_bwd(const T* da, int64_t ldda, const T* gu, int64_t ldgu, int64_t n, int64_t nfeat, T* dgu,
+               int64_t lddgu, cudaStream_t s) {
+  if (nfeat % 64) return set_error(TTT_ERR_INVALID_ARG, "swiglu_bwd: features must be a multiple of 64");
+  dim3 grid(ceil_div(nfeat, 256), (unsigned)n);
+  swiglu_bwd_kernel<T><<<grid, 256, 0, s>>>(da, ldda, gu, ldgu, n, nfeat, dgu, lddgu);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+int ce_finalize(const float* pmax, const float* psum, int64_t part_ld, int tiles, const float* zt, int64_t n,
+                int64_t n_valid, float inv_nc, float* loss_out, float* lse, float* scale, cudaStream_t s) {
+  ce_finalize_kernel<<<ceil_div(n, 128), 128, 0, s>>>(pmax, psum, part_ld, tiles, zt, n, n_valid, inv_nc, loss_out,
+                                                      lse, scale);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+int check_tokens(const int32_t* tok, int64_t T, int V, int* err, cudaStream_t s) {
+  check_tokens_kernel<<<ceil_div(T, 256), 256, 0, s>>>(tok, T, V, err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+int chunk_targets(const int32_t* tok, int64_t T, int64_t p0, int64_t n, int32_t* targets, cudaStream_t s) {
+  chunk_targets_kernel<<<ceil_div(n, 256), 256, 0, s>>>(tok, T, p0, n, targets);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename TS, typename TD>
+int interleave_gate_up(const TS* gate, const TS* up, int f, int d, TD* out, cudaStream_t s) {
+  if (f % 64) return set_error(TTT_ERR_INVALID_ARG, "interleave: d_ff must be a multiple of 64");
+  interleave_kernel<TS, TD><<<ceil_div((int64_t)2 * f * d, 256), 256, 0, s>>>(gate, up, f, d, out);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+template int interleave_gate_up<float, float>(const float*, const float*, int, int, float*, cudaStream_t);
+template int interleave_gate_up<bf16, bf16>(const bf16*, const bf16*, int, int, bf16*, cudaStream_t);
+
+int deinterleave_gate_up(const float* in, int f, int d, float* gate, float* up, cudaStream_t s) {
+  deinterleave_kernel<<<ceil_div((int64_t)2 * f * d, 256), 256, 0, s>>>(in, f, d, gate, up);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int copy2d_from_f32(const float* src, int64_t lds, T* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s) {
+  copy2d_kernel<float, T><<<ceil_div(rows * cols, 256), 256, 0, s>>>(src, lds, dst, ldd, rows, cols);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+template <typename T>
+int copy2d(const T* src, int64_t lds, T* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s) {
+  copy2d_kernel<T, T><<<ceil_div(rows * cols, 256), 256, 0, s>>>(src, lds, dst, ldd, rows, cols);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+#define TTT_INST(T)                                                                                              \
+  template int embed_gather<T>(const int32_t*, const T*, int64_t, int, int, float*, int*, cudaStream_t);        \
+  template int rmsnorm_fwd<T>(const float*, int64_t, const float*, float, int64_t, int, T*, int64_t, float*,    \
+                              cudaStream_t);                                                                    \
+  template int rmsnorm_bwd<T>(const float*, int64_t, const float*, const float*, const float*, int64_t,         \
+                              const float*, int64_t, int64_t, int, float*, int64_t, T*, int64_t, cudaStream_t); \
+  template int qknorm_rope_fwd<T>(const T*, int64_t, const float*, const float*, int64_t, int64_t, int, int,    \
+                                  float, double, T*, int64_t, T*, T*, int64_t, int64_t, float*, float*,         \
+                                  cudaStream_t);                                                                \
+  template int qknorm_rope_bwd<T>(T*, int64_t, const T*, int64_t, const float*, const float*, const float*,     \
+                                  const float*, int64_t, int64_t, int, int, double, cudaStream_t);              \
+  template int swiglu_bwd<T>(const T*, int64_t, const T*, int64_t, int64_t, int64_t, T*, int64_t, cudaStream_t); \
+  template int copy2d_from_f32<T>(const float*, int64_t, T*, int64_t, int64_t, int64_t, cudaStream_t);          \
+  template int copy2d<T>(const T*, int64_t, T*, int64_t, int64_t, int64_t, cudaStream_t);
+
+TTT_INST(float)
+TTT_INST(bf16)
+
+}  // namespace ttt

@@ -1,3 +1,653 @@
-// placeholder, replaced below
-#include "common.cuh"
-extern "C" const char* ttt_last_error(ttt_ctx*) { return ttt::last_error_message(); }
+// The TTT-E2E prefill engine behind include/ttt.h.
+//
+// Schedule of ttt_prefill (算法 1 of the reading notes, eq. (9)):
+//   Blocks 0 .. L-n_u-1 have no fast weights, so their outputs depend only
+//   on the tokens.  They run over a super-chunk of S = spc*b positions at a
+//   time (large-M GEMMs), with their own KV rings of S + k slots.
+//   Blocks L-n_u .. L-1 then run chunk by chunk (b positions): forward with
+//   the current fast weights, per-token losses recorded, then - for every
+//   full chunk - the backward through these blocks and one SGD step on each
+//   block's fast MLP, applied right after that block's data gradients.
+// Everything in the loop is device work on one stream; the host only
+// enqueues.
+#include <cmath>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "../../include/ttt.h"
+#include "attention.cuh"
+#include "elementwise.cuh"
+#include "gemm.cuh"
+
+struct ttt_ctx {
+  virtual ~ttt_ctx() = default;
+  virtual int prefill(const int32_t* tok, int64_t T, float* losses, float* const* fast_out) = 0;
+  virtual int reset() = 0;
+  virtual int sync() = 0;
+  std::string last_error = "no error";
+  int64_t launches = 0;
+};
+
+namespace ttt {
+namespace {
+
+// Device allocations owned by a context, released together.
+struct Arena {
+  std::vector<void*> blocks;
+  cudaStream_t stream = nullptr;
+  ~Arena() {
+    for (void* p : blocks) cudaFree(p);
+  }
+  template <typename T>
+  int alloc(T** out, int64_t count) {
+    void* p = nullptr;
+    const size_t bytes = (size_t)(count > 0 ? count : 1) * sizeof(T);
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return set_error(TTT_ERR_OOM, "cudaMalloc of " + std::to_string(bytes) + " bytes failed");
+    }
+    blocks.push_back(p);
+    e = cudaMemsetAsync(p, 0, bytes, stream);
+    if (e != cudaSuccess) return set_cuda_error(e, "cudaMemsetAsync", __FILE__, __LINE__);
+    *out = reinterpret_cast<T*>(p);
+    return TTT_OK;
+  }
+};
+
+#define TRY(expr)                 \
+  do {                            \
+    int rc_ = (expr);             \
+    if (rc_ != TTT_OK) return rc_; \
+  } while (0)
+
+template <typename T>
+struct ActTraits;
+template <>
+struct ActTraits<float> {
+  static constexpr bool bf = false;
+  static constexpr int store_epi = EPI_STORE_F32;
+};
+template <>
+struct ActTraits<bf16> {
+  static constexpr bool bf = true;
+  static constexpr int store_epi = EPI_STORE_BF16;
+};
+
+// One GEMM of the schedule, with its tensor maps built once (bf16 mode).
+struct Gemm {
+  GemmShape shape;
+  int epi = 0;
+  EpiArgs args;
+  TcGemm tc;
+  bool bf = false;
+};
+
+template <typename T>
+class Engine final : public ttt_ctx {
+ public:
+  Engine(const ttt_config& cfg, const ttt_weights& w, float eta, int k, int b, int nu, cudaStream_t s)
+      : cfg_(cfg), eta_(eta), k_(k), b_(b), nu_(nu), st_(s) {
+    wt_ = w;
+    layers_.assign(w.layers, w.layers + cfg.n_layers);
+    fast_init_.assign(w.fast, w.fast + nu);
+    wt_.layers = layers_.data();
+    wt_.fast = fast_init_.data();
+  }
+
+  int init();
+  int prefill(const int32_t* tok, int64_t T_, float* losses, float* const* fast_out) override;
+  int reset() override;
+  int sync() override;
+
+ private:
+  static constexpr bool BF = ActTraits<T>::bf;
+  static constexpr int STORE = ActTraits<T>::store_epi;
+
+  int prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, const EpiArgs& args);
+  int run(Gemm& g, int64_t rows);  // rows overrides the M extent (chunk/super-chunk length)
+  int bottom_layers(const int32_t* tok, int64_t s0, int64_t S);
+  int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
+  int count(int rc) {
+    ++launches;
+    return rc;
+  }
+  SwaArgs swa_args(const T* q, int64_t n, int64_t p0, const T* kr, const T* vr, int64_t ring, T* o, float* lse,
+                   int64_t ld_lse) const {
+    SwaArgs a;
+    a.heads = (int)H_;
+    a.head_dim = (int)HD_;
+    a.n = n;
+    a.p0 = p0;
+    a.window = k_;
+    a.scale = scale_;
+    a.q = q;
+    a.ldq = d_;
+    a.k = kr;
+    a.v = vr;
+    a.ldkv = d_;
+    a.ring = ring;
+    a.o = o;
+    a.ldo = d_;
+    a.lse = lse;
+    a.ld_lse = ld_lse;
+    return a;
+  }
+  float* master_gu(int i) { return BF ? m_gu_[i] : reinterpret_cast<float*>(wgu_[nbot_ + i]) + 2 * f_ * d_; }
+  float* master_d(int i) { return BF ? m_d_[i] : reinterpret_cast<float*>(wd_[nbot_ + i]) + f_; }
+  int64_t master_d_ld() const { return BF ? f_ : 2 * f_; }
+
+  ttt_config cfg_;
+  float eta_;
+  int k_, b_, nu_;
+  cudaStream_t st_;
+  ttt_weights wt_;
+  std::vector<ttt_layer_weights> layers_;
+  std::vector<ttt_fast_weights> fast_init_;
+  Arena arena_;
+  bool fresh_ = true;
+  int* err_ = nullptr;
+
+  int64_t d_ = 0, f_ = 0, H_ = 0, HD_ = 0, V_ = 0, L_ = 0, nbot_ = 0;
+  int64_t S_ = 0, R1_ = 0, R_ = 0, Vc_ = 0, nvc_ = 0, ce_tiles_ = 0;
+  float scale_ = 1.f;
+
+  // weights rearranged for the GEMMs
+  std::vector<T*> wqkv_;   // [3d, d] per block
+  std::vector<T*> wgu_;    // bottom: [2f, d]; top: [4f, d] (static | fast), interleaved gate/up
+  std::vector<T*> wd_;     // top: [d, 2f] (static | fast); bottom: caller's [d, f]
+  std::vector<float*> m_gu_, m_d_;        // fp32 masters (bf16 mode) per top block
+  std::vector<float*> init_gu_, init_d_;  // W_init copies per top block
+  // phase-1 buffers
+  float* xs_ = nullptr;
+  T *hs_ = nullptr, *qkvs_ = nullptr, *qs_ = nullptr, *os_ = nullptr, *as_ = nullptr;
+  float *rs_ = nullptr, *rqs_ = nullptr, *rks_ = nullptr, *lses_ = nullptr;
+  std::vector<T*> kb_, vb_;  // bottom rings [R1, d]
+  // top blocks, per block i
+  std::vector<float*> xin_, r1_, xmid_, r2_, rq_, rk_, lse_;
+  std::vector<T*> h_, qkv_, q_, o_, h2_, gu_, a_, kt_, vt_;
+  float *xf_ = nullptr, *rf_ = nullptr;
+  T* hf_ = nullptr;
+  float *pmax_ = nullptr, *psum_ = nullptr, *zt_ = nullptr, *lsef_ = nullptr, *scl_ = nullptr;
+  int32_t* tgt_ = nullptr;
+  // backward
+  float *dx_ = nullptr, *dxm_ = nullptr, *dhf_ = nullptr, *dh2_ = nullptr, *dh_ = nullptr, *Dbuf_ = nullptr;
+  T *dx16_ = nullptr, *dxm16_ = nullptr, *dz_ = nullptr, *da_ = nullptr, *dgu_ = nullptr, *do_ = nullptr,
+    *dqkv_ = nullptr;
+  // GEMM plans
+  std::vector<Gemm> g_bot_;  // 4 per bottom block: qkv, o, gu, down
+  std::vector<Gemm> g_top_;  // 10 per top block: qkv, o, gu, down, da, dh2, wd, wgu, do, dh
+  Gemm g_head_;
+  std::vector<Gemm> g_ce_dz_, g_ce_dh_;
+};
+
+template <typename T>
+int Engine<T>::prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, const EpiArgs& args) {
+  g.shape.a_mn = a_mn;
+  g.shape.b_mn = b_mn;
+  g.shape.a = a;
+  g.shape.b = b;
+  g.epi = epi;
+  g.args = args;
+  g.bf = BF;
+  if (BF) {
+    g.tc.act_bf16 = 1;
+    TRY(tc_gemm_prepare(&g.tc, g.shape, epi, args));
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::run(Gemm& g, int64_t rows) {
+  ++launches;
+  if (BF) {
+    TcGemm tc = g.tc;
+    tc.args = g.args;
+    if (rows > 0 && !tc.a_mn) tc.M = rows;
+    return tc_gemm_launch(tc, st_, err_);
+  }
+  GemmShape s = g.shape;
+  if (rows > 0 && !s.a_mn) s.a.rows = rows;
+  return simt_gemm(s, g.epi, g.args, st_);
+}
+
+template <typename T>
+int Engine<T>::init() {
+  L_ = cfg_.n_layers;
+  d_ = cfg_.d_model;
+  f_ = cfg_.d_ff;
+  H_ = cfg_.n_heads;
+  HD_ = cfg_.head_dim;
+  V_ = cfg_.vocab;
+  nbot_ = L_ - nu_;
+  scale_ = 1.f / std::sqrt((float)HD_);
+  const int64_t d = d_, f = f_, b = b_;
+  arena_.stream = st_;
+  TRY(arena_.alloc(&err_, 1));
+
+  // Super-chunk length for the fast-weight-free blocks: about 16K positions.
+  int64_t spc = std::max<int64_t>(1, 16384 / b);
+  S_ = spc * b;
+  R1_ = S_ + k_;
+  R_ = k_ + b;
+
+  // ---- weights ----------------------------------------------------------------------------
+  wqkv_.resize(L_);
+  wgu_.resize(L_);
+  wd_.resize(L_);
+  for (int64_t l = 0; l < L_; ++l) {
+    const ttt_layer_weights& lw = wt_.layers[l];
+    TRY(arena_.alloc(&wqkv_[l], 3 * d * d));
+    TTT_CUDA_TRY(cudaMemcpyAsync(wqkv_[l], lw.wq, d * d * sizeof(T), cudaMemcpyDeviceToDevice, st_));
+    TTT_CUDA_TRY(cudaMemcpyAsync(wqkv_[l] + d * d, lw.wk, d * d * sizeof(T), cudaMemcpyDeviceToDevice, st_));
+    TTT_CUDA_TRY(cudaMemcpyAsync(wqkv_[l] + 2 * d * d, lw.wv, d * d * sizeof(T), cudaMemcpyDeviceToDevice, st_));
+  }
+  // gate/up rows interleaved in (gate 64 | up 64) blocks; the top blocks append the fast half
+  m_gu_.assign(nu_, nullptr);
+  m_d_.assign(nu_, nullptr);
+  init_gu_.assign(nu_, nullptr);
+  init_d_.assign(nu_, nullptr);
+  for (int64_t l = 0; l < L_; ++l) {
+    const ttt_layer_weights& lw = wt_.layers[l];
+    const bool top = l >= nbot_;
+    TRY(arena_.alloc(&wgu_[l], (top ? 4 : 2) * f * d));
+    TRY((interleave_gate_up<T, T>(reinterpret_cast<const T*>(lw.w_gate), reinterpret_cast<const T*>(lw.w_up), (int)f,
+                                 (int)d, wgu_[l], st_)));
+    if (top) {
+      const int64_t i = l - nbot_;
+      const ttt_fast_weights& fw = wt_.fast[i];
+      TRY(arena_.alloc(&init_gu_[i], 2 * f * d));
+      TRY(arena_.alloc(&init_d_[i], d * f));
+      TRY((interleave_gate_up<float, float>(fw.w_gate, fw.w_up, (int)f, (int)d, init_gu_[i], st_)));
+      TTT_CUDA_TRY(cudaMemcpyAsync(init_d_[i], fw.w_down, d * f * sizeof(float), cudaMemcpyDeviceToDevice, st_));
+      TRY(arena_.alloc(&wd_[l], d * 2 * f));
+      TRY(copy2d<T>(reinterpret_cast<const T*>(lw.w_down), f, wd_[l], 2 * f, d, f, st_));
+      if (BF) {
+        TRY(arena_.alloc(&m_gu_[i], 2 * f * d));
+        TRY(arena_.alloc(&m_d_[i], d * f));
+      }
+    } else {
+      wd_[l] = const_cast<T*>(reinterpret_cast<const T*>(lw.w_down));
+    }
+  }
+  TRY(reset());
+
+  // ---- activations ------------------------------------------------------------------------
+  if (nbot_ > 0) {
+    TRY(arena_.alloc(&hs_, S_ * d));
+    TRY(arena_.alloc(&qkvs_, S_ * 3 * d));
+    TRY(arena_.alloc(&qs_, S_ * d));
+    TRY(arena_.alloc(&os_, S_ * d));
+    TRY(arena_.alloc(&as_, S_ * f));
+    TRY(arena_.alloc(&rs_, S_));
+    TRY(arena_.alloc(&rqs_, S_ * H_));
+    TRY(arena_.alloc(&rks_, S_ * H_));
+    TRY(arena_.alloc(&lses_, H_ * S_));
+    kb_.resize(nbot_);
+    vb_.resize(nbot_);
+    for (int64_t l = 0; l < nbot_; ++l) {
+      TRY(arena_.alloc(&kb_[l], R1_ * d));
+      TRY(arena_.alloc(&vb_[l], R1_ * d));
+    }
+  }
+  TRY(arena_.alloc(&xs_, S_ * d));
+  auto per = [&](auto& vec) { vec.assign(nu_, nullptr); };
+  per(xin_); per(r1_); per(xmid_); per(r2_); per(rq_); per(rk_); per(lse_);
+  per(h_); per(qkv_); per(q_); per(o_); per(h2_); per(gu_); per(a_); per(kt_); per(vt_);
+  for (int i = 0; i < nu_; ++i) {
+    if (i > 0) TRY(arena_.alloc(&xin_[i], b * d));  // xin_[0] points into xs_
+    TRY(arena_.alloc(&r1_[i], b));
+    TRY(arena_.alloc(&xmid_[i], b * d));
+    TRY(arena_.alloc(&r2_[i], b));
+    TRY(arena_.alloc(&rq_[i], b * H_));
+    TRY(arena_.alloc(&rk_[i], b * H_));
+    TRY(arena_.alloc(&lse_[i], H_ * b));
+    TRY(arena_.alloc(&h_[i], b * d));
+    TRY(arena_.alloc(&qkv_[i], b * 3 * d));
+    TRY(arena_.alloc(&q_[i], b * d));
+    TRY(arena_.alloc(&o_[i], b * d));
+    TRY(arena_.alloc(&h2_[i], b * d));
+    TRY(arena_.alloc(&gu_[i], b * 4 * f));
+    TRY(arena_.alloc(&a_[i], b * 2 * f));
+    TRY(arena_.alloc(&kt_[i], R_ * d));
+    TRY(arena_.alloc(&vt_[i], R_ * d));
+  }
+  TRY(arena_.alloc(&xf_, b * d));
+  TRY(arena_.alloc(&rf_, b));
+  TRY(arena_.alloc(&hf_, b * d));
+  ce_tiles_ = BF ? tc_ce_tiles(V_, tc_pick_bn(b, V_, 0)) : (V_ + 127) / 128;
+  TRY(arena_.alloc(&pmax_, ce_tiles_ * b));
+  TRY(arena_.alloc(&psum_, ce_tiles_ * b));
+  TRY(arena_.alloc(&zt_, b));
+  TRY(arena_.alloc(&lsef_, b));
+  TRY(arena_.alloc(&scl_, b));
+  TRY(arena_.alloc(&tgt_, b));
+  TRY(arena_.alloc(&dx_, b * d));
+  TRY(arena_.alloc(&dxm_, b * d));
+  TRY(arena_.alloc(&dhf_, b * d));
+  TRY(arena_.alloc(&dh2_, b * d));
+  TRY(arena_.alloc(&dh_, b * d));
+  TRY(arena_.alloc(&Dbuf_, H_ * b));
+  TRY(arena_.alloc(&dx16_, b * d));
+  TRY(arena_.alloc(&dxm16_, b * d));
+  // vocab chunk of the LM-head backward: the dz chunk stays L2-sized (<= 48 MB)
+  {
+    const int64_t max_cols = std::max<int64_t>(256, (48ll << 20) / (b * (int64_t)sizeof(T)) / 256 * 256);
+    nvc_ = (V_ + max_cols - 1) / max_cols;
+    Vc_ = ((V_ + nvc_ - 1) / nvc_ + 255) / 256 * 256;
+    nvc_ = (V_ + Vc_ - 1) / Vc_;
+  }
+  TRY(arena_.alloc(&dz_, b * Vc_));
+  TRY(arena_.alloc(&da_, b * 2 * f));
+  TRY(arena_.alloc(&dgu_, b * 4 * f));
+  TRY(arena_.alloc(&do_, b * d));
+  TRY(arena_.alloc(&dqkv_, b * 3 * d));
+
+  // ---- GEMM plans -------------------------------------------------------------------------
+  EpiArgs e;
+  g_bot_.resize(4 * nbot_);
+  for (int64_t l = 0; l < nbot_; ++l) {
+    Gemm* g = &g_bot_[4 * l];
+    e = EpiArgs{}; e.c = qkvs_; e.ldc = 3 * d;
+    TRY(prep(g[0], 0, MatView{hs_, S_, d, d}, 0, MatView{wqkv_[l], 3 * d, d, d}, STORE, e));
+    e = EpiArgs{}; e.c = xs_; e.ldc = d;
+    TRY(prep(g[1], 0, MatView{os_, S_, d, d}, 0, MatView{wt_.layers[l].wo, d, d, d}, EPI_ADD_F32, e));
+    e = EpiArgs{}; e.c = as_; e.ldc = f;
+    TRY(prep(g[2], 0, MatView{hs_, S_, d, d}, 0, MatView{wgu_[l], 2 * f, d, d}, EPI_SWIGLU, e));
+    e = EpiArgs{}; e.c = xs_; e.ldc = d;
+    TRY(prep(g[3], 0, MatView{as_, S_, f, f}, 0, MatView{wd_[l], d, f, f}, EPI_ADD_F32, e));
+  }
+  g_top_.resize(10 * nu_);
+  for (int i = 0; i < nu_; ++i) {
+    const int64_t l = nbot_ + i;
+    Gemm* g = &g_top_[10 * i];
+    e = EpiArgs{}; e.c = qkv_[i]; e.ldc = 3 * d;
+    TRY(prep(g[0], 0, MatView{h_[i], b, d, d}, 0, MatView{wqkv_[l], 3 * d, d, d}, STORE, e));
+    e = EpiArgs{}; e.c = xmid_[i]; e.ldc = d; e.ldc2 = d;  // c2 = x_in, set per chunk
+    TRY(prep(g[1], 0, MatView{o_[i], b, d, d}, 0, MatView{wt_.layers[l].wo, d, d, d}, EPI_ADD_F32, e));
+    e = EpiArgs{}; e.c = a_[i]; e.ldc = 2 * f; e.c2 = gu_[i]; e.ldc2 = 4 * f;
+    TRY(prep(g[2], 0, MatView{h2_[i], b, d, d}, 0, MatView{wgu_[l], 4 * f, d, d}, EPI_SWIGLU, e));
+    e = EpiArgs{}; e.c = (i + 1 < nu_) ? xin_[i + 1] : xf_; e.ldc = d; e.c2 = xmid_[i]; e.ldc2 = d;
+    TRY(prep(g[3], 0, MatView{a_[i], b, 2 * f, 2 * f}, 0, MatView{wd_[l], d, 2 * f, 2 * f}, EPI_ADD_F32, e));
+    // backward: da (fast half only in the lowest updated block)
+    if (i == 0) {
+      e = EpiArgs{}; e.c = da_ + f; e.ldc = 2 * f;
+      TRY(prep(g[4], 0, MatView{dx16_, b, d, d}, 1, MatView{wd_[l] + f, d, f, 2 * f}, STORE, e));
+    } else {
+      e = EpiArgs{}; e.c = da_; e.ldc = 2 * f;
+      TRY(prep(g[4], 0, MatView{dx16_, b, d, d}, 1, MatView{wd_[l], d, 2 * f, 2 * f}, STORE, e));
+      e = EpiArgs{}; e.c = dh2_; e.ldc = d;
+      TRY(prep(g[5], 0, MatView{dgu_, b, 4 * f, 4 * f}, 1, MatView{wgu_[l], 4 * f, d, d}, EPI_STORE_F32, e));
+    }
+    // weight gradients + SGD on the fast halves
+    e = EpiArgs{}; e.alpha = eta_;
+    if (BF) { e.c = m_d_[i]; e.ldc = f; e.c2 = wd_[l] + f; e.ldc2 = 2 * f; }
+    else { e.c = wd_[l] + f; e.ldc = 2 * f; }
+    TRY(prep(g[6], 1, MatView{dx16_, b, d, d}, 1, MatView{a_[i] + f, b, f, 2 * f}, EPI_SGD, e));
+    e = EpiArgs{}; e.alpha = eta_;
+    if (BF) { e.c = m_gu_[i]; e.ldc = d; e.c2 = wgu_[l] + 2 * f * d; e.ldc2 = d; }
+    else { e.c = wgu_[l] + 2 * f * d; e.ldc = d; }
+    TRY(prep(g[7], 1, MatView{dgu_ + 2 * f, b, 2 * f, 4 * f}, 1, MatView{h2_[i], b, d, d}, EPI_SGD, e));
+    if (i > 0) {
+      e = EpiArgs{}; e.c = do_; e.ldc = d;
+      TRY(prep(g[8], 0, MatView{dxm16_, b, d, d}, 1, MatView{wt_.layers[l].wo, d, d, d}, STORE, e));
+      e = EpiArgs{}; e.c = dh_; e.ldc = d;
+      TRY(prep(g[9], 0, MatView{dqkv_, b, 3 * d, 3 * d}, 1, MatView{wqkv_[l], 3 * d, d, d}, EPI_STORE_F32, e));
+    }
+  }
+  e = EpiArgs{}; e.row_i = tgt_; e.part_max = pmax_; e.part_sum = psum_; e.target_logit = zt_; e.part_ld = b;
+  TRY(prep(g_head_, 0, MatView{hf_, b, d, d}, 0, MatView{wt_.lm_head, V_, d, d}, EPI_CE_FWD, e));
+  g_ce_dz_.resize(nvc_);
+  g_ce_dh_.resize(nvc_);
+  for (int64_t c = 0; c < nvc_; ++c) {
+    const int64_t v0 = c * Vc_, vn = std::min<int64_t>(Vc_, V_ - v0);
+    const T* hv = reinterpret_cast<const T*>(wt_.lm_head) + v0 * d;
+    e = EpiArgs{}; e.c = dz_; e.ldc = Vc_; e.row_f = lsef_; e.row_g = scl_; e.row_i = tgt_; e.col_offset = v0;
+    TRY(prep(g_ce_dz_[c], 0, MatView{hf_, b, d, d}, 0, MatView{hv, vn, d, d}, EPI_CE_BWD, e));
+    e = EpiArgs{}; e.c = dhf_; e.ldc = d;
+    TRY(prep(g_ce_dh_[c], 0, MatView{dz_, b, vn, Vc_}, 1, MatView{hv, vn, d, d}, c == 0 ? EPI_STORE_F32 : EPI_ADD_F32,
+             e));
+  }
+  TTT_CUDA_TRY(cudaStreamSynchronize(st_));
+  return TTT_OK;
+}
+
+
+template <typename T>
+int Engine<T>::reset() {
+  const int64_t d = d_, f = f_;
+  for (int i = 0; i < nu_; ++i) {
+    const int64_t l = nbot_ + i;
+    TTT_CUDA_TRY(cudaMemcpyAsync(master_gu(i), init_gu_[i], 2 * f * d * sizeof(float), cudaMemcpyDeviceToDevice, st_));
+    TRY(count(copy2d<float>(init_d_[i], f, master_d(i), master_d_ld(), d, f, st_)));
+    if (BF) {
+      TRY(count(copy2d_from_f32<T>(init_gu_[i], d, wgu_[l] + 2 * f * d, d, 2 * f, d, st_)));
+      TRY(count(copy2d_from_f32<T>(init_d_[i], f, wd_[l] + f, 2 * f, d, f, st_)));
+    }
+  }
+  fresh_ = true;
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::sync() {
+  TTT_CUDA_TRY(cudaStreamSynchronize(st_));
+  int h = 0;
+  TTT_CUDA_TRY(cudaMemcpy(&h, err_, sizeof(int), cudaMemcpyDeviceToHost));
+  if (h) {
+    TTT_CUDA_TRY(cudaMemset(err_, 0, sizeof(int)));
+    TTT_CUDA_TRY(cudaDeviceSynchronize());
+    if (h & DEV_ERR_BAD_TOKEN) return set_error(TTT_ERR_INVALID_ARG, "a token id lies outside [0, vocab)");
+    return set_error(TTT_ERR_TIMEOUT, "a kernel's bounded wait timed out (device watchdog)");
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
+  const int64_t d = d_;
+  const float eps = cfg_.norm_eps;
+  const double theta = cfg_.rope_theta;
+  TRY(count(embed_gather<T>(tok + s0, reinterpret_cast<const T*>(wt_.embed), S, (int)d, (int)V_, xs_, err_, st_)));
+  for (int64_t l = 0; l < nbot_; ++l) {
+    const ttt_layer_weights& lw = wt_.layers[l];
+    Gemm* g = &g_bot_[4 * l];
+    TRY(count(rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_)));
+    TRY(run(g[0], S));
+    TRY(count(qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
+                                 kb_[l], vb_[l], d, R1_, rqs_, rks_, st_)));
+    TRY(count(swa_forward(swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_), BF, st_)));
+    TRY(run(g[1], S));
+    TRY(count(rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_)));
+    TRY(run(g[2], S));
+    TRY(run(g[3], S));
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses) {
+  const int64_t d = d_, f = f_, b = b_;
+  const float eps = cfg_.norm_eps;
+  const double theta = cfg_.rope_theta;
+  const int64_t n_valid = std::max<int64_t>(0, std::min<int64_t>(n, T_ - 1 - p0));
+  TRY(count(chunk_targets(tok, T_, p0, n, tgt_, st_)));
+  // ---- forward of the updated blocks with the current fast weights ----
+  for (int i = 0; i < nu_; ++i) {
+    const int64_t l = nbot_ + i;
+    const ttt_layer_weights& lw = wt_.layers[l];
+    Gemm* g = &g_top_[10 * i];
+    const float* xin = i == 0 ? x0 : xin_[i];
+    TRY(count(rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_)));
+    TRY(run(g[0], n));
+    TRY(count(qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
+                                 kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_)));
+    TRY(count(swa_forward(swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b), BF, st_)));
+    g[1].args.c2 = const_cast<float*>(xin);
+    TRY(run(g[1], n));
+    TRY(count(rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_)));
+    TRY(run(g[2], n));
+    TRY(run(g[3], n));
+  }
+  TRY(count(rmsnorm_fwd<T>(xf_, d, wt_.final_norm, eps, n, (int)d, hf_, d, rf_, st_)));
+  TRY(run(g_head_, n));
+  TRY(count(ce_finalize(pmax_, psum_, b, (int)ce_tiles_, zt_, n, n_valid, n_valid ? 1.f / (float)n_valid : 0.f,
+                        losses + p0, lsef_, scl_, st_)));
+  if (n < b || n_valid == 0) return TTT_OK;  // a trailing partial chunk is scored only
+
+  // ---- backward through the updated blocks, SGD on each fast MLP ----
+  for (int64_t c = 0; c < nvc_; ++c) {
+    TRY(run(g_ce_dz_[c], n));
+    TRY(run(g_ce_dh_[c], n));
+  }
+  TRY(count(rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_)));
+  for (int i = nu_ - 1; i >= 0; --i) {
+    const int64_t l = nbot_ + i;
+    const ttt_layer_weights& lw = wt_.layers[l];
+    Gemm* g = &g_top_[10 * i];
+    TRY(run(g[4], n));
+    if (i == 0) {
+      TRY(count(swiglu_bwd<T>(da_ + f, 2 * f, gu_[i] + 2 * f, 4 * f, n, f, dgu_ + 2 * f, 4 * f, st_)));
+    } else {
+      TRY(count(swiglu_bwd<T>(da_, 2 * f, gu_[i], 4 * f, n, 2 * f, dgu_, 4 * f, st_)));
+      TRY(run(g[5], n));  // reads the fast shadow before its update
+    }
+    TRY(run(g[6], 0));  // W_down fast -= eta * dx^T a_f
+    TRY(run(g[7], 0));  // W_gate/up fast -= eta * dgu_f^T h2
+    if (i == 0) break;  // nothing below the lowest fast block depends on W
+    TRY(count(rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_)));
+    TRY(run(g[8], n));
+    SwaArgs a = swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b);
+    a.dout = do_;
+    a.lddo = d;
+    a.dq = dqkv_;
+    a.lddq = 3 * d;
+    a.dk = dqkv_ + d;
+    a.dv = dqkv_ + 2 * d;
+    a.lddkv = 3 * d;
+    a.D = Dbuf_;
+    TRY(count(swa_backward(a, BF, st_)));
+    launches += 2;  // the backward launches three kernels
+    TRY(count(qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
+                                 (int)HD_, theta, st_)));
+    TRY(run(g[9], n));
+    TRY(count(rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_)));
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* const* fast_out) {
+  if (!fresh_) return set_error(TTT_ERR_STATE, "ttt_prefill needs a fresh context (call ttt_reset)");
+  if (!tok || !losses || T_ < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: bad argument");
+  fresh_ = false;
+  launches = 0;
+  TRY(count(check_tokens(tok, T_, (int)V_, err_, st_)));
+  for (int64_t s0 = 0; s0 < T_; s0 += S_) {
+    const int64_t S = std::min<int64_t>(S_, T_ - s0);
+    TRY(bottom_layers(tok, s0, S));
+    for (int64_t p0 = s0; p0 < s0 + S; p0 += b_) {
+      const int64_t n = std::min<int64_t>(b_, T_ - p0);
+      TRY(chunk(tok, T_, p0, n, xs_ + (p0 - s0) * d_, losses));
+    }
+  }
+  if (fast_out) {
+    const int64_t d = d_, f = f_;
+    for (int i = 0; i < nu_; ++i) {
+      float* og = fast_out[3 * i];
+      float* ou = fast_out[3 * i + 1];
+      float* od = fast_out[3 * i + 2];
+      if (!og || !ou || !od) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: NULL entry in fast_out");
+      TRY(count(deinterleave_gate_up(master_gu(i), (int)f, (int)d, og, ou, st_)));
+      TRY(count(copy2d<float>(master_d(i), master_d_ld(), od, f, d, f, st_)));
+    }
+  }
+  return TTT_OK;
+}
+
+}  // namespace
+}  // namespace ttt
+
+// ---- C ABI ----------------------------------------------------------------------------------------
+
+using namespace ttt;
+
+static int fail(ttt_ctx* ctx, int rc) {
+  if (rc != TTT_OK && ctx) ctx->last_error = last_error_message();
+  return rc;
+}
+
+extern "C" int ttt_init(const ttt_config* c, const ttt_weights* w, float eta, int32_t k, int32_t b, int32_t nu,
+                        void* stream, ttt_ctx** out) {
+  if (out) *out = nullptr;
+  if (!c || !w || !out) return set_error(TTT_ERR_INVALID_ARG, "ttt_init: NULL argument");
+  const bool hd_ok = c->head_dim == 32 || c->head_dim == 64 || c->head_dim == 80 || c->head_dim == 96 ||
+                     c->head_dim == 128;
+  if (c->n_layers < 1 || c->n_heads < 1 || c->d_model != c->n_heads * c->head_dim || c->d_model % 8 ||
+      c->d_ff < 64 || c->d_ff % 64 || c->vocab < 1 || !(c->norm_eps > 0.f) || !(c->rope_theta > 0.f))
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_init: bad model configuration");
+  if (!hd_ok) return set_error(TTT_ERR_UNSUPPORTED, "ttt_init: head_dim must be 32, 64, 80, 96 or 128");
+  if (c->dtype != TTT_F32 && c->dtype != TTT_BF16) return set_error(TTT_ERR_INVALID_ARG, "ttt_init: bad dtype");
+  if (!std::isfinite(eta) || k < 1 || b < 1 || nu < 1 || nu > c->n_layers)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_init: need finite eta, k >= 1, b >= 1, 1 <= n_updated <= n_layers");
+  if (!w->embed || !w->layers || !w->fast || !w->final_norm || !w->lm_head)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_init: NULL weight pointer");
+  for (int l = 0; l < c->n_layers; ++l) {
+    const ttt_layer_weights& lw = w->layers[l];
+    if (!lw.attn_norm || !lw.wq || !lw.wk || !lw.wv || !lw.wo || !lw.q_norm || !lw.k_norm || !lw.mlp_norm ||
+        !lw.w_gate || !lw.w_up || !lw.w_down)
+      return set_error(TTT_ERR_INVALID_ARG, "ttt_init: NULL weight pointer in block " + std::to_string(l));
+  }
+  for (int i = 0; i < nu; ++i)
+    if (!w->fast[i].w_gate || !w->fast[i].w_up || !w->fast[i].w_down)
+      return set_error(TTT_ERR_INVALID_ARG, "ttt_init: NULL fast weight pointer");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  std::unique_ptr<ttt_ctx> ctx;
+  int rc;
+  if (c->dtype == TTT_BF16) {
+    auto* e = new Engine<bf16>(*c, *w, eta, k, b, nu, s);
+    ctx.reset(e);
+    rc = e->init();
+  } else {
+    auto* e = new Engine<float>(*c, *w, eta, k, b, nu, s);
+    ctx.reset(e);
+    rc = e->init();
+  }
+  if (rc != TTT_OK) return rc;
+  *out = ctx.release();
+  return TTT_OK;
+}
+
+extern "C" int ttt_prefill(ttt_ctx* ctx, const int32_t* tokens_dev, int64_t T, float* losses_dev,
+                           float* const* fast_out_dev) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: NULL context");
+  return fail(ctx, ctx->prefill(tokens_dev, T, losses_dev, fast_out_dev));
+}
+
+extern "C" int ttt_decode_step(ttt_ctx* ctx, int32_t* next_token_dev) {
+  (void)next_token_dev;
+  return fail(ctx, set_error(TTT_ERR_UNSUPPORTED, "ttt_decode_step is not provided by this build"));
+}
+
+extern "C" int ttt_reset(ttt_ctx* ctx) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_reset: NULL context");
+  return fail(ctx, ctx->reset());
+}
+
+extern "C" int ttt_sync(ttt_ctx* ctx) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_sync: NULL context");
+  return fail(ctx, ctx->sync());
+}
+
+extern "C" const char* ttt_last_error(ttt_ctx* ctx) {
+  return ctx ? ctx->last_error.c_str() : last_error_message();
+}
+
+extern "C" void ttt_free(ttt_ctx* ctx) {
+  if (!ctx) return;
+  ctx->sync();
+  delete ctx;
+}
+
+extern "C" int64_t ttt_launch_count(ttt_ctx* ctx) { return ctx ? ctx->launches : 0; }

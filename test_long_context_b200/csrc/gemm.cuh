@@ -17,7 +17,7 @@ namespace ttt {
 enum Epi : int {
   EPI_STORE_F32 = 0,   // C (fp32) = acc
   EPI_STORE_BF16 = 1,  // C (bf16) = acc
-  EPI_ADD_F32 = 2,     // C (fp32) += acc
+  EPI_ADD_F32 = 2,     // C (fp32) = R + acc, R = C2 (fp32) when given, else C itself
   EPI_SWIGLU = 3,      // columns come in (gate 64 | up 64) pairs: C[:, pair*64 + i] = silu(g) * u
                        // (activation dtype); C2 (optional) = raw acc (activation dtype)
   EPI_CE_FWD = 4,      // per row and N tile: part_max, part_sum of exp; target_logit[row] if the

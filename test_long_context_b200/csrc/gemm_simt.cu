@@ -108,7 +108,9 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
         } else if constexpr (EPI == EPI_STORE_BF16) {
           reinterpret_cast<bf16*>(ep.c)[row * ep.ldc + col] = __float2bfloat16_rn(v);
         } else if constexpr (EPI == EPI_ADD_F32) {
-          reinterpret_cast<float*>(ep.c)[row * ep.ldc + col] += v;
+          const float r = ep.c2 ? reinterpret_cast<const float*>(ep.c2)[row * ep.ldc2 + col]
+                                : reinterpret_cast<float*>(ep.c)[row * ep.ldc + col];
+          reinterpret_cast<float*>(ep.c)[row * ep.ldc + col] = r + v;
         } else if constexpr (EPI == EPI_CE_BWD) {
           const float p = expf(v - ep.row_f[row]);
           const float onehot = (col + ep.col_offset == (int64_t)ep.row_i[row]) ? 1.f : 0.f;

@@ -148,7 +148,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
         store32<bf16>(reinterpret_cast<bf16*>(ep.c) + row * ep.ldc + col0, v, nval);
       } else if constexpr (EPI == EPI_ADD_F32) {
         float* dst = reinterpret_cast<float*>(ep.c) + row * ep.ldc + col0;
-        for (int i = 0; i < nval; ++i) v[i] += dst[i];
+        const float* src = ep.c2 ? reinterpret_cast<const float*>(ep.c2) + row * ep.ldc2 + col0 : dst;
+        for (int i = 0; i < nval; ++i) v[i] += src[i];
         store32<float>(dst, v, nval);
       } else if constexpr (EPI == EPI_CE_BWD) {
         constexpr float LOG2E = 1.4426950408889634f;

@@ -1,6 +1,7 @@
 // Op-level entry points (include/ttt_ops.h): thin wrappers that validate the
 // arguments and launch one kernel family each.
 #include "../../include/ttt_ops.h"
+#include "attention.cuh"
 #include "gemm.cuh"
 
 namespace ttt {
@@ -77,4 +78,57 @@ extern "C" int ttt_op_sync(void* stream) {
     return set_error(TTT_ERR_CUDA, "kernel error word " + std::to_string(h));
   }
   return TTT_OK;
+}
+
+static SwaArgs swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t window, const void* q, int64_t ldq,
+                        const void* k, const void* v, int64_t ring, void* o, int64_t ldo, const float* lse) {
+  SwaArgs a;
+  a.heads = H;
+  a.head_dim = HD;
+  a.n = n;
+  a.p0 = p0;
+  a.window = window;
+  a.scale = 1.f / sqrtf((float)HD);
+  a.q = q;
+  a.ldq = ldq;
+  a.k = k;
+  a.v = v;
+  a.ldkv = (int64_t)H * HD;
+  a.ring = ring;
+  a.o = o;
+  a.ldo = ldo;
+  a.lse = const_cast<float*>(lse);
+  a.ld_lse = n;
+  return a;
+}
+
+extern "C" int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
+                                  int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
+                                  int64_t ring_slots, void* o, int64_t ldo, float* lse, void* stream) {
+  if (!q || !k_ring || !v_ring || !o || !lse || n_q < 1 || q_pos0 < 0 || window < 1 || ring_slots < 1 ||
+      n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_forward: bad argument");
+  SwaArgs a = swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots, o, ldo, lse);
+  return swa_forward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
+                                   int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
+                                   int64_t ring_slots, const void* o, int64_t ldo, const float* lse, const void* dout,
+                                   int64_t lddo, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv,
+                                   float* D_scratch, void* stream) {
+  if (!q || !k_ring || !v_ring || !o || !lse || !dout || !dq || !dk || !dv || !D_scratch || n_q < 1 || q_pos0 < 0 ||
+      window < 1 || ring_slots < 1 || n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_backward: bad argument");
+  SwaArgs a = swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots,
+                       const_cast<void*>(o), ldo, lse);
+  a.dout = dout;
+  a.lddo = lddo;
+  a.dq = dq;
+  a.lddq = lddq;
+  a.dk = dk;
+  a.dv = dv;
+  a.lddkv = lddkv;
+  a.D = D_scratch;
+  return swa_backward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
 }
