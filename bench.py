@@ -1,0 +1,363 @@
+#!/usr/bin/env python
+"""Prefill throughput of the TTT-E2E loop on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config 2.7b] [--tokens T] [--no-cpu-baseline]
+
+A step is one full ttt_reset + ttt_prefill over one synthetic sequence of the
+workload (every row of the hot path: bottom blocks, chunked forward, loss,
+backward through the updated blocks, SGD on the fast MLPs).  Inputs are
+seeded synthetic tokens and N(0, 0.02) weights (synth/); the weights (7+ GB
+at 2.7B) are far larger than L2, so no flush is needed between steps.
+
+With N > 1 (torchrun) every rank runs an independent replica on its own
+sequence (the path does not shard: replicas only); value = tokens of all
+ranks / max over ranks of the device time.
+
+--impl reference times the CPU oracle (oracle/) on this machine's host cores on
+a bounded sample of the same workload (the first b tokens: one full chunk
+with its backward and update).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s (2.7B, SWA k=8K, TTT b=1K, T=128K) and % of bf16 tensor peak"
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default="2.7b")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (testing only; not a bench line)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def algorithmic_flops(cfg, T):
+    """Algorithmic flops of one prefill (2 flops per MAC; attention over the
+    eq. (1) band only; backward only for what the method needs; no flash
+    recompute):  forward L*(8d^2 + 6df) + n_u*6df + 2dV per token plus
+    4d * sum_p min(p+1, k) per block; backward per full chunk: 2dV +
+    (n_u-1)(8d^2 + 6df + 12df) + 8df per token (the lowest updated block needs
+    only its fast MLP), plus attention 4d*(band + b(b+1)/2) in n_u-1 blocks."""
+    L, d, f, V, nu, k, b = cfg.n_layers, cfg.d_model, cfg.d_ff, cfg.vocab, cfg.n_updated, cfg.k, cfg.b
+    band = sum(min(p + 1, k) for p in range(T)) if T < 4 * k else (k * (k + 1) // 2 + (T - k) * k)
+    fwd = T * (L * (8 * d * d + 6 * d * f) + nu * 6 * d * f + 2 * d * V) + 4 * d * band * L
+    full = T // b if T % b == 0 else T // b
+    tb = full * b
+    bwd = tb * (2 * d * V + (nu - 1) * (8 * d * d + 6 * d * f + 12 * d * f) + 8 * d * f)
+    band_full = sum(min(p + 1, k) for p in range(tb)) if tb < 4 * k else (k * (k + 1) // 2 + (tb - k) * k)
+    bwd += (nu - 1) * 4 * d * (band_full + full * b * (b + 1) // 2)
+    return float(fwd + bwd)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}, "fallback"
+
+
+def kernel_source_hash(kc):
+    files = {"gemm": ["gemm_tc.cu", "ptx.cuh"], "attn_fwd": ["attention.cu"], "attn_bwd": ["attention.cu"],
+             "other": ["elementwise.cu"]}[kc]
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "test_long_context_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kc, workload):
+    """DRAM bytes per launch of the kernel class from the committed ncu
+    summary, if it was taken on the current source of that kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            t = json.load(fh)
+    except OSError:
+        return None
+    e = t.get(workload, {}).get(kc)
+    if not e or e.get("source_hash") != kernel_source_hash(kc):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ttt_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", self.uuid], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as fh:
+            for line in fh:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx = max(mx, float(parts[1]))
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def workload_name(cfg, T):
+    return (f"{cfg.name} TTT-E2E prefill: L={cfg.n_layers} d={cfg.d_model} H={cfg.n_heads}x{cfg.head_dim} "
+            f"f={cfg.d_ff} V={cfg.vocab} n_u={cfg.n_updated} T={T} k={cfg.k} b={cfg.b} batch=1")
+
+
+def config_dict(cfg, T, n):
+    return {"workload": workload_name(cfg, T), "tokens_per_sequence": T, "window": cfg.k, "chunk": cfg.b,
+            "updated_blocks": cfg.n_updated, "sequences_per_gpu": 1, "parallelism": f"replicas{n}",
+            "l2": "inputs larger than L2 (7 GB of bf16 weights streamed per step), no flush"}
+
+
+def cpu_baseline(cfg, weights_arrays, toks, sample_tokens):
+    import numpy as np
+
+    import oracle
+    m = oracle.Model(cfg, weights_arrays)
+    t0 = time.perf_counter()
+    oracle.prefill(m, np.asarray(toks[:sample_tokens]))
+    dt = time.perf_counter() - t0
+    cores = os.cpu_count()
+    return {"value": sample_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"oracle (fp64 numpy, BLAS threads = {cores}) prefill of the first {sample_tokens} tokens of "
+                       f"the same sequence: one full chunk with backward and SGD update; "
+                       f"window not yet full, so this favours the CPU"),
+            "seconds": dt}
+
+
+def run_reference(args, cfg, T):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.make_weights(cfg, keep_bits=False)
+    toks = synth.tokens(cfg, T)
+    sample = min(cfg.b, T)
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, w.arrays, toks, sample)
+    times = []
+    for _ in range(args.steps):
+        times.append(cpu_baseline(cfg, w.arrays, toks, sample)["seconds"])
+    tot = sum(times)
+    value = args.steps * sample / tot
+    cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded Zipf + repeated spans; N(0,0.02) weights)", "config": config_dict(cfg, T, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"first {sample} tokens per step (one full chunk with backward and update)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    import synth
+    cfg = synth.get_config(args.config)
+    T = args.tokens or cfg.T
+    if args.impl == "reference":
+        return run_reference(args, cfg, T)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from test_long_context_b200.context import Context, upload_weights
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=torch.device("cuda", local))
+
+    want_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    keep = {}
+    gw = {}
+    for name, arr, bits in synth.iter_weights(cfg):
+        gw.update(upload_weights([(name, arr, bits)], cfg.dtype))
+        if want_cpu:
+            keep[name] = arr
+    toks = synth.tokens(cfg, T, seed=cfg.seed + 7919 * rank)
+    tok_dev = torch.from_numpy(toks).cuda()
+    stream = torch.cuda.current_stream()
+    ctx = Context(cfg, gw, stream=stream)
+    losses = torch.empty(T, device="cuda")
+
+    def step():
+        ctx.reset()
+        ctx.prefill(tok_dev, losses, sync=False)
+
+    for _ in range(args.warmup):
+        step()
+    ctx.sync()
+    if not torch.isfinite(losses[:-1]).all():
+        raise SystemExit("non-finite losses")
+
+    uuid = str(torch.cuda.get_device_properties(local).uuid)
+    uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    clocks = ClockSampler(uuid)
+    ctx.timing_enable(True)
+    n0 = ctx.launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    ctx.sync()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches = ctx.launch_count() - n0
+    timing = ctx.timing_read()
+    ctx.timing_enable(False)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # end to end through the public API: pinned host tokens in, losses out
+    e2e = None
+    if not args.no_e2e:
+        tok_host = torch.from_numpy(toks).pin_memory()
+        loss_host = torch.empty(T, dtype=torch.float32).pin_memory()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            tok_dev.copy_(tok_host, non_blocking=True)
+            ctx.reset()
+            ctx.prefill(tok_dev, losses, sync=False)
+            loss_host.copy_(losses, non_blocking=True)
+        e1.record(stream)
+        ctx.sync()
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": world * args.steps * T / (ems / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(tok_host.numel() * 4), "d2h_bytes_per_step": int(loss_host.numel() * 4),
+               "ms_per_step": ems / args.steps}
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        value = world * args.steps * T / (ms / 1000.0)
+        flops_step = algorithmic_flops(cfg, T)
+        tensor_peak = peaks["bf16_tflops_sustained"]
+        classes = {}
+        for name in KC_NAMES:
+            tms, tn, tfl = timing[name]
+            classes[name] = {"ms_per_step": tms / args.steps, "launches_per_step": tn / args.steps,
+                             "share": tms / max(1e-9, sum(v[0] for v in timing.values())),
+                             "tflops": (tfl / (tms / 1000.0) / 1e12) if tms > 0 and tfl > 0 else None}
+        dom = max(KC_NAMES[:3], key=lambda n: timing[n][0])
+        tms, tn, tfl = timing[dom]
+        achieved = tfl / (tms / 1000.0) / 1e12
+        simt_attn = dom.startswith("attn")
+        if simt_attn:
+            # SIMT fp32 FMA kernels: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock
+            peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            bound, note = "alu", "fp32 FMA peak from unit counts and the max SM clock"
+        else:
+            peak, bound, note = tensor_peak, "tensor", f"bf16 dense, sustained ({peak_src})"
+        per_launch_flops = tfl / max(tn, 1)
+        traffic = traffic_for(dom, args.config)
+        roof = {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "algorithmic_flops_per_launch": per_launch_flops,
+                "avg_launch_ms": tms / max(tn, 1), "peak_source": note}
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": cfg.dtype,
+                "data": "synthetic (seeded Zipf(1.1) tokens + repeated 64-token spans; N(0,0.02) weights)",
+                "config": config_dict(cfg, T, world),
+                "ms_per_1k_tokens": (ms / args.steps) / (T / 1000.0),
+                "tensor_peak_frac": flops_step * world * args.steps / (ms / 1000.0) / 1e12 / tensor_peak,
+                "algorithmic_tflop_per_step": flops_step / 1e12,
+                "roofline": roof, "kernel_classes": classes, "gpu_launches": int(launches),
+                "clocks": clk, "e2e": e2e}
+        if want_cpu:
+            line["cpu_baseline"] = cpu_baseline(cfg, keep, toks, min(cfg.b, T))
+            line["cpu_baseline"].pop("seconds", None)
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

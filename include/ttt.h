@@ -166,8 +166,24 @@ const char* ttt_last_error(ttt_ctx* ctx);
 /* Release everything the context owns.  NULL is ignored. */
 void ttt_free(ttt_ctx* ctx);
 
-/* Number of kernel launches issued by the last ttt_prefill on this context. */
+/* Number of kernel launches issued on this context since ttt_init. */
 int64_t ttt_launch_count(ttt_ctx* ctx);
+
+/* ---- optional per-kernel-class timing ----
+ * When enabled, every launch is bracketed by CUDA events recorded on the
+ * context's stream, and the launch's algorithmic work is accumulated:
+ *   GEMM: 2*M*N*K flops;  ATTN_FWD: 4 * d_model * (query-key pairs admitted by
+ *   the window, eq. (1));  ATTN_BWD: 4 * d_model * (band pairs + causal pairs
+ *   among the chunk's own positions).  OTHER: memory-bound kernels (no flops).
+ * ttt_timing_read synchronises the stream and returns the totals since the
+ * last ttt_timing_enable(ctx, 1). */
+#define TTT_KC_GEMM 0
+#define TTT_KC_ATTN_FWD 1
+#define TTT_KC_ATTN_BWD 2
+#define TTT_KC_OTHER 3
+#define TTT_KC_COUNT 4
+int ttt_timing_enable(ttt_ctx* ctx, int32_t enable);
+int ttt_timing_read(ttt_ctx* ctx, int32_t kernel_class, double* total_ms, int64_t* launches, double* flops);
 
 #ifdef __cplusplus
 }

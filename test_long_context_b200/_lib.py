@@ -20,6 +20,8 @@ TTT_ERR_UNSUPPORTED = -6
 TTT_F32 = 0
 TTT_BF16 = 1
 
+KC_GEMM, KC_ATTN_FWD, KC_ATTN_BWD, KC_OTHER = range(4)
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other")
 EPI_STORE_F32, EPI_STORE_BF16, EPI_ADD_F32, EPI_SWIGLU, EPI_CE_FWD, EPI_CE_BWD, EPI_SGD = range(7)
 
 c_i32, c_i64, c_f32, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -70,6 +72,9 @@ def lib():
             "ttt_last_error": (ctypes.c_char_p, [c_vp]),
             "ttt_free": (None, [c_vp]),
             "ttt_launch_count": (c_i64, [c_vp]),
+            "ttt_timing_enable": (c_i32, [c_vp, c_i32]),
+            "ttt_timing_read": (c_i32, [c_vp, c_i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(c_i64),
+                                        ctypes.POINTER(ctypes.c_double)]),
             "ttt_op_gemm": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
                                     ctypes.POINTER(ttt_epilogue_args), c_i32, c_vp]),
             "ttt_op_gemm_ce_tiles": (c_i64, [c_i32, c_i64, c_i64, c_i32]),
@@ -107,7 +112,7 @@ def exported_symbols():
     L = lib()
     names = []
     for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
-              "ttt_launch_count", "ttt_op_gemm", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
+              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
               "ttt_op_swa_backward"):
         if hasattr(L, n):
             names.append(n)

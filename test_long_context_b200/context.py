@@ -95,6 +95,18 @@ class Context:
     def launch_count(self):
         return int(L.lib().ttt_launch_count(self.h))
 
+    def timing_enable(self, on=True):
+        L.check(L.lib().ttt_timing_enable(self.h, 1 if on else 0), self.h)
+
+    def timing_read(self):
+        """{class name: (total_ms, launches, algorithmic flops)} since timing_enable."""
+        out = {}
+        for kc, name in enumerate(L.KC_NAMES):
+            ms, n, fl = ctypes.c_double(), ctypes.c_int64(), ctypes.c_double()
+            L.check(L.lib().ttt_timing_read(self.h, kc, ctypes.byref(ms), ctypes.byref(n), ctypes.byref(fl)), self.h)
+            out[name] = (ms.value, n.value, fl.value)
+        return out
+
     def close(self):
         if getattr(self, "h", None):
             L.lib().ttt_free(self.h)

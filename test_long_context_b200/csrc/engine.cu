@@ -25,6 +25,8 @@ struct ttt_ctx {
   virtual int prefill(const int32_t* tok, int64_t T, float* losses, float* const* fast_out) = 0;
   virtual int reset() = 0;
   virtual int sync() = 0;
+  virtual int timing_enable(bool on) = 0;
+  virtual int timing_read(int kc, double* ms, int64_t* n, double* flops) = 0;
   std::string last_error = "no error";
   int64_t launches = 0;
 };
@@ -84,6 +86,53 @@ struct Gemm {
   bool bf = false;
 };
 
+// Event-pair timing of launches, per kernel class (opt-in).
+struct LaunchTimer {
+  struct Rec {
+    int kc;
+    cudaEvent_t a, b;
+    double flops;
+  };
+  bool on = false;
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  double ms[TTT_KC_COUNT] = {}, flops[TTT_KC_COUNT] = {};
+  int64_t n[TTT_KC_COUNT] = {};
+  ~LaunchTimer() {
+    for (auto& r : pending) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+    for (auto e : pool) cudaEventDestroy(e);
+  }
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+  int drain() {
+    for (auto& r : pending) {
+      float t = 0.f;
+      TTT_CUDA_TRY(cudaEventElapsedTime(&t, r.a, r.b));
+      ms[r.kc] += t;
+      flops[r.kc] += r.flops;
+      n[r.kc] += 1;
+      pool.push_back(r.a);
+      pool.push_back(r.b);
+    }
+    pending.clear();
+    return TTT_OK;
+  }
+  void clear() {
+    for (int i = 0; i < TTT_KC_COUNT; ++i) ms[i] = flops[i] = 0, n[i] = 0;
+  }
+};
+
 template <typename T>
 class Engine final : public ttt_ctx {
  public:
@@ -100,6 +149,22 @@ class Engine final : public ttt_ctx {
   int prefill(const int32_t* tok, int64_t T_, float* losses, float* const* fast_out) override;
   int reset() override;
   int sync() override;
+  int timing_enable(bool on) override {
+    TTT_CUDA_TRY(cudaStreamSynchronize(st_));
+    TRY(timer_.drain());
+    timer_.clear();
+    timer_.on = on;
+    return TTT_OK;
+  }
+  int timing_read(int kc, double* ms, int64_t* n, double* flops) override {
+    if (kc < 0 || kc >= TTT_KC_COUNT) return set_error(TTT_ERR_INVALID_ARG, "ttt_timing_read: bad class");
+    TTT_CUDA_TRY(cudaStreamSynchronize(st_));
+    TRY(timer_.drain());
+    if (ms) *ms = timer_.ms[kc];
+    if (n) *n = timer_.n[kc];
+    if (flops) *flops = timer_.flops[kc];
+    return TTT_OK;
+  }
 
  private:
   static constexpr bool BF = ActTraits<T>::bf;
@@ -109,9 +174,31 @@ class Engine final : public ttt_ctx {
   int run(Gemm& g, int64_t rows);  // rows overrides the M extent (chunk/super-chunk length)
   int bottom_layers(const int32_t* tok, int64_t s0, int64_t S);
   int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
-  int count(int rc) {
+  // Launch `f` (returns a status); bracket it with events when timing is on.
+  template <typename F>
+  int timed(int kc, double flops, F&& f) {
     ++launches;
+    if (!timer_.on) return f();
+    cudaEvent_t a = timer_.get(), b = timer_.get();
+    TTT_CUDA_TRY(cudaEventRecord(a, st_));
+    const int rc = f();
+    TTT_CUDA_TRY(cudaEventRecord(b, st_));
+    timer_.pending.push_back({kc, a, b, flops});
     return rc;
+  }
+  // Query-key pairs admitted by the window for queries p0 .. p0+n-1 (eq. (1)).
+  double band_pairs(int64_t p0, int64_t n) const {
+    const int64_t k = k_;
+    double s = 0;
+    // queries with p + 1 <= k see p + 1 keys, the rest see k
+    const int64_t full_from = std::max<int64_t>(p0, k - 1);
+    const int64_t e = p0 + n;
+    if (full_from > p0) {
+      const int64_t a = p0 + 1, z = std::min<int64_t>(full_from, e);  // keys p+1 for p in [p0, z)
+      s += (double)(a + z) * (double)(z - p0) / 2.0;
+    }
+    if (e > full_from) s += (double)(e - full_from) * (double)k;
+    return s;
   }
   SwaArgs swa_args(const T* q, int64_t n, int64_t p0, const T* kr, const T* vr, int64_t ring, T* o, float* lse,
                    int64_t ld_lse) const {
@@ -146,6 +233,7 @@ class Engine final : public ttt_ctx {
   std::vector<ttt_layer_weights> layers_;
   std::vector<ttt_fast_weights> fast_init_;
   Arena arena_;
+  LaunchTimer timer_;
   bool fresh_ = true;
   int* err_ = nullptr;
 
@@ -200,16 +288,16 @@ int Engine<T>::prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, 
 
 template <typename T>
 int Engine<T>::run(Gemm& g, int64_t rows) {
-  ++launches;
+  GemmShape s = g.shape;
+  if (rows > 0 && !s.a_mn) s.a.rows = rows;
+  const double flops = 2.0 * (double)s.M() * (double)s.N() * (double)s.K();
   if (BF) {
     TcGemm tc = g.tc;
     tc.args = g.args;
     if (rows > 0 && !tc.a_mn) tc.M = rows;
-    return tc_gemm_launch(tc, st_, err_);
+    return timed(TTT_KC_GEMM, flops, [&] { return tc_gemm_launch(tc, st_, err_); });
   }
-  GemmShape s = g.shape;
-  if (rows > 0 && !s.a_mn) s.a.rows = rows;
-  return simt_gemm(s, g.epi, g.args, st_);
+  return timed(TTT_KC_GEMM, flops, [&] { return simt_gemm(s, g.epi, g.args, st_); });
 }
 
 template <typename T>
@@ -420,10 +508,10 @@ int Engine<T>::reset() {
   for (int i = 0; i < nu_; ++i) {
     const int64_t l = nbot_ + i;
     TTT_CUDA_TRY(cudaMemcpyAsync(master_gu(i), init_gu_[i], 2 * f * d * sizeof(float), cudaMemcpyDeviceToDevice, st_));
-    TRY(count(copy2d<float>(init_d_[i], f, master_d(i), master_d_ld(), d, f, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d<float>(init_d_[i], f, master_d(i), master_d_ld(), d, f, st_); }));
     if (BF) {
-      TRY(count(copy2d_from_f32<T>(init_gu_[i], d, wgu_[l] + 2 * f * d, d, 2 * f, d, st_)));
-      TRY(count(copy2d_from_f32<T>(init_d_[i], f, wd_[l] + f, 2 * f, d, f, st_)));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d_from_f32<T>(init_gu_[i], d, wgu_[l] + 2 * f * d, d, 2 * f, d, st_); }));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d_from_f32<T>(init_d_[i], f, wd_[l] + f, 2 * f, d, f, st_); }));
     }
   }
   fresh_ = true;
@@ -449,17 +537,18 @@ int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
   const int64_t d = d_;
   const float eps = cfg_.norm_eps;
   const double theta = cfg_.rope_theta;
-  TRY(count(embed_gather<T>(tok + s0, reinterpret_cast<const T*>(wt_.embed), S, (int)d, (int)V_, xs_, err_, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return embed_gather<T>(tok + s0, reinterpret_cast<const T*>(wt_.embed), S, (int)d, (int)V_, xs_, err_, st_); }));
   for (int64_t l = 0; l < nbot_; ++l) {
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_bot_[4 * l];
-    TRY(count(rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[0], S));
-    TRY(count(qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
-                                 kb_[l], vb_[l], d, R1_, rqs_, rks_, st_)));
-    TRY(count(swa_forward(swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_), BF, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
+                                 kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }));
+    TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(s0, S),
+              [&] { return swa_forward(swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_), BF, st_); }));
     TRY(run(g[1], S));
-    TRY(count(rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[2], S));
     TRY(run(g[3], S));
   }
@@ -472,28 +561,29 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
   const float eps = cfg_.norm_eps;
   const double theta = cfg_.rope_theta;
   const int64_t n_valid = std::max<int64_t>(0, std::min<int64_t>(n, T_ - 1 - p0));
-  TRY(count(chunk_targets(tok, T_, p0, n, tgt_, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return chunk_targets(tok, T_, p0, n, tgt_, st_); }));
   // ---- forward of the updated blocks with the current fast weights ----
   for (int i = 0; i < nu_; ++i) {
     const int64_t l = nbot_ + i;
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_top_[10 * i];
     const float* xin = i == 0 ? x0 : xin_[i];
-    TRY(count(rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_); }));
     TRY(run(g[0], n));
-    TRY(count(qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
-                                 kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_)));
-    TRY(count(swa_forward(swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b), BF, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
+                                 kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_); }));
+    TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(p0, n),
+              [&] { return swa_forward(swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b), BF, st_); }));
     g[1].args.c2 = const_cast<float*>(xin);
     TRY(run(g[1], n));
-    TRY(count(rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_); }));
     TRY(run(g[2], n));
     TRY(run(g[3], n));
   }
-  TRY(count(rmsnorm_fwd<T>(xf_, d, wt_.final_norm, eps, n, (int)d, hf_, d, rf_, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xf_, d, wt_.final_norm, eps, n, (int)d, hf_, d, rf_, st_); }));
   TRY(run(g_head_, n));
-  TRY(count(ce_finalize(pmax_, psum_, b, (int)ce_tiles_, zt_, n, n_valid, n_valid ? 1.f / (float)n_valid : 0.f,
-                        losses + p0, lsef_, scl_, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return ce_finalize(pmax_, psum_, b, (int)ce_tiles_, zt_, n, n_valid, n_valid ? 1.f / (float)n_valid : 0.f,
+                        losses + p0, lsef_, scl_, st_); }));
   if (n < b || n_valid == 0) return TTT_OK;  // a trailing partial chunk is scored only
 
   // ---- backward through the updated blocks, SGD on each fast MLP ----
@@ -501,22 +591,22 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     TRY(run(g_ce_dz_[c], n));
     TRY(run(g_ce_dh_[c], n));
   }
-  TRY(count(rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_); }));
   for (int i = nu_ - 1; i >= 0; --i) {
     const int64_t l = nbot_ + i;
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_top_[10 * i];
     TRY(run(g[4], n));
     if (i == 0) {
-      TRY(count(swiglu_bwd<T>(da_ + f, 2 * f, gu_[i] + 2 * f, 4 * f, n, f, dgu_ + 2 * f, 4 * f, st_)));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return swiglu_bwd<T>(da_ + f, 2 * f, gu_[i] + 2 * f, 4 * f, n, f, dgu_ + 2 * f, 4 * f, st_); }));
     } else {
-      TRY(count(swiglu_bwd<T>(da_, 2 * f, gu_[i], 4 * f, n, 2 * f, dgu_, 4 * f, st_)));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return swiglu_bwd<T>(da_, 2 * f, gu_[i], 4 * f, n, 2 * f, dgu_, 4 * f, st_); }));
       TRY(run(g[5], n));  // reads the fast shadow before its update
     }
     TRY(run(g[6], 0));  // W_down fast -= eta * dx^T a_f
     TRY(run(g[7], 0));  // W_gate/up fast -= eta * dgu_f^T h2
     if (i == 0) break;  // nothing below the lowest fast block depends on W
-    TRY(count(rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_); }));
     TRY(run(g[8], n));
     SwaArgs a = swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b);
     a.dout = do_;
@@ -527,12 +617,13 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     a.dv = dqkv_ + 2 * d;
     a.lddkv = 3 * d;
     a.D = Dbuf_;
-    TRY(count(swa_backward(a, BF, st_)));
+    TRY(timed(TTT_KC_ATTN_BWD, 4.0 * d * (band_pairs(p0, n) + (double)n * (double)(n + 1) / 2.0),
+              [&] { return swa_backward(a, BF, st_); }));
     launches += 2;  // the backward launches three kernels
-    TRY(count(qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
-                                 (int)HD_, theta, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
+                                 (int)HD_, theta, st_); }));
     TRY(run(g[9], n));
-    TRY(count(rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_)));
+    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_); }));
   }
   return TTT_OK;
 }
@@ -542,8 +633,7 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
   if (!fresh_) return set_error(TTT_ERR_STATE, "ttt_prefill needs a fresh context (call ttt_reset)");
   if (!tok || !losses || T_ < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: bad argument");
   fresh_ = false;
-  launches = 0;
-  TRY(count(check_tokens(tok, T_, (int)V_, err_, st_)));
+  TRY(timed(TTT_KC_OTHER, 0, [&] { return check_tokens(tok, T_, (int)V_, err_, st_); }));
   for (int64_t s0 = 0; s0 < T_; s0 += S_) {
     const int64_t S = std::min<int64_t>(S_, T_ - s0);
     TRY(bottom_layers(tok, s0, S));
@@ -559,8 +649,8 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
       float* ou = fast_out[3 * i + 1];
       float* od = fast_out[3 * i + 2];
       if (!og || !ou || !od) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: NULL entry in fast_out");
-      TRY(count(deinterleave_gate_up(master_gu(i), (int)f, (int)d, og, ou, st_)));
-      TRY(count(copy2d<float>(master_d(i), master_d_ld(), od, f, d, f, st_)));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return deinterleave_gate_up(master_gu(i), (int)f, (int)d, og, ou, st_); }));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d<float>(master_d(i), master_d_ld(), od, f, d, f, st_); }));
     }
   }
   return TTT_OK;
@@ -651,3 +741,13 @@ extern "C" void ttt_free(ttt_ctx* ctx) {
 }
 
 extern "C" int64_t ttt_launch_count(ttt_ctx* ctx) { return ctx ? ctx->launches : 0; }
+
+extern "C" int ttt_timing_enable(ttt_ctx* ctx, int32_t enable) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_timing_enable: NULL context");
+  return fail(ctx, ctx->timing_enable(enable != 0));
+}
+
+extern "C" int ttt_timing_read(ttt_ctx* ctx, int32_t kc, double* total_ms, int64_t* launches, double* flops) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_timing_read: NULL context");
+  return fail(ctx, ctx->timing_read(kc, total_ms, launches, flops));
+}
