@@ -212,6 +212,9 @@ def run_reference(args, cfg, T):
 
 def main():
     args = parse_args()
+    if os.environ.get("TTT_BENCH_WATCHDOG"):
+        import faulthandler
+        faulthandler.dump_traceback_later(int(os.environ["TTT_BENCH_WATCHDOG"]), repeat=True, file=sys.stderr)
     import synth
     cfg = synth.get_config(args.config)
     T = args.tokens or cfg.T

@@ -70,12 +70,15 @@ int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hin
  *   in slot j % ring_slots, so ring_slots >= window + n_q - 1 is required
  *   when the ring holds earlier positions as well.
  *   lse: [n_heads, n_q] fp32 natural-log log-sum-exp of the scaled scores.
- * dtype TTT_F32 (all fp32) or TTT_BF16 (bf16 tensors, fp32 math).
- * Scores are scaled by 1/sqrt(head_dim).
+ * dtype TTT_F32 (all fp32, SIMT) or TTT_BF16 (bf16 tensors).  With TTT_BF16,
+ * head_dim in {64, 80, 96, 128}, ring_slots a multiple of 128 and flags bit 0
+ * clear, the tcgen05 tensor-core kernel runs (fp32 softmax, bf16 P); otherwise
+ * the SIMT kernel (fp32 math).  Scores are scaled by 1/sqrt(head_dim).
  */
+#define TTT_SWA_FORCE_SIMT 1
 int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
                        const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
-                       void* o, int64_t ldo, float* lse, void* stream);
+                       void* o, int64_t ldo, float* lse, int32_t flags, void* stream);
 
 /*
  * Backward of ttt_op_swa_forward given dout = dL/do: dq for every query (over
@@ -88,6 +91,12 @@ int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_
                         const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
                         const void* o, int64_t ldo, const float* lse, const void* dout, int64_t lddo, void* dq,
                         int64_t lddq, void* dk, void* dv, int64_t lddkv, float* D_scratch, void* stream);
+
+/* Device watchdog self-test: launches one thread that waits on an mbarrier
+ * nothing ever arrives at.  The bounded wait gives up (about 2 s) and records
+ * a timeout, so the following ttt_op_sync returns TTT_ERR_TIMEOUT and the
+ * context stays usable. */
+int ttt_op_watchdog_selftest(void* stream);
 
 /* Wait for `stream`; return TTT_ERR_TIMEOUT if a kernel launched through this
  * header recorded a bounded-wait timeout since the last call (then clears it). */

@@ -1,0 +1,462 @@
+// Tensor-core (tcgen05) flash attention forward for the banded causal window
+// of eq. (1) (query p sees keys p-k+1 .. p), bf16 operands, fp32 softmax.
+//
+// CTA = one tile of 128 queries x one head; 8 warps:
+//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys (2 stages)
+//   warp 1      TMEM owner; lane 0 issues every tcgen05.mma
+//   warps 4..7  softmax: thread = query row = TMEM lane; writes P (bf16) to
+//               128B-swizzled smem, keeps the running max / sum, rescales O in
+//               TMEM only when the max grows by more than 2^8 (log2 domain),
+//               and finally normalises O and writes it with the LSE.
+// S = Q K^T goes to one of two TMEM buffers (128 columns each) so that the
+// next tile's QK^T overlaps this tile's softmax; O (head_dim columns) lives
+// in TMEM for the whole key loop.
+//
+// head_dim = 64*A + R with R in {0, 16, 32}: the first 64*A columns of Q, K,
+// V use 128-byte swizzled tiles, the remaining R columns a 2R-byte swizzle, so
+// every TMA box starts on a 16-byte boundary and matches a canonical UMMA
+// layout (K-major for Q and K, MN-major for V as the B operand of P V).
+#include <mutex>
+#include <set>
+
+#include "attention_tc.cuh"
+#include "ptx.cuh"
+
+namespace ttt {
+namespace {
+
+constexpr int QT = 128;   // queries per CTA
+constexpr int KT = 128;   // keys per tile
+constexpr int NST = 2;    // K/V stages
+constexpr float RESCALE_LOG2 = 8.f;
+
+__host__ __device__ constexpr int rem_swizzle_layout(int rem) { return rem == 16 ? 6 : (rem == 32 ? 4 : 2); }
+
+template <int HD>
+struct Geo {
+  static constexpr int A = HD / 64;          // 128B-swizzled atoms along head_dim
+  static constexpr int R = HD % 64;          // remainder columns (0, 16, 32)
+  static constexpr int RB = R * 2;           // remainder row bytes (32 or 64)
+  static constexpr int TILE = 128 * HD * 2;  // bytes of a 128-row tile
+  static constexpr int REM_OFF = A * 16384;  // offset of the remainder region in a tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = TILE;        // stage s: K at KV_OFF + s*2*TILE, V after it
+  static constexpr int P_OFF = KV_OFF + NST * 2 * TILE;
+  static constexpr int P_BYTES = 128 * 128 * 2;
+  static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(R == 0 || R == 16 || R == 32, "head_dim must be 64*A + {0,16,32}");
+  static_assert(TILE % 1024 == 0, "tiles must stay 1024-byte aligned");
+};
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Load one 128-row tile (rows row0.., head columns col0 .. col0+HD) into smem.
+template <int HD>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m128, const CUtensorMap* mrem,
+                                          uint64_t* bar, int col0, int row0) {
+  using G = Geo<HD>;
+#pragma unroll
+  for (int a = 0; a < G::A; ++a) ptx::tma_load_2d(dst + a * 16384, m128, bar, col0 + 64 * a, row0);
+  if constexpr (G::R > 0) ptx::tma_load_2d(dst + G::REM_OFF, mrem, bar, col0 + 64 * G::A, row0);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(256, 1)
+    swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
+                      const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
+                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r, SwaArgs a,
+                      int* err) {
+  using G = Geo<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;    // [NST]
+  uint64_t* kv_empty = bars + 3;   // [NST]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_empty = bars + 7;    // [2]
+  uint64_t* p_full = bars + 9;     // [2]
+  uint64_t* pv_done = bars + 11;   // [2]
+  uint64_t* o_full = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int64_t q0 = a.p0 + (int64_t)blockIdx.x * QT;            // absolute position of row 0
+  const int64_t qlast = imin64(q0 + QT, a.p0 + a.n) - 1;          // last valid query position
+  const int64_t kfirst = imax64(0, q0 - a.window + 1);
+  const int64_t j_begin = (kfirst / KT) * KT;                     // aligned key tile start
+  const int ntiles = (int)((qlast - j_begin) / KT + 1);
+  const int col0 = h * HD;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&s_empty[s], 128);
+      ptx::mbar_init(&p_full[s], 128);
+      ptx::mbar_init(&pv_done[s], 1);
+    }
+    ptx::mbar_init(o_full, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s0 = tmem, t_o = tmem + 256;  // S buffers at columns 0 and 128, O at 256
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(q_full, G::TILE);
+      load_tile<HD>(sm + G::Q_OFF, &tq, &tq_r, q_full, col0, (int)(q0 - a.p0));
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % NST;
+        if (!ptx::mbar_wait(&kv_empty[s], ((j / NST) & 1) ^ 1, err)) break;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], 2 * G::TILE);
+        const int slot = (int)((j_begin + (int64_t)j * KT) % a.ring);
+        uint8_t* kd = sm + G::KV_OFF + s * 2 * G::TILE;
+        load_tile<HD>(kd, &tk, &tk_r, &kv_full[s], col0, slot);
+        load_tile<HD>(kd + G::TILE, &tv, &tv_r, &kv_full[s], col0, slot);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, KT, false, false);
+      constexpr uint32_t id_pv64 = ptx::idesc_bf16_f32(128, 64, false, true);
+      constexpr uint32_t id_pvr = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
+      const uint32_t q_addr = ptx::smem_u32(sm + G::Q_OFF);
+      bool ok = ptx::mbar_wait(q_full, 0, err);
+      auto issue_s = [&](int j) {
+        const int s = j % NST;
+        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE);
+        const uint32_t d = t_s0 + (j & 1) * 128;
+        int step = 0;
+#pragma unroll
+        for (int at = 0; at < G::A; ++at)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk, ++step)
+            ptx::umma_bf16(d, sdesc(q_addr + at * 16384 + kk * 32, 16, 1024, 2),
+                           sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2), id_s, step > 0);
+        if constexpr (G::R > 0) {
+#pragma unroll
+          for (int kk = 0; kk < G::R / 16; ++kk, ++step)
+            ptx::umma_bf16(d, sdesc(q_addr + G::REM_OFF + kk * 32, 16, 8 * G::RB, rem_swizzle_layout(G::R)),
+                           sdesc(k_addr + G::REM_OFF + kk * 32, 16, 8 * G::RB, rem_swizzle_layout(G::R)), id_s,
+                           step > 0);
+        }
+        ptx::umma_commit(&s_full[j & 1]);
+      };
+      if (ok && ntiles > 0) {
+        if ((ok = ptx::mbar_wait(&kv_full[0], 0, err))) {
+          ptx::tc_fence_after();
+          issue_s(0);
+        }
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles) {
+          const int s1 = (j + 1) % NST;
+          if (!(ok = ptx::mbar_wait(&kv_full[s1], ((j + 1) / NST) & 1, err))) break;
+          if (j + 1 >= 2 && !(ok = ptx::mbar_wait(&s_empty[(j + 1) & 1], (((j + 1) / 2) - 1) & 1, err))) break;
+          ptx::tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (!(ok = ptx::mbar_wait(&p_full[j & 1], (j / 2) & 1, err))) break;
+        ptx::tc_fence_after();
+        const int s = j % NST;
+        const uint32_t v_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE + G::TILE);
+        const uint32_t p_addr = ptx::smem_u32(sm + G::P_OFF + (j & 1) * G::P_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk) {
+          const uint64_t pd = sdesc(p_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, 2);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+#pragma unroll
+          for (int at = 0; at < G::A; ++at)
+            ptx::umma_bf16(t_o + 64 * at, pd, sdesc(v_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_pv64, acc);
+          if constexpr (G::R > 0)
+            ptx::umma_bf16(t_o + 64 * G::A, pd,
+                           sdesc(v_addr + G::REM_OFF + kk * 16 * G::RB, 16, 8 * G::RB, rem_swizzle_layout(G::R)),
+                           id_pvr, acc);
+        }
+        ptx::umma_commit(&kv_empty[s]);
+        ptx::umma_commit(&pv_done[j & 1]);
+      }
+      ptx::umma_commit(o_full);
+      ptx::mbar_drain(o_full, 0);  // no MMA may still write TMEM when it is released
+    }
+  } else if (warp >= 4) {
+    // ---- softmax: one query row per thread ----
+    const int r = (warp - 4) * 32 + lane;                  // row in the tile (== TMEM lane)
+    const int64_t p = q0 + r;                               // absolute query position
+    const bool row_ok = p <= qlast;
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const float sl2 = a.scale * 1.4426950408889634f;        // scale * log2(e)
+    float m = -INFINITY, l = 0.f;
+    uint8_t* pbase = sm + G::P_OFF;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int64_t j0 = j_begin + (int64_t)j * KT;
+      ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
+      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads follow
+      ptx::tc_fence_after();
+      float s[KT];
+#pragma unroll
+      for (int c = 0; c < KT; c += 32) {
+        uint32_t rr[32];
+        ptx::tmem_ld32(t_s0 + (j & 1) * 128 + c + lane_off, rr);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(rr[i]) * sl2;
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&s_empty[j & 1]);
+      // mask: key c valid iff j0 + c in [p - window + 1, p]
+      const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
+      const bool full = row_ok && lo <= 0 && hi >= KT - 1;
+      float tmax = -INFINITY;
+      if (full) {
+#pragma unroll
+        for (int c = 0; c < KT; ++c) tmax = fmaxf(tmax, s[c]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < KT; ++c) {
+          const bool v = row_ok && c >= lo && c <= hi;
+          s[c] = v ? s[c] : -INFINITY;
+          tmax = fmaxf(tmax, s[c]);
+        }
+      }
+      // running max with lazy rescaling of O (needs PV_{j-1} complete).  The
+      // TMEM load/store of O is warp-collective, so a warp rescales together
+      // when any of its rows needs it; rows that do not use corr = 1.
+      float mu = m, corr = 1.f;
+      if (tmax > -INFINITY) {
+        if (m == -INFINITY) {
+          mu = tmax;
+        } else if (tmax > m + RESCALE_LOG2) {
+          mu = tmax;
+          corr = exp2f(m - mu);
+          l *= corr;
+        }
+      }
+      m = mu;
+      if (__any_sync(0xffffffffu, corr != 1.f)) {
+        ok = ptx::mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, err);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HD; c += 16) {
+          uint32_t o[16];
+          tmem_ld16(t_o + c + lane_off, o);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+          tmem_st16(t_o + c + lane_off, o);
+        }
+        tmem_st_wait();
+      }
+      // P buffer (j & 1) is free once PV_{j-2} completed
+      if (j >= 2) {
+        ok = ptx::mbar_wait(&pv_done[j & 1], ((j - 2) / 2) & 1, err);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      uint8_t* prow = pbase + (j & 1) * G::P_BYTES + r * 128;
+      float lsum = 0.f;
+#pragma unroll
+      for (int g = 0; g < KT / 8; ++g) {  // 16 granules of 8 keys
+        float pv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          pv[i] = (m == -INFINITY) ? 0.f : exp2f(s[g * 8 + i] - m);
+          lsum += pv[i];
+        }
+        uint4 w;
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(pv[0], pv[1]), b1 = __floats2bfloat162_rn(pv[2], pv[3]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(pv[4], pv[5]), b3 = __floats2bfloat162_rn(pv[6], pv[7]);
+        w.x = *reinterpret_cast<uint32_t*>(&b0);
+        w.y = *reinterpret_cast<uint32_t*>(&b1);
+        w.z = *reinterpret_cast<uint32_t*>(&b2);
+        w.w = *reinterpret_cast<uint32_t*>(&b3);
+        const int atom = g / 8, gr = g % 8;
+        *reinterpret_cast<uint4*>(prow + atom * 16384 + ((gr ^ (r & 7)) << 4)) = w;
+      }
+      l += lsum;
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&p_full[j & 1]);
+    }
+    // ---- epilogue: O / l and the natural-log LSE ----
+    if (ok) ok = ptx::mbar_wait(o_full, 0, err);
+    if (__all_sync(0xffffffffu, ok)) {
+      ptx::tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t i = p - a.p0;
+      bf16* orow = reinterpret_cast<bf16*>(a.o) + i * a.ldo + col0;
+#pragma unroll
+      for (int c = 0; c < HD; c += 16) {
+        uint32_t o[16];
+        tmem_ld16(t_o + c + lane_off, o);
+        ptx::tmem_ld_wait();
+        if (row_ok) {
+          uint4 w0, w1;
+          uint32_t* pw = &w0.x;
+          uint32_t* pw1 = &w1.x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(__uint_as_float(o[8 + 2 * e]) * inv,
+                                                      __uint_as_float(o[8 + 2 * e + 1]) * inv);
+            pw[e] = *reinterpret_cast<uint32_t*>(&t0);
+            pw1[e] = *reinterpret_cast<uint32_t*>(&t1);
+          }
+          *reinterpret_cast<uint4*>(orow + c) = w0;
+          *reinterpret_cast<uint4*>(orow + c + 8) = w1;
+        }
+      }
+      if (row_ok) a.lse[(int64_t)h * a.ld_lse + i] = (m + log2f(l)) * 0.6931471805599453f;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();  // tcgen05.dealloc is warp-collective: reconverge lane 0 with the others
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 [rows, cols] with row pitch ld; box = box_cols x 128 rows; swizzle by box width.
+int tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols) {
+  EncodeTiledFn enc = encode();
+  if (!enc) return set_error(TTT_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((ld * 2) & 15))
+    return set_error(TTT_ERR_INVALID_ARG, "attention: operands must be 16-byte aligned");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, 128u};
+  cuuint32_t es[2] = {1u, 1u};
+  const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(TTT_ERR_CUDA, "attention tensor map: " + std::to_string((int)r));
+  return TTT_OK;
+}
+
+template <int HD>
+int launch(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  using G = Geo<HD>;
+  auto fn = &swa_fwd_tc_kernel<HD>;
+  {
+    static std::mutex mu;
+    static std::set<int> done;
+    int dev = 0;
+    TTT_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done.count(dev)) {
+      TTT_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+      done.insert(dev);
+    }
+  }
+  dim3 grid(ceil_div(a.n, QT), a.heads);
+  fn<<<grid, 256, G::SMEM, s>>>(p.q128, p.qr, p.k128, p.kr, p.v128, p.vr, a, err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // namespace
+
+bool swa_tc_supported(int head_dim) {
+  return head_dim == 64 || head_dim == 80 || head_dim == 96 || head_dim == 128;
+}
+
+int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t q_rows, int64_t ldq, const void* k,
+                   const void* v, int64_t ring, int64_t ldkv) {
+  if (!swa_tc_supported(head_dim)) return set_error(TTT_ERR_UNSUPPORTED, "attention: head_dim not supported");
+  if (ring % KT) return set_error(TTT_ERR_INVALID_ARG, "attention: ring slots must be a multiple of 128");
+  p->head_dim = head_dim;
+  p->ring = ring;
+  const int64_t cols = (int64_t)heads * head_dim;
+  const int rem = head_dim % 64;
+  int rc = tmap(&p->q128, q, q_rows, cols, ldq, 64);
+  if (!rc) rc = tmap(&p->k128, k, ring, cols, ldkv, 64);
+  if (!rc) rc = tmap(&p->v128, v, ring, cols, ldkv, 64);
+  if (rc) return rc;
+  if (rem) {
+    rc = tmap(&p->qr, q, q_rows, cols, ldq, rem);
+    if (!rc) rc = tmap(&p->kr, k, ring, cols, ldkv, rem);
+    if (!rc) rc = tmap(&p->vr, v, ring, cols, ldkv, rem);
+  } else {
+    p->qr = p->q128;
+    p->kr = p->k128;
+    p->vr = p->v128;
+  }
+  return rc;
+}
+
+int swa_tc_forward(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  if (a.ring != p.ring || a.head_dim != p.head_dim) return set_error(TTT_ERR_INVALID_ARG, "attention: plan mismatch");
+  switch (a.head_dim) {
+    case 64: return launch<64>(p, a, s, err);
+    case 80: return launch<80>(p, a, s, err);
+    case 96: return launch<96>(p, a, s, err);
+    case 128: return launch<128>(p, a, s, err);
+  }
+  return set_error(TTT_ERR_UNSUPPORTED, "attention (tensor cores): head_dim must be 64, 80, 96 or 128");
+}
+
+}  // namespace ttt

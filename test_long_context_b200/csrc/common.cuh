@@ -23,6 +23,8 @@ enum : int {
 
 // Bounded waits give up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// ... or after this many polls of the barrier (each poll may suspend briefly).
+constexpr uint32_t kWaitLimitIters = 1u << 26;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;

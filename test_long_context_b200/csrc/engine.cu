@@ -11,12 +11,15 @@
 // Everything in the loop is device work on one stream; the host only
 // enqueues.
 #include <cmath>
+#include <cstdio>
+#include <cstdlib>
 #include <memory>
 #include <string>
 #include <vector>
 
 #include "../../include/ttt.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
 
@@ -178,12 +181,35 @@ class Engine final : public ttt_ctx {
   template <typename F>
   int timed(int kc, double flops, F&& f) {
     ++launches;
+    if (trace_) return traced(kc, f);
     if (!timer_.on) return f();
     cudaEvent_t a = timer_.get(), b = timer_.get();
     TTT_CUDA_TRY(cudaEventRecord(a, st_));
     const int rc = f();
     TTT_CUDA_TRY(cudaEventRecord(b, st_));
     timer_.pending.push_back({kc, a, b, flops});
+    return rc;
+  }
+  // TTT_TRACE=1: synchronise after every launch and log it to stderr (debugging aid).
+  template <typename F>
+  int traced(int kc, F&& f) {
+    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other"};
+    if (trace_verbose_) fprintf(stderr, "[ttt trace] launching %lld %s\n", (long long)launches, names[kc]);
+    cudaEvent_t a = timer_.get(), b = timer_.get();
+    TTT_CUDA_TRY(cudaEventRecord(a, st_));
+    const int rc = f();
+    TTT_CUDA_TRY(cudaEventRecord(b, st_));
+    const cudaError_t e = cudaStreamSynchronize(st_);
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, a, b);
+    timer_.pool.push_back(a);
+    timer_.pool.push_back(b);
+    int h = 0;
+    cudaMemcpy(&h, err_, sizeof(int), cudaMemcpyDeviceToHost);
+    if (ms > trace_ms_ || h || e != cudaSuccess || rc != TTT_OK)
+      fprintf(stderr, "[ttt trace] launch %lld %s %.3f ms rc=%d cuda=%d err_word=%d\n", (long long)launches,
+              names[kc], ms, rc, (int)e, h);
+    if (e != cudaSuccess) return set_cuda_error(e, "trace sync", __FILE__, __LINE__);
     return rc;
   }
   // Query-key pairs admitted by the window for queries p0 .. p0+n-1 (eq. (1)).
@@ -234,6 +260,8 @@ class Engine final : public ttt_ctx {
   std::vector<ttt_fast_weights> fast_init_;
   Arena arena_;
   LaunchTimer timer_;
+  bool trace_ = false, trace_verbose_ = false;
+  float trace_ms_ = 0.f;
   bool fresh_ = true;
   int* err_ = nullptr;
 
@@ -268,6 +296,13 @@ class Engine final : public ttt_ctx {
   std::vector<Gemm> g_top_;  // 10 per top block: qkv, o, gu, down, da, dh2, wd, wgu, do, dh
   Gemm g_head_;
   std::vector<Gemm> g_ce_dz_, g_ce_dh_;
+  // tensor-core attention plans (bf16, supported head_dim)
+  bool tc_attn_ = false;
+  std::vector<SwaTcPlan> att_bot_, att_top_;
+  int attn_fwd(const SwaTcPlan* plan, const SwaArgs& a) {
+    if (tc_attn_) return swa_tc_forward(*plan, a, st_, err_);
+    return swa_forward(a, BF, st_);
+  }
 };
 
 template <typename T>
@@ -312,13 +347,20 @@ int Engine<T>::init() {
   scale_ = 1.f / std::sqrt((float)HD_);
   const int64_t d = d_, f = f_, b = b_;
   arena_.stream = st_;
+  if (const char* t = getenv("TTT_TRACE")) {
+    trace_ = t[0] && t[0] != '0';
+    trace_verbose_ = t[0] == 'v';
+    trace_ms_ = (float)atof(t) > 1.f ? (float)atof(t) : 0.f;  // TTT_TRACE=<ms>: log launches slower than that
+  }
   TRY(arena_.alloc(&err_, 1));
 
   // Super-chunk length for the fast-weight-free blocks: about 16K positions.
   int64_t spc = std::max<int64_t>(1, 16384 / b);
   S_ = spc * b;
-  R1_ = S_ + k_;
-  R_ = k_ + b;
+  // ring slots: at least window + chunk - 1, a multiple of 128 (key tiles of the
+  // tensor-core attention start on 128-aligned positions)
+  R1_ = (S_ + k_ + 127) / 128 * 128;
+  R_ = (k_ + b + 127) / 128 * 128;
 
   // ---- weights ----------------------------------------------------------------------------
   wqkv_.resize(L_);
@@ -431,6 +473,17 @@ int Engine<T>::init() {
   TRY(arena_.alloc(&dgu_, b * 4 * f));
   TRY(arena_.alloc(&do_, b * d));
   TRY(arena_.alloc(&dqkv_, b * 3 * d));
+
+  // ---- attention plans ----------------------------------------------------------------------
+  tc_attn_ = BF && swa_tc_supported((int)HD_);
+  if (tc_attn_) {
+    att_bot_.resize(nbot_);
+    att_top_.resize(nu_);
+    for (int64_t l = 0; l < nbot_; ++l)
+      TRY(swa_tc_prepare(&att_bot_[l], (int)H_, (int)HD_, qs_, S_, d, kb_[l], vb_[l], R1_, d));
+    for (int i = 0; i < nu_; ++i)
+      TRY(swa_tc_prepare(&att_top_[i], (int)H_, (int)HD_, q_[i], b, d, kt_[i], vt_[i], R_, d));
+  }
 
   // ---- GEMM plans -------------------------------------------------------------------------
   EpiArgs e;
@@ -546,7 +599,8 @@ int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
     TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
                                  kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(s0, S),
-              [&] { return swa_forward(swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_), BF, st_); }));
+              [&] { return attn_fwd(tc_attn_ ? &att_bot_[l] : nullptr,
+                                    swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_)); }));
     TRY(run(g[1], S));
     TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[2], S));
@@ -573,7 +627,8 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
                                  kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(p0, n),
-              [&] { return swa_forward(swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b), BF, st_); }));
+              [&] { return attn_fwd(tc_attn_ ? &att_top_[i] : nullptr,
+                                    swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b)); }));
     g[1].args.c2 = const_cast<float*>(xin);
     TRY(run(g[1], n));
     TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_); }));

@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(192, 1)
     ptx::prefetch_tmap(&tmb);
   }
   if (warp == 1) {
+    __syncwarp();
     ptx::tmem_alloc(tmem_slot, BN);
     ptx::tmem_relinquish();
   }
@@ -254,9 +255,10 @@ __global__ void __launch_bounds__(192, 1)
       }
       // Arrives once every MMA issued above has completed (also on a bail-out).
       ptx::umma_commit(accf);
+      ptx::mbar_drain(accf, 0);  // no MMA may still write TMEM when it is released
     }
   } else {
-    const bool ok = ptx::mbar_wait(accf, 0, err);
+    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(accf, 0, err));  // warp-uniform before tcgen05.ld
     ptx::tc_fence_after();
     if (ok) {
       const int q = warp & 3;
@@ -268,6 +270,7 @@ __global__ void __launch_bounds__(192, 1)
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    __syncwarp();  // tcgen05.dealloc is warp-collective: reconverge lane 0 with the others
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, BN);
   }

@@ -2,7 +2,9 @@
 // arguments and launch one kernel family each.
 #include "../../include/ttt_ops.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "gemm.cuh"
+#include "ptx.cuh"
 
 namespace ttt {
 
@@ -104,12 +106,22 @@ static SwaArgs swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t wi
 
 extern "C" int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
                                   int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
-                                  int64_t ring_slots, void* o, int64_t ldo, float* lse, void* stream) {
+                                  int64_t ring_slots, void* o, int64_t ldo, float* lse, int32_t flags, void* stream) {
   if (!q || !k_ring || !v_ring || !o || !lse || n_q < 1 || q_pos0 < 0 || window < 1 || ring_slots < 1 ||
       n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
     return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_forward: bad argument");
   SwaArgs a = swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots, o, ldo, lse);
-  return swa_forward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0) {
+    SwaTcPlan plan;
+    int rc = swa_tc_prepare(&plan, n_heads, head_dim, q, n_q, ldq, k_ring, v_ring, ring_slots,
+                            (int64_t)n_heads * head_dim);
+    if (rc) return rc;
+    int* err = op_err_word();
+    if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_swa_forward: no device error word");
+    return swa_tc_forward(plan, a, st, err);
+  }
+  return swa_forward(a, dtype == TTT_BF16, st);
 }
 
 extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
@@ -131,4 +143,23 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
   a.lddkv = lddkv;
   a.D = D_scratch;
   return swa_backward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace ttt {
+namespace {
+__global__ void watchdog_selftest_kernel(int* err) {
+  __shared__ uint64_t bar;
+  ptx::mbar_init(&bar, 1);
+  ptx::fence_mbar_init();
+  ptx::mbar_wait(&bar, 0, err);  // nobody arrives: must give up and set the error word
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" int ttt_op_watchdog_selftest(void* stream) {
+  int* err = op_err_word();
+  if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_watchdog_selftest: no device error word");
+  watchdog_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
 }

@@ -51,8 +51,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait on an mbarrier phase.  Gives up (returns false) when the
-// device error word is already set by another thread, or after
-// kWaitLimitNs; in the latter case it sets DEV_ERR_TIMEOUT.
+// device error word is already set by another thread, after kWaitLimitNs of
+// %globaltimer, or after kWaitLimitIters polls (a second bound that does not
+// depend on the timer); on a timeout it sets DEV_ERR_TIMEOUT.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -60,11 +61,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0) {
       if (*(volatile int*)err != 0) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > kWaitLimitNs || i >= kWaitLimitIters) {
         atomicOr(err, DEV_ERR_TIMEOUT);
         return false;
       }
     }
+  }
+}
+
+// Bounded wait that ignores the error word: used on bail-out paths to let
+// in-flight asynchronous work drain before shared memory or TMEM is released.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 0; !mbar_try_wait(bar, parity); ++i) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs || i >= kWaitLimitIters) return;
   }
 }
 

@@ -50,11 +50,11 @@ def sync(stream=None):
     L.check(L.lib().ttt_op_sync(_stream(stream)))
 
 
-def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, stream=None):
+def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, force_simt=False, stream=None):
     """ttt_op_swa_forward; q/o [n, H*hd], rings [R, H*hd], lse [H, n]."""
     rc = L.lib().ttt_op_swa_forward(_dtype(q), n_heads, head_dim, q.shape[0], q_pos0, window, _p(q), q.stride(0),
                                     _p(k_ring), _p(v_ring), k_ring.shape[0], _p(o), o.stride(0), _p(lse),
-                                    _stream(stream))
+                                    1 if force_simt else 0, _stream(stream))
     L.check(rc)
 
 
@@ -65,3 +65,8 @@ def swa_backward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, d
                                      dout.stride(0), _p(dq), dq.stride(0), _p(dk), _p(dv), dk.stride(0), _p(D),
                                      _stream(stream))
     L.check(rc)
+
+
+def watchdog_selftest(stream=None):
+    """Launch the bounded-wait self-test; ops.sync() afterwards must raise TTT_ERR_TIMEOUT."""
+    L.check(L.lib().ttt_op_watchdog_selftest(_stream(stream)))
