@@ -92,6 +92,31 @@ int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_
                         const void* o, int64_t ldo, const float* lse, const void* dout, int64_t lddo, void* dq,
                         int64_t lddq, void* dk, void* dv, int64_t lddkv, float* D_scratch, void* stream);
 
+/*
+ * Allocation-free variant of ttt_op_swa_backward.  The paper has no
+ * counterpart: this is an addition for callers that may not allocate device
+ * memory, because their memory belongs to another allocator (a framework's
+ * caching pool, a fixed budget) and cudaMalloc would bypass it and
+ * synchronise the whole device.
+ * Same arguments and results as ttt_op_swa_backward without D_scratch: the
+ * work array lives inside the library as a fixed 1 MiB array per GPU that
+ * loads the library (held until the process exits), so n_heads * n_q must
+ * not exceed 262144; larger calls return TTT_ERR_INVALID_ARG and change
+ * nothing.  It calls no cudaMalloc or cudaFree.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.
+ * Every call uses the same array and leaves its last contents there (each
+ * entry is rewritten before it is read, so nothing needs clearing); calls
+ * whose work overlaps on the GPU (other streams, other host threads) race
+ * on it and must be serialised by the caller.
+ */
+int ttt_op_swa_backward_noalloc(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
+                                int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
+                                int64_t ring_slots, const void* o, int64_t ldo, const float* lse, const void* dout,
+                                int64_t lddo, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv,
+                                void* stream);
+
 /* Device watchdog self-test: launches one thread that waits on an mbarrier
  * nothing ever arrives at.  The bounded wait gives up (about 2 s) and records
  * a timeout, so the following ttt_op_sync returns TTT_ERR_TIMEOUT and the

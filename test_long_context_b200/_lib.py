@@ -80,6 +80,9 @@ def lib():
             "ttt_op_gemm_ce_tiles": (c_i64, [c_i32, c_i64, c_i64, c_i32]),
             "ttt_op_sync": (c_i32, [c_vp]),
             "ttt_op_watchdog_selftest": (c_i32, [c_vp]),
+            "ttt_op_swa_backward_noalloc": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp,
+                                                    c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
+                                                    c_vp, c_i64, c_vp]),
             "ttt_op_swa_forward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp, c_i64,
                                            c_vp, c_i64, c_vp, c_i32, c_vp]),
             "ttt_op_swa_backward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp,
@@ -114,7 +117,8 @@ def exported_symbols():
     names = []
     for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
               "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
-              "ttt_op_swa_backward", "ttt_op_watchdog_selftest"):
+              "ttt_op_swa_backward", "ttt_op_watchdog_selftest",
+              "ttt_op_swa_backward_noalloc"):
         if hasattr(L, n):
             names.append(n)
     return names

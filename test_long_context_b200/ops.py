@@ -70,3 +70,14 @@ def swa_backward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, d
 def watchdog_selftest(stream=None):
     """Launch the bounded-wait self-test; ops.sync() afterwards must raise TTT_ERR_TIMEOUT."""
     L.check(L.lib().ttt_op_watchdog_selftest(_stream(stream)))
+
+
+def swa_backward_noalloc(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, dout, dq, dk, dv,
+                         stream=None):
+    """ttt_op_swa_backward_noalloc: like swa_backward, with the library's own
+    fixed work array instead of caller scratch (no device allocation)."""
+    rc = L.lib().ttt_op_swa_backward_noalloc(_dtype(q), n_heads, head_dim, q.shape[0], q_pos0, window, _p(q),
+                                             q.stride(0), _p(k_ring), _p(v_ring), k_ring.shape[0], _p(o),
+                                             o.stride(0), _p(lse), _p(dout), dout.stride(0), _p(dq), dq.stride(0),
+                                             _p(dk), _p(dv), dk.stride(0), _stream(stream))
+    L.check(rc)
