@@ -85,12 +85,16 @@ int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t
  * the full band, cached keys included) and dk, dv for the keys at positions
  * q_pos0 .. q_pos0+n_q-1 only (row i = position q_pos0 + i); keys of earlier
  * positions are treated as constants.  dq: [n_q, lddq]; dk, dv: [n_q, lddkv].
- * D_scratch: fp32 [n_heads * n_q] work space.
+ * D_scratch: fp32 [n_heads * n_q] work space.  With TTT_BF16, head_dim in
+ * {64, 80, 96, 128}, ring_slots a multiple of 128, q and dout with the same
+ * row pitch, and flags bit 0 (TTT_SWA_FORCE_SIMT) clear, dq is computed on
+ * the tensor cores; everything else uses the SIMT kernels.
  */
 int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
                         const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
                         const void* o, int64_t ldo, const float* lse, const void* dout, int64_t lddo, void* dq,
-                        int64_t lddq, void* dk, void* dv, int64_t lddkv, float* D_scratch, void* stream);
+                        int64_t lddq, void* dk, void* dv, int64_t lddkv, float* D_scratch, int32_t flags,
+                        void* stream);
 
 /*
  * Allocation-free variant of ttt_op_swa_backward.  The paper has no

@@ -87,7 +87,7 @@ def lib():
                                            c_vp, c_i64, c_vp, c_i32, c_vp]),
             "ttt_op_swa_backward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp,
                                             c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64,
-                                            c_vp, c_vp]),
+                                            c_vp, c_i32, c_vp]),
         }
         for name, (res, args) in sig.items():
             if hasattr(L, name):

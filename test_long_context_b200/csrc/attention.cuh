@@ -1,5 +1,7 @@
 // Sliding-window attention launch interface.
 #pragma once
+#include <functional>
+
 #include "common.cuh"
 
 namespace ttt {
@@ -36,5 +38,7 @@ struct SwaArgs {
 int swa_forward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
 // Needs a.o, a.lse from the forward; writes D, dq, dk, dv.
 int swa_backward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
+// Same, with the dq part replaced by `dq` (launched after D is written).
+int swa_backward_with_dq(const SwaArgs& a, bool use_bf16, cudaStream_t s, const std::function<int()>& dq);
 
 }  // namespace ttt

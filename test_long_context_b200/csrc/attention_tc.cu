@@ -360,6 +360,283 @@ __global__ void __launch_bounds__(256, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------------------------
+// Backward, dq part: dQ = scale * sum_j dS_j K_j over the band, with
+// dS = P o (dP - D), P = exp(S*scale - lse), S = Q K^T, dP = dO V^T.
+// CTA = 128 queries x one head; key tiles of 64 keys (2 K/V stages).
+//   warp 0      TMA: Q and dO once, then K/V tiles
+//   warp 1      TMEM owner; lane 0 issues S_j = Q K_j^T and dP_j = dO V_j^T into
+//               one of two TMEM buffers (64 + 64 columns), then dQ += dS_j K_j
+//   warps 4..7  one query row per thread: P, dS in fp32 -> bf16 dS tile in
+//               128B-swizzled smem (K-major A operand of the dQ product)
+// The softmax statistics come from the forward (lse), so there is no online
+// rescaling and every TMEM access is warp-uniform.
+constexpr int BKT = 64;  // keys per tile in the backward
+constexpr int BNST = 3;  // K/V stages in the backward (also keeps one CTA per SM: each takes all of TMEM)
+
+template <int HD>
+struct BGeo {
+  static constexpr int A = HD / 64;
+  static constexpr int R = HD % 64;
+  static constexpr int RB = R * 2;
+  static constexpr int QTILE = 128 * HD * 2;   // Q or dO tile (128 rows)
+  static constexpr int KTILE = BKT * HD * 2;   // K or V tile (64 rows)
+  static constexpr int KREM = A * 8192;        // remainder offset inside a 64-row tile
+  static constexpr int QREM = A * 16384;       // remainder offset inside a 128-row tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int DO_OFF = QTILE;
+  static constexpr int KV_OFF = 2 * QTILE;     // stage s: K at KV_OFF + s*2*KTILE, V after
+  static constexpr int DS_OFF = KV_OFF + BNST * 2 * KTILE;
+  static constexpr int DS_BYTES = 128 * BKT * 2;  // one 128B-swizzled atom column (64 keys)
+  static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(KTILE % 1024 == 0 && QTILE % 1024 == 0, "1024-byte aligned tiles");
+};
+
+template <int HD>
+__device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m64, const CUtensorMap* mrem,
+                                          uint64_t* bar, int col0, int row0, int atom_bytes, int rem_off) {
+  constexpr int A = HD / 64, R = HD % 64;
+#pragma unroll
+  for (int a = 0; a < A; ++a) ptx::tma_load_2d(dst + a * atom_bytes, m64, bar, col0 + 64 * a, row0);
+  if constexpr (R > 0) ptx::tma_load_2d(dst + rem_off, mrem, bar, col0 + 64 * A, row0);
+}
+
+template <int HD>
+__global__ void __launch_bounds__(256, 1)
+    swa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
+                         const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tdo_r,
+                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
+                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r, SwaArgs a,
+                         int* err) {
+  using G = BGeo<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* kv_full = bars + 1;   // [BNST]
+  uint64_t* kv_empty = bars + 4;  // [BNST]
+  uint64_t* s_full = bars + 7;    // [2]  S_j, dP_j in TMEM buffer j&1
+  uint64_t* ds_full = bars + 9;   // [2]  dS_j written (and TMEM buffer j&1 read)
+  uint64_t* ds_free = bars + 11;  // [2]  dQ_j consumed dS buffer j&1
+  uint64_t* dq_full = bars + 13;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int64_t q0 = a.p0 + (int64_t)blockIdx.x * QT;
+  const int64_t qlast = imin64(q0 + QT, a.p0 + a.n) - 1;
+  const int64_t kfirst = imax64(0, q0 - a.window + 1);
+  const int64_t j_begin = (kfirst / BKT) * BKT;
+  const int ntiles = (int)((qlast - j_begin) / BKT + 1);
+  const int col0 = h * HD;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int s = 0; s < BNST; ++s) {
+      ptx::mbar_init(&kv_full[s], 1);
+      ptx::mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&s_full[s], 1);
+      ptx::mbar_init(&ds_full[s], 128);
+      ptx::mbar_init(&ds_free[s], 1);
+    }
+    ptx::mbar_init(dq_full, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_dq = tmem + 256;  // S/dP buffers at columns [0,128) and [128,256)
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(q_full, 2 * G::QTILE);
+      const int qrow = (int)(q0 - a.p0);
+      load_rows<HD>(sm + G::Q_OFF, &tq, &tq_r, q_full, col0, qrow, 16384, G::QREM);
+      load_rows<HD>(sm + G::DO_OFF, &tdo, &tdo_r, q_full, col0, qrow, 16384, G::QREM);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j % BNST;
+        if (!ptx::mbar_wait(&kv_empty[s], ((j / BNST) & 1) ^ 1, err)) break;
+        ptx::mbar_arrive_expect_tx(&kv_full[s], 2 * G::KTILE);
+        const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
+        uint8_t* kd = sm + G::KV_OFF + s * 2 * G::KTILE;
+        load_rows<HD>(kd, &tk, &tk_r, &kv_full[s], col0, slot, 8192, G::KREM);
+        load_rows<HD>(kd + G::KTILE, &tv, &tv_r, &kv_full[s], col0, slot, 8192, G::KREM);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, BKT, false, false);
+      constexpr uint32_t id_q64 = ptx::idesc_bf16_f32(128, 64, false, true);
+      constexpr uint32_t id_qr = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
+      const uint32_t q_addr = ptx::smem_u32(sm + G::Q_OFF), do_addr = ptx::smem_u32(sm + G::DO_OFF);
+      constexpr uint32_t rl = rem_swizzle_layout(G::R);
+      bool ok = ptx::mbar_wait(q_full, 0, err);
+      // S_j = Q K_j^T and dP_j = dO V_j^T into TMEM buffer j&1
+      auto issue_s = [&](int j) {
+        const int s = j % BNST;
+        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::KTILE);
+        const uint32_t v_addr = k_addr + G::KTILE;
+        const uint32_t dS = tmem + (j & 1) * 128, dP = dS + 64;
+        int step = 0;
+#pragma unroll
+        for (int at = 0; at < G::A; ++at)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk, ++step) {
+            ptx::umma_bf16(dS, sdesc(q_addr + at * 16384 + kk * 32, 16, 1024, 2),
+                           sdesc(k_addr + at * 8192 + kk * 32, 16, 1024, 2), id_s, step > 0);
+            ptx::umma_bf16(dP, sdesc(do_addr + at * 16384 + kk * 32, 16, 1024, 2),
+                           sdesc(v_addr + at * 8192 + kk * 32, 16, 1024, 2), id_s, step > 0);
+          }
+        if constexpr (G::R > 0) {
+#pragma unroll
+          for (int kk = 0; kk < G::R / 16; ++kk, ++step) {
+            ptx::umma_bf16(dS, sdesc(q_addr + G::QREM + kk * 32, 16, 8 * G::RB, rl),
+                           sdesc(k_addr + G::KREM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
+            ptx::umma_bf16(dP, sdesc(do_addr + G::QREM + kk * 32, 16, 8 * G::RB, rl),
+                           sdesc(v_addr + G::KREM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
+          }
+        }
+        ptx::umma_commit(&s_full[j & 1]);
+      };
+      if (ok && ntiles > 0 && (ok = ptx::mbar_wait(&kv_full[0], 0, err))) {
+        ptx::tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; ok && j < ntiles; ++j) {
+        // TMEM buffer (j+1)&1 was read by the softmax of tile j-1 (waited below in the previous iteration)
+        if (j + 1 < ntiles) {
+          if (!(ok = ptx::mbar_wait(&kv_full[(j + 1) % BNST], ((j + 1) / BNST) & 1, err))) break;
+          ptx::tc_fence_after();
+          issue_s(j + 1);
+        }
+        if (!(ok = ptx::mbar_wait(&ds_full[j & 1], (j / 2) & 1, err))) break;
+        ptx::tc_fence_after();
+        const int s = j % BNST;
+        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::KTILE);
+        const uint32_t ds_addr = ptx::smem_u32(sm + G::DS_OFF + (j & 1) * G::DS_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BKT / 16; ++kk) {  // dQ += dS_j K_j, K over the 64 keys
+          const uint64_t ad = sdesc(ds_addr + kk * 32, 16, 1024, 2);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+#pragma unroll
+          for (int at = 0; at < G::A; ++at)
+            ptx::umma_bf16(t_dq + 64 * at, ad, sdesc(k_addr + at * 8192 + kk * 2048, 16, 1024, 2), id_q64, acc);
+          if constexpr (G::R > 0)
+            ptx::umma_bf16(t_dq + 64 * G::A, ad, sdesc(k_addr + G::KREM + kk * 16 * G::RB, 16, 8 * G::RB, rl),
+                           id_qr, acc);
+        }
+        ptx::umma_commit(&kv_empty[s]);
+        ptx::umma_commit(&ds_free[j & 1]);
+      }
+      ptx::umma_commit(dq_full);
+      ptx::mbar_drain(dq_full, 0);
+    }
+  } else if (warp >= 4) {
+    const int r = (warp - 4) * 32 + lane;
+    const int64_t p = q0 + r;
+    const bool row_ok = p <= qlast;
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const float L2E = 1.4426950408889634f;
+    const float sl2 = a.scale * L2E;
+    const int64_t i = p - a.p0;
+    const float lse2 = row_ok ? a.lse[(int64_t)h * a.ld_lse + i] * L2E : 0.f;
+    const float Di = row_ok ? a.D[(int64_t)h * a.ld_lse + i] : 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int64_t j0 = j_begin + (int64_t)j * BKT;
+      ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      ptx::tc_fence_after();
+      float sv[BKT], dp[BKT];
+#pragma unroll
+      for (int c = 0; c < BKT; c += 32) {
+        uint32_t rs[32], rd[32];
+        ptx::tmem_ld32(tmem + (j & 1) * 128 + c + lane_off, rs);
+        ptx::tmem_ld32(tmem + (j & 1) * 128 + 64 + c + lane_off, rd);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          sv[c + e] = __uint_as_float(rs[e]);
+          dp[c + e] = __uint_as_float(rd[e]);
+        }
+      }
+      ptx::tc_fence_before();
+      if (j >= 2) {  // dS buffer j&1 is free once dQ_{j-2} consumed it
+        ok = ptx::mbar_wait(&ds_free[j & 1], ((j - 2) / 2) & 1, err);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
+      uint8_t* drow = sm + G::DS_OFF + (j & 1) * G::DS_BYTES + r * 128;
+#pragma unroll
+      for (int g = 0; g < BKT / 8; ++g) {
+        float ds[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = g * 8 + e;
+          const bool v = row_ok && c >= lo && c <= hi;
+          const float pr = v ? exp2f(sv[c] * sl2 - lse2) : 0.f;
+          ds[e] = pr * (dp[c] - Di);
+        }
+        uint4 w;
+        __nv_bfloat162 b0 = __floats2bfloat162_rn(ds[0], ds[1]), b1 = __floats2bfloat162_rn(ds[2], ds[3]);
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(ds[4], ds[5]), b3 = __floats2bfloat162_rn(ds[6], ds[7]);
+        w.x = *reinterpret_cast<uint32_t*>(&b0);
+        w.y = *reinterpret_cast<uint32_t*>(&b1);
+        w.z = *reinterpret_cast<uint32_t*>(&b2);
+        w.w = *reinterpret_cast<uint32_t*>(&b3);
+        *reinterpret_cast<uint4*>(drow + ((g ^ (r & 7)) << 4)) = w;
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&ds_full[j & 1]);
+    }
+    if (ok) ok = ptx::mbar_wait(dq_full, 0, err);
+    if (__all_sync(0xffffffffu, ok)) {
+      ptx::tc_fence_after();
+      bf16* out = reinterpret_cast<bf16*>(a.dq) + i * a.lddq + col0;
+#pragma unroll
+      for (int c = 0; c < HD; c += 16) {
+        uint32_t o[16];
+        tmem_ld16(t_dq + c + lane_off, o);
+        ptx::tmem_ld_wait();
+        if (row_ok) {
+          uint4 w0, w1;
+          uint32_t* pw = &w0.x;
+          uint32_t* pw1 = &w1.x;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 t0 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * a.scale,
+                                                      __uint_as_float(o[2 * e + 1]) * a.scale);
+            __nv_bfloat162 t1 = __floats2bfloat162_rn(__uint_as_float(o[8 + 2 * e]) * a.scale,
+                                                      __uint_as_float(o[9 + 2 * e]) * a.scale);
+            pw[e] = *reinterpret_cast<uint32_t*>(&t0);
+            pw1[e] = *reinterpret_cast<uint32_t*>(&t1);
+          }
+          *reinterpret_cast<uint4*>(out + c) = w0;
+          *reinterpret_cast<uint4*>(out + c + 8) = w1;
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -378,14 +655,14 @@ EncodeTiledFn encode() {
 }
 
 // bf16 [rows, cols] with row pitch ld; box = box_cols x 128 rows; swizzle by box width.
-int tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols) {
+int tmap(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int64_t ld, int box_cols, int box_rows = 128) {
   EncodeTiledFn enc = encode();
   if (!enc) return set_error(TTT_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || ((ld * 2) & 15))
     return set_error(TTT_ERR_INVALID_ARG, "attention: operands must be 16-byte aligned");
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, 128u};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t es[2] = {1u, 1u};
   const CUtensorMapSwizzle sw = box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B
                                 : box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
@@ -418,6 +695,69 @@ int launch(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
   return TTT_OK;
 }
 
+
+template <int HD>
+int launch_bwd_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  using G = BGeo<HD>;
+  auto fn = &swa_bwd_dq_tc_kernel<HD>;
+  {
+    static std::mutex mu;
+    static std::set<int> done;
+    int dev = 0;
+    TTT_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done.count(dev)) {
+      TTT_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+      done.insert(dev);
+    }
+  }
+  dim3 grid(ceil_div(a.n, QT), a.heads);
+  fn<<<grid, 256, G::SMEM, s>>>(p.q128, p.qr, p.do128, p.dor, p.k64, p.kr, p.v64, p.vr, a, err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+}  // namespace
+
+int swa_tc_bwd_prepare(SwaTcBwdPlan* p, int heads, int head_dim, const void* q, const void* dout, int64_t rows,
+                       int64_t ld, const void* k, const void* v, int64_t ring, int64_t ldkv) {
+  if (!swa_tc_supported(head_dim)) return set_error(TTT_ERR_UNSUPPORTED, "attention: head_dim not supported");
+  if (ring % 128) return set_error(TTT_ERR_INVALID_ARG, "attention: ring slots must be a multiple of 128");
+  p->head_dim = head_dim;
+  p->ring = ring;
+  const int64_t cols = (int64_t)heads * head_dim;
+  const int rem = head_dim % 64;
+  int rc = tmap(&p->q128, q, rows, cols, ld, 64);
+  if (!rc) rc = tmap(&p->do128, dout, rows, cols, ld, 64);
+  if (!rc) rc = tmap(&p->k64, k, ring, cols, ldkv, 64, 64);
+  if (!rc) rc = tmap(&p->v64, v, ring, cols, ldkv, 64, 64);
+  if (rc) return rc;
+  if (rem) {
+    rc = tmap(&p->qr, q, rows, cols, ld, rem);
+    if (!rc) rc = tmap(&p->dor, dout, rows, cols, ld, rem);
+    if (!rc) rc = tmap(&p->kr, k, ring, cols, ldkv, rem, 64);
+    if (!rc) rc = tmap(&p->vr, v, ring, cols, ldkv, rem, 64);
+  } else {
+    p->qr = p->q128;
+    p->dor = p->do128;
+    p->kr = p->k64;
+    p->vr = p->v64;
+  }
+  return rc;
+}
+
+int swa_tc_backward_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  if (a.ring != p.ring || a.head_dim != p.head_dim) return set_error(TTT_ERR_INVALID_ARG, "attention: plan mismatch");
+  switch (a.head_dim) {
+    case 64: return launch_bwd_dq<64>(p, a, s, err);
+    case 80: return launch_bwd_dq<80>(p, a, s, err);
+    case 96: return launch_bwd_dq<96>(p, a, s, err);
+    case 128: return launch_bwd_dq<128>(p, a, s, err);
+  }
+  return set_error(TTT_ERR_UNSUPPORTED, "attention (tensor cores): head_dim must be 64, 80, 96 or 128");
+}
+
+namespace {
 }  // namespace
 
 bool swa_tc_supported(int head_dim) {

@@ -16,7 +16,27 @@ struct SwaTcPlan {
   int64_t ring = 0;
 };
 
+// Backward (dq over the band) on tensor cores: q and dout share a layout
+// ([rows, heads*head_dim], pitch ld); the rings as in the forward.
+struct SwaTcBwdPlan {
+  alignas(64) CUtensorMap q128;
+  alignas(64) CUtensorMap qr;
+  alignas(64) CUtensorMap do128;
+  alignas(64) CUtensorMap dor;
+  alignas(64) CUtensorMap k64;
+  alignas(64) CUtensorMap kr;
+  alignas(64) CUtensorMap v64;
+  alignas(64) CUtensorMap vr;
+  int head_dim = 0;
+  int64_t ring = 0;
+};
+
 bool swa_tc_supported(int head_dim);
+int swa_tc_bwd_prepare(SwaTcBwdPlan* p, int heads, int head_dim, const void* q, const void* dout, int64_t rows,
+                       int64_t ld, const void* k, const void* v, int64_t ring, int64_t ldkv);
+// Writes a.dq (bf16) from a.q, a.dout, the rings, a.lse and a.D (the row dot
+// products dO . O, computed beforehand).
+int swa_tc_backward_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err);
 // q: [q_rows, heads*head_dim] (pitch ldq); k, v rings: [ring, heads*head_dim]
 // (pitch ldkv); ring must be a multiple of 128.
 int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t q_rows, int64_t ldq, const void* k,

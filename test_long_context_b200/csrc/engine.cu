@@ -299,6 +299,7 @@ class Engine final : public ttt_ctx {
   // tensor-core attention plans (bf16, supported head_dim)
   bool tc_attn_ = false;
   std::vector<SwaTcPlan> att_bot_, att_top_;
+  std::vector<SwaTcBwdPlan> att_bwd_;
   int attn_fwd(const SwaTcPlan* plan, const SwaArgs& a) {
     if (tc_attn_) return swa_tc_forward(*plan, a, st_, err_);
     return swa_forward(a, BF, st_);
@@ -483,6 +484,9 @@ int Engine<T>::init() {
       TRY(swa_tc_prepare(&att_bot_[l], (int)H_, (int)HD_, qs_, S_, d, kb_[l], vb_[l], R1_, d));
     for (int i = 0; i < nu_; ++i)
       TRY(swa_tc_prepare(&att_top_[i], (int)H_, (int)HD_, q_[i], b, d, kt_[i], vt_[i], R_, d));
+    att_bwd_.resize(nu_);
+    for (int i = 1; i < nu_; ++i)
+      TRY(swa_tc_bwd_prepare(&att_bwd_[i], (int)H_, (int)HD_, q_[i], do_, b, d, kt_[i], vt_[i], R_, d));
   }
 
   // ---- GEMM plans -------------------------------------------------------------------------
@@ -672,8 +676,10 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     a.dv = dqkv_ + 2 * d;
     a.lddkv = 3 * d;
     a.D = Dbuf_;
-    TRY(timed(TTT_KC_ATTN_BWD, 4.0 * d * (band_pairs(p0, n) + (double)n * (double)(n + 1) / 2.0),
-              [&] { return swa_backward(a, BF, st_); }));
+    TRY(timed(TTT_KC_ATTN_BWD, 4.0 * d * (band_pairs(p0, n) + (double)n * (double)(n + 1) / 2.0), [&] {
+      if (tc_attn_) return swa_backward_with_dq(a, true, st_, [&] { return swa_tc_backward_dq(att_bwd_[i], a, st_, err_); });
+      return swa_backward(a, BF, st_);
+    }));
     launches += 2;  // the backward launches three kernels
     TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
                                  (int)HD_, theta, st_); }));

@@ -128,7 +128,7 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
                                    int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
                                    int64_t ring_slots, const void* o, int64_t ldo, const float* lse, const void* dout,
                                    int64_t lddo, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv,
-                                   float* D_scratch, void* stream) {
+                                   float* D_scratch, int32_t flags, void* stream) {
   if (!q || !k_ring || !v_ring || !o || !lse || !dout || !dq || !dk || !dv || !D_scratch || n_q < 1 || q_pos0 < 0 ||
       window < 1 || ring_slots < 1 || n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
     return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_backward: bad argument");
@@ -142,7 +142,18 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
   a.dv = dv;
   a.lddkv = lddkv;
   a.D = D_scratch;
-  return swa_backward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0 &&
+      ldq == lddo) {
+    SwaTcBwdPlan plan;
+    int rc = swa_tc_bwd_prepare(&plan, n_heads, head_dim, q, dout, n_q, ldq, k_ring, v_ring, ring_slots,
+                                (int64_t)n_heads * head_dim);
+    if (rc) return rc;
+    int* err = op_err_word();
+    if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_swa_backward: no device error word");
+    return swa_backward_with_dq(a, true, st, [&] { return swa_tc_backward_dq(plan, a, st, err); });
+  }
+  return swa_backward(a, dtype == TTT_BF16, st);
 }
 
 namespace ttt {

@@ -58,12 +58,13 @@ def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, fo
     L.check(rc)
 
 
-def swa_backward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, dout, dq, dk, dv, D, stream=None):
+def swa_backward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, dout, dq, dk, dv, D,
+                 force_simt=False, stream=None):
     """ttt_op_swa_backward; dk/dv rows are the keys at q_pos0 .. q_pos0+n-1."""
     rc = L.lib().ttt_op_swa_backward(_dtype(q), n_heads, head_dim, q.shape[0], q_pos0, window, _p(q), q.stride(0),
                                      _p(k_ring), _p(v_ring), k_ring.shape[0], _p(o), o.stride(0), _p(lse), _p(dout),
                                      dout.stride(0), _p(dq), dq.stride(0), _p(dk), _p(dv), dk.stride(0), _p(D),
-                                     _stream(stream))
+                                     1 if force_simt else 0, _stream(stream))
     L.check(rc)
 
 

@@ -66,7 +66,7 @@ def test_swa_forward_backward_vs_oracle(impl, hd, n, p0, window, ring):
     dk = torch.empty_like(o)
     dv = torch.empty_like(o)
     D = torch.empty(H * n, device="cuda")
-    ops.swa_backward(qd, krd, vrd, H, hd, p0, window, o, lse, dd, dq, dk, dv, D)
+    ops.swa_backward(qd, krd, vrd, H, hd, p0, window, o, lse, dd, dq, dk, dv, D, force_simt=(impl == "bf16-simt"))
     ops.sync()
     tol = 2e-2 if dtype == "bf16" else 1e-5
 

@@ -29,7 +29,7 @@ def test_noalloc_backward_matches_scratch_entry_point_twice(dtype):
         ops.swa_forward(q, kr, vr, H, hd, p0, window, o, lse, force_simt=True)
         ref = [torch.empty_like(q) for _ in range(3)]
         D = torch.empty(H * n, device="cuda")
-        ops.swa_backward(q, kr, vr, H, hd, p0, window, o, lse, dout, *ref, D)
+        ops.swa_backward(q, kr, vr, H, hd, p0, window, o, lse, dout, *ref, D, force_simt=True)
         got = [torch.full_like(q, float("nan")) for _ in range(3)]
         ops.swa_backward_noalloc(q, kr, vr, H, hd, p0, window, o, lse, dout, *got)
         ops.sync()
