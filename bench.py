@@ -33,7 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill tokens/s (2.7B, SWA k=8K, TTT b=1K, T=128K) and % of bf16 tensor peak"
-KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other")
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope")
 
 
 def parse_args():
@@ -79,8 +79,9 @@ def load_peaks():
 
 
 def kernel_source_hash(kc):
-    files = {"gemm": ["gemm_tc.cu", "ptx.cuh"], "attn_fwd": ["attention.cu"], "attn_bwd": ["attention.cu"],
-             "other": ["elementwise.cu"]}[kc]
+    files = {"gemm": ["gemm_tc.cu", "ptx.cuh"], "attn_fwd": ["attention_tc.cu", "ptx.cuh"],
+             "attn_bwd": ["attention_tc.cu", "attention.cu", "ptx.cuh"], "other": ["elementwise.cu"],
+             "norm": ["elementwise.cu"], "rope": ["elementwise.cu"]}[kc]
     h = hashlib.sha256()
     for f in files:
         with open(os.path.join(ROOT, "test_long_context_b200", "csrc", f), "rb") as fh:

@@ -180,8 +180,10 @@ int64_t ttt_launch_count(ttt_ctx* ctx);
 #define TTT_KC_GEMM 0
 #define TTT_KC_ATTN_FWD 1
 #define TTT_KC_ATTN_BWD 2
-#define TTT_KC_OTHER 3
-#define TTT_KC_COUNT 4
+#define TTT_KC_OTHER 3 /* embedding, SwiGLU backward, CE finalise, targets, copies */
+#define TTT_KC_NORM 4  /* RMSNorm forward and backward */
+#define TTT_KC_ROPE 5  /* QK-norm + RoPE forward (with the KV-ring write) and backward */
+#define TTT_KC_COUNT 6
 int ttt_timing_enable(ttt_ctx* ctx, int32_t enable);
 int ttt_timing_read(ttt_ctx* ctx, int32_t kernel_class, double* total_ms, int64_t* launches, double* flops);
 

@@ -59,6 +59,18 @@ int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N,
                 int64_t lda, const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args,
                 int32_t bn_hint, void* stream);
 
+/*
+ * ttt_op_gemm (TTT_BF16 only) with the K range split into ksplit parts: each
+ * part's fp32 partial product goes to `workspace` (caller-owned, at least
+ * ksplit * M * N floats), then one kernel sums the parts in a fixed order
+ * (run-to-run identical results) and applies the epilogue.  Epilogues:
+ * TTT_EPI_STORE_F32, TTT_EPI_STORE_BF16, TTT_EPI_ADD_F32.  ksplit <= 1 is the
+ * plain GEMM.  Useful when the output alone has too few tiles to fill the GPU.
+ */
+int ttt_op_gemm_split(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                      const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args, int32_t bn_hint,
+                      int32_t ksplit, float* workspace, void* stream);
+
 /* Number of N tiles a CE_FWD ttt_op_gemm of width N writes partials for. */
 int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint);
 

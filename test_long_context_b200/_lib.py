@@ -20,8 +20,8 @@ TTT_ERR_UNSUPPORTED = -6
 TTT_F32 = 0
 TTT_BF16 = 1
 
-KC_GEMM, KC_ATTN_FWD, KC_ATTN_BWD, KC_OTHER = range(4)
-KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other")
+KC_GEMM, KC_ATTN_FWD, KC_ATTN_BWD, KC_OTHER, KC_NORM, KC_ROPE = range(6)
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope")
 EPI_STORE_F32, EPI_STORE_BF16, EPI_ADD_F32, EPI_SWIGLU, EPI_CE_FWD, EPI_CE_BWD, EPI_SGD = range(7)
 
 c_i32, c_i64, c_f32, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -78,6 +78,8 @@ def lib():
             "ttt_op_gemm": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
                                     ctypes.POINTER(ttt_epilogue_args), c_i32, c_vp]),
             "ttt_op_gemm_ce_tiles": (c_i64, [c_i32, c_i64, c_i64, c_i32]),
+            "ttt_op_gemm_split": (c_i32, [c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
+                                          ctypes.POINTER(ttt_epilogue_args), c_i32, c_i32, c_vp, c_vp]),
             "ttt_op_sync": (c_i32, [c_vp]),
             "ttt_op_watchdog_selftest": (c_i32, [c_vp]),
             "ttt_op_swa_backward_noalloc": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp,
@@ -116,7 +118,7 @@ def exported_symbols():
     L = lib()
     names = []
     for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
-              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
+              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
               "ttt_op_swa_backward", "ttt_op_watchdog_selftest",
               "ttt_op_swa_backward_noalloc"):
         if hasattr(L, n):

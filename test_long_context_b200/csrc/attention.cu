@@ -270,7 +270,8 @@ int launch_fwd(const SwaArgs& a, cudaStream_t s) {
 }
 
 template <typename T, int HD>
-int launch_bwd(const SwaArgs& a, cudaStream_t s, const std::function<int()>& dq_override) {
+int launch_bwd(const SwaArgs& a, cudaStream_t s, const std::function<int()>& dq_override,
+               const std::function<int()>& dkdv_override) {
   swa_bwd_dot<T, HD><<<ceil_div(a.n * a.heads, 256), 256, 0, s>>>(a);
   TTT_CUDA_TRY(cudaGetLastError());
   if (dq_override) {
@@ -281,6 +282,7 @@ int launch_bwd(const SwaArgs& a, cudaStream_t s, const std::function<int()>& dq_
     swa_bwd_dq_simt<T, HD, 2><<<g1, ATT_THREADS, 0, s>>>(a);
     TTT_CUDA_TRY(cudaGetLastError());
   }
+  if (dkdv_override) return dkdv_override();
   dim3 g2(ceil_div(a.n, ATT_THREADS / 4), a.heads);
   swa_bwd_dkdv_simt<T, HD, 4><<<g2, ATT_THREADS, 0, s>>>(a);
   TTT_CUDA_TRY(cudaGetLastError());
@@ -300,13 +302,14 @@ int dispatch_fwd(const SwaArgs& a, cudaStream_t s) {
 }
 
 template <typename T>
-int dispatch_bwd(const SwaArgs& a, cudaStream_t s, const std::function<int()>& dq) {
+int dispatch_bwd(const SwaArgs& a, cudaStream_t s, const std::function<int()>& dq,
+                 const std::function<int()>& dkdv) {
   switch (a.head_dim) {
-    case 32: return launch_bwd<T, 32>(a, s, dq);
-    case 64: return launch_bwd<T, 64>(a, s, dq);
-    case 80: return launch_bwd<T, 80>(a, s, dq);
-    case 96: return launch_bwd<T, 96>(a, s, dq);
-    case 128: return launch_bwd<T, 128>(a, s, dq);
+    case 32: return launch_bwd<T, 32>(a, s, dq, dkdv);
+    case 64: return launch_bwd<T, 64>(a, s, dq, dkdv);
+    case 80: return launch_bwd<T, 80>(a, s, dq, dkdv);
+    case 96: return launch_bwd<T, 96>(a, s, dq, dkdv);
+    case 128: return launch_bwd<T, 128>(a, s, dq, dkdv);
   }
   return set_error(TTT_ERR_UNSUPPORTED, "attention: head_dim must be 32, 64, 80, 96 or 128");
 }
@@ -320,12 +323,13 @@ int swa_forward(const SwaArgs& a, bool use_bf16, cudaStream_t s) {
 
 int swa_backward(const SwaArgs& a, bool use_bf16, cudaStream_t s) {
   if (a.n < 1 || a.window < 1 || a.ring < 1) return set_error(TTT_ERR_INVALID_ARG, "attention: bad sizes");
-  return use_bf16 ? dispatch_bwd<bf16>(a, s, {}) : dispatch_bwd<float>(a, s, {});
+  return use_bf16 ? dispatch_bwd<bf16>(a, s, {}, {}) : dispatch_bwd<float>(a, s, {}, {});
 }
 
-int swa_backward_with_dq(const SwaArgs& a, bool use_bf16, cudaStream_t s, const std::function<int()>& dq) {
+int swa_backward_with_dq(const SwaArgs& a, bool use_bf16, cudaStream_t s, const std::function<int()>& dq,
+                         const std::function<int()>& dkdv) {
   if (a.n < 1 || a.window < 1 || a.ring < 1) return set_error(TTT_ERR_INVALID_ARG, "attention: bad sizes");
-  return use_bf16 ? dispatch_bwd<bf16>(a, s, dq) : dispatch_bwd<float>(a, s, dq);
+  return use_bf16 ? dispatch_bwd<bf16>(a, s, dq, dkdv) : dispatch_bwd<float>(a, s, dq, dkdv);
 }
 
 }  // namespace ttt

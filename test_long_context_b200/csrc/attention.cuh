@@ -38,7 +38,9 @@ struct SwaArgs {
 int swa_forward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
 // Needs a.o, a.lse from the forward; writes D, dq, dk, dv.
 int swa_backward(const SwaArgs& a, bool use_bf16, cudaStream_t s);
-// Same, with the dq part replaced by `dq` (launched after D is written).
-int swa_backward_with_dq(const SwaArgs& a, bool use_bf16, cudaStream_t s, const std::function<int()>& dq);
+// Same, with the dq part replaced by `dq` (launched after D is written) and,
+// when `dkdv` is given, the dk/dv part replaced by it.
+int swa_backward_with_dq(const SwaArgs& a, bool use_bf16, cudaStream_t s, const std::function<int()>& dq,
+                         const std::function<int()>& dkdv = {});
 
 }  // namespace ttt

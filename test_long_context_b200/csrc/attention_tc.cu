@@ -1,13 +1,15 @@
 // Tensor-core (tcgen05) flash attention forward for the banded causal window
 // of eq. (1) (query p sees keys p-k+1 .. p), bf16 operands, fp32 softmax.
 //
-// CTA = one tile of 128 queries x one head; 8 warps:
-//   warp 0      TMA producer: Q once, then K/V tiles of 128 keys (2 stages)
-//   warp 1      TMEM owner; lane 0 issues every tcgen05.mma
-//   warps 4..7  softmax: thread = query row = TMEM lane; writes P (bf16) to
-//               128B-swizzled smem, keeps the running max / sum, rescales O in
-//               TMEM only when the max grows by more than 2^8 (log2 domain),
-//               and finally normalises O and writes it with the LSE.
+// CTA = one tile of 128 queries x one head; 12 warps:
+//   warp 0       TMA producer: Q once, then K/V tiles of 128 keys (2 stages)
+//   warp 1       TMEM owner; lane 0 issues every tcgen05.mma
+//   warps 4..11  softmax: a query row (= TMEM lane) is shared by two threads,
+//                one per warpgroup, each owning 64 key columns; they combine
+//                row maxima through smem, write P (bf16) to 128B-swizzled
+//                smem, keep the running max / partial sums, rescale O in TMEM
+//                only when the max grows by more than 2^8 (log2 domain), and
+//                finally normalise O and write it with the LSE.
 // S = Q K^T goes to one of two TMEM buffers (128 columns each) so that the
 // next tile's QK^T overlaps this tile's softmax; O (head_dim columns) lives
 // in TMEM for the whole key loop.
@@ -39,14 +41,17 @@ struct Geo {
   static constexpr int RB = R * 2;           // remainder row bytes (32 or 64)
   static constexpr int TILE = 128 * HD * 2;  // bytes of a 128-row tile
   static constexpr int REM_OFF = A * 16384;  // offset of the remainder region in a tile
+  static constexpr int NSTF = NST;  // K/V stages
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = TILE;        // stage s: K at KV_OFF + s*2*TILE, V after it
-  static constexpr int P_OFF = KV_OFF + NST * 2 * TILE;
+  static constexpr int P_OFF = KV_OFF + NSTF * 2 * TILE;
   static constexpr int P_BYTES = 128 * 128 * 2;
-  static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
+  static constexpr int X_OFF = P_OFF + 2 * P_BYTES;  // row-statistics exchange, 2 x 128 fp32
+  static constexpr int BAR_OFF = X_OFF + 1024;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
   static_assert(R == 0 || R == 16 || R == 32, "head_dim must be 64*A + {0,16,32}");
   static_assert(TILE % 1024 == 0, "tiles must stay 1024-byte aligned");
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
@@ -77,6 +82,28 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// AND of `v` over the `n` threads that meet at named barrier `id` (all of them
+// must call it): lets a group agree on a bail-out before a later bar.sync.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+// 2^x with the hardware approximation (one MUFU op; -inf -> 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Load one 128-row tile (rows row0.., head columns col0 .. col0+HD) into smem.
 template <int HD>
 __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m128, const CUtensorMap* mrem,
@@ -88,7 +115,7 @@ __device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m128,
 }
 
 template <int HD>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r, SwaArgs a,
@@ -118,14 +145,14 @@ __global__ void __launch_bounds__(256, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < G::NSTF; ++s) {
       ptx::mbar_init(&kv_full[s], 1);
       ptx::mbar_init(&kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
-      ptx::mbar_init(&s_empty[s], 128);
-      ptx::mbar_init(&p_full[s], 128);
+      ptx::mbar_init(&s_empty[s], 256);
+      ptx::mbar_init(&p_full[s], 256);
       ptx::mbar_init(&pv_done[s], 1);
     }
     ptx::mbar_init(o_full, 1);
@@ -147,8 +174,8 @@ __global__ void __launch_bounds__(256, 1)
       ptx::mbar_arrive_expect_tx(q_full, G::TILE);
       load_tile<HD>(sm + G::Q_OFF, &tq, &tq_r, q_full, col0, (int)(q0 - a.p0));
       for (int j = 0; j < ntiles; ++j) {
-        const int s = j % NST;
-        if (!ptx::mbar_wait(&kv_empty[s], ((j / NST) & 1) ^ 1, err)) break;
+        const int s = j % G::NSTF;
+        if (!ptx::mbar_wait(&kv_empty[s], ((j / G::NSTF) & 1) ^ 1, err)) break;
         ptx::mbar_arrive_expect_tx(&kv_full[s], 2 * G::TILE);
         const int slot = (int)((j_begin + (int64_t)j * KT) % a.ring);
         uint8_t* kd = sm + G::KV_OFF + s * 2 * G::TILE;
@@ -164,7 +191,7 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t q_addr = ptx::smem_u32(sm + G::Q_OFF);
       bool ok = ptx::mbar_wait(q_full, 0, err);
       auto issue_s = [&](int j) {
-        const int s = j % NST;
+        const int s = j % G::NSTF;
         const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE);
         const uint32_t d = t_s0 + (j & 1) * 128;
         int step = 0;
@@ -191,15 +218,15 @@ __global__ void __launch_bounds__(256, 1)
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         if (j + 1 < ntiles) {
-          const int s1 = (j + 1) % NST;
-          if (!(ok = ptx::mbar_wait(&kv_full[s1], ((j + 1) / NST) & 1, err))) break;
+          const int s1 = (j + 1) % G::NSTF;
+          if (!(ok = ptx::mbar_wait(&kv_full[s1], ((j + 1) / G::NSTF) & 1, err))) break;
           if (j + 1 >= 2 && !(ok = ptx::mbar_wait(&s_empty[(j + 1) & 1], (((j + 1) / 2) - 1) & 1, err))) break;
           ptx::tc_fence_after();
           issue_s(j + 1);
         }
         if (!(ok = ptx::mbar_wait(&p_full[j & 1], (j / 2) & 1, err))) break;
         ptx::tc_fence_after();
-        const int s = j % NST;
+        const int s = j % G::NSTF;
         const uint32_t v_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE + G::TILE);
         const uint32_t p_addr = ptx::smem_u32(sm + G::P_OFF + (j & 1) * G::P_BYTES);
 #pragma unroll
@@ -221,66 +248,75 @@ __global__ void __launch_bounds__(256, 1)
       ptx::mbar_drain(o_full, 0);  // no MMA may still write TMEM when it is released
     }
   } else if (warp >= 4) {
-    // ---- softmax: one query row per thread ----
-    const int r = (warp - 4) * 32 + lane;                  // row in the tile (== TMEM lane)
+    // ---- softmax: 8 warps; a row is shared by two threads (warpgroups g = 0, 1),
+    // each owning 64 of the tile's 128 key columns; row statistics are combined
+    // through shared memory once per tile ----
+    const int g = (warp - 4) >> 2;                          // column half
+    const int r = ((warp - 4) & 3) * 32 + lane;            // row in the tile (== TMEM lane)
     const int64_t p = q0 + r;                               // absolute query position
     const bool row_ok = p <= qlast;
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
     const float sl2 = a.scale * 1.4426950408889634f;        // scale * log2(e)
-    float m = -INFINITY, l = 0.f;
+    float* xmax = reinterpret_cast<float*>(sm + G::X_OFF);  // [2][128] partial row maxima
+    float* xsum = xmax;  // [2][128] partial row sums in the epilogue (xmax is dead after the last tile)
+    float m = -INFINITY, l = 0.f;                           // l: this thread's half of the row sum
     uint8_t* pbase = sm + G::P_OFF;
-    bool ok = true;
+    bool ok = true;  // failures inside an iteration only clear `ok`; the whole group leaves together at the
+                     // agreement at the top of the next iteration (no thread is left at a named barrier)
     for (int j = 0; j < ntiles; ++j) {
       const int64_t j0 = j_begin + (int64_t)j * KT;
-      ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
-      if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: TMEM loads follow
+      if (ok) ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
+      ok = bar_and(1, 256, ok);  // all 256 softmax threads agree before the exchanges below
+      if (!ok) break;
       ptx::tc_fence_after();
-      float s[KT];
+      float s[64];  // raw scores of columns 64g .. 64g+63; the scale is folded into the exponent
 #pragma unroll
-      for (int c = 0; c < KT; c += 32) {
+      for (int c = 0; c < 64; c += 32) {
         uint32_t rr[32];
-        ptx::tmem_ld32(t_s0 + (j & 1) * 128 + c + lane_off, rr);
+        ptx::tmem_ld32(t_s0 + (j & 1) * 128 + 64 * g + c + lane_off, rr);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(rr[i]) * sl2;
+        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(rr[i]);
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&s_empty[j & 1]);
-      // mask: key c valid iff j0 + c in [p - window + 1, p]
-      const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
-      const bool full = row_ok && lo <= 0 && hi >= KT - 1;
-      float tmax = -INFINITY;
-      if (full) {
+      // mask: key 64g + c valid iff j0 + 64g + c in [p - window + 1, p]
+      const int64_t lo = p - a.window + 1 - j0 - 64 * g, hi = p - j0 - 64 * g;
+      if (!(row_ok && lo <= 0 && hi >= 63)) {
 #pragma unroll
-        for (int c = 0; c < KT; ++c) tmax = fmaxf(tmax, s[c]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < KT; ++c) {
-          const bool v = row_ok && c >= lo && c <= hi;
-          s[c] = v ? s[c] : -INFINITY;
-          tmax = fmaxf(tmax, s[c]);
-        }
+        for (int c = 0; c < 64; ++c) s[c] = (row_ok && c >= lo && c <= hi) ? s[c] : -INFINITY;
       }
-      // running max with lazy rescaling of O (needs PV_{j-1} complete).  The
-      // TMEM load/store of O is warp-collective, so a warp rescales together
-      // when any of its rows needs it; rows that do not use corr = 1.
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
+      }
+      xmax[g * 128 + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float tmax = fmaxf(xmax[r], xmax[128 + r]) * sl2;  // whole-row tile max, log2 domain
+      asm volatile("bar.sync 1, 256;" ::: "memory");           // xmax may be rewritten next tile
+      // running max with lazy rescaling of O (needs PV_{j-1} complete).  Both
+      // threads of a row take the same decision; each rescales its own O columns
+      // (16-column groups of parity g).  TMEM access is warp-collective, so a warp
+      // rescales together when any of its rows needs it (corr = 1 otherwise).
       float mu = m, corr = 1.f;
       if (tmax > -INFINITY) {
         if (m == -INFINITY) {
           mu = tmax;
         } else if (tmax > m + RESCALE_LOG2) {
           mu = tmax;
-          corr = exp2f(m - mu);
+          corr = ex2(m - mu);
           l *= corr;
         }
       }
       m = mu;
       if (__any_sync(0xffffffffu, corr != 1.f)) {
-        ok = ptx::mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, err);
-        if (!__all_sync(0xffffffffu, ok)) break;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, err));
+        if (!ok) continue;  // skip to the agreement
         ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < HD; c += 16) {
+        for (int c = 16 * g; c < HD; c += 32) {
           uint32_t o[16];
           tmem_ld16(t_o + c + lane_off, o);
           ptx::tmem_ld_wait();
@@ -292,18 +328,19 @@ __global__ void __launch_bounds__(256, 1)
       }
       // P buffer (j & 1) is free once PV_{j-2} completed
       if (j >= 2) {
-        ok = ptx::mbar_wait(&pv_done[j & 1], ((j - 2) / 2) & 1, err);
-        if (!__all_sync(0xffffffffu, ok)) break;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[j & 1], ((j - 2) / 2) & 1, err));
+        if (!ok) continue;  // skip to the agreement
       }
-      uint8_t* prow = pbase + (j & 1) * G::P_BYTES + r * 128;
-      float lsum = 0.f;
+      uint8_t* prow = pbase + (j & 1) * G::P_BYTES + g * 16384 + r * 128;  // this half = one 64-key atom
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;  // m = -inf only while every score so far is masked
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int g = 0; g < KT / 8; ++g) {  // 16 granules of 8 keys
+      for (int gr = 0; gr < 8; ++gr) {  // 8 granules of 8 keys
         float pv[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          pv[i] = (m == -INFINITY) ? 0.f : exp2f(s[g * 8 + i] - m);
-          lsum += pv[i];
+          pv[i] = ex2(fmaf(s[gr * 8 + i], sl2, neg_m));
+          ls[i & 3] += pv[i];
         }
         uint4 w;
         __nv_bfloat162 b0 = __floats2bfloat162_rn(pv[0], pv[1]), b1 = __floats2bfloat162_rn(pv[2], pv[3]);
@@ -312,23 +349,26 @@ __global__ void __launch_bounds__(256, 1)
         w.y = *reinterpret_cast<uint32_t*>(&b1);
         w.z = *reinterpret_cast<uint32_t*>(&b2);
         w.w = *reinterpret_cast<uint32_t*>(&b3);
-        const int atom = g / 8, gr = g % 8;
-        *reinterpret_cast<uint4*>(prow + atom * 16384 + ((gr ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4*>(prow + ((gr ^ (r & 7)) << 4)) = w;
       }
-      l += lsum;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&p_full[j & 1]);
     }
-    // ---- epilogue: O / l and the natural-log LSE ----
+    // ---- epilogue: O / l (l = both halves) and the natural-log LSE ----
     if (ok) ok = ptx::mbar_wait(o_full, 0, err);
-    if (__all_sync(0xffffffffu, ok)) {
+    ok = bar_and(1, 256, ok);
+    if (ok) {
+      xsum[g * 128 + r] = l;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      const float lt = xsum[r] + xsum[128 + r];
       ptx::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
       const int64_t i = p - a.p0;
       bf16* orow = reinterpret_cast<bf16*>(a.o) + i * a.ldo + col0;
 #pragma unroll
-      for (int c = 0; c < HD; c += 16) {
+      for (int c = 16 * g; c < HD; c += 32) {
         uint32_t o[16];
         tmem_ld16(t_o + c + lane_off, o);
         ptx::tmem_ld_wait();
@@ -348,7 +388,7 @@ __global__ void __launch_bounds__(256, 1)
           *reinterpret_cast<uint4*>(orow + c + 8) = w1;
         }
       }
-      if (row_ok) a.lse[(int64_t)h * a.ld_lse + i] = (m + log2f(l)) * 0.6931471805599453f;
+      if (row_ok && g == 0) a.lse[(int64_t)h * a.ld_lse + i] = (m + log2f(lt)) * 0.6931471805599453f;
     }
   }
   ptx::tc_fence_before();
@@ -576,6 +616,10 @@ __global__ void __launch_bounds__(256, 1)
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
+      if (!(row_ok && lo <= 0 && hi >= BKT - 1)) {  // edge tile: masked scores give P = 0
+#pragma unroll
+        for (int c = 0; c < BKT; ++c) sv[c] = (row_ok && c >= lo && c <= hi) ? sv[c] : -INFINITY;
+      }
       uint8_t* drow = sm + G::DS_OFF + (j & 1) * G::DS_BYTES + r * 128;
 #pragma unroll
       for (int g = 0; g < BKT / 8; ++g) {
@@ -583,8 +627,7 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int c = g * 8 + e;
-          const bool v = row_ok && c >= lo && c <= hi;
-          const float pr = v ? exp2f(sv[c] * sl2 - lse2) : 0.f;
+          const float pr = ex2(fmaf(sv[c], sl2, -lse2));
           ds[e] = pr * (dp[c] - Di);
         }
         uint4 w;
@@ -624,6 +667,280 @@ __global__ void __launch_bounds__(256, 1)
           }
           *reinterpret_cast<uint4*>(out + c) = w0;
           *reinterpret_cast<uint4*>(out + c + 8) = w1;
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Backward, dk/dv part for the chunk's own keys (earlier keys are constants):
+//   dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i dS_ij Q_i  over queries i >= j in the chunk.
+// CTA = 128 keys x one head; query tiles of 128 from the key tile to the end of the chunk.
+//   warp 0      TMA: K, V once; Q and dO tiles (2 stages)
+//   warp 1      TMEM owner; lane 0 issues S^T = K Q^T and dP^T = V dO^T (128 + 128
+//               columns), then dV += P^T dO and dK += dS^T Q (head_dim columns each)
+//   warps 4..7  one key row per thread: P^T = exp(S^T*scale - lse_i), dS^T = P^T o
+//               (dP^T - D_i), written as K-major (query-contiguous) swizzled operands
+template <int HD>
+struct KVGeo {
+  static constexpr int A = HD / 64;
+  static constexpr int R = HD % 64;
+  static constexpr int RB = R * 2;
+  static constexpr int TILE = 128 * HD * 2;    // any 128-row tile
+  static constexpr int REM = A * 16384;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = TILE;
+  static constexpr int QDST = HD <= 96 ? 2 : 1;  // Q/dO stages (shared memory bound at head_dim 128)
+  static constexpr int QD_OFF = 2 * TILE;      // stage s: Q at QD_OFF + s*2*TILE, dO after it
+  static constexpr int PT_OFF = QD_OFF + QDST * 2 * TILE;
+  static constexpr int OP_BYTES = 128 * 128 * 2;  // P^T or dS^T tile (two 64-query atoms)
+  static constexpr int DST_OFF = PT_OFF + OP_BYTES;
+  static constexpr int LD_OFF = DST_OFF + OP_BYTES;  // lse*log2e [128] then D [128], fp32
+  static constexpr int BAR_OFF = LD_OFF + 1024;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(256, 1)
+    swa_bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
+                           const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tdo_r,
+                           const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
+                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r,
+                           SwaArgs a, int* err) {
+  using G = KVGeo<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* qd_full = bars + 1;   // [2]
+  uint64_t* qd_empty = bars + 3;  // [2]
+  uint64_t* s_full = bars + 5;
+  uint64_t* s_read = bars + 6;    // 128 arrivals: S^T/dP^T read and P^T/dS^T written
+  uint64_t* pv_done = bars + 7;   // dV/dK products of the tile done (operands free)
+  uint64_t* o_full = bars + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  float* lse_s = reinterpret_cast<float*>(sm + G::LD_OFF);
+  float* d_s = lse_s + 128;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int64_t kb0 = (int64_t)blockIdx.x * 128;                   // first key row (chunk-local)
+  const int64_t klast = imin64(kb0 + 128, a.n) - 1;
+  const int64_t qend = imin64(a.n, klast + a.window);              // queries i < qend can see some key
+  const int ntiles = (int)((qend - kb0 + 127) / 128);
+  const int col0 = h * HD;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&qd_full[s], 1);
+      ptx::mbar_init(&qd_empty[s], 1);
+    }
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(s_read, 128);
+    ptx::mbar_init(pv_done, 1);
+    ptx::mbar_init(o_full, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_dp = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 384;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(kv_full, 2 * G::TILE);
+      const int slot = (int)((a.p0 + kb0) % a.ring);
+      load_rows<HD>(sm + G::K_OFF, &tk, &tk_r, kv_full, col0, slot, 16384, G::REM);
+      load_rows<HD>(sm + G::V_OFF, &tv, &tv_r, kv_full, col0, slot, 16384, G::REM);
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % G::QDST;
+        if (!ptx::mbar_wait(&qd_empty[s], ((t / G::QDST) & 1) ^ 1, err)) break;
+        ptx::mbar_arrive_expect_tx(&qd_full[s], 2 * G::TILE);
+        const int qrow = (int)(kb0 + (int64_t)t * 128);
+        uint8_t* qd = sm + G::QD_OFF + s * 2 * G::TILE;
+        load_rows<HD>(qd, &tq, &tq_r, &qd_full[s], col0, qrow, 16384, G::REM);
+        load_rows<HD>(qd + G::TILE, &tdo, &tdo_r, &qd_full[s], col0, qrow, 16384, G::REM);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t id_o64 = ptx::idesc_bf16_f32(128, 64, false, true);
+      constexpr uint32_t id_or = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
+      constexpr uint32_t rl = rem_swizzle_layout(G::R);
+      const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF), v_addr = ptx::smem_u32(sm + G::V_OFF);
+      const uint32_t pt_addr = ptx::smem_u32(sm + G::PT_OFF), dst_addr = ptx::smem_u32(sm + G::DST_OFF);
+      bool ok = ptx::mbar_wait(kv_full, 0, err);
+      for (int t = 0; ok && t < ntiles; ++t) {
+        const int s = t % G::QDST;
+        if (!(ok = ptx::mbar_wait(&qd_full[s], (t / G::QDST) & 1, err))) break;
+        ptx::tc_fence_after();
+        const uint32_t q_addr = ptx::smem_u32(sm + G::QD_OFF + s * 2 * G::TILE), do_addr = q_addr + G::TILE;
+        // S^T = K Q^T and dP^T = V dO^T (K over head_dim)
+        int step = 0;
+#pragma unroll
+        for (int at = 0; at < G::A; ++at)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk, ++step) {
+            ptx::umma_bf16(t_s, sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2),
+                           sdesc(q_addr + at * 16384 + kk * 32, 16, 1024, 2), id_s, step > 0);
+            ptx::umma_bf16(t_dp, sdesc(v_addr + at * 16384 + kk * 32, 16, 1024, 2),
+                           sdesc(do_addr + at * 16384 + kk * 32, 16, 1024, 2), id_s, step > 0);
+          }
+        if constexpr (G::R > 0) {
+#pragma unroll
+          for (int kk = 0; kk < G::R / 16; ++kk, ++step) {
+            ptx::umma_bf16(t_s, sdesc(k_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
+                           sdesc(q_addr + G::REM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
+            ptx::umma_bf16(t_dp, sdesc(v_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
+                           sdesc(do_addr + G::REM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
+          }
+        }
+        ptx::umma_commit(s_full);
+        if (!(ok = ptx::mbar_wait(s_read, t & 1, err))) break;
+        ptx::tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q (K over the tile's 128 queries)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t pd = sdesc(pt_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, 2);
+          const uint64_t dd = sdesc(dst_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, 2);
+          const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+#pragma unroll
+          for (int at = 0; at < G::A; ++at) {
+            ptx::umma_bf16(t_dv + 64 * at, pd, sdesc(do_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
+            ptx::umma_bf16(t_dk + 64 * at, dd, sdesc(q_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
+          }
+          if constexpr (G::R > 0) {
+            ptx::umma_bf16(t_dv + 64 * G::A, pd, sdesc(do_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
+                           acc);
+            ptx::umma_bf16(t_dk + 64 * G::A, dd, sdesc(q_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
+                           acc);
+          }
+        }
+        ptx::umma_commit(&qd_empty[s]);
+        ptx::umma_commit(pv_done);
+      }
+      ptx::umma_commit(o_full);
+      ptx::mbar_drain(o_full, 0);
+    }
+  } else if (warp >= 4) {
+    const int r = (warp - 4) * 32 + lane;     // key row in the tile (== TMEM lane)
+    const int64_t jl = kb0 + r;               // chunk-local key row
+    const bool key_ok = jl < a.n;
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const float L2E = 1.4426950408889634f;
+    const float sl2 = a.scale * L2E;
+    bool ok = true;
+    for (int t = 0; t < ntiles; ++t) {
+      const int64_t qb0 = kb0 + (int64_t)t * 128;
+      ok = ptx::mbar_wait(s_full, t & 1, err);
+      if (t > 0 && ok) ok = ptx::mbar_wait(pv_done, (t - 1) & 1, err);  // P^T/dS^T buffers free
+      // all 128 key-row threads agree before the named barrier below (no one waits alone)
+      ok = bar_and(1, 128, ok);
+      if (!ok) break;
+      // per-query statistics of this tile (thread r fetches query qb0 + r)
+      {
+        const int64_t i = qb0 + r;
+        const bool q_ok = i < a.n;
+        lse_s[r] = q_ok ? a.lse[(int64_t)h * a.ld_lse + i] * L2E : INFINITY;  // +inf: P = 0
+        d_s[r] = q_ok ? a.D[(int64_t)h * a.ld_lse + i] : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      ptx::tc_fence_after();
+      uint8_t* prow = sm + G::PT_OFF + r * 128;
+      uint8_t* drow = sm + G::DST_OFF + r * 128;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        float sv[64], dp[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t rs[32], rd[32];
+          ptx::tmem_ld32(t_s + half * 64 + c + lane_off, rs);
+          ptx::tmem_ld32(t_dp + half * 64 + c + lane_off, rd);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            sv[c + e] = __uint_as_float(rs[e]);
+            dp[c + e] = __uint_as_float(rd[e]);
+          }
+        }
+        // query i = qb0 + half*64 + c sees key jl iff jl <= i < jl + window
+        const int64_t lo = jl - qb0 - half * 64, hi = jl + a.window - 1 - qb0 - half * 64;
+        if (!(key_ok && lo <= 0 && hi >= 63)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] = (key_ok && c >= lo && c <= hi) ? sv[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          float pv[8], dv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = g * 8 + e, q = half * 64 + c;
+            pv[e] = ex2(fmaf(sv[c], sl2, -lse_s[q]));
+            dv[e] = pv[e] * (dp[c] - d_s[q]);
+          }
+          uint4 w, x;
+          __nv_bfloat162 p0 = __floats2bfloat162_rn(pv[0], pv[1]), p1 = __floats2bfloat162_rn(pv[2], pv[3]);
+          __nv_bfloat162 p2 = __floats2bfloat162_rn(pv[4], pv[5]), p3 = __floats2bfloat162_rn(pv[6], pv[7]);
+          __nv_bfloat162 d0 = __floats2bfloat162_rn(dv[0], dv[1]), d1 = __floats2bfloat162_rn(dv[2], dv[3]);
+          __nv_bfloat162 d2 = __floats2bfloat162_rn(dv[4], dv[5]), d3 = __floats2bfloat162_rn(dv[6], dv[7]);
+          w.x = *reinterpret_cast<uint32_t*>(&p0);
+          w.y = *reinterpret_cast<uint32_t*>(&p1);
+          w.z = *reinterpret_cast<uint32_t*>(&p2);
+          w.w = *reinterpret_cast<uint32_t*>(&p3);
+          x.x = *reinterpret_cast<uint32_t*>(&d0);
+          x.y = *reinterpret_cast<uint32_t*>(&d1);
+          x.z = *reinterpret_cast<uint32_t*>(&d2);
+          x.w = *reinterpret_cast<uint32_t*>(&d3);
+          const int off = half * 16384 + ((g ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(prow + off) = w;
+          *reinterpret_cast<uint4*>(drow + off) = x;
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(s_read);
+    }
+    if (ok) ok = ptx::mbar_wait(o_full, 0, err);
+    if (__all_sync(0xffffffffu, ok)) {
+      ptx::tc_fence_after();
+      bf16* ov = reinterpret_cast<bf16*>(a.dv) + jl * a.lddkv + col0;
+      bf16* ok_ = reinterpret_cast<bf16*>(a.dk) + jl * a.lddkv + col0;
+#pragma unroll
+      for (int c = 0; c < HD; c += 16) {
+        uint32_t v[16], kx[16];
+        tmem_ld16(t_dv + c + lane_off, v);
+        tmem_ld16(t_dk + c + lane_off, kx);
+        ptx::tmem_ld_wait();
+        if (key_ok) {
+          uint32_t pv_[8], pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            __nv_bfloat162 tv2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            __nv_bfloat162 tk2 = __floats2bfloat162_rn(__uint_as_float(kx[2 * e]) * a.scale,
+                                                       __uint_as_float(kx[2 * e + 1]) * a.scale);
+            pv_[e] = *reinterpret_cast<uint32_t*>(&tv2);
+            pk[e] = *reinterpret_cast<uint32_t*>(&tk2);
+          }
+          *reinterpret_cast<uint4*>(ov + c) = make_uint4(pv_[0], pv_[1], pv_[2], pv_[3]);
+          *reinterpret_cast<uint4*>(ov + c + 8) = make_uint4(pv_[4], pv_[5], pv_[6], pv_[7]);
+          *reinterpret_cast<uint4*>(ok_ + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(ok_ + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
     }
@@ -690,7 +1007,7 @@ int launch(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
     }
   }
   dim3 grid(ceil_div(a.n, QT), a.heads);
-  fn<<<grid, 256, G::SMEM, s>>>(p.q128, p.qr, p.k128, p.kr, p.v128, p.vr, a, err);
+  fn<<<grid, 384, G::SMEM, s>>>(p.q128, p.qr, p.k128, p.kr, p.v128, p.vr, a, err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -717,6 +1034,27 @@ int launch_bwd_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* 
   return TTT_OK;
 }
 
+template <int HD>
+int launch_bwd_dkdv(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  using G = KVGeo<HD>;
+  auto fn = &swa_bwd_dkdv_tc_kernel<HD>;
+  {
+    static std::mutex mu;
+    static std::set<int> done;
+    int dev = 0;
+    TTT_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lock(mu);
+    if (!done.count(dev)) {
+      TTT_CUDA_TRY(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM));
+      done.insert(dev);
+    }
+  }
+  dim3 grid(ceil_div(a.n, 128), a.heads);
+  fn<<<grid, 256, G::SMEM, s>>>(p.q128, p.qr, p.do128, p.dor, p.k128, p.kr128, p.v128, p.vr128, a, err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
 }  // namespace
 
 int swa_tc_bwd_prepare(SwaTcBwdPlan* p, int heads, int head_dim, const void* q, const void* dout, int64_t rows,
@@ -731,19 +1069,39 @@ int swa_tc_bwd_prepare(SwaTcBwdPlan* p, int heads, int head_dim, const void* q, 
   if (!rc) rc = tmap(&p->do128, dout, rows, cols, ld, 64);
   if (!rc) rc = tmap(&p->k64, k, ring, cols, ldkv, 64, 64);
   if (!rc) rc = tmap(&p->v64, v, ring, cols, ldkv, 64, 64);
+  if (!rc) rc = tmap(&p->k128, k, ring, cols, ldkv, 64, 128);
+  if (!rc) rc = tmap(&p->v128, v, ring, cols, ldkv, 64, 128);
   if (rc) return rc;
   if (rem) {
     rc = tmap(&p->qr, q, rows, cols, ld, rem);
     if (!rc) rc = tmap(&p->dor, dout, rows, cols, ld, rem);
     if (!rc) rc = tmap(&p->kr, k, ring, cols, ldkv, rem, 64);
     if (!rc) rc = tmap(&p->vr, v, ring, cols, ldkv, rem, 64);
+    if (!rc) rc = tmap(&p->kr128, k, ring, cols, ldkv, rem, 128);
+    if (!rc) rc = tmap(&p->vr128, v, ring, cols, ldkv, rem, 128);
   } else {
     p->qr = p->q128;
     p->dor = p->do128;
     p->kr = p->k64;
     p->vr = p->v64;
+    p->kr128 = p->k128;
+    p->vr128 = p->v128;
   }
   return rc;
+}
+
+bool swa_tc_dkdv_supported(const SwaArgs& a) { return a.p0 % 128 == 0 && a.ring % 128 == 0; }
+
+int swa_tc_backward_dkdv(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+  if (a.ring != p.ring || a.head_dim != p.head_dim) return set_error(TTT_ERR_INVALID_ARG, "attention: plan mismatch");
+  if (!swa_tc_dkdv_supported(a)) return set_error(TTT_ERR_INVALID_ARG, "attention: dk/dv needs 128-aligned chunks");
+  switch (a.head_dim) {
+    case 64: return launch_bwd_dkdv<64>(p, a, s, err);
+    case 80: return launch_bwd_dkdv<80>(p, a, s, err);
+    case 96: return launch_bwd_dkdv<96>(p, a, s, err);
+    case 128: return launch_bwd_dkdv<128>(p, a, s, err);
+  }
+  return set_error(TTT_ERR_UNSUPPORTED, "attention (tensor cores): head_dim must be 64, 80, 96 or 128");
 }
 
 int swa_tc_backward_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {

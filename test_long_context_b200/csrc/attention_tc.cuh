@@ -27,6 +27,10 @@ struct SwaTcBwdPlan {
   alignas(64) CUtensorMap kr;
   alignas(64) CUtensorMap v64;
   alignas(64) CUtensorMap vr;
+  alignas(64) CUtensorMap k128;  // 128-row boxes of the rings (dk/dv kernel)
+  alignas(64) CUtensorMap kr128;
+  alignas(64) CUtensorMap v128;
+  alignas(64) CUtensorMap vr128;
   int head_dim = 0;
   int64_t ring = 0;
 };
@@ -37,6 +41,10 @@ int swa_tc_bwd_prepare(SwaTcBwdPlan* p, int heads, int head_dim, const void* q, 
 // Writes a.dq (bf16) from a.q, a.dout, the rings, a.lse and a.D (the row dot
 // products dO . O, computed beforehand).
 int swa_tc_backward_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err);
+// dk, dv (bf16) for the chunk's own keys; needs a.p0 % 128 == 0 (the chunk's
+// keys start a ring tile); reads a.lse and a.D.
+bool swa_tc_dkdv_supported(const SwaArgs& a);
+int swa_tc_backward_dkdv(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err);
 // q: [q_rows, heads*head_dim] (pitch ldq); k, v rings: [ring, heads*head_dim]
 // (pitch ldkv); ring must be a multiple of 128.
 int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t q_rows, int64_t ldq, const void* k,

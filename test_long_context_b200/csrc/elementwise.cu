@@ -82,12 +82,20 @@ template <typename T>
 __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n,
                                        int64_t p0, int H, int HD, float eps, double theta, T* qout, int64_t ldq,
                                        T* kring, T* vring, int64_t ldkv, int64_t R, float* rq, float* rk) {
-  const int64_t w = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  // one block per token: the position's rotation table is computed once (fp64
+  // angles) and shared by all heads; warp w handles heads w, w + 8, ...
+  __shared__ float2 cs[32 * MAXP];
+  const int64_t i = blockIdx.x;
   const int lane = threadIdx.x % 32;
-  if (w >= n * H) return;
-  const int64_t i = w / H;
-  const int h = (int)(w % H);
   const int h2 = HD / 2;
+  if (i >= n) return;
+  for (int t = threadIdx.x; t < h2; t += blockDim.x) {
+    float c, sn;
+    rope_cs(p0 + i, t, HD, theta, c, sn);
+    cs[t] = make_float2(c, sn);
+  }
+  __syncthreads();
+  for (int h = threadIdx.x / 32; h < H; h += blockDim.x / 32) {
   const int D = H * HD;
   const T* q = qkv + i * ldqkv + h * HD;
   const T* k = q + D;
@@ -120,8 +128,7 @@ __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float*
   for (int u = 0; u < MAXP; ++u) {
     const int t = lane + 32 * u;
     if (t < h2) {
-      float c, s;
-      rope_cs(pos, t, HD, theta, c, s);
+      const float c = cs[t].x, s = cs[t].y;
       const float a1 = q1[u] * rqv * gq[t], a2 = q2[u] * rqv * gq[t + h2];
       const float b1 = k1[u] * rkv * gk[t], b2 = k2[u] * rkv * gk[t + h2];
       qo[t] = from_f32<T>(a1 * c - a2 * s);
@@ -135,20 +142,28 @@ __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float*
     rq[i * H + h] = rqv;
     rk[i * H + h] = rkv;
   }
+  }
 }
 
 template <typename T>
 __global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq,
                                        const float* gk, const float* rq, const float* rk, int64_t n, int64_t p0,
                                        int H, int HD, double theta) {
-  const int64_t w = (int64_t)blockIdx.x * ROW_WARPS + threadIdx.x / 32;
+  // one block per token, rotation table shared by the 2H (q, k) heads
+  __shared__ float2 cs[32 * MAXP];
+  const int64_t i = blockIdx.x;
   const int lane = threadIdx.x % 32;
-  if (w >= n * H * 2) return;
-  const int which = (int)(w % 2);  // 0: q, 1: k
-  const int64_t ih = w / 2;
-  const int64_t i = ih / H;
-  const int h = (int)(ih % H);
   const int h2 = HD / 2;
+  if (i >= n) return;
+  for (int t = threadIdx.x; t < h2; t += blockDim.x) {
+    float c, sn;
+    rope_cs(p0 + i, t, HD, theta, c, sn);
+    cs[t] = make_float2(c, sn);
+  }
+  __syncthreads();
+  for (int w = threadIdx.x / 32; w < 2 * H; w += blockDim.x / 32) {
+  const int which = w % 2;  // 0: q, 1: k
+  const int h = w / 2;
   const int D = H * HD;
   T* dv = dqkv + i * ld + which * D + h * HD;
   const T* xv = qkv + i * ldqkv + which * D + h * HD;
@@ -162,8 +177,7 @@ __global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_
     const int t = lane + 32 * u;
     u1[u] = u2[u] = x1[u] = x2[u] = 0.f;
     if (t < h2) {
-      float c, s;
-      rope_cs(pos, t, HD, theta, c, s);
+      const float c = cs[t].x, s = cs[t].y;
       const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
       // transpose of the rotation, then the gain
       u1[u] = (d1 * c + d2 * s) * g[t];
@@ -181,6 +195,7 @@ __global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_
       dv[t] = from_f32<T>(r * (u1[u] - x1[u] * dot));
       dv[t + h2] = from_f32<T>(r * (u2[u] - x2[u] * dot));
     }
+  }
   }
 }
 
@@ -291,7 +306,7 @@ int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* g
                     int HD, float eps, double theta, T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv,
                     int64_t R, float* rq, float* rk, cudaStream_t s) {
   if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
-  qknorm_rope_fwd_kernel<T><<<row_blocks(n * H), 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, theta,
+  qknorm_rope_fwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, theta,
                                                                           qout, ldq, kring, vring, ldkv, R, rq, rk);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
@@ -302,7 +317,7 @@ int qknorm_rope_bwd(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const floa
                     const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, double theta,
                     cudaStream_t s) {
   if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
-  qknorm_rope_bwd_kernel<T><<<row_blocks(n * H * 2), 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n,
+  qknorm_rope_bwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n,
                                                                               p0, H, HD, theta);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;

@@ -87,6 +87,7 @@ struct Gemm {
   EpiArgs args;
   TcGemm tc;
   bool bf = false;
+  int64_t split = 1;  // deterministic split-K count (bf16 mode)
 };
 
 // Event-pair timing of launches, per kernel class (opt-in).
@@ -193,7 +194,7 @@ class Engine final : public ttt_ctx {
   // TTT_TRACE=1: synchronise after every launch and log it to stderr (debugging aid).
   template <typename F>
   int traced(int kc, F&& f) {
-    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other"};
+    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope"};
     if (trace_verbose_) fprintf(stderr, "[ttt trace] launching %lld %s\n", (long long)launches, names[kc]);
     cudaEvent_t a = timer_.get(), b = timer_.get();
     TTT_CUDA_TRY(cudaEventRecord(a, st_));
@@ -296,6 +297,20 @@ class Engine final : public ttt_ctx {
   std::vector<Gemm> g_top_;  // 10 per top block: qkv, o, gu, down, da, dh2, wd, wgu, do, dh
   Gemm g_head_;
   std::vector<Gemm> g_ce_dz_, g_ce_dh_;
+  // split-K workspace shared by every split GEMM (they run one after another on the stream)
+  int64_t ws_floats_ = 0;
+  float* ws_ = nullptr;
+  int finalize_splits() {
+    if (!ws_floats_) return TTT_OK;
+    TRY(arena_.alloc(&ws_, ws_floats_));
+    auto fix = [&](Gemm& g) { return g.split > 1 ? tc_gemm_set_split(&g.tc, g.split, ws_) : TTT_OK; };
+    for (auto& g : g_bot_) TRY(fix(g));
+    for (auto& g : g_top_) TRY(fix(g));
+    TRY(fix(g_head_));
+    for (auto& g : g_ce_dz_) TRY(fix(g));
+    for (auto& g : g_ce_dh_) TRY(fix(g));
+    return TTT_OK;
+  }
   // tensor-core attention plans (bf16, supported head_dim)
   bool tc_attn_ = false;
   std::vector<SwaTcPlan> att_bot_, att_top_;
@@ -317,7 +332,13 @@ int Engine<T>::prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, 
   g.bf = BF;
   if (BF) {
     g.tc.act_bf16 = 1;
-    TRY(tc_gemm_prepare(&g.tc, g.shape, epi, args));
+    int bn = 0;
+    const int64_t S = tc_split_plan(g.shape.M(), g.shape.N(), g.shape.K(), epi, &bn);
+    TRY(tc_gemm_prepare(&g.tc, g.shape, epi, args, bn));
+    if (S > 1) {
+      g.split = S;
+      ws_floats_ = std::max<int64_t>(ws_floats_, S * g.shape.M() * g.shape.N());
+    }
   }
   return TTT_OK;
 }
@@ -554,6 +575,7 @@ int Engine<T>::init() {
     TRY(prep(g_ce_dh_[c], 0, MatView{dz_, b, vn, Vc_}, 1, MatView{hv, vn, d, d}, c == 0 ? EPI_STORE_F32 : EPI_ADD_F32,
              e));
   }
+  TRY(finalize_splits());
   TTT_CUDA_TRY(cudaStreamSynchronize(st_));
   return TTT_OK;
 }
@@ -598,15 +620,15 @@ int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
   for (int64_t l = 0; l < nbot_; ++l) {
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_bot_[4 * l];
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[0], S));
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
+    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
                                  kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(s0, S),
               [&] { return attn_fwd(tc_attn_ ? &att_bot_[l] : nullptr,
                                     swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_)); }));
     TRY(run(g[1], S));
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[2], S));
     TRY(run(g[3], S));
   }
@@ -626,20 +648,20 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_top_[10 * i];
     const float* xin = i == 0 ? x0 : xin_[i];
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_); }));
     TRY(run(g[0], n));
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
+    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
                                  kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(p0, n),
               [&] { return attn_fwd(tc_attn_ ? &att_top_[i] : nullptr,
                                     swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b)); }));
     g[1].args.c2 = const_cast<float*>(xin);
     TRY(run(g[1], n));
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_); }));
     TRY(run(g[2], n));
     TRY(run(g[3], n));
   }
-  TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_fwd<T>(xf_, d, wt_.final_norm, eps, n, (int)d, hf_, d, rf_, st_); }));
+  TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xf_, d, wt_.final_norm, eps, n, (int)d, hf_, d, rf_, st_); }));
   TRY(run(g_head_, n));
   TRY(timed(TTT_KC_OTHER, 0, [&] { return ce_finalize(pmax_, psum_, b, (int)ce_tiles_, zt_, n, n_valid, n_valid ? 1.f / (float)n_valid : 0.f,
                         losses + p0, lsef_, scl_, st_); }));
@@ -650,7 +672,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     TRY(run(g_ce_dz_[c], n));
     TRY(run(g_ce_dh_[c], n));
   }
-  TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_); }));
+  TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_); }));
   for (int i = nu_ - 1; i >= 0; --i) {
     const int64_t l = nbot_ + i;
     const ttt_layer_weights& lw = wt_.layers[l];
@@ -665,7 +687,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     TRY(run(g[6], 0));  // W_down fast -= eta * dx^T a_f
     TRY(run(g[7], 0));  // W_gate/up fast -= eta * dgu_f^T h2
     if (i == 0) break;  // nothing below the lowest fast block depends on W
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_); }));
     TRY(run(g[8], n));
     SwaArgs a = swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b);
     a.dout = do_;
@@ -677,14 +699,19 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     a.lddkv = 3 * d;
     a.D = Dbuf_;
     TRY(timed(TTT_KC_ATTN_BWD, 4.0 * d * (band_pairs(p0, n) + (double)n * (double)(n + 1) / 2.0), [&] {
-      if (tc_attn_) return swa_backward_with_dq(a, true, st_, [&] { return swa_tc_backward_dq(att_bwd_[i], a, st_, err_); });
+      if (tc_attn_) {
+        std::function<int()> dkdv;
+        if (swa_tc_dkdv_supported(a)) dkdv = [&] { return swa_tc_backward_dkdv(att_bwd_[i], a, st_, err_); };
+        return swa_backward_with_dq(a, true, st_, [&] { return swa_tc_backward_dq(att_bwd_[i], a, st_, err_); },
+                                    dkdv);
+      }
       return swa_backward(a, BF, st_);
     }));
     launches += 2;  // the backward launches three kernels
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
+    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
                                  (int)HD_, theta, st_); }));
     TRY(run(g[9], n));
-    TRY(timed(TTT_KC_OTHER, 0, [&] { return rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_); }));
+    TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_); }));
   }
   return TTT_OK;
 }

@@ -42,6 +42,7 @@ struct EpiArgs {
   int64_t part_ld = 0;  // stride between N tiles in part_max/part_sum
   float alpha = 0.f;
   int64_t col_offset = 0;
+  int64_t split_stride = 0;  // split-K partials: elements between consecutive splits (EPI_STORE_F32 only)
 };
 
 // Row-major matrix view in storage order (element type given by the GEMM).
@@ -68,7 +69,17 @@ struct TcGemm {
   int64_t M = 0, N = 0, K = 0;
   EpiArgs args;
   int act_bf16 = 1;  // activation dtype of EPI_SWIGLU / EPI_CE_BWD outputs
+  // deterministic split-K (ksplit > 1): partials to ws [ksplit][M][N] fp32, then an ordered reduction
+  int ksplit = 1;
+  int64_t kps = 0;  // K per split, a multiple of 64
+  float* ws = nullptr;
 };
+
+// Split-K count for an M x N x K GEMM with this epilogue (1 = no split); sets
+// *bn_out to the tile width to use when splitting (0 = default).
+int64_t tc_split_plan(int64_t M, int64_t N, int64_t K, int epi, int* bn_out);
+// Enable split-K on a prepared GEMM: ws must hold ksplit * M * N floats.
+int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws);
 
 // Returns TTT_OK or an error code (bad shapes, tensor-map failure).
 int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args, int bn_hint = 0);

@@ -26,7 +26,8 @@ struct TcCfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int WBUF = 4 * 32 * 33 * 4;  // epilogue transpose tiles, one per epilogue warp
+  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + WBUF;
 };
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
@@ -77,7 +78,8 @@ __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
 // Epilogue of one accumulator row (thread) over the tile's BN columns.
 template <int BN, int EPI, typename TACT>
 __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool row_ok, int64_t n0, int64_t N,
-                                             const EpiArgs& ep, int tile_n) {
+                                             const EpiArgs& ep, int tile_n, int split, float* wbuf, int64_t row0,
+                                             int64_t M) {
   float v[32];
   if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll 1
@@ -135,6 +137,50 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
       ep.part_sum[(int64_t)tile_n * ep.part_ld + row] = sm;
       if (found) ep.target_logit[row] = zt;
     }
+  } else if constexpr (EPI == EPI_ADD_F32 || EPI == EPI_SGD) {
+    // Read-modify-write epilogues: transpose each 32 x 32 chunk through this
+    // warp's padded smem tile so that global accesses walk rows with lane =
+    // column (coalesced 128-byte loads/stores, 8 rows in flight).
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      ld32f(t_row + c, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) wbuf[lane * 33 + i] = v[i];
+      __syncwarp();
+      const int64_t col = n0 + c + lane;
+      const bool col_ok = col < N;
+#pragma unroll 1
+      for (int r0 = 0; r0 < 32; r0 += 8) {
+        float cur[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t rr = row0 + r0 + u;
+          cur[u] = 0.f;
+          if (col_ok && rr < M) {
+            if constexpr (EPI == EPI_ADD_F32)
+              cur[u] = ep.c2 ? reinterpret_cast<const float*>(ep.c2)[rr * ep.ldc2 + col]
+                             : reinterpret_cast<const float*>(ep.c)[rr * ep.ldc + col];
+            else
+              cur[u] = reinterpret_cast<const float*>(ep.c)[rr * ep.ldc + col];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t rr = row0 + r0 + u;
+          if (!(col_ok && rr < M)) continue;
+          const float acc = wbuf[(r0 + u) * 33 + lane];
+          if constexpr (EPI == EPI_ADD_F32) {
+            reinterpret_cast<float*>(ep.c)[rr * ep.ldc + col] = cur[u] + acc;
+          } else {
+            const float w = cur[u] - ep.alpha * acc;
+            reinterpret_cast<float*>(ep.c)[rr * ep.ldc + col] = w;
+            if (ep.c2) reinterpret_cast<bf16*>(ep.c2)[rr * ep.ldc2 + col] = __float2bfloat16_rn(w);
+          }
+        }
+      }
+      __syncwarp();
+    }
   } else {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
@@ -143,7 +189,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
       if (!row_ok || col0 >= N) continue;
       const int nval = (int)(N - col0 < 32 ? N - col0 : 32);
       if constexpr (EPI == EPI_STORE_F32) {
-        store32<float>(reinterpret_cast<float*>(ep.c) + row * ep.ldc + col0, v, nval);
+        store32<float>(reinterpret_cast<float*>(ep.c) + (int64_t)split * ep.split_stride + row * ep.ldc + col0, v,
+                       nval);
       } else if constexpr (EPI == EPI_STORE_BF16) {
         store32<bf16>(reinterpret_cast<bf16*>(ep.c) + row * ep.ldc + col0, v, nval);
       } else if constexpr (EPI == EPI_ADD_F32) {
@@ -171,10 +218,16 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
   }
 }
 
+// Persistent kernel: one CTA per SM walks the work units u = blockIdx.x,
+// blockIdx.x + gridDim.x, ...  A unit is (m-tile, n-tile, k-split) with the
+// m-tile fastest, so CTAs running at the same time share weight (B) tiles in
+// L2.  The accumulator is double-buffered in TMEM (2 x BN columns): the
+// epilogue warps drain unit i while the MMA thread already accumulates unit
+// i+1.  The smem ring's stage/phase counters run on across units.
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, int64_t M,
-                   int64_t N, int64_t K, EpiArgs ep, int* err) {
+                   int64_t N, int64_t K, int64_t kps, int n_mt, int n_nt, int n_split, EpiArgs ep, int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,26 +235,40 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sB = smem + C::STAGES * C::A_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* accf = empty + C::STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* acc_full = empty + C::STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  float* wbufs = reinterpret_cast<float*>(sB + C::STAGES * C::B_BYTES + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t n0 = (int64_t)blockIdx.x * BN, m0 = (int64_t)blockIdx.y * BM;
-  const int nkb = (int)((K + BK - 1) / BK);
+  const int64_t units = (int64_t)n_mt * n_nt * n_split;
+  auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int64_t& k_begin) {
+    m0 = (u % n_mt) * BM;
+    const int64_t nt = (u / n_mt) % n_nt;
+    n0 = nt * BN;
+    split = (int)(u / ((int64_t)n_mt * n_nt));
+    k_begin = (int64_t)split * kps;
+    nkb = (int)((imin64(kps, K - k_begin) + BK - 1) / BK);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
-    ptx::mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 128);
+    }
+    ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tma);
     ptx::prefetch_tmap(&tmb);
   }
   if (warp == 1) {
     __syncwarp();
-    ptx::tmem_alloc(tmem_slot, BN);
+    ptx::tmem_alloc(tmem_slot, 2 * BN);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -211,60 +278,90 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t ph = (uint32_t)(kb / C::STAGES) & 1u;
-        if (!ptx::mbar_wait(&empty[s], ph ^ 1u, err)) break;
-        ptx::mbar_arrive_expect_tx(&full[s], C::STAGE);
-        uint8_t* a = sA + s * C::A_BYTES;
-        uint8_t* b = sB + s * C::B_BYTES;
-        const int k0 = kb * BK;
-        if constexpr (!A_MN) {
-          ptx::tma_load_2d(a, &tma, &full[s], k0, (int)m0);
-        } else {
-          ptx::tma_load_2d(a, &tma, &full[s], (int)m0, k0);
-          ptx::tma_load_2d(a + 8192, &tma, &full[s], (int)m0 + 64, k0);
-        }
-        if constexpr (!B_MN) {
-          ptx::tma_load_2d(b, &tmb, &full[s], k0, (int)n0);
-        } else {
+      uint32_t kbg = 0;  // k-blocks issued by this CTA so far (ring position)
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        int64_t m0, n0, k_begin;
+        int split, nkb;
+        decode(u, m0, n0, split, nkb, k_begin);
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = (int)(kbg % C::STAGES);
+          const uint32_t ph = (kbg / C::STAGES) & 1u;
+          if (!(ok = ptx::mbar_wait(&empty[s], ph ^ 1u, err))) break;
+          ptx::mbar_arrive_expect_tx(&full[s], C::STAGE);
+          uint8_t* a = sA + s * C::A_BYTES;
+          uint8_t* b = sB + s * C::B_BYTES;
+          const int k0 = (int)(k_begin + (int64_t)kb * BK);
+          if constexpr (!A_MN) {
+            ptx::tma_load_2d(a, &tma, &full[s], k0, (int)m0);
+          } else {
+            ptx::tma_load_2d(a, &tma, &full[s], (int)m0, k0);
+            ptx::tma_load_2d(a + 8192, &tma, &full[s], (int)m0 + 64, k0);
+          }
+          if constexpr (!B_MN) {
+            ptx::tma_load_2d(b, &tmb, &full[s], k0, (int)n0);
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j) ptx::tma_load_2d(b + j * 8192, &tmb, &full[s], (int)n0 + 64 * j, k0);
+            for (int j = 0; j < BN / 64; ++j) ptx::tma_load_2d(b + j * 8192, &tmb, &full[s], (int)n0 + 64 * j, k0);
+          }
         }
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN, A_MN, B_MN);
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % C::STAGES;
-        const uint32_t ph = (uint32_t)(kb / C::STAGES) & 1u;
-        if (!ptx::mbar_wait(&full[s], ph, err)) break;
+      uint32_t kbg = 0, it = 0;
+      bool ok = true;
+      for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++it) {
+        int64_t m0, n0, k_begin;
+        int split, nkb;
+        decode(u, m0, n0, split, nkb, k_begin);
+        const uint32_t b = it & 1u, use = it >> 1;
+        // the epilogue must have drained this accumulator buffer's previous unit
+        if (!(ok = ptx::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
         ptx::tc_fence_after();
-        const uint32_t a_addr = ptx::smem_u32(sA + s * C::A_BYTES);
-        const uint32_t b_addr = ptx::smem_u32(sB + s * C::B_BYTES);
+        const uint32_t d_tmem = tmem + b * BN;
+        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+          const int s = (int)(kbg % C::STAGES);
+          const uint32_t ph = (kbg / C::STAGES) & 1u;
+          if (!(ok = ptx::mbar_wait(&full[s], ph, err))) break;
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(sA + s * C::A_BYTES);
+          const uint32_t b_addr = ptx::smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = A_MN ? ptx::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
-                                   : ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
-                                   : ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-          ptx::umma_bf16(tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? ptx::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                     : ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                     : ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            ptx::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          ptx::umma_commit(&empty[s]);
         }
-        ptx::umma_commit(&empty[s]);
+        if (!ok) break;
+        ptx::umma_commit(&acc_full[b]);
       }
       // Arrives once every MMA issued above has completed (also on a bail-out).
-      ptx::umma_commit(accf);
-      ptx::mbar_drain(accf, 0);  // no MMA may still write TMEM when it is released
+      ptx::umma_commit(drain);
+      ptx::mbar_drain(drain, 0);  // no MMA may still write TMEM when it is released
     }
   } else {
-    const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(accf, 0, err));  // warp-uniform before tcgen05.ld
-    ptx::tc_fence_after();
-    if (ok) {
-      const int q = warp & 3;
+    const int q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    uint32_t it = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      int64_t m0, n0, k_begin;
+      int split, nkb;
+      decode(u, m0, n0, split, nkb, k_begin);
+      const uint32_t b = it & 1u, use = it >> 1;
+      const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));  // warp-uniform
+      if (!ok) break;
+      ptx::tc_fence_after();
       const int64_t row = m0 + q * 32 + lane;
-      const uint32_t t_row = tmem + ((uint32_t)(q * 32) << 16);
-      epilogue_row<BN, EPI, TACT>(t_row, row, row < M, n0, N, ep, (int)blockIdx.x);
+      epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split,
+                                  wbufs + q * 32 * 33, m0 + q * 32, M);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&acc_empty[b]);
     }
   }
   ptx::tc_fence_before();
@@ -272,7 +369,7 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     __syncwarp();  // tcgen05.dealloc is warp-collective: reconverge lane 0 with the others
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, BN);
+    ptx::tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -312,7 +409,33 @@ int make_tmap(CUtensorMap* tm, const MatView& v, int box_rows) {
   return TTT_OK;
 }
 
-using KernelFn = void (*)(CUtensorMap, CUtensorMap, int64_t, int64_t, int64_t, EpiArgs, int*);
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, int64_t, int64_t, int64_t, int64_t, int, int, int, EpiArgs, int*);
+
+// Sum of split-K partials in a fixed order (deterministic), then the epilogue.
+template <int EPI>
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int S, int64_t M, int64_t N, int64_t stride,
+                                     EpiArgs ep) {
+  const int64_t idx4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  if (idx4 >= M * N) return;
+  const int64_t row = idx4 / N, col = idx4 % N;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  const int cnt = (int)imin64(4, N - col);
+  for (int s = 0; s < S; ++s) {
+    const float* p = ws + s * stride + row * N + col;
+    for (int e = 0; e < cnt; ++e) v[e] += p[e];
+  }
+  for (int e = 0; e < cnt; ++e) {
+    if constexpr (EPI == EPI_STORE_F32) {
+      reinterpret_cast<float*>(ep.c)[row * ep.ldc + col + e] = v[e];
+    } else if constexpr (EPI == EPI_STORE_BF16) {
+      reinterpret_cast<bf16*>(ep.c)[row * ep.ldc + col + e] = __float2bfloat16_rn(v[e]);
+    } else {  // EPI_ADD_F32
+      const float r = ep.c2 ? reinterpret_cast<const float*>(ep.c2)[row * ep.ldc2 + col + e]
+                            : reinterpret_cast<const float*>(ep.c)[row * ep.ldc + col + e];
+      reinterpret_cast<float*>(ep.c)[row * ep.ldc + col + e] = r + v[e];
+    }
+  }
+}
 
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 KernelFn kernel_ptr() {
@@ -354,6 +477,30 @@ int tc_pick_bn(int64_t M, int64_t N, int hint) {
   return (tiles256 >= 148 || N > 4096) ? 256 : 128;
 }
 
+int64_t tc_split_plan(int64_t M, int64_t N, int64_t K, int epi, int* bn_out) {
+  // Split K when the output alone gives fewer than two waves of 256-wide tiles
+  // and the reduction is long: pick the split count (2..8, >= 1024 of K each)
+  // whose work units fill the 148 SMs best.
+  *bn_out = 0;
+  if (epi != EPI_STORE_F32 && epi != EPI_STORE_BF16 && epi != EPI_ADD_F32) return 1;
+  const int64_t tiles = ((N + 255) / 256) * ((M + BM - 1) / BM);
+  if (tiles >= 2 * 148 || K < 2048) return 1;
+  auto fill = [](int64_t units) { return (double)units / (double)(((units + 147) / 148) * 148); };
+  const int bn0 = tc_pick_bn(M, N, 0);
+  const double eff0 = fill(((N + bn0 - 1) / bn0) * ((M + BM - 1) / BM));
+  double best_eff = eff0 + 0.1;  // the extra workspace pass must buy a clear gain
+  int64_t best = 1;
+  for (int64_t S = 2; S <= 8 && K / S >= 1024; ++S) {
+    const double eff = fill(tiles * S);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = S;
+    }
+  }
+  if (best > 1) *bn_out = 256;
+  return best;
+}
+
 int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args, int bn_hint) {
   const int64_t M = s.M(), N = s.N(), K = s.K();
   if (M < 1 || N < 1 || K < 1 || s.KB() != K) return set_error(TTT_ERR_INVALID_ARG, "gemm: inconsistent shapes");
@@ -369,14 +516,34 @@ int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args,
   g->N = N;
   g->K = K;
   g->args = args;
+  g->ksplit = 1;
+  g->kps = K;
+  g->ws = nullptr;
   int rc = make_tmap(&g->ta, s.a, s.a_mn ? 64 : BM);
   if (rc) return rc;
   rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : bn);
   return rc;
 }
 
+int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws) {
+  if (ksplit <= 1) {
+    g->ksplit = 1;
+    g->kps = g->K;
+    return TTT_OK;
+  }
+  if (!ws) return set_error(TTT_ERR_INVALID_ARG, "gemm: split-K needs a workspace");
+  if (g->epi != EPI_STORE_F32 && g->epi != EPI_STORE_BF16 && g->epi != EPI_ADD_F32)
+    return set_error(TTT_ERR_INVALID_ARG, "gemm: split-K only for store/add epilogues");
+  const int64_t kps = ((g->K + ksplit - 1) / ksplit + BK - 1) / BK * BK;
+  g->ksplit = (int)((g->K + kps - 1) / kps);
+  g->kps = kps;
+  g->ws = ws;
+  return TTT_OK;
+}
+
 int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
-  KernelFn fn = g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, g.epi, g.act_bf16) : pick<128>(g.a_mn, g.b_mn, g.epi, g.act_bf16);
+  const int kepi = g.ksplit > 1 ? EPI_STORE_F32 : g.epi;
+  KernelFn fn = g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, kepi, g.act_bf16) : pick<128>(g.a_mn, g.b_mn, kepi, g.act_bf16);
   if (!fn) return set_error(TTT_ERR_INVALID_ARG, "gemm: no kernel for this combination");
   const int smem = g.bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM;
   {
@@ -391,8 +558,38 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
       configured.insert({dev, fn});
     }
   }
-  dim3 grid((unsigned)((g.N + g.bn - 1) / g.bn), (unsigned)((g.M + BM - 1) / BM));
-  fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.M, g.N, g.K, g.args, dev_err);
+  const int n_mt = (int)((g.M + BM - 1) / BM), n_nt = (int)((g.N + g.bn - 1) / g.bn);
+  const int64_t units = (int64_t)n_mt * n_nt * g.ksplit;
+  static int n_sm = 0;
+  if (!n_sm) {
+    int dev = 0;
+    TTT_CUDA_TRY(cudaGetDevice(&dev));
+    TTT_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
+  }
+  const dim3 grid((unsigned)std::min<int64_t>(units, n_sm));
+  if (g.ksplit <= 1) {
+    fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.M, g.N, g.K, g.K, n_mt, n_nt, 1, g.args, dev_err);
+    TTT_CUDA_TRY(cudaGetLastError());
+    return TTT_OK;
+  }
+  // split-K: partial accumulators to the workspace, then the ordered sum + epilogue
+  EpiArgs part;
+  part.c = g.ws;
+  part.ldc = g.N;
+  part.split_stride = g.M * g.N;
+  fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.M, g.N, g.K, g.kps, n_mt, n_nt, g.ksplit, part, dev_err);
+  TTT_CUDA_TRY(cudaGetLastError());
+  const unsigned blocks = ceil_div((g.M * g.N + 3) / 4, 256);
+  switch (g.epi) {
+    case EPI_STORE_F32:
+      splitk_reduce_kernel<EPI_STORE_F32><<<blocks, 256, 0, stream>>>(g.ws, g.ksplit, g.M, g.N, g.M * g.N, g.args);
+      break;
+    case EPI_STORE_BF16:
+      splitk_reduce_kernel<EPI_STORE_BF16><<<blocks, 256, 0, stream>>>(g.ws, g.ksplit, g.M, g.N, g.M * g.N, g.args);
+      break;
+    default:
+      splitk_reduce_kernel<EPI_ADD_F32><<<blocks, 256, 0, stream>>>(g.ws, g.ksplit, g.M, g.N, g.M * g.N, g.args);
+  }
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }

@@ -62,6 +62,27 @@ extern "C" int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M,
   return tc_gemm_launch(g, st, err);
 }
 
+extern "C" int ttt_op_gemm_split(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A,
+                                 int64_t lda, const void* B, int64_t ldb, int32_t epilogue,
+                                 const ttt_epilogue_args* args, int32_t bn_hint, int32_t ksplit, float* workspace,
+                                 void* stream) {
+  if (!A || !B || !args || M < 1 || N < 1 || K < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_op_gemm_split: bad argument");
+  if (a_mn && !b_mn) return set_error(TTT_ERR_UNSUPPORTED, "ttt_op_gemm_split: (a_mn, b_mn) = (1, 0) not built");
+  GemmShape s;
+  s.a_mn = a_mn ? 1 : 0;
+  s.b_mn = b_mn ? 1 : 0;
+  s.a = a_mn ? MatView{A, K, M, lda} : MatView{A, M, K, lda};
+  s.b = b_mn ? MatView{B, K, N, ldb} : MatView{B, N, K, ldb};
+  TcGemm g;
+  int rc = tc_gemm_prepare(&g, s, epilogue, to_epi(args), bn_hint);
+  if (rc) return rc;
+  rc = tc_gemm_set_split(&g, ksplit, workspace);
+  if (rc) return rc;
+  int* err = op_err_word();
+  if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_gemm_split: no device error word");
+  return tc_gemm_launch(g, reinterpret_cast<cudaStream_t>(stream), err);
+}
+
 extern "C" int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint) {
   if (dtype == TTT_F32) return (N + 127) / 128;
   return tc_ce_tiles(N, tc_pick_bn(M, N, bn_hint));
@@ -151,7 +172,9 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
     if (rc) return rc;
     int* err = op_err_word();
     if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_swa_backward: no device error word");
-    return swa_backward_with_dq(a, true, st, [&] { return swa_tc_backward_dq(plan, a, st, err); });
+    std::function<int()> dkdv;
+    if (swa_tc_dkdv_supported(a) && lddkv == ldq) dkdv = [&] { return swa_tc_backward_dkdv(plan, a, st, err); };
+    return swa_backward_with_dq(a, true, st, [&] { return swa_tc_backward_dq(plan, a, st, err); }, dkdv);
   }
   return swa_backward(a, dtype == TTT_BF16, st);
 }

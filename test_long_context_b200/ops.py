@@ -42,6 +42,18 @@ def gemm(A, B, a_mn, b_mn, epi, c=None, c2=None, row_f=None, row_g=None, row_i=N
     L.check(rc)
 
 
+def gemm_split(A, B, a_mn, b_mn, epi, ksplit, workspace, c=None, c2=None, bn=0, stream=None):
+    """ttt_op_gemm_split: bf16 GEMM with a deterministic split-K reduction."""
+    M = A.shape[1] if a_mn else A.shape[0]
+    K = A.shape[0] if a_mn else A.shape[1]
+    N = B.shape[1] if b_mn else B.shape[0]
+    args = L.ttt_epilogue_args(_p(c), c.stride(0) if c is not None else 0, _p(c2), c2.stride(0) if c2 is not None else 0,
+                               None, None, None, None, None, None, 0, 0.0, 0)
+    rc = L.lib().ttt_op_gemm_split(int(a_mn), int(b_mn), M, N, K, _p(A), A.stride(0), _p(B), B.stride(0), epi,
+                                   ctypes.byref(args), bn, ksplit, _p(workspace), _stream(stream))
+    L.check(rc)
+
+
 def gemm_ce_tiles(dtype_is_bf16, M, N, bn=0):
     return int(L.lib().ttt_op_gemm_ce_tiles(L.TTT_BF16 if dtype_is_bf16 else L.TTT_F32, M, N, bn))
 

@@ -30,7 +30,8 @@ def _case(H, hd, n, p0, window, ring, dtype, seed):
 
 
 CASES = [(100, 350, 120, 256), (64, 0, 1000, 64), (37, 5, 1, 64), (130, 900, 64, 200), (300, 1000, 700, 1152),
-         (129, 0, 5000, 256), (200, 4000, 4096, 4352), (1, 77, 3, 128), (256, 2048, 128, 384)]
+         (129, 0, 5000, 256), (200, 4000, 4096, 4352), (1, 77, 3, 128), (256, 2048, 128, 384),
+         (384, 1024, 300, 1792), (200, 512, 64, 896)]
 
 
 @pytest.mark.parametrize("impl", ["f32", "bf16-simt", "bf16"])

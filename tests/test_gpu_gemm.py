@@ -110,3 +110,29 @@ def test_gemm_cross_entropy_epilogues(dtype):
     oh = torch.nn.functional.one_hot(tgt.long(), V).double()
     want = ((p - oh) * scale.double()[:, None])[:, off:]
     assert (dz.double() - want).abs().max().item() <= (1e-2 if bf else 2e-5) * want.abs().max().item()
+
+
+@pytest.mark.parametrize("combo", [(0, 0), (0, 1)])
+@pytest.mark.parametrize("ksplit", [2, 3, 7])
+def test_split_k_matches_and_is_deterministic(combo, ksplit):
+    """Split-K partials summed in a fixed order: equal to the product within
+    fp32 accumulation error, with every epilogue, and bit-identical on rerun."""
+    from test_long_context_b200 import ops
+    M, N, K = 300, 640, 4160   # ragged rows; K not a multiple of the split
+    A, B, ref = _operands(M, N, K, *combo, torch.bfloat16, seed=9)
+    ws = torch.empty(ksplit * M * N, device="cuda")
+    c = torch.empty(M, N, device="cuda")
+    ops.gemm_split(A, B, *combo, ops.L.EPI_STORE_F32, ksplit, ws, c=c)
+    c_again = torch.empty_like(c)
+    ops.gemm_split(A, B, *combo, ops.L.EPI_STORE_F32, ksplit, ws, c=c_again)
+    x0 = torch.randn(M, N, device="cuda")
+    x = torch.empty_like(x0)
+    ops.gemm_split(A, B, *combo, ops.L.EPI_ADD_F32, ksplit, ws, c=x, c2=x0)
+    cb = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    ops.gemm_split(A, B, *combo, ops.L.EPI_STORE_BF16, ksplit, ws, c=cb)
+    ops.sync()
+    scale = ref.abs().max().item()
+    assert (c.double() - ref).abs().max().item() <= 1e-4 * scale + 1e-4
+    assert torch.equal(c, c_again)
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * scale + 1e-4
+    assert (cb.double() - ref).abs().max().item() <= 1e-2 * scale
