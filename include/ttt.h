@@ -151,7 +151,7 @@ int ttt_prefill(ttt_ctx* ctx, const int32_t* tokens_dev, int64_t T, float* losse
  */
 int ttt_decode_step(ttt_ctx* ctx, int32_t* next_token_dev);
 
-/* Restore W_init (a fresh copy for a new document, 算法 2 step 1), empty the
+/* Restore W_init (a fresh copy for a new document, as 算法 2 starts each document), empty the
  * attention state and set the position to 0.  Asynchronous on the stream. */
 int ttt_reset(ttt_ctx* ctx);
 

@@ -26,7 +26,8 @@ extern "C" {
                                 c2 (optional) = raw acc.  Output dtype = the GEMM's dtype. */
 #define TTT_EPI_CE_FWD 4     /* softmax-CE partials per row and N tile (see below) */
 #define TTT_EPI_CE_BWD 5     /* c = (exp(acc - row_f[m]) - [n + col_offset == row_i[m]]) * row_g[m] */
-#define TTT_EPI_SGD 6        /* c (fp32) -= alpha * acc;  c2 (optional, bf16) = new c */
+#define TTT_EPI_SGD 6        /* c (fp32) -= alpha * acc;  c2 (optional, bf16) = hi = bf16(new c);
+                                c3 (optional, with c2) = lo = bf16(new c - hi) */
 
 typedef struct ttt_epilogue_args {
   void* c;
@@ -42,6 +43,8 @@ typedef struct ttt_epilogue_args {
   int64_t part_ld;
   float alpha;             /* SGD: learning rate */
   int64_t col_offset;      /* global column index of output column 0 (vocab chunks) */
+  void* c3;                /* SGD: low bf16 half of the new master (NULL: none) */
+  int64_t ldc3;
 } ttt_epilogue_args;
 
 /*
@@ -67,6 +70,22 @@ int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N,
  * TTT_EPI_STORE_F32, TTT_EPI_STORE_BF16, TTT_EPI_ADD_F32.  ksplit <= 1 is the
  * plain GEMM.  Useful when the output alone has too few tiles to fill the GPU.
  */
+/*
+ * Two products into one accumulator (TTT_BF16 only):
+ *   acc[m][n] = sum_k A(m,k) B(n,k)  +  [n >= n_ext] sum_k' A2(m,k') B2(n - n_ext, k')
+ * then the epilogue.  A2 / B2 take the orientation of A / B (a_mn, b_mn) and
+ * have K2 columns of reduction; B2 covers the N - n_ext outputs from n_ext
+ * on, and n_ext must be a multiple of the tile width (bn_hint; 128 always
+ * works).  ksplit > 1 (workspace as in ttt_op_gemm_split) needs n_ext = 0.
+ * The prefill uses it for the fast MLP: a fast weight is kept as a bf16 pair
+ * hi + lo of its fp32 master, and h (W_hi + W_lo)^T is h W_hi^T + h W_lo^T.
+ * Not an operation of the method itself: a precision device of this library.
+ */
+int ttt_op_gemm_dual(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+                     const void* B, int64_t ldb, int64_t K2, const void* A2, int64_t lda2, const void* B2,
+                     int64_t ldb2, int64_t n_ext, int32_t epilogue, const ttt_epilogue_args* args, int32_t bn_hint,
+                     int32_t ksplit, float* workspace, void* stream);
+
 int ttt_op_gemm_split(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
                       const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args, int32_t bn_hint,
                       int32_t ksplit, float* workspace, void* stream);

@@ -13,11 +13,11 @@ reading notes by Zhongzhu Zhou, "算法 1：因果预填充与内层适应" and 
   2. for each chunk of b tokens, in order:
        forward every position with the current W (the Transformer with
        sliding-window attention, eq. (1)); record the next-token loss of
-       every position *before* any update (section 7, step 3.3);
+       every position *before* any update (reading notes §7, 算法 1);
        A_c = mean loss over the chunk's targets, eq. (9);
        G = dA_c/dW by an explicit, hand-derived backward;
        W <- W - eta * G (plain SGD, eq. (9));
-       keep the keys/values the window still needs (step 3.6);
+       keep the keys/values the window still needs (算法 1);
   3. return the per-token losses and the adapted W.
 
 Only the MLPs of the last n_u blocks carry fast weights ("只更新最后四分之一
@@ -31,7 +31,7 @@ Readings where the pages are silent (each one also listed in the design doc):
   * keys of earlier chunks are the values cached when those positions were
     processed; they are constants of the current chunk's gradient;
   * a trailing partial chunk is scored but does not update W (its update
-    would wait for more tokens, as in generation, 算法 3 step 2);
+    would wait for more tokens, as in generation, 算法 3);
   * RMSNorm y = x / sqrt(mean(x^2) + eps) * g, eps = 1e-5; QK-norm is a
     per-head RMSNorm over head_dim applied before RoPE; RoPE pairs element i
     with i + hd/2 at absolute position p, theta = 10000; attention scale is
@@ -194,7 +194,7 @@ class Model:
 
 
 def init_fast(model):
-    """W <- W_init (step 1): float64 copies of every fast tensor."""
+    """W <- W_init (start of 算法 1): float64 copies of every fast tensor."""
     return {l: {"w_gate": np.array(model.w[f"fast.{l}.w_gate"], dtype=F),
                 "w_up": np.array(model.w[f"fast.{l}.w_up"], dtype=F),
                 "w_down": np.array(model.w[f"fast.{l}.w_down"], dtype=F)} for l in model.top}
@@ -347,7 +347,7 @@ def prefill(model, toks, eta=None, b=None, k=None, keep_grads=False, count_pairs
         if nt > 0:
             tgt[:nt] = toks[p0 + 1:p0 + 1 + nt]
         loss, fwd = forward_chunk(model, W, state, toks[p0:p0 + n], p0, tgt, count_pairs=count_pairs)
-        losses[p0:p0 + n] = loss          # recorded before the update (step 3.3)
+        losses[p0:p0 + n] = loss          # recorded before the update
         n_c = int((tgt >= 0).sum())
         means.append(float(np.nanmean(loss)) if n_c else float("nan"))
         if n == b and n_c > 0 and W:

@@ -49,7 +49,7 @@ class ttt_weights(ctypes.Structure):
 class ttt_epilogue_args(ctypes.Structure):
     _fields_ = [("c", c_vp), ("ldc", c_i64), ("c2", c_vp), ("ldc2", c_i64), ("row_f", c_vp), ("row_g", c_vp),
                 ("row_i", c_vp), ("part_max", c_vp), ("part_sum", c_vp), ("target_logit", c_vp),
-                ("part_ld", c_i64), ("alpha", c_f32), ("col_offset", c_i64)]
+                ("part_ld", c_i64), ("alpha", c_f32), ("col_offset", c_i64), ("c3", c_vp), ("ldc3", c_i64)]
 
 
 _lib = None
@@ -78,6 +78,9 @@ def lib():
             "ttt_op_gemm": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
                                     ctypes.POINTER(ttt_epilogue_args), c_i32, c_vp]),
             "ttt_op_gemm_ce_tiles": (c_i64, [c_i32, c_i64, c_i64, c_i32]),
+            "ttt_op_gemm_dual": (c_i32, [c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i64, c_vp,
+                                         c_i64, c_vp, c_i64, c_i64, c_i32, ctypes.POINTER(ttt_epilogue_args), c_i32,
+                                         c_i32, c_vp, c_vp]),
             "ttt_op_gemm_split": (c_i32, [c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
                                           ctypes.POINTER(ttt_epilogue_args), c_i32, c_i32, c_vp, c_vp]),
             "ttt_op_sync": (c_i32, [c_vp]),
@@ -118,7 +121,7 @@ def exported_symbols():
     L = lib()
     names = []
     for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
-              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
+              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_dual", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
               "ttt_op_swa_backward", "ttt_op_watchdog_selftest",
               "ttt_op_swa_backward_noalloc"):
         if hasattr(L, n):

@@ -4,12 +4,12 @@
 // CTA = one tile of 128 queries x one head; 12 warps:
 //   warp 0       TMA producer: Q once, then K/V tiles of 128 keys (2 stages)
 //   warp 1       TMEM owner; lane 0 issues every tcgen05.mma
-//   warps 4..11  softmax: a query row (= TMEM lane) is shared by two threads,
-//                one per warpgroup, each owning 64 key columns; they combine
-//                row maxima through smem, write P (bf16) to 128B-swizzled
-//                smem, keep the running max / partial sums, rescale O in TMEM
-//                only when the max grows by more than 2^8 (log2 domain), and
-//                finally normalise O and write it with the LSE.
+//   warps 4..11  softmax: two independent warpgroups; warpgroup g owns key
+//                columns 64g..64g+63 of each tile and runs its own online
+//                softmax into its own TMEM accumulator O_g (thread = query
+//                row = TMEM lane), writes P (bf16) to 128B-swizzled smem and
+//                rescales O_g only when its max grows by more than 2^8 (log2
+//                domain); the epilogue combines O_0 and O_1 and writes O, LSE.
 // S = Q K^T goes to one of two TMEM buffers (128 columns each) so that the
 // next tile's QK^T overlaps this tile's softmax; O (head_dim columns) lives
 // in TMEM for the whole key loop.
@@ -41,13 +41,18 @@ struct Geo {
   static constexpr int RB = R * 2;           // remainder row bytes (32 or 64)
   static constexpr int TILE = 128 * HD * 2;  // bytes of a 128-row tile
   static constexpr int REM_OFF = A * 16384;  // offset of the remainder region in a tile
-  static constexpr int NSTF = NST;  // K/V stages
+  // V tiles are whole 128B-swizzled atoms (the last one partly past the head),
+  // so that one MMA of N = HD covers a P V step
+  static constexpr int VA = (HD + 63) / 64;
+  static constexpr int VTILE = VA * 16384;
+  static constexpr int NK = HD <= 64 ? 4 : (HD <= 96 ? 3 : 2);  // K ring stages (released after S)
+  static constexpr int NV = HD <= 64 ? 3 : 2;                    // V ring stages (released after P V)
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = TILE;        // stage s: K at KV_OFF + s*2*TILE, V after it
-  static constexpr int P_OFF = KV_OFF + NSTF * 2 * TILE;
+  static constexpr int K_OFF = TILE;
+  static constexpr int V_OFF = K_OFF + NK * TILE;
+  static constexpr int P_OFF = V_OFF + NV * VTILE;
   static constexpr int P_BYTES = 128 * 128 * 2;
-  static constexpr int X_OFF = P_OFF + 2 * P_BYTES;  // row-statistics exchange, 2 x 128 fp32
-  static constexpr int BAR_OFF = X_OFF + 1024;
+  static constexpr int BAR_OFF = P_OFF + 2 * P_BYTES;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
   static_assert(R == 0 || R == 16 || R == 32, "head_dim must be 64*A + {0,16,32}");
   static_assert(TILE % 1024 == 0, "tiles must stay 1024-byte aligned");
@@ -118,21 +123,22 @@ template <int HD>
 __global__ void __launch_bounds__(384, 1)
     swa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
                       const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
-                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r, SwaArgs a,
-                      int* err) {
+                      const __grid_constant__ CUtensorMap tv, SwaArgs a, int* err) {
   using G = Geo<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;    // [NST]
-  uint64_t* kv_empty = bars + 3;   // [NST]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_empty = bars + 7;    // [2]
-  uint64_t* p_full = bars + 9;     // [2]
-  uint64_t* pv_done = bars + 11;   // [2]
-  uint64_t* o_full = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* k_full = bars + 1;              // [NK]
+  uint64_t* k_empty = k_full + G::NK;       // [NK]
+  uint64_t* v_full = k_empty + G::NK;       // [NV]
+  uint64_t* v_empty = v_full + G::NV;       // [NV]
+  uint64_t* s_full = v_empty + G::NV;       // [2]
+  uint64_t* s_empty = s_full + 2;           // [2]
+  uint64_t* p_full = s_empty + 2;           // [2]
+  uint64_t* pv_done = p_full + 2;           // [2]
+  uint64_t* o_full = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -145,9 +151,13 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 1);
-    for (int s = 0; s < G::NSTF; ++s) {
-      ptx::mbar_init(&kv_full[s], 1);
-      ptx::mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < G::NK; ++s) {
+      ptx::mbar_init(&k_full[s], 1);
+      ptx::mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < G::NV; ++s) {
+      ptx::mbar_init(&v_full[s], 1);
+      ptx::mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
@@ -167,32 +177,43 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s0 = tmem, t_o = tmem + 256;  // S buffers at columns 0 and 128, O at 256
+  // S buffers at columns 0 and 128; O_0, O_1 (one per key half / softmax warpgroup) at 256 and 384
+  const uint32_t t_s0 = tmem, t_o0 = tmem + 256, t_o1 = tmem + 384;
 
   if (warp == 0) {
     if (lane == 0) {
       ptx::mbar_arrive_expect_tx(q_full, G::TILE);
       load_tile<HD>(sm + G::Q_OFF, &tq, &tq_r, q_full, col0, (int)(q0 - a.p0));
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j % G::NSTF;
-        if (!ptx::mbar_wait(&kv_empty[s], ((j / G::NSTF) & 1) ^ 1, err)) break;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], 2 * G::TILE);
+      // K runs one tile ahead of V: K_{j+1} is wanted for S_{j+1} before P_j V_j
+      auto load_k = [&](int j) {
+        const int s = j % G::NK;
+        if (!ptx::mbar_wait(&k_empty[s], ((j / G::NK) & 1) ^ 1, err)) return false;
+        ptx::mbar_arrive_expect_tx(&k_full[s], G::TILE);
         const int slot = (int)((j_begin + (int64_t)j * KT) % a.ring);
-        uint8_t* kd = sm + G::KV_OFF + s * 2 * G::TILE;
-        load_tile<HD>(kd, &tk, &tk_r, &kv_full[s], col0, slot);
-        load_tile<HD>(kd + G::TILE, &tv, &tv_r, &kv_full[s], col0, slot);
+        load_tile<HD>(sm + G::K_OFF + s * G::TILE, &tk, &tk_r, &k_full[s], col0, slot);
+        return true;
+      };
+      bool ok = ntiles > 0 ? load_k(0) : true;
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles && !(ok = load_k(j + 1))) break;
+        const int s = j % G::NV;
+        if (!(ok = ptx::mbar_wait(&v_empty[s], ((j / G::NV) & 1) ^ 1, err))) break;
+        ptx::mbar_arrive_expect_tx(&v_full[s], G::VTILE);
+        const int slot = (int)((j_begin + (int64_t)j * KT) % a.ring);
+        uint8_t* vd = sm + G::V_OFF + s * G::VTILE;
+#pragma unroll
+        for (int at = 0; at < G::VA; ++at) ptx::tma_load_2d(vd + at * 16384, &tv, &v_full[s], col0 + 64 * at, slot);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, KT, false, false);
-      constexpr uint32_t id_pv64 = ptx::idesc_bf16_f32(128, 64, false, true);
-      constexpr uint32_t id_pvr = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
+      constexpr uint32_t id_pv = ptx::idesc_bf16_f32(128, HD, false, true);
       const uint32_t q_addr = ptx::smem_u32(sm + G::Q_OFF);
       bool ok = ptx::mbar_wait(q_full, 0, err);
       auto issue_s = [&](int j) {
-        const int s = j % G::NSTF;
-        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE);
+        const int s = j % G::NK;
+        const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + s * G::TILE);
         const uint32_t d = t_s0 + (j & 1) * 128;
         int step = 0;
 #pragma unroll
@@ -209,67 +230,65 @@ __global__ void __launch_bounds__(384, 1)
                            step > 0);
         }
         ptx::umma_commit(&s_full[j & 1]);
+        ptx::umma_commit(&k_empty[s]);
       };
       if (ok && ntiles > 0) {
-        if ((ok = ptx::mbar_wait(&kv_full[0], 0, err))) {
+        if ((ok = ptx::mbar_wait(&k_full[0], 0, err))) {
           ptx::tc_fence_after();
           issue_s(0);
         }
       }
       for (int j = 0; ok && j < ntiles; ++j) {
         if (j + 1 < ntiles) {
-          const int s1 = (j + 1) % G::NSTF;
-          if (!(ok = ptx::mbar_wait(&kv_full[s1], ((j + 1) / G::NSTF) & 1, err))) break;
+          const int s1 = (j + 1) % G::NK;
+          if (!(ok = ptx::mbar_wait(&k_full[s1], ((j + 1) / G::NK) & 1, err))) break;
           if (j + 1 >= 2 && !(ok = ptx::mbar_wait(&s_empty[(j + 1) & 1], (((j + 1) / 2) - 1) & 1, err))) break;
           ptx::tc_fence_after();
           issue_s(j + 1);
         }
+        const int sv = j % G::NV;
         if (!(ok = ptx::mbar_wait(&p_full[j & 1], (j / 2) & 1, err))) break;
+        if (!(ok = ptx::mbar_wait(&v_full[sv], (j / G::NV) & 1, err))) break;
         ptx::tc_fence_after();
-        const int s = j % G::NSTF;
-        const uint32_t v_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::TILE + G::TILE);
+        const uint32_t v_addr = ptx::smem_u32(sm + G::V_OFF + sv * G::VTILE);
         const uint32_t p_addr = ptx::smem_u32(sm + G::P_OFF + (j & 1) * G::P_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < KT / 16; ++kk) {
+        for (int kk = 0; kk < KT / 16; ++kk) {  // keys 0..63 -> O_0, keys 64..127 -> O_1
           const uint64_t pd = sdesc(p_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, 2);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-#pragma unroll
-          for (int at = 0; at < G::A; ++at)
-            ptx::umma_bf16(t_o + 64 * at, pd, sdesc(v_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_pv64, acc);
-          if constexpr (G::R > 0)
-            ptx::umma_bf16(t_o + 64 * G::A, pd,
-                           sdesc(v_addr + G::REM_OFF + kk * 16 * G::RB, 16, 8 * G::RB, rem_swizzle_layout(G::R)),
-                           id_pvr, acc);
+          const uint32_t acc = (j > 0 || (kk % 4) > 0) ? 1u : 0u;
+          // V: MN-major, VA atoms 16384 bytes apart along head_dim (LBO), 8-key groups 1024 apart (SBO)
+          ptx::umma_bf16(kk < 4 ? t_o0 : t_o1, pd, sdesc(v_addr + kk * 2048, 16384, 1024, 2), id_pv, acc);
         }
-        ptx::umma_commit(&kv_empty[s]);
+        ptx::umma_commit(&v_empty[sv]);
         ptx::umma_commit(&pv_done[j & 1]);
       }
       ptx::umma_commit(o_full);
       ptx::mbar_drain(o_full, 0);  // no MMA may still write TMEM when it is released
     }
   } else if (warp >= 4) {
-    // ---- softmax: 8 warps; a row is shared by two threads (warpgroups g = 0, 1),
-    // each owning 64 of the tile's 128 key columns; row statistics are combined
-    // through shared memory once per tile ----
-    const int g = (warp - 4) >> 2;                          // column half
-    const int r = ((warp - 4) & 3) * 32 + lane;            // row in the tile (== TMEM lane)
-    const int64_t p = q0 + r;                               // absolute query position
+    // ---- softmax: two independent warpgroups.  Warpgroup g owns key columns
+    // 64g .. 64g+63 of every tile and runs its own online softmax (max m, sum l)
+    // into its own accumulator O_g; thread = query row (= TMEM lane).  The two
+    // halves are combined once, in the epilogue. ----
+    const int g = (warp - 4) >> 2;
+    const int r = ((warp - 4) & 3) * 32 + lane;
+    const int64_t p = q0 + r;
     const bool row_ok = p <= qlast;
     const uint32_t lane_off = (uint32_t)(((warp - 4) & 3) * 32) << 16;
+    const uint32_t t_og = g ? t_o1 : t_o0;
     const float sl2 = a.scale * 1.4426950408889634f;        // scale * log2(e)
-    float* xmax = reinterpret_cast<float*>(sm + G::X_OFF);  // [2][128] partial row maxima
-    float* xsum = xmax;  // [2][128] partial row sums in the epilogue (xmax is dead after the last tile)
-    float m = -INFINITY, l = 0.f;                           // l: this thread's half of the row sum
+    // epilogue exchange of the halves' row statistics, in P buffer 0 (free once O is final)
+    float* xm = reinterpret_cast<float*>(sm + G::P_OFF);  // [2][128] row max per half
+    float* xl = xm + 256;                                 // [2][128] row sum per half
+    float m = -INFINITY, l = 0.f;
     uint8_t* pbase = sm + G::P_OFF;
-    bool ok = true;  // failures inside an iteration only clear `ok`; the whole group leaves together at the
-                     // agreement at the top of the next iteration (no thread is left at a named barrier)
+    bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
-      const int64_t j0 = j_begin + (int64_t)j * KT;
-      if (ok) ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
-      ok = bar_and(1, 256, ok);  // all 256 softmax threads agree before the exchanges below
-      if (!ok) break;
+      const int64_t j0 = j_begin + (int64_t)j * KT + 64 * g;  // position of this half's first key
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err));
+      if (!ok) break;  // warp-uniform: TMEM loads follow
       ptx::tc_fence_after();
-      float s[64];  // raw scores of columns 64g .. 64g+63; the scale is folded into the exponent
+      float s[64];  // raw scores; the scale is folded into the exponent
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
         uint32_t rr[32];
@@ -280,8 +299,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&s_empty[j & 1]);
-      // mask: key 64g + c valid iff j0 + 64g + c in [p - window + 1, p]
-      const int64_t lo = p - a.window + 1 - j0 - 64 * g, hi = p - j0 - 64 * g;
+      const int64_t lo = p - a.window + 1 - j0, hi = p - j0;  // key c valid iff lo <= c <= hi
       if (!(row_ok && lo <= 0 && hi >= 63)) {
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = (row_ok && c >= lo && c <= hi) ? s[c] : -INFINITY;
@@ -292,14 +310,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u) mx[u] = fmaxf(mx[u], s[c + u]);
       }
-      xmax[g * 128 + r] = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float tmax = fmaxf(xmax[r], xmax[128 + r]) * sl2;  // whole-row tile max, log2 domain
-      asm volatile("bar.sync 1, 256;" ::: "memory");           // xmax may be rewritten next tile
-      // running max with lazy rescaling of O (needs PV_{j-1} complete).  Both
-      // threads of a row take the same decision; each rescales its own O columns
-      // (16-column groups of parity g).  TMEM access is warp-collective, so a warp
-      // rescales together when any of its rows needs it (corr = 1 otherwise).
+      const float tmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;  // log2 domain
+      // lazy rescaling of O_g (needs PV_{j-1} complete); warp-collective TMEM
+      // access, so a warp rescales together when any of its rows needs it
       float mu = m, corr = 1.f;
       if (tmax > -INFINITY) {
         if (m == -INFINITY) {
@@ -313,23 +326,22 @@ __global__ void __launch_bounds__(384, 1)
       m = mu;
       if (__any_sync(0xffffffffu, corr != 1.f)) {
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) / 2) & 1, err));
-        if (!ok) continue;  // skip to the agreement
+        if (!ok) break;
         ptx::tc_fence_after();
 #pragma unroll
-        for (int c = 16 * g; c < HD; c += 32) {
+        for (int c = 0; c < HD; c += 16) {
           uint32_t o[16];
-          tmem_ld16(t_o + c + lane_off, o);
+          tmem_ld16(t_og + c + lane_off, o);
           ptx::tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-          tmem_st16(t_o + c + lane_off, o);
+          tmem_st16(t_og + c + lane_off, o);
         }
         tmem_st_wait();
       }
-      // P buffer (j & 1) is free once PV_{j-2} completed
-      if (j >= 2) {
+      if (j >= 2) {  // P buffer (j & 1) is free once PV_{j-2} completed
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[j & 1], ((j - 2) / 2) & 1, err));
-        if (!ok) continue;  // skip to the agreement
+        if (!ok) break;
       }
       uint8_t* prow = pbase + (j & 1) * G::P_BYTES + g * 16384 + r * 128;  // this half = one 64-key atom
       const float neg_m = (m == -INFINITY) ? 0.f : -m;  // m = -inf only while every score so far is masked
@@ -356,39 +368,42 @@ __global__ void __launch_bounds__(384, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&p_full[j & 1]);
     }
-    // ---- epilogue: O / l (l = both halves) and the natural-log LSE ----
+    // ---- epilogue: combine the halves, O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / l ----
     if (ok) ok = ptx::mbar_wait(o_full, 0, err);
-    ok = bar_and(1, 256, ok);
+    ok = bar_and(1, 256, ok);  // every softmax thread arrives here exactly once
     if (ok) {
-      xsum[g * 128 + r] = l;
+      xm[g * 128 + r] = m;
+      xl[g * 128 + r] = l;
       asm volatile("bar.sync 1, 256;" ::: "memory");
-      const float lt = xsum[r] + xsum[128 + r];
+      const float m0 = xm[r], m1 = xm[128 + r];
+      const float M = fmaxf(m0, m1);
+      const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M), f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+      const float lt = xl[r] * f0 + xl[128 + r] * f1;
       ptx::tc_fence_after();
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float c0 = f0 * inv, c1 = f1 * inv;
       const int64_t i = p - a.p0;
       bf16* orow = reinterpret_cast<bf16*>(a.o) + i * a.ldo + col0;
 #pragma unroll
-      for (int c = 16 * g; c < HD; c += 32) {
-        uint32_t o[16];
-        tmem_ld16(t_o + c + lane_off, o);
+      for (int c = 16 * g; c < HD; c += 32) {  // this thread writes the 16-column groups of parity g
+        uint32_t o0[16], o1[16];
+        tmem_ld16(t_o0 + c + lane_off, o0);
+        tmem_ld16(t_o1 + c + lane_off, o1);
         ptx::tmem_ld_wait();
         if (row_ok) {
-          uint4 w0, w1;
-          uint32_t* pw = &w0.x;
-          uint32_t* pw1 = &w1.x;
+          uint32_t pw[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 t0 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-            __nv_bfloat162 t1 = __floats2bfloat162_rn(__uint_as_float(o[8 + 2 * e]) * inv,
-                                                      __uint_as_float(o[8 + 2 * e + 1]) * inv);
-            pw[e] = *reinterpret_cast<uint32_t*>(&t0);
-            pw1[e] = *reinterpret_cast<uint32_t*>(&t1);
+          for (int e = 0; e < 8; ++e) {
+            const float v0 = __uint_as_float(o0[2 * e]) * c0 + __uint_as_float(o1[2 * e]) * c1;
+            const float v1 = __uint_as_float(o0[2 * e + 1]) * c0 + __uint_as_float(o1[2 * e + 1]) * c1;
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(v0, v1);
+            pw[e] = *reinterpret_cast<uint32_t*>(&t2);
           }
-          *reinterpret_cast<uint4*>(orow + c) = w0;
-          *reinterpret_cast<uint4*>(orow + c + 8) = w1;
+          *reinterpret_cast<uint4*>(orow + c) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+          *reinterpret_cast<uint4*>(orow + c + 8) = make_uint4(pw[4], pw[5], pw[6], pw[7]);
         }
       }
-      if (row_ok && g == 0) a.lse[(int64_t)h * a.ld_lse + i] = (m + log2f(lt)) * 0.6931471805599453f;
+      if (row_ok && g == 0) a.lse[(int64_t)h * a.ld_lse + i] = (M + log2f(lt)) * 0.6931471805599453f;
     }
   }
   ptx::tc_fence_before();
@@ -1007,7 +1022,7 @@ int launch(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
     }
   }
   dim3 grid(ceil_div(a.n, QT), a.heads);
-  fn<<<grid, 384, G::SMEM, s>>>(p.q128, p.qr, p.k128, p.kr, p.v128, p.vr, a, err);
+  fn<<<grid, 384, G::SMEM, s>>>(p.q128, p.qr, p.k128, p.kr, p.v128, a, err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }

@@ -1,6 +1,7 @@
-// Memory-bound kernels of the prefill loop (see elementwise.cuh).  Row
-// reductions use one warp per row and warp shuffles; everything else is one
-// thread per element.
+// Memory-bound kernels of the prefill loop (see elementwise.cuh).  RMSNorm
+// uses one 128-thread block per row with float4 access (one warp per row when
+// the layout is not vector-aligned); everything else is one thread per
+// element or one warp per row.
 #include "elementwise.cuh"
 
 namespace ttt {
@@ -66,6 +67,113 @@ __global__ void rmsnorm_bwd_kernel(const float* x, int64_t ldx, const float* rst
     if (dx16) dx16[row * ld16 + c] = from_f32<T>(v);
   }
 }
+
+// Vectorised RMSNorm: one 128-thread block per row, the row held in
+// registers as float4 (d <= 4 * 128 * VN), so x is read once and each block
+// reduces with 4 warps.  Used when d and every leading dimension are
+// multiples of 4 and the pointers are 16-byte (fp32) / 8-byte (bf16) aligned.
+constexpr int VT = 128;  // threads per row
+constexpr int VN = 8;    // float4 per thread: d <= 4096
+
+__device__ __forceinline__ float block_sum128(float v, float* red) {
+  v = warp_sum(v);
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  const float t = (red[0] + red[1]) + (red[2] + red[3]);
+  __syncthreads();  // red may be reused by the caller
+  return t;
+}
+
+template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) {
+  *reinterpret_cast<float4*>(p) = v;
+}
+template <> __device__ __forceinline__ void store4<bf16>(bf16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(VT) rmsnorm_fwd_vec_kernel(const float* x, int64_t ldx, const float* g, float eps,
+                                                             int d, T* y, int64_t ldy, float* rstd) {
+  __shared__ float red[4];
+  const int64_t row = blockIdx.x;
+  const int d4 = d >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * ldx);
+  float4 v[VN];
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < VN; ++u) {
+    const int c = threadIdx.x + u * VT;
+    v[u] = c < d4 ? xr[c] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss = fmaf(v[u].x, v[u].x, fmaf(v[u].y, v[u].y, fmaf(v[u].z, v[u].z, fmaf(v[u].w, v[u].w, ss))));
+  }
+  ss = block_sum128(ss, red);
+  const float r = 1.f / sqrtf(ss / (float)d + eps);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  T* yr = y + row * ldy;
+#pragma unroll
+  for (int u = 0; u < VN; ++u) {
+    const int c = threadIdx.x + u * VT;
+    if (c < d4) {
+      const float4 gg = g4[c];
+      store4<T>(yr + 4 * c, make_float4(v[u].x * r * gg.x, v[u].y * r * gg.y, v[u].z * r * gg.z, v[u].w * r * gg.w));
+    }
+  }
+  if (threadIdx.x == 0 && rstd) rstd[row] = r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(VT) rmsnorm_bwd_vec_kernel(const float* x, int64_t ldx, const float* rstd,
+                                                             const float* g, const float* dy, int64_t lddy,
+                                                             const float* dres, int64_t ldres, int d, float* dx,
+                                                             int64_t lddx, T* dx16, int64_t ld16) {
+  __shared__ float red[4];
+  const int64_t row = blockIdx.x;
+  const int d4 = d >> 2;
+  const float r = rstd[row];
+  const float4* xr = reinterpret_cast<const float4*>(x + row * ldx);
+  const float4* dyr = reinterpret_cast<const float4*>(dy + row * lddy);
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  float4 xv[VN], uv[VN];  // x and u = dy * g
+  float dot = 0.f;
+#pragma unroll
+  for (int u = 0; u < VN; ++u) {
+    const int c = threadIdx.x + u * VT;
+    xv[u] = uv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (c < d4) {
+      xv[u] = xr[c];
+      const float4 dd = dyr[c], gg = g4[c];
+      uv[u] = make_float4(dd.x * gg.x, dd.y * gg.y, dd.z * gg.z, dd.w * gg.w);
+    }
+    dot = fmaf(xv[u].x * r, uv[u].x, fmaf(xv[u].y * r, uv[u].y, fmaf(xv[u].z * r, uv[u].z, fmaf(xv[u].w * r, uv[u].w, dot))));
+  }
+  dot = block_sum128(dot, red) / (float)d;
+  const float rd = r * dot;
+#pragma unroll
+  for (int u = 0; u < VN; ++u) {
+    const int c = threadIdx.x + u * VT;
+    if (c < d4) {
+      float4 o = make_float4(r * (uv[u].x - xv[u].x * rd), r * (uv[u].y - xv[u].y * rd),
+                             r * (uv[u].z - xv[u].z * rd), r * (uv[u].w - xv[u].w * rd));
+      if (dres) {
+        const float4 e = reinterpret_cast<const float4*>(dres + row * ldres)[c];
+        o.x += e.x;
+        o.y += e.y;
+        o.z += e.z;
+        o.w += e.w;
+      }
+      reinterpret_cast<float4*>(dx + row * lddx)[c] = o;
+      if (dx16) store4<T>(dx16 + row * ld16 + 4 * c, o);
+    }
+  }
+}
+
+__host__ __forceinline__ bool al(const void* p, int b) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) % b) == 0; }
 
 // One warp per (token, head); lane t handles rotation pairs t and t + 32.
 constexpr int MAXP = 2;  // pairs per lane (head_dim <= 128)
@@ -272,6 +380,15 @@ __global__ void copy2d_kernel(const TS* src, int64_t lds, TD* dst, int64_t ldd, 
   dst[r * ldd + c] = from_f32<TD>(to_f32(src[r * lds + c]));
 }
 
+// lo = bf16(x - bf16(x)): the low half of a two-term bf16 representation of x
+__global__ void bf16_lo_kernel(const float* src, int64_t lds, bf16* dst, int64_t ldd, int64_t rows, int64_t cols) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * cols) return;
+  const int64_t r = idx / cols, c = idx % cols;
+  const float x = src[r * lds + c];
+  dst[r * ldd + c] = __float2bfloat16_rn(x - __bfloat162float(__float2bfloat16_rn(x)));
+}
+
 inline unsigned row_blocks(int64_t rows) { return ceil_div(rows, ROW_WARPS); }
 
 }  // namespace
@@ -286,7 +403,11 @@ int embed_gather(const int32_t* tok, const T* E, int64_t n, int d, int V, float*
 template <typename T>
 int rmsnorm_fwd(const float* x, int64_t ldx, const float* g, float eps, int64_t n, int d, T* y, int64_t ldy,
                 float* rstd, cudaStream_t s) {
-  rmsnorm_fwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, g, eps, n, d, y, ldy, rstd);
+  if (n <= 0) return TTT_OK;
+  if (d % 4 == 0 && d <= 4 * VT * VN && ldx % 4 == 0 && ldy % 4 == 0 && al(x, 16) && al(g, 16) && al(y, 4 * sizeof(T)))
+    rmsnorm_fwd_vec_kernel<T><<<(unsigned)n, VT, 0, s>>>(x, ldx, g, eps, d, y, ldy, rstd);
+  else
+    rmsnorm_fwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, g, eps, n, d, y, ldy, rstd);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -295,8 +416,15 @@ template <typename T>
 int rmsnorm_bwd(const float* x, int64_t ldx, const float* rstd, const float* g, const float* dy, int64_t lddy,
                 const float* dres, int64_t ldres, int64_t n, int d, float* dx, int64_t lddx, T* dx16, int64_t ld16,
                 cudaStream_t s) {
-  rmsnorm_bwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, rstd, g, dy, lddy, dres, ldres, n, d, dx,
-                                                                  lddx, dx16, ld16);
+  if (n <= 0) return TTT_OK;
+  if (d % 4 == 0 && d <= 4 * VT * VN && ldx % 4 == 0 && lddy % 4 == 0 && lddx % 4 == 0 && (!dres || ldres % 4 == 0) &&
+      (!dx16 || ld16 % 4 == 0) && al(x, 16) && al(g, 16) && al(dy, 16) && al(dres, 16) && al(dx, 16) &&
+      al(dx16, 4 * sizeof(T)))
+    rmsnorm_bwd_vec_kernel<T><<<(unsigned)n, VT, 0, s>>>(x, ldx, rstd, g, dy, lddy, dres, ldres, d, dx, lddx, dx16,
+                                                         ld16);
+  else
+    rmsnorm_bwd_kernel<T><<<row_blocks(n), 32 * ROW_WARPS, 0, s>>>(x, ldx, rstd, g, dy, lddy, dres, ldres, n, d, dx,
+                                                                    lddx, dx16, ld16);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -372,6 +500,13 @@ int deinterleave_gate_up(const float* in, int f, int d, float* gate, float* up, 
 template <typename T>
 int copy2d_from_f32(const float* src, int64_t lds, T* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s) {
   copy2d_kernel<float, T><<<ceil_div(rows * cols, 256), 256, 0, s>>>(src, lds, dst, ldd, rows, cols);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
+int bf16_lo2d(const float* src, int64_t lds, bf16* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s) {
+  if (rows * cols == 0) return TTT_OK;
+  bf16_lo_kernel<<<ceil_div(rows * cols, 256), 256, 0, s>>>(src, lds, dst, ldd, rows, cols);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }

@@ -61,6 +61,8 @@ template <typename TS, typename TD>
 int interleave_gate_up(const TS* gate, const TS* up, int f, int d, TD* out, cudaStream_t s);
 int deinterleave_gate_up(const float* in, int f, int d, float* gate, float* up, cudaStream_t s);
 
+// dst = bf16(src - bf16(src)) (fp32 source): with bf16(src) it represents src to ~2^-17 relative.
+int bf16_lo2d(const float* src, int64_t lds, bf16* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s);
 // dst[r, c] = src[r, c] for r < rows, c < cols (fp32 -> T).
 template <typename T>
 int copy2d_from_f32(const float* src, int64_t lds, T* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s);

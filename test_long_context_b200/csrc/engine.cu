@@ -175,6 +175,8 @@ class Engine final : public ttt_ctx {
   static constexpr int STORE = ActTraits<T>::store_epi;
 
   int prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, const EpiArgs& args);
+  // bf16 mode: add the second product A2 B2^T on output columns >= n_ext (re-plans split-K)
+  int prep_ext(Gemm& g, MatView a2, MatView b2, int64_t n_ext);
   int run(Gemm& g, int64_t rows);  // rows overrides the M extent (chunk/super-chunk length)
   int bottom_layers(const int32_t* tok, int64_t s0, int64_t S);
   int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
@@ -275,6 +277,10 @@ class Engine final : public ttt_ctx {
   std::vector<T*> wgu_;    // bottom: [2f, d]; top: [4f, d] (static | fast), interleaved gate/up
   std::vector<T*> wd_;     // top: [d, 2f] (static | fast); bottom: caller's [d, f]
   std::vector<float*> m_gu_, m_d_;        // fp32 masters (bf16 mode) per top block
+  // bf16 mode: the fast shadow is a two-term bf16 pair hi + lo of the master
+  // (hi inside wgu_/wd_, lo here), so the forward sees updates far below one
+  // bf16 ulp of W
+  std::vector<bf16*> gu_lo_, d_lo_;       // [2f, d] interleaved, [d, f]
   std::vector<float*> init_gu_, init_d_;  // W_init copies per top block
   // phase-1 buffers
   float* xs_ = nullptr;
@@ -344,6 +350,21 @@ int Engine<T>::prep(Gemm& g, int a_mn, MatView a, int b_mn, MatView b, int epi, 
 }
 
 template <typename T>
+int Engine<T>::prep_ext(Gemm& g, MatView a2, MatView b2, int64_t n_ext) {
+  if (!BF) return TTT_OK;
+  const int64_t K2 = g.shape.a_mn ? a2.rows : a2.cols;
+  const int64_t M = g.shape.M(), N = g.shape.N(), K = g.shape.K();
+  int bn = 0;
+  int64_t S = n_ext == 0 ? tc_split_plan(M, N, K + K2, g.epi, &bn) : 1;
+  if (n_ext > 0 && n_ext % tc_pick_bn(M, N, 0)) bn = 128;  // tiles must not straddle n_ext
+  TRY(tc_gemm_prepare(&g.tc, g.shape, g.epi, g.args, bn));
+  TRY(tc_gemm_set_ext(&g.tc, a2, b2, n_ext));
+  g.split = S;
+  if (S > 1) ws_floats_ = std::max<int64_t>(ws_floats_, S * M * N);
+  return TTT_OK;
+}
+
+template <typename T>
 int Engine<T>::run(Gemm& g, int64_t rows) {
   GemmShape s = g.shape;
   if (rows > 0 && !s.a_mn) s.a.rows = rows;
@@ -398,6 +419,8 @@ int Engine<T>::init() {
   // gate/up rows interleaved in (gate 64 | up 64) blocks; the top blocks append the fast half
   m_gu_.assign(nu_, nullptr);
   m_d_.assign(nu_, nullptr);
+  gu_lo_.assign(nu_, nullptr);
+  d_lo_.assign(nu_, nullptr);
   init_gu_.assign(nu_, nullptr);
   init_d_.assign(nu_, nullptr);
   for (int64_t l = 0; l < L_; ++l) {
@@ -418,6 +441,8 @@ int Engine<T>::init() {
       if (BF) {
         TRY(arena_.alloc(&m_gu_[i], 2 * f * d));
         TRY(arena_.alloc(&m_d_[i], d * f));
+        TRY(arena_.alloc(&gu_lo_[i], 2 * f * d));
+        TRY(arena_.alloc(&d_lo_[i], d * f));
       }
     } else {
       wd_[l] = const_cast<T*>(reinterpret_cast<const T*>(lw.w_down));
@@ -534,8 +559,12 @@ int Engine<T>::init() {
     TRY(prep(g[1], 0, MatView{o_[i], b, d, d}, 0, MatView{wt_.layers[l].wo, d, d, d}, EPI_ADD_F32, e));
     e = EpiArgs{}; e.c = a_[i]; e.ldc = 2 * f; e.c2 = gu_[i]; e.ldc2 = 4 * f;
     TRY(prep(g[2], 0, MatView{h2_[i], b, d, d}, 0, MatView{wgu_[l], 4 * f, d, d}, EPI_SWIGLU, e));
+    // fast half: + h2 W_lo^T
+    TRY(prep_ext(g[2], MatView{h2_[i], b, d, d}, MatView{gu_lo_[i], 2 * f, d, d}, 2 * f));
     e = EpiArgs{}; e.c = (i + 1 < nu_) ? xin_[i + 1] : xf_; e.ldc = d; e.c2 = xmid_[i]; e.ldc2 = d;
     TRY(prep(g[3], 0, MatView{a_[i], b, 2 * f, 2 * f}, 0, MatView{wd_[l], d, 2 * f, 2 * f}, EPI_ADD_F32, e));
+    // + a_fast W_down,lo^T
+    TRY(prep_ext(g[3], MatView{a_[i] + f, b, f, 2 * f}, MatView{d_lo_[i], d, f, f}, 0));
     // backward: da (fast half only in the lowest updated block)
     if (i == 0) {
       e = EpiArgs{}; e.c = da_ + f; e.ldc = 2 * f;
@@ -548,11 +577,11 @@ int Engine<T>::init() {
     }
     // weight gradients + SGD on the fast halves
     e = EpiArgs{}; e.alpha = eta_;
-    if (BF) { e.c = m_d_[i]; e.ldc = f; e.c2 = wd_[l] + f; e.ldc2 = 2 * f; }
+    if (BF) { e.c = m_d_[i]; e.ldc = f; e.c2 = wd_[l] + f; e.ldc2 = 2 * f; e.c3 = d_lo_[i]; e.ldc3 = f; }
     else { e.c = wd_[l] + f; e.ldc = 2 * f; }
     TRY(prep(g[6], 1, MatView{dx16_, b, d, d}, 1, MatView{a_[i] + f, b, f, 2 * f}, EPI_SGD, e));
     e = EpiArgs{}; e.alpha = eta_;
-    if (BF) { e.c = m_gu_[i]; e.ldc = d; e.c2 = wgu_[l] + 2 * f * d; e.ldc2 = d; }
+    if (BF) { e.c = m_gu_[i]; e.ldc = d; e.c2 = wgu_[l] + 2 * f * d; e.ldc2 = d; e.c3 = gu_lo_[i]; e.ldc3 = d; }
     else { e.c = wgu_[l] + 2 * f * d; e.ldc = d; }
     TRY(prep(g[7], 1, MatView{dgu_ + 2 * f, b, 2 * f, 4 * f}, 1, MatView{h2_[i], b, d, d}, EPI_SGD, e));
     if (i > 0) {
@@ -591,6 +620,8 @@ int Engine<T>::reset() {
     if (BF) {
       TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d_from_f32<T>(init_gu_[i], d, wgu_[l] + 2 * f * d, d, 2 * f, d, st_); }));
       TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d_from_f32<T>(init_d_[i], f, wd_[l] + f, 2 * f, d, f, st_); }));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return bf16_lo2d(init_gu_[i], d, gu_lo_[i], d, 2 * f, d, st_); }));
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return bf16_lo2d(init_d_[i], f, d_lo_[i], f, d, f, st_); }));
     }
   }
   fresh_ = true;

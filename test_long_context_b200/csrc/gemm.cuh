@@ -24,7 +24,8 @@ enum Epi : int {
                        // target column (row_i[row] - col_offset) is in this GEMM's columns
   EPI_CE_BWD = 5,      // C (activation dtype) = (exp(acc - row_f[row]) - [col + col_offset ==
                        // row_i[row]]) * row_g[row]
-  EPI_SGD = 6,         // C (fp32 master) -= alpha * acc; C2 (optional, bf16) = bf16(new master)
+  EPI_SGD = 6,         // C (fp32 master) -= alpha * acc; C2 (optional, bf16) = hi = bf16(new master);
+                       // C3 (optional, bf16, with C2) = lo = bf16(new master - hi)
   EPI_COUNT = 7
 };
 
@@ -43,6 +44,8 @@ struct EpiArgs {
   float alpha = 0.f;
   int64_t col_offset = 0;
   int64_t split_stride = 0;  // split-K partials: elements between consecutive splits (EPI_STORE_F32 only)
+  void* c3 = nullptr;  // EPI_SGD: low bf16 half of the new master
+  int64_t ldc3 = 0;
 };
 
 // Row-major matrix view in storage order (element type given by the GEMM).
@@ -71,8 +74,12 @@ struct TcGemm {
   int act_bf16 = 1;  // activation dtype of EPI_SWIGLU / EPI_CE_BWD outputs
   // deterministic split-K (ksplit > 1): partials to ws [ksplit][M][N] fp32, then an ordered reduction
   int ksplit = 1;
-  int64_t kps = 0;  // K per split, a multiple of 64
+  int64_t kps = 0;  // k per split (of the concatenated reduction), a multiple of 64
   float* ws = nullptr;
+  // second product A2 B2^T, added on output tiles with n0 >= n_ext (K2 = 0: none)
+  alignas(64) CUtensorMap ta2;
+  alignas(64) CUtensorMap tb2;
+  int64_t K2 = 0, n_ext = 0;
 };
 
 // Split-K count for an M x N x K GEMM with this epilogue (1 = no split); sets
@@ -80,6 +87,12 @@ struct TcGemm {
 int64_t tc_split_plan(int64_t M, int64_t N, int64_t K, int epi, int* bn_out);
 // Enable split-K on a prepared GEMM: ws must hold ksplit * M * N floats.
 int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws);
+// Add a second product: acc += A2 B2^T on output tiles with n0 >= n_ext (a
+// multiple of the tile width; B2's rows/cols are counted from n_ext).  A2 and
+// B2 take the main operands' orientation; A2 has the same M, B2 covers
+// N - n_ext outputs, and they share their own reduction length K2.  Call
+// before tc_gemm_set_split; split-K then needs n_ext = 0.
+int tc_gemm_set_ext(TcGemm* g, const MatView& a2, const MatView& b2, int64_t n_ext);
 
 // Returns TTT_OK or an error code (bad shapes, tensor-map failure).
 int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args, int bn_hint = 0);

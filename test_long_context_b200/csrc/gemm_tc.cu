@@ -175,7 +175,11 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
           } else {
             const float w = cur[u] - ep.alpha * acc;
             reinterpret_cast<float*>(ep.c)[rr * ep.ldc + col] = w;
-            if (ep.c2) reinterpret_cast<bf16*>(ep.c2)[rr * ep.ldc2 + col] = __float2bfloat16_rn(w);
+            if (ep.c2) {
+              const bf16 hi = __float2bfloat16_rn(w);
+              reinterpret_cast<bf16*>(ep.c2)[rr * ep.ldc2 + col] = hi;
+              if (ep.c3) reinterpret_cast<bf16*>(ep.c3)[rr * ep.ldc3 + col] = __float2bfloat16_rn(w - __bfloat162float(hi));
+            }
           }
         }
       }
@@ -224,10 +228,16 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
 // L2.  The accumulator is double-buffered in TMEM (2 x BN columns): the
 // epilogue warps drain unit i while the MMA thread already accumulates unit
 // i+1.  The smem ring's stage/phase counters run on across units.
+//
+// Second product: output tiles with n0 >= n_ext accumulate A2 B2^T after
+// A B^T (k-blocks KB1 .. KB1+KB2-1 of the concatenated reduction; B2's row is
+// n0 - n_ext).  The k-splits cut the concatenated range.
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 __global__ void __launch_bounds__(192, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb, int64_t M,
-                   int64_t N, int64_t K, int64_t kps, int n_mt, int n_nt, int n_split, EpiArgs ep, int* err) {
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                   const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2, int64_t M,
+                   int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt, int n_split, EpiArgs ep,
+                   int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -243,13 +253,16 @@ __global__ void __launch_bounds__(192, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t units = (int64_t)n_mt * n_nt * n_split;
-  auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int64_t& k_begin) {
+  // k-blocks [kb_begin, kb_begin + nkb) of this unit's concatenated reduction
+  auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int& kb_begin) {
     m0 = (u % n_mt) * BM;
     const int64_t nt = (u / n_mt) % n_nt;
     n0 = nt * BN;
     split = (int)(u / ((int64_t)n_mt * n_nt));
-    k_begin = (int64_t)split * kps;
-    nkb = (int)((imin64(kps, K - k_begin) + BK - 1) / BK);
+    const int total = KB1 + (n0 >= n_ext ? KB2 : 0);
+    kb_begin = split * kpsb;
+    nkb = total - kb_begin < kpsb ? total - kb_begin : kpsb;
+    if (nkb < 0) nkb = 0;
   };
 
   if (threadIdx.x == 0) {
@@ -265,6 +278,10 @@ __global__ void __launch_bounds__(192, 1)
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tma);
     ptx::prefetch_tmap(&tmb);
+    if (KB2 > 0) {
+      ptx::prefetch_tmap(&tma2);
+      ptx::prefetch_tmap(&tmb2);
+    }
   }
   if (warp == 1) {
     __syncwarp();
@@ -281,28 +298,33 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t kbg = 0;  // k-blocks issued by this CTA so far (ring position)
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
-        int64_t m0, n0, k_begin;
-        int split, nkb;
-        decode(u, m0, n0, split, nkb, k_begin);
-        for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+        int64_t m0, n0;
+        int split, nkb, kb_begin;
+        decode(u, m0, n0, split, nkb, kb_begin);
+        for (int j = 0; j < nkb; ++j, ++kbg) {
           const int s = (int)(kbg % C::STAGES);
           const uint32_t ph = (kbg / C::STAGES) & 1u;
           if (!(ok = ptx::mbar_wait(&empty[s], ph ^ 1u, err))) break;
           ptx::mbar_arrive_expect_tx(&full[s], C::STAGE);
           uint8_t* a = sA + s * C::A_BYTES;
           uint8_t* b = sB + s * C::B_BYTES;
-          const int k0 = (int)(k_begin + (int64_t)kb * BK);
+          const int kb = kb_begin + j;
+          const bool second = kb >= KB1;  // block of the second product
+          const CUtensorMap* ta = second ? &tma2 : &tma;
+          const CUtensorMap* tb = second ? &tmb2 : &tmb;
+          const int k0 = (second ? kb - KB1 : kb) * BK;
+          const int nb = (int)(second ? n0 - n_ext : n0);
           if constexpr (!A_MN) {
-            ptx::tma_load_2d(a, &tma, &full[s], k0, (int)m0);
+            ptx::tma_load_2d(a, ta, &full[s], k0, (int)m0);
           } else {
-            ptx::tma_load_2d(a, &tma, &full[s], (int)m0, k0);
-            ptx::tma_load_2d(a + 8192, &tma, &full[s], (int)m0 + 64, k0);
+            ptx::tma_load_2d(a, ta, &full[s], (int)m0, k0);
+            ptx::tma_load_2d(a + 8192, ta, &full[s], (int)m0 + 64, k0);
           }
           if constexpr (!B_MN) {
-            ptx::tma_load_2d(b, &tmb, &full[s], k0, (int)n0);
+            ptx::tma_load_2d(b, tb, &full[s], k0, nb);
           } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) ptx::tma_load_2d(b + j * 8192, &tmb, &full[s], (int)n0 + 64 * j, k0);
+            for (int jj = 0; jj < BN / 64; ++jj) ptx::tma_load_2d(b + jj * 8192, tb, &full[s], nb + 64 * jj, k0);
           }
         }
       }
@@ -313,9 +335,9 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t kbg = 0, it = 0;
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x, ++it) {
-        int64_t m0, n0, k_begin;
-        int split, nkb;
-        decode(u, m0, n0, split, nkb, k_begin);
+        int64_t m0, n0;
+        int split, nkb, kb_begin;
+        decode(u, m0, n0, split, nkb, kb_begin);
         const uint32_t b = it & 1u, use = it >> 1;
         // the epilogue must have drained this accumulator buffer's previous unit
         if (!(ok = ptx::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
@@ -350,9 +372,9 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     uint32_t it = 0;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
-      int64_t m0, n0, k_begin;
-      int split, nkb;
-      decode(u, m0, n0, split, nkb, k_begin);
+      int64_t m0, n0;
+      int split, nkb, kb_begin;
+      decode(u, m0, n0, split, nkb, kb_begin);
       const uint32_t b = it & 1u, use = it >> 1;
       const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));  // warp-uniform
       if (!ok) break;
@@ -409,15 +431,17 @@ int make_tmap(CUtensorMap* tm, const MatView& v, int box_rows) {
   return TTT_OK;
 }
 
-using KernelFn = void (*)(CUtensorMap, CUtensorMap, int64_t, int64_t, int64_t, int64_t, int, int, int, EpiArgs, int*);
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, int64_t, int64_t, int, int, int64_t, int,
+                          int, int, int, EpiArgs, int*);
 
 // Sum of split-K partials in a fixed order (deterministic), then the epilogue.
 template <int EPI>
 __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int S, int64_t M, int64_t N, int64_t stride,
                                      EpiArgs ep) {
-  const int64_t idx4 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
-  if (idx4 >= M * N) return;
-  const int64_t row = idx4 / N, col = idx4 % N;
+  const int64_t gpr = (N + 3) / 4;  // 4-column groups per row
+  const int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= M * gpr) return;
+  const int64_t row = gi / gpr, col = (gi % gpr) * 4;
   float v[4] = {0.f, 0.f, 0.f, 0.f};
   const int cnt = (int)imin64(4, N - col);
   for (int s = 0; s < S; ++s) {
@@ -519,10 +543,30 @@ int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args,
   g->ksplit = 1;
   g->kps = K;
   g->ws = nullptr;
+  g->K2 = 0;
+  g->n_ext = 0;
   int rc = make_tmap(&g->ta, s.a, s.a_mn ? 64 : BM);
   if (rc) return rc;
   rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : bn);
+  g->ta2 = g->ta;
+  g->tb2 = g->tb;
   return rc;
+}
+
+int tc_gemm_set_ext(TcGemm* g, const MatView& a2, const MatView& b2, int64_t n_ext) {
+  const int64_t M2 = g->a_mn ? a2.cols : a2.rows, K2 = g->a_mn ? a2.rows : a2.cols;
+  const int64_t N2 = g->b_mn ? b2.cols : b2.rows, KB = g->b_mn ? b2.rows : b2.cols;
+  if (g->ksplit > 1) return set_error(TTT_ERR_STATE, "gemm: set the second product before split-K");
+  if (K2 < 1 || KB != K2 || M2 != g->M || n_ext < 0 || n_ext % g->bn || N2 < g->N - n_ext)
+    return set_error(TTT_ERR_INVALID_ARG, "gemm: inconsistent second product");
+  if (g->epi == EPI_CE_FWD) return set_error(TTT_ERR_INVALID_ARG, "gemm: no second product with CE partials");
+  int rc = make_tmap(&g->ta2, a2, g->a_mn ? 64 : BM);
+  if (rc) return rc;
+  rc = make_tmap(&g->tb2, b2, g->b_mn ? 64 : g->bn);
+  if (rc) return rc;
+  g->K2 = K2;
+  g->n_ext = n_ext;
+  return TTT_OK;
 }
 
 int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws) {
@@ -534,9 +578,13 @@ int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws) {
   if (!ws) return set_error(TTT_ERR_INVALID_ARG, "gemm: split-K needs a workspace");
   if (g->epi != EPI_STORE_F32 && g->epi != EPI_STORE_BF16 && g->epi != EPI_ADD_F32)
     return set_error(TTT_ERR_INVALID_ARG, "gemm: split-K only for store/add epilogues");
-  const int64_t kps = ((g->K + ksplit - 1) / ksplit + BK - 1) / BK * BK;
-  g->ksplit = (int)((g->K + kps - 1) / kps);
-  g->kps = kps;
+  if (g->K2 > 0 && g->n_ext > 0)
+    return set_error(TTT_ERR_INVALID_ARG, "gemm: split-K needs the second product on every tile");
+  // split the concatenated reduction in whole k-blocks
+  const int64_t kblocks = (g->K + BK - 1) / BK + (g->K2 + BK - 1) / BK;
+  const int64_t kpsb = (kblocks + ksplit - 1) / ksplit;
+  g->ksplit = (int)((kblocks + kpsb - 1) / kpsb);
+  g->kps = kpsb * BK;
   g->ws = ws;
   return TTT_OK;
 }
@@ -567,8 +615,11 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
     TTT_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
   }
   const dim3 grid((unsigned)std::min<int64_t>(units, n_sm));
+  const int KB1 = (int)((g.K + BK - 1) / BK), KB2 = (int)((g.K2 + BK - 1) / BK);
+  const int64_t n_ext = g.K2 > 0 ? g.n_ext : INT64_MAX;
   if (g.ksplit <= 1) {
-    fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.M, g.N, g.K, g.K, n_mt, n_nt, 1, g.args, dev_err);
+    fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1,
+                                    g.args, dev_err);
     TTT_CUDA_TRY(cudaGetLastError());
     return TTT_OK;
   }
@@ -577,9 +628,10 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   part.c = g.ws;
   part.ldc = g.N;
   part.split_stride = g.M * g.N;
-  fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.M, g.N, g.K, g.kps, n_mt, n_nt, g.ksplit, part, dev_err);
+  fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, (int)(g.kps / BK), n_mt, n_nt,
+                                  g.ksplit, part, dev_err);
   TTT_CUDA_TRY(cudaGetLastError());
-  const unsigned blocks = ceil_div((g.M * g.N + 3) / 4, 256);
+  const unsigned blocks = ceil_div(g.M * ((g.N + 3) / 4), 256);
   switch (g.epi) {
     case EPI_STORE_F32:
       splitk_reduce_kernel<EPI_STORE_F32><<<blocks, 256, 0, stream>>>(g.ws, g.ksplit, g.M, g.N, g.M * g.N, g.args);

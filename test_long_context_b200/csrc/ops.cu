@@ -33,6 +33,8 @@ static EpiArgs to_epi(const ttt_epilogue_args* a) {
   e.part_ld = a->part_ld;
   e.alpha = a->alpha;
   e.col_offset = a->col_offset;
+  e.c3 = a->c3;
+  e.ldc3 = a->ldc3;
   return e;
 }
 
@@ -80,6 +82,33 @@ extern "C" int ttt_op_gemm_split(int32_t a_mn, int32_t b_mn, int64_t M, int64_t 
   if (rc) return rc;
   int* err = op_err_word();
   if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_gemm_split: no device error word");
+  return tc_gemm_launch(g, reinterpret_cast<cudaStream_t>(stream), err);
+}
+
+extern "C" int ttt_op_gemm_dual(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A,
+                                int64_t lda, const void* B, int64_t ldb, int64_t K2, const void* A2, int64_t lda2,
+                                const void* B2, int64_t ldb2, int64_t n_ext, int32_t epilogue,
+                                const ttt_epilogue_args* args, int32_t bn_hint, int32_t ksplit, float* workspace,
+                                void* stream) {
+  if (!A || !B || !A2 || !B2 || !args || M < 1 || N < 1 || K < 1 || K2 < 1 || n_ext < 0 || n_ext >= N)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_gemm_dual: bad argument");
+  if (a_mn && !b_mn) return set_error(TTT_ERR_UNSUPPORTED, "ttt_op_gemm_dual: (a_mn, b_mn) = (1, 0) not built");
+  GemmShape s;
+  s.a_mn = a_mn ? 1 : 0;
+  s.b_mn = b_mn ? 1 : 0;
+  s.a = a_mn ? MatView{A, K, M, lda} : MatView{A, M, K, lda};
+  s.b = b_mn ? MatView{B, K, N, ldb} : MatView{B, N, K, ldb};
+  const MatView a2 = a_mn ? MatView{A2, K2, M, lda2} : MatView{A2, M, K2, lda2};
+  const MatView b2 = b_mn ? MatView{B2, K2, N - n_ext, ldb2} : MatView{B2, N - n_ext, K2, ldb2};
+  TcGemm g;
+  int rc = tc_gemm_prepare(&g, s, epilogue, to_epi(args), bn_hint);
+  if (rc) return rc;
+  rc = tc_gemm_set_ext(&g, a2, b2, n_ext);
+  if (rc) return rc;
+  rc = tc_gemm_set_split(&g, ksplit, workspace);
+  if (rc) return rc;
+  int* err = op_err_word();
+  if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_gemm_dual: no device error word");
   return tc_gemm_launch(g, reinterpret_cast<cudaStream_t>(stream), err);
 }
 

@@ -26,17 +26,23 @@ def _dtype(t):
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _epi_args(c=None, c2=None, row_f=None, row_g=None, row_i=None, part_max=None, part_sum=None,
+              target_logit=None, part_ld=0, alpha=0.0, col_offset=0, c3=None):
+    return L.ttt_epilogue_args(
+        _p(c), c.stride(0) if c is not None else 0, _p(c2), c2.stride(0) if c2 is not None else 0,
+        _p(row_f), _p(row_g), _p(row_i), _p(part_max), _p(part_sum), _p(target_logit), part_ld, alpha, col_offset,
+        _p(c3), c3.stride(0) if c3 is not None else 0)
+
+
 def gemm(A, B, a_mn, b_mn, epi, c=None, c2=None, row_f=None, row_g=None, row_i=None, part_max=None,
          part_sum=None, target_logit=None, part_ld=0, alpha=0.0, col_offset=0, bn=0, M=None, N=None, K=None,
-         stream=None):
+         c3=None, stream=None):
     """ttt_op_gemm on 2-D tensors in storage order (see ttt_ops.h)."""
     dt = _dtype(A)
     M = (A.shape[1] if a_mn else A.shape[0]) if M is None else M
     K = (A.shape[0] if a_mn else A.shape[1]) if K is None else K
     N = (B.shape[1] if b_mn else B.shape[0]) if N is None else N
-    args = L.ttt_epilogue_args(
-        _p(c), c.stride(0) if c is not None else 0, _p(c2), c2.stride(0) if c2 is not None else 0,
-        _p(row_f), _p(row_g), _p(row_i), _p(part_max), _p(part_sum), _p(target_logit), part_ld, alpha, col_offset)
+    args = _epi_args(c, c2, row_f, row_g, row_i, part_max, part_sum, target_logit, part_ld, alpha, col_offset, c3)
     rc = L.lib().ttt_op_gemm(dt, int(a_mn), int(b_mn), M, N, K, _p(A), A.stride(0), _p(B), B.stride(0), epi,
                              ctypes.byref(args), bn, _stream(stream))
     L.check(rc)
@@ -47,10 +53,22 @@ def gemm_split(A, B, a_mn, b_mn, epi, ksplit, workspace, c=None, c2=None, bn=0, 
     M = A.shape[1] if a_mn else A.shape[0]
     K = A.shape[0] if a_mn else A.shape[1]
     N = B.shape[1] if b_mn else B.shape[0]
-    args = L.ttt_epilogue_args(_p(c), c.stride(0) if c is not None else 0, _p(c2), c2.stride(0) if c2 is not None else 0,
-                               None, None, None, None, None, None, 0, 0.0, 0)
+    args = _epi_args(c, c2)
     rc = L.lib().ttt_op_gemm_split(int(a_mn), int(b_mn), M, N, K, _p(A), A.stride(0), _p(B), B.stride(0), epi,
                                    ctypes.byref(args), bn, ksplit, _p(workspace), _stream(stream))
+    L.check(rc)
+
+
+def gemm_dual(A, B, A2, B2, a_mn, b_mn, epi, n_ext=0, ksplit=1, workspace=None, bn=0, stream=None, **epi_kw):
+    """ttt_op_gemm_dual: acc = A B^T, plus A2 B2^T on output columns >= n_ext (bf16)."""
+    M = A.shape[1] if a_mn else A.shape[0]
+    K = A.shape[0] if a_mn else A.shape[1]
+    K2 = A2.shape[0] if a_mn else A2.shape[1]
+    N = B.shape[1] if b_mn else B.shape[0]
+    args = _epi_args(**epi_kw)
+    rc = L.lib().ttt_op_gemm_dual(int(a_mn), int(b_mn), M, N, K, _p(A), A.stride(0), _p(B), B.stride(0), K2, _p(A2),
+                                  A2.stride(0), _p(B2), B2.stride(0), n_ext, epi, ctypes.byref(args), bn, ksplit,
+                                  _p(workspace), _stream(stream))
     L.check(rc)
 
 

@@ -136,3 +136,86 @@ def test_split_k_matches_and_is_deterministic(combo, ksplit):
     assert torch.equal(c, c_again)
     assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * scale + 1e-4
     assert (cb.double() - ref).abs().max().item() <= 1e-2 * scale
+
+
+def _dual_ref(A, B, A2, B2, a_mn, b_mn, n_ext):
+    Am = A.double().T if a_mn else A.double()
+    Bm = B.double() if b_mn else B.double().T
+    A2m = A2.double().T if a_mn else A2.double()
+    B2m = B2.double() if b_mn else B2.double().T
+    ref = Am @ Bm
+    ref[:, n_ext:] += A2m @ B2m
+    return ref
+
+
+@pytest.mark.parametrize("combo", [(0, 0), (0, 1)])
+def test_dual_product_swiglu_mixed_tiles(combo):
+    """Second product on the columns from n_ext on only (the fast half of a
+    [static | fast] gate/up GEMM), a different reduction length K2."""
+    from test_long_context_b200 import ops
+    M, N, K, K2, n_ext = 300, 768, 192, 136, 384
+    g = torch.Generator(device="cuda").manual_seed(21)
+    a_mn, b_mn = combo
+    A = torch.randn((M, K), device="cuda", generator=g).bfloat16()
+    B = torch.randn((K, N) if b_mn else (N, K), device="cuda", generator=g).bfloat16()
+    A2 = torch.randn((M, K2), device="cuda", generator=g).bfloat16()
+    B2 = torch.randn((K2, N - n_ext) if b_mn else (N - n_ext, K2), device="cuda", generator=g).bfloat16()
+    ref = _dual_ref(A, B, A2, B2, a_mn, b_mn, n_ext)
+    a = torch.empty(M, N // 2, device="cuda", dtype=torch.bfloat16)
+    raw = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    ops.gemm_dual(A, B, A2, B2, a_mn, b_mn, ops.L.EPI_SWIGLU, n_ext=n_ext, bn=128, c=a, c2=raw)
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm_dual(A, B, A2, B2, a_mn, b_mn, ops.L.EPI_STORE_F32, n_ext=n_ext, bn=128, c=c)
+    ops.sync()
+    assert (c.double() - ref).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
+    r = ref.view(M, N // 128, 2, 64)
+    want = (torch.nn.functional.silu(r[:, :, 0]) * r[:, :, 1]).reshape(M, N // 2)
+    assert (a.double() - want).abs().max().item() <= 2e-2 * want.abs().max().item()
+    assert (raw.double() - ref).abs().max().item() <= 2e-2 * ref.abs().max().item()
+
+
+@pytest.mark.parametrize("ksplit", [1, 3, 5])
+def test_dual_product_add_split_k(ksplit):
+    """Second product on every tile with split-K over the concatenated
+    reduction: ragged K (a partial last k-block before the second product
+    starts) and ragged K2; deterministic on rerun."""
+    from test_long_context_b200 import ops
+    M, N, K, K2 = 300, 640, 4104, 1000
+    g = torch.Generator(device="cuda").manual_seed(22)
+    A = torch.randn((M, K), device="cuda", generator=g).bfloat16()
+    B = torch.randn((N, K), device="cuda", generator=g).bfloat16()
+    A2 = torch.randn((M, K2), device="cuda", generator=g).bfloat16()
+    B2 = torch.randn((N, K2), device="cuda", generator=g).bfloat16()
+    ref = _dual_ref(A, B, A2, B2, 0, 0, 0)
+    ws = torch.empty(max(ksplit, 1) * M * N, device="cuda")
+    x0 = torch.randn(M, N, device="cuda")
+    x, x_again = torch.empty_like(x0), torch.empty_like(x0)
+    ops.gemm_dual(A, B, A2, B2, 0, 0, ops.L.EPI_ADD_F32, ksplit=ksplit, workspace=ws, c=x, c2=x0)
+    ops.gemm_dual(A, B, A2, B2, 0, 0, ops.L.EPI_ADD_F32, ksplit=ksplit, workspace=ws, c=x_again, c2=x0)
+    ops.sync()
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
+    assert torch.equal(x, x_again)
+
+
+def test_sgd_two_term_bf16_shadow():
+    """SGD epilogue with hi and lo shadows: hi = bf16(W), lo = bf16(W - hi),
+    so hi + lo follows an update far below one bf16 ulp of W."""
+    from test_long_context_b200 import ops
+    Aw, Bw, G = _operands(160, 384, 256, 1, 1, torch.bfloat16, seed=3)
+    W = (0.02 * torch.randn(160, 384, device="cuda")).bfloat16().float()  # weight-sized, bf16-exact start
+    W0 = W.clone()
+    hi = torch.empty(160, 384, device="cuda", dtype=torch.bfloat16)
+    lo = torch.empty_like(hi)
+    alpha = 1e-6
+    ops.gemm(Aw, Bw, 1, 1, ops.L.EPI_SGD, c=W, c2=hi, c3=lo, alpha=alpha)
+    ops.sync()
+    want = W0.double() - alpha * G
+    assert (W.double() - want).abs().max().item() <= 1e-6
+    assert torch.equal(hi, W.to(torch.bfloat16))
+    assert torch.equal(lo, (W - hi.float()).to(torch.bfloat16))
+    two = hi.double() + lo.double()
+    step = (want - W0.double()).abs()
+    # hi + lo carries W to ~|W| 2^-18, well inside 1% of the largest step
+    assert (two - want).abs().max().item() <= 1e-2 * step.max().item()
+    # a single bf16 copy would lose most of the step (half an ulp of 0.02 is ~6e-5)
+    assert (hi.double() - W0.double()).abs().mean().item() < 0.5 * step.mean().item()

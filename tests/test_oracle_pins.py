@@ -288,7 +288,7 @@ def test_golden_pair_counts():
 
 def test_causality_predict_before_update(micro_cfg):
     """Changing tokens[q:] leaves losses[:q-1] bit-identical: a position is
-    scored before any label at or after its target is used (算法 1 step 3.3;
+    scored before any label at or after its target is used (算法 1;
     eq. (3) ordering).  q inside a chunk catches an update-before-score."""
     cfg = micro_cfg.with_(eta=0.3)
     m, _ = _model(cfg)
