@@ -178,31 +178,32 @@ __host__ __forceinline__ bool al(const void* p, int b) { return p == nullptr || 
 // One warp per (token, head); lane t handles rotation pairs t and t + 32.
 constexpr int MAXP = 2;  // pairs per lane (head_dim <= 128)
 
-__device__ __forceinline__ void rope_cs(int64_t pos, int t, int HD, double theta, float& c, float& s) {
+// Rotation table of positions p0 .. p0+n-1: tab[i * HD/2 + t] = (cos, sin) of
+// (p0 + i) * theta^(-2t/HD), angles in fp64, stored as fp32.
+__global__ void rope_table_kernel(float2* tab, int64_t p0, int64_t n, int HD, double theta) {
+  const int h2 = HD / 2;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * h2) return;
+  const int64_t i = idx / h2;
+  const int t = (int)(idx % h2);
   const double inv = pow(theta, -2.0 * (double)t / (double)HD);
   double sd, cd;
-  sincos((double)pos * inv, &sd, &cd);
-  c = (float)cd;
-  s = (float)sd;
+  sincos((double)(p0 + i) * inv, &sd, &cd);
+  tab[idx] = make_float2((float)cd, (float)sd);
 }
 
 template <typename T>
 __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n,
-                                       int64_t p0, int H, int HD, float eps, double theta, T* qout, int64_t ldq,
-                                       T* kring, T* vring, int64_t ldkv, int64_t R, float* rq, float* rk) {
-  // one block per token: the position's rotation table is computed once (fp64
-  // angles) and shared by all heads; warp w handles heads w, w + 8, ...
-  __shared__ float2 cs[32 * MAXP];
+                                       int64_t p0, int H, int HD, float eps, const float2* tab, int64_t tab_p0,
+                                       T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv, int64_t R, float* rq,
+                                       float* rk) {
+  // one block per token, the position's row of the rotation table shared by
+  // all heads; warp w handles heads w, w + 8, ...
   const int64_t i = blockIdx.x;
   const int lane = threadIdx.x % 32;
   const int h2 = HD / 2;
   if (i >= n) return;
-  for (int t = threadIdx.x; t < h2; t += blockDim.x) {
-    float c, sn;
-    rope_cs(p0 + i, t, HD, theta, c, sn);
-    cs[t] = make_float2(c, sn);
-  }
-  __syncthreads();
+  const float2* cs = tab + (p0 + i - tab_p0) * h2;
   for (int h = threadIdx.x / 32; h < H; h += blockDim.x / 32) {
   const int D = H * HD;
   const T* q = qkv + i * ldqkv + h * HD;
@@ -236,7 +237,8 @@ __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float*
   for (int u = 0; u < MAXP; ++u) {
     const int t = lane + 32 * u;
     if (t < h2) {
-      const float c = cs[t].x, s = cs[t].y;
+      const float2 csv = cs[t];
+      const float c = csv.x, s = csv.y;
       const float a1 = q1[u] * rqv * gq[t], a2 = q2[u] * rqv * gq[t + h2];
       const float b1 = k1[u] * rkv * gk[t], b2 = k2[u] * rkv * gk[t + h2];
       qo[t] = from_f32<T>(a1 * c - a2 * s);
@@ -256,19 +258,13 @@ __global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float*
 template <typename T>
 __global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq,
                                        const float* gk, const float* rq, const float* rk, int64_t n, int64_t p0,
-                                       int H, int HD, double theta) {
-  // one block per token, rotation table shared by the 2H (q, k) heads
-  __shared__ float2 cs[32 * MAXP];
+                                       int H, int HD, const float2* tab, int64_t tab_p0) {
+  // one block per token, the position's table row shared by the 2H (q, k) heads
   const int64_t i = blockIdx.x;
   const int lane = threadIdx.x % 32;
   const int h2 = HD / 2;
   if (i >= n) return;
-  for (int t = threadIdx.x; t < h2; t += blockDim.x) {
-    float c, sn;
-    rope_cs(p0 + i, t, HD, theta, c, sn);
-    cs[t] = make_float2(c, sn);
-  }
-  __syncthreads();
+  const float2* cs = tab + (p0 + i - tab_p0) * h2;
   for (int w = threadIdx.x / 32; w < 2 * H; w += blockDim.x / 32) {
   const int which = w % 2;  // 0: q, 1: k
   const int h = w / 2;
@@ -285,7 +281,8 @@ __global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_
     const int t = lane + 32 * u;
     u1[u] = u2[u] = x1[u] = x2[u] = 0.f;
     if (t < h2) {
-      const float c = cs[t].x, s = cs[t].y;
+      const float2 csv = cs[t];
+      const float c = csv.x, s = csv.y;
       const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
       // transpose of the rotation, then the gain
       u1[u] = (d1 * c + d2 * s) * g[t];
@@ -321,19 +318,85 @@ __global__ void swiglu_bwd_kernel(const T* da, int64_t ldda, const T* gu, int64_
   dgu[row * lddgu + uc] = from_f32<T>(a * g * sg);
 }
 
-__global__ void ce_finalize_kernel(const float* pmax, const float* psum, int64_t part_ld, int tiles, const float* zt,
-                                   int64_t n, int64_t n_valid, float inv_nc, float* loss_out, float* lse_out,
-                                   float* scale) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  float M = -INFINITY;
-  for (int t = 0; t < tiles; ++t) M = fmaxf(M, pmax[(int64_t)t * part_ld + i]);
-  float S = 0.f;
-  for (int t = 0; t < tiles; ++t) {
-    const float m = pmax[(int64_t)t * part_ld + i];
-    if (m > -INFINITY) S += psum[(int64_t)t * part_ld + i] * expf(m - M);
+// Four consecutive features per thread (one 8- or 16-byte access per operand).
+template <typename T> struct Vec4;
+template <> struct Vec4<float> { using type = float4; };
+template <> struct Vec4<bf16> { using type = uint2; };
+__device__ __forceinline__ void unpack4(float4 v, float (&f)[4]) { f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w; }
+__device__ __forceinline__ void unpack4(uint2 v, float (&f)[4]) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&v.y));
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+template <typename V> __device__ __forceinline__ V pack4(const float (&f)[4]);
+template <> __device__ __forceinline__ float4 pack4<float4>(const float (&f)[4]) { return make_float4(f[0], f[1], f[2], f[3]); }
+template <> __device__ __forceinline__ uint2 pack4<uint2>(const float (&f)[4]) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(f[0], f[1]), b = __floats2bfloat162_rn(f[2], f[3]);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  return u;
+}
+
+template <typename T>
+__global__ void swiglu_bwd_vec_kernel(const T* da, int64_t ldda, const T* gu, int64_t ldgu, int64_t n, int64_t nfeat,
+                                      T* dgu, int64_t lddgu) {
+  using V = typename Vec4<T>::type;
+  const int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 4;
+  const int64_t row = blockIdx.y;
+  if (j >= nfeat || row >= n) return;
+  const int64_t gc = 128 * (j / 64) + (j % 64), uc = gc + 64;
+  float g[4], u[4], a[4], dg[4], du[4];
+  unpack4(*reinterpret_cast<const V*>(gu + row * ldgu + gc), g);
+  unpack4(*reinterpret_cast<const V*>(gu + row * ldgu + uc), u);
+  unpack4(*reinterpret_cast<const V*>(da + row * ldda + j), a);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float sg = 1.f / (1.f + expf(-g[e]));
+    dg[e] = a[e] * u[e] * sg * (1.f + g[e] * (1.f - sg));
+    du[e] = a[e] * g[e] * sg;
   }
-  const float lse = M + logf(S);
+  *reinterpret_cast<V*>(dgu + row * lddgu + gc) = pack4<V>(dg);
+  *reinterpret_cast<V*>(dgu + row * lddgu + uc) = pack4<V>(du);
+}
+
+// Combines the per-tile softmax partials of each row: a block covers 32 rows
+// (threadIdx.x) and splits the tiles over CE_SLICES slices (threadIdx.y),
+// each slice keeping an online (max, sum) pair, merged through smem.
+constexpr int CE_SLICES = 16;
+
+__global__ void __launch_bounds__(32 * CE_SLICES) ce_finalize_kernel(const float* pmax, const float* psum,
+                                                                     int64_t part_ld, int tiles, const float* zt,
+                                                                     int64_t n, int64_t n_valid, float inv_nc,
+                                                                     float* loss_out, float* lse_out, float* scale) {
+  __shared__ float sm_m[CE_SLICES][32], sm_s[CE_SLICES][32];
+  const int64_t i = (int64_t)blockIdx.x * 32 + threadIdx.x;
+  float M = -INFINITY, S = 0.f;
+  if (i < n) {
+#pragma unroll 4
+    for (int t = threadIdx.y; t < tiles; t += CE_SLICES) {
+      const float m = pmax[(int64_t)t * part_ld + i], ps = psum[(int64_t)t * part_ld + i];
+      if (m == -INFINITY) continue;
+      if (m > M) {
+        S = S * expf(M - m) + ps;
+        M = m;
+      } else {
+        S += ps * expf(m - M);
+      }
+    }
+  }
+  sm_m[threadIdx.y][threadIdx.x] = M;
+  sm_s[threadIdx.y][threadIdx.x] = S;
+  __syncthreads();
+  if (threadIdx.y != 0 || i >= n) return;
+  float Mt = -INFINITY;
+  for (int y = 0; y < CE_SLICES; ++y) Mt = fmaxf(Mt, sm_m[y][threadIdx.x]);
+  float St = 0.f;
+  for (int y = 0; y < CE_SLICES; ++y) {
+    const float m = sm_m[y][threadIdx.x];
+    if (m > -INFINITY) St += sm_s[y][threadIdx.x] * expf(m - Mt);
+  }
+  const float lse = Mt + logf(St);
   lse_out[i] = lse;
   const bool ok = i < n_valid;
   loss_out[i] = ok ? lse - zt[i] : __int_as_float(0x7fc00000);
@@ -431,22 +494,24 @@ int rmsnorm_bwd(const float* x, int64_t ldx, const float* rstd, const float* g, 
 
 template <typename T>
 int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n, int64_t p0, int H,
-                    int HD, float eps, double theta, T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv,
-                    int64_t R, float* rq, float* rk, cudaStream_t s) {
+                    int HD, float eps, const float2* tab, int64_t tab_p0, T* qout, int64_t ldq, T* kring, T* vring,
+                    int64_t ldkv, int64_t R, float* rq, float* rk, cudaStream_t s) {
   if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
-  qknorm_rope_fwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, theta,
-                                                                          qout, ldq, kring, vring, ldkv, R, rq, rk);
+  if (n <= 0) return TTT_OK;
+  qknorm_rope_fwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, tab, tab_p0,
+                                                                   qout, ldq, kring, vring, ldkv, R, rq, rk);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
 
 template <typename T>
 int qknorm_rope_bwd(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq, const float* gk,
-                    const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, double theta,
-                    cudaStream_t s) {
+                    const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, const float2* tab,
+                    int64_t tab_p0, cudaStream_t s) {
   if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
-  qknorm_rope_bwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n,
-                                                                              p0, H, HD, theta);
+  if (n <= 0) return TTT_OK;
+  qknorm_rope_bwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n, p0, H,
+                                                                   HD, tab, tab_p0);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -456,15 +521,24 @@ int swiglu_bwd(const T* da, int64_t ldda, const T* gu, int64_t ldgu, int64_t n, 
                int64_t lddgu, cudaStream_t s) {
   if (nfeat % 64) return set_error(TTT_ERR_INVALID_ARG, "swiglu_bwd: features must be a multiple of 64");
   dim3 grid(ceil_div(nfeat, 256), (unsigned)n);
-  swiglu_bwd_kernel<T><<<grid, 256, 0, s>>>(da, ldda, gu, ldgu, n, nfeat, dgu, lddgu);
+  constexpr int VB = 4 * (int)sizeof(T);  // bytes of a 4-feature access
+  const bool vec = ldda % 4 == 0 && ldgu % 4 == 0 && lddgu % 4 == 0 && reinterpret_cast<uintptr_t>(da) % VB == 0 &&
+                   reinterpret_cast<uintptr_t>(gu) % VB == 0 && reinterpret_cast<uintptr_t>(dgu) % VB == 0;
+  if (vec) {
+    dim3 g4(ceil_div(nfeat / 4, 256), (unsigned)n);
+    swiglu_bwd_vec_kernel<T><<<g4, 256, 0, s>>>(da, ldda, gu, ldgu, n, nfeat, dgu, lddgu);
+  } else {
+    swiglu_bwd_kernel<T><<<grid, 256, 0, s>>>(da, ldda, gu, ldgu, n, nfeat, dgu, lddgu);
+  }
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
 
 int ce_finalize(const float* pmax, const float* psum, int64_t part_ld, int tiles, const float* zt, int64_t n,
                 int64_t n_valid, float inv_nc, float* loss_out, float* lse, float* scale, cudaStream_t s) {
-  ce_finalize_kernel<<<ceil_div(n, 128), 128, 0, s>>>(pmax, psum, part_ld, tiles, zt, n, n_valid, inv_nc, loss_out,
-                                                      lse, scale);
+  if (n <= 0) return TTT_OK;
+  ce_finalize_kernel<<<ceil_div(n, 32), dim3(32, CE_SLICES), 0, s>>>(pmax, psum, part_ld, tiles, zt, n, n_valid,
+                                                                     inv_nc, loss_out, lse, scale);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -504,6 +578,14 @@ int copy2d_from_f32(const float* src, int64_t lds, T* dst, int64_t ldd, int64_t 
   return TTT_OK;
 }
 
+int rope_table(float2* tab, int64_t p0, int64_t n, int HD, double theta, cudaStream_t s) {
+  if (n <= 0) return TTT_OK;
+  if (HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "rope_table: odd head_dim");
+  rope_table_kernel<<<ceil_div(n * (HD / 2), 256), 256, 0, s>>>(tab, p0, n, HD, theta);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+
 int bf16_lo2d(const float* src, int64_t lds, bf16* dst, int64_t ldd, int64_t rows, int64_t cols, cudaStream_t s) {
   if (rows * cols == 0) return TTT_OK;
   bf16_lo_kernel<<<ceil_div(rows * cols, 256), 256, 0, s>>>(src, lds, dst, ldd, rows, cols);
@@ -525,10 +607,11 @@ int copy2d(const T* src, int64_t lds, T* dst, int64_t ldd, int64_t rows, int64_t
   template int rmsnorm_bwd<T>(const float*, int64_t, const float*, const float*, const float*, int64_t,         \
                               const float*, int64_t, int64_t, int, float*, int64_t, T*, int64_t, cudaStream_t); \
   template int qknorm_rope_fwd<T>(const T*, int64_t, const float*, const float*, int64_t, int64_t, int, int,    \
-                                  float, double, T*, int64_t, T*, T*, int64_t, int64_t, float*, float*,         \
-                                  cudaStream_t);                                                                \
+                                  float, const float2*, int64_t, T*, int64_t, T*, T*, int64_t, int64_t, float*, \
+                                  float*, cudaStream_t);                                                        \
   template int qknorm_rope_bwd<T>(T*, int64_t, const T*, int64_t, const float*, const float*, const float*,     \
-                                  const float*, int64_t, int64_t, int, int, double, cudaStream_t);              \
+                                  const float*, int64_t, int64_t, int, int, const float2*, int64_t,             \
+                                  cudaStream_t);                                                                \
   template int swiglu_bwd<T>(const T*, int64_t, const T*, int64_t, int64_t, int64_t, T*, int64_t, cudaStream_t); \
   template int copy2d_from_f32<T>(const float*, int64_t, T*, int64_t, int64_t, int64_t, cudaStream_t);          \
   template int copy2d<T>(const T*, int64_t, T*, int64_t, int64_t, int64_t, cudaStream_t);

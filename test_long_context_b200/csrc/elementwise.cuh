@@ -28,15 +28,20 @@ int rmsnorm_bwd(const float* x, int64_t ldx, const float* rstd, const float* g, 
 // and the per-head RMS factors rq, rk [n, H].
 template <typename T>
 int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n, int64_t p0, int H,
-                    int HD, float eps, double theta, T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv,
-                    int64_t R, float* rq, float* rk, cudaStream_t s);
+                    int HD, float eps, const float2* tab, int64_t tab_p0, T* qout, int64_t ldq, T* kring, T* vring,
+                    int64_t ldkv, int64_t R, float* rq, float* rk, cudaStream_t s);
 
 // In place on dqkv's q and k parts: gradient w.r.t. rotated q,k -> gradient
 // w.r.t. the raw projections (RoPE transpose, then per-head RMSNorm backward).
 template <typename T>
 int qknorm_rope_bwd(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq, const float* gk,
-                    const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, double theta,
-                    cudaStream_t s);
+                    const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, const float2* tab,
+                    int64_t tab_p0, cudaStream_t s);
+
+// RoPE rotation table of positions p0 .. p0+n-1 (row i = position p0 + i):
+// tab[i * HD/2 + t] = (cos, sin)((p0 + i) * theta^(-2t/HD)), angles in fp64.
+// qknorm_rope_fwd/bwd read the rows of their positions (tab_p0 = the table's p0).
+int rope_table(float2* tab, int64_t p0, int64_t n, int HD, double theta, cudaStream_t s);
 
 // SwiGLU backward on (gate 64 | up 64) interleaved columns: for feature j
 // (pair j/64, lane j%64) with g, u from gu and da from da:

@@ -13,6 +13,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <map>
 #include <memory>
 #include <string>
 #include <vector>
@@ -88,6 +89,7 @@ struct Gemm {
   TcGemm tc;
   bool bf = false;
   int64_t split = 1;  // deterministic split-K count (bf16 mode)
+  const char* label = "gemm";
 };
 
 // Event-pair timing of launches, per kernel class (opt-in).
@@ -96,7 +98,14 @@ struct LaunchTimer {
     int kc;
     cudaEvent_t a, b;
     double flops;
+    std::string label;
   };
+  struct Stat {
+    double ms = 0, flops = 0;
+    int64_t n = 0;
+  };
+  std::map<std::string, Stat> by_label;  // filled when `labels` is set (TTT_PROFILE=1)
+  bool labels = false;
   bool on = false;
   std::vector<Rec> pending;
   std::vector<cudaEvent_t> pool;
@@ -126,6 +135,12 @@ struct LaunchTimer {
       ms[r.kc] += t;
       flops[r.kc] += r.flops;
       n[r.kc] += 1;
+      if (labels && !r.label.empty()) {
+        Stat& st = by_label[r.label];
+        st.ms += t;
+        st.flops += r.flops;
+        st.n += 1;
+      }
       pool.push_back(r.a);
       pool.push_back(r.b);
     }
@@ -134,6 +149,15 @@ struct LaunchTimer {
   }
   void clear() {
     for (int i = 0; i < TTT_KC_COUNT; ++i) ms[i] = flops[i] = 0, n[i] = 0;
+    by_label.clear();
+  }
+  // TTT_PROFILE=1: per-label table on stderr (launches, ms, TFLOP/s) of what was timed.
+  void report() const {
+    if (!labels || by_label.empty()) return;
+    fprintf(stderr, "[ttt profile] %-22s %8s %10s %9s\n", "label", "launches", "ms", "TFLOP/s");
+    for (const auto& kv : by_label)
+      fprintf(stderr, "[ttt profile] %-22s %8lld %10.3f %9.1f\n", kv.first.c_str(), (long long)kv.second.n,
+              kv.second.ms, kv.second.ms > 0 ? kv.second.flops / kv.second.ms / 1e9 : 0.0);
   }
 };
 
@@ -153,9 +177,13 @@ class Engine final : public ttt_ctx {
   int prefill(const int32_t* tok, int64_t T_, float* losses, float* const* fast_out) override;
   int reset() override;
   int sync() override;
+  ~Engine() override {
+    if (timer_.labels && cudaStreamSynchronize(st_) == cudaSuccess && timer_.drain() == TTT_OK) timer_.report();
+  }
   int timing_enable(bool on) override {
     TTT_CUDA_TRY(cudaStreamSynchronize(st_));
     TRY(timer_.drain());
+    timer_.report();  // TTT_PROFILE: what was timed since the last enable
     timer_.clear();
     timer_.on = on;
     return TTT_OK;
@@ -182,15 +210,18 @@ class Engine final : public ttt_ctx {
   int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
   // Launch `f` (returns a status); bracket it with events when timing is on.
   template <typename F>
-  int timed(int kc, double flops, F&& f) {
+  int timed(int kc, double flops, F&& f, const char* label = nullptr) {
     ++launches;
     if (trace_) return traced(kc, f);
     if (!timer_.on) return f();
+    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope"};
     cudaEvent_t a = timer_.get(), b = timer_.get();
     TTT_CUDA_TRY(cudaEventRecord(a, st_));
     const int rc = f();
     TTT_CUDA_TRY(cudaEventRecord(b, st_));
-    timer_.pending.push_back({kc, a, b, flops});
+    std::string lab;
+    if (timer_.labels) lab = label ? std::string(label) : std::string(phase_) + "." + names[kc];
+    timer_.pending.push_back({kc, a, b, flops, std::move(lab)});
     return rc;
   }
   // TTT_TRACE=1: synchronise after every launch and log it to stderr (debugging aid).
@@ -264,6 +295,7 @@ class Engine final : public ttt_ctx {
   Arena arena_;
   LaunchTimer timer_;
   bool trace_ = false, trace_verbose_ = false;
+  const char* phase_ = "misc";  // label prefix of untagged launches under TTT_PROFILE
   float trace_ms_ = 0.f;
   bool fresh_ = true;
   int* err_ = nullptr;
@@ -284,6 +316,8 @@ class Engine final : public ttt_ctx {
   std::vector<float*> init_gu_, init_d_;  // W_init copies per top block
   // phase-1 buffers
   float* xs_ = nullptr;
+  float2* rope_tab_ = nullptr;  // RoPE (cos, sin) of the current super-chunk's positions, from tab_p0_
+  int64_t tab_p0_ = 0;
   T *hs_ = nullptr, *qkvs_ = nullptr, *qs_ = nullptr, *os_ = nullptr, *as_ = nullptr;
   float *rs_ = nullptr, *rqs_ = nullptr, *rks_ = nullptr, *lses_ = nullptr;
   std::vector<T*> kb_, vb_;  // bottom rings [R1, d]
@@ -373,9 +407,9 @@ int Engine<T>::run(Gemm& g, int64_t rows) {
     TcGemm tc = g.tc;
     tc.args = g.args;
     if (rows > 0 && !tc.a_mn) tc.M = rows;
-    return timed(TTT_KC_GEMM, flops, [&] { return tc_gemm_launch(tc, st_, err_); });
+    return timed(TTT_KC_GEMM, flops, [&] { return tc_gemm_launch(tc, st_, err_); }, g.label);
   }
-  return timed(TTT_KC_GEMM, flops, [&] { return simt_gemm(s, g.epi, g.args, st_); });
+  return timed(TTT_KC_GEMM, flops, [&] { return simt_gemm(s, g.epi, g.args, st_); }, g.label);
 }
 
 template <typename T>
@@ -395,6 +429,7 @@ int Engine<T>::init() {
     trace_verbose_ = t[0] == 'v';
     trace_ms_ = (float)atof(t) > 1.f ? (float)atof(t) : 0.f;  // TTT_TRACE=<ms>: log launches slower than that
   }
+  if (const char* t = getenv("TTT_PROFILE")) timer_.labels = t[0] && t[0] != '0';
   TRY(arena_.alloc(&err_, 1));
 
   // Super-chunk length for the fast-weight-free blocks: about 16K positions.
@@ -469,6 +504,7 @@ int Engine<T>::init() {
     }
   }
   TRY(arena_.alloc(&xs_, S_ * d));
+  TRY(arena_.alloc(&rope_tab_, S_ * (HD_ / 2)));
   auto per = [&](auto& vec) { vec.assign(nu_, nullptr); };
   per(xin_); per(r1_); per(xmid_); per(r2_); per(rq_); per(rk_); per(lse_);
   per(h_); per(qkv_); per(q_); per(o_); per(h2_); per(gu_); per(a_); per(kt_); per(vt_);
@@ -542,12 +578,16 @@ int Engine<T>::init() {
     Gemm* g = &g_bot_[4 * l];
     e = EpiArgs{}; e.c = qkvs_; e.ldc = 3 * d;
     TRY(prep(g[0], 0, MatView{hs_, S_, d, d}, 0, MatView{wqkv_[l], 3 * d, d, d}, STORE, e));
+    g[0].label = "bot.qkv";
     e = EpiArgs{}; e.c = xs_; e.ldc = d;
     TRY(prep(g[1], 0, MatView{os_, S_, d, d}, 0, MatView{wt_.layers[l].wo, d, d, d}, EPI_ADD_F32, e));
+    g[1].label = "bot.o";
     e = EpiArgs{}; e.c = as_; e.ldc = f;
     TRY(prep(g[2], 0, MatView{hs_, S_, d, d}, 0, MatView{wgu_[l], 2 * f, d, d}, EPI_SWIGLU, e));
+    g[2].label = "bot.gateup";
     e = EpiArgs{}; e.c = xs_; e.ldc = d;
     TRY(prep(g[3], 0, MatView{as_, S_, f, f}, 0, MatView{wd_[l], d, f, f}, EPI_ADD_F32, e));
+    g[3].label = "bot.down";
   }
   g_top_.resize(10 * nu_);
   for (int i = 0; i < nu_; ++i) {
@@ -555,44 +595,56 @@ int Engine<T>::init() {
     Gemm* g = &g_top_[10 * i];
     e = EpiArgs{}; e.c = qkv_[i]; e.ldc = 3 * d;
     TRY(prep(g[0], 0, MatView{h_[i], b, d, d}, 0, MatView{wqkv_[l], 3 * d, d, d}, STORE, e));
+    g[0].label = "top.qkv";
     e = EpiArgs{}; e.c = xmid_[i]; e.ldc = d; e.ldc2 = d;  // c2 = x_in, set per chunk
     TRY(prep(g[1], 0, MatView{o_[i], b, d, d}, 0, MatView{wt_.layers[l].wo, d, d, d}, EPI_ADD_F32, e));
+    g[1].label = "top.o";
     e = EpiArgs{}; e.c = a_[i]; e.ldc = 2 * f; e.c2 = gu_[i]; e.ldc2 = 4 * f;
     TRY(prep(g[2], 0, MatView{h2_[i], b, d, d}, 0, MatView{wgu_[l], 4 * f, d, d}, EPI_SWIGLU, e));
+    g[2].label = "top.gateup";
     // fast half: + h2 W_lo^T
     TRY(prep_ext(g[2], MatView{h2_[i], b, d, d}, MatView{gu_lo_[i], 2 * f, d, d}, 2 * f));
     e = EpiArgs{}; e.c = (i + 1 < nu_) ? xin_[i + 1] : xf_; e.ldc = d; e.c2 = xmid_[i]; e.ldc2 = d;
     TRY(prep(g[3], 0, MatView{a_[i], b, 2 * f, 2 * f}, 0, MatView{wd_[l], d, 2 * f, 2 * f}, EPI_ADD_F32, e));
+    g[3].label = "top.down";
     // + a_fast W_down,lo^T
     TRY(prep_ext(g[3], MatView{a_[i] + f, b, f, 2 * f}, MatView{d_lo_[i], d, f, f}, 0));
     // backward: da (fast half only in the lowest updated block)
     if (i == 0) {
       e = EpiArgs{}; e.c = da_ + f; e.ldc = 2 * f;
       TRY(prep(g[4], 0, MatView{dx16_, b, d, d}, 1, MatView{wd_[l] + f, d, f, 2 * f}, STORE, e));
+      g[4].label = "top.da";
     } else {
       e = EpiArgs{}; e.c = da_; e.ldc = 2 * f;
       TRY(prep(g[4], 0, MatView{dx16_, b, d, d}, 1, MatView{wd_[l], d, 2 * f, 2 * f}, STORE, e));
+      g[4].label = "top.da";
       e = EpiArgs{}; e.c = dh2_; e.ldc = d;
       TRY(prep(g[5], 0, MatView{dgu_, b, 4 * f, 4 * f}, 1, MatView{wgu_[l], 4 * f, d, d}, EPI_STORE_F32, e));
+      g[5].label = "top.dgrad_gu";
     }
     // weight gradients + SGD on the fast halves
     e = EpiArgs{}; e.alpha = eta_;
     if (BF) { e.c = m_d_[i]; e.ldc = f; e.c2 = wd_[l] + f; e.ldc2 = 2 * f; e.c3 = d_lo_[i]; e.ldc3 = f; }
     else { e.c = wd_[l] + f; e.ldc = 2 * f; }
     TRY(prep(g[6], 1, MatView{dx16_, b, d, d}, 1, MatView{a_[i] + f, b, f, 2 * f}, EPI_SGD, e));
+    g[6].label = "top.sgd_down";
     e = EpiArgs{}; e.alpha = eta_;
     if (BF) { e.c = m_gu_[i]; e.ldc = d; e.c2 = wgu_[l] + 2 * f * d; e.ldc2 = d; e.c3 = gu_lo_[i]; e.ldc3 = d; }
     else { e.c = wgu_[l] + 2 * f * d; e.ldc = d; }
     TRY(prep(g[7], 1, MatView{dgu_ + 2 * f, b, 2 * f, 4 * f}, 1, MatView{h2_[i], b, d, d}, EPI_SGD, e));
+    g[7].label = "top.sgd_gu";
     if (i > 0) {
       e = EpiArgs{}; e.c = do_; e.ldc = d;
       TRY(prep(g[8], 0, MatView{dxm16_, b, d, d}, 1, MatView{wt_.layers[l].wo, d, d, d}, STORE, e));
+      g[8].label = "top.dgrad_o";
       e = EpiArgs{}; e.c = dh_; e.ldc = d;
       TRY(prep(g[9], 0, MatView{dqkv_, b, 3 * d, 3 * d}, 1, MatView{wqkv_[l], 3 * d, d, d}, EPI_STORE_F32, e));
+      g[9].label = "top.dgrad_qkv";
     }
   }
   e = EpiArgs{}; e.row_i = tgt_; e.part_max = pmax_; e.part_sum = psum_; e.target_logit = zt_; e.part_ld = b;
   TRY(prep(g_head_, 0, MatView{hf_, b, d, d}, 0, MatView{wt_.lm_head, V_, d, d}, EPI_CE_FWD, e));
+  g_head_.label = "head.ce_fwd";
   g_ce_dz_.resize(nvc_);
   g_ce_dh_.resize(nvc_);
   for (int64_t c = 0; c < nvc_; ++c) {
@@ -600,9 +652,11 @@ int Engine<T>::init() {
     const T* hv = reinterpret_cast<const T*>(wt_.lm_head) + v0 * d;
     e = EpiArgs{}; e.c = dz_; e.ldc = Vc_; e.row_f = lsef_; e.row_g = scl_; e.row_i = tgt_; e.col_offset = v0;
     TRY(prep(g_ce_dz_[c], 0, MatView{hf_, b, d, d}, 0, MatView{hv, vn, d, d}, EPI_CE_BWD, e));
+    g_ce_dz_[c].label = "head.ce_dz";
     e = EpiArgs{}; e.c = dhf_; e.ldc = d;
     TRY(prep(g_ce_dh_[c], 0, MatView{dz_, b, vn, Vc_}, 1, MatView{hv, vn, d, d}, c == 0 ? EPI_STORE_F32 : EPI_ADD_F32,
              e));
+    g_ce_dh_[c].label = "head.ce_dh";
   }
   TRY(finalize_splits());
   TTT_CUDA_TRY(cudaStreamSynchronize(st_));
@@ -644,16 +698,20 @@ int Engine<T>::sync() {
 
 template <typename T>
 int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
+  phase_ = "bot";
   const int64_t d = d_;
   const float eps = cfg_.norm_eps;
   const double theta = cfg_.rope_theta;
   TRY(timed(TTT_KC_OTHER, 0, [&] { return embed_gather<T>(tok + s0, reinterpret_cast<const T*>(wt_.embed), S, (int)d, (int)V_, xs_, err_, st_); }));
+  // rotation table of this super-chunk's positions: every block and chunk inside it reads it
+  tab_p0_ = s0;
+  TRY(timed(TTT_KC_ROPE, 0, [&] { return rope_table(rope_tab_, s0, S, (int)HD_, theta, st_); }));
   for (int64_t l = 0; l < nbot_; ++l) {
     const ttt_layer_weights& lw = wt_.layers[l];
     Gemm* g = &g_bot_[4 * l];
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.attn_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[0], S));
-    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, theta, qs_, d,
+    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, S, s0, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, qs_, d,
                                  kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(s0, S),
               [&] { return attn_fwd(tc_attn_ ? &att_bot_[l] : nullptr,
@@ -668,6 +726,7 @@ int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
 
 template <typename T>
 int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses) {
+  phase_ = "top";
   const int64_t d = d_, f = f_, b = b_;
   const float eps = cfg_.norm_eps;
   const double theta = cfg_.rope_theta;
@@ -681,7 +740,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     const float* xin = i == 0 ? x0 : xin_[i];
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, n, (int)d, h_[i], d, r1_[i], st_); }));
     TRY(run(g[0], n));
-    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, theta, q_[i], d,
+    TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_fwd<T>(qkv_[i], 3 * d, lw.q_norm, lw.k_norm, n, p0, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, q_[i], d,
                                  kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(p0, n),
               [&] { return attn_fwd(tc_attn_ ? &att_top_[i] : nullptr,
@@ -699,6 +758,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
   if (n < b || n_valid == 0) return TTT_OK;  // a trailing partial chunk is scored only
 
   // ---- backward through the updated blocks, SGD on each fast MLP ----
+  phase_ = "bwd";
   for (int64_t c = 0; c < nvc_; ++c) {
     TRY(run(g_ce_dz_[c], n));
     TRY(run(g_ce_dh_[c], n));
@@ -740,7 +800,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
     }));
     launches += 2;  // the backward launches three kernels
     TRY(timed(TTT_KC_ROPE, 0, [&] { return qknorm_rope_bwd<T>(dqkv_, 3 * d, qkv_[i], 3 * d, lw.q_norm, lw.k_norm, rq_[i], rk_[i], n, p0, (int)H_,
-                                 (int)HD_, theta, st_); }));
+                                 (int)HD_, rope_tab_, tab_p0_, st_); }));
     TRY(run(g[9], n));
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xin_[i], d, r1_[i], lw.attn_norm, dh_, d, dxm_, d, n, (int)d, dx_, d, dx16_, d, st_); }));
   }
@@ -752,6 +812,7 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
   if (!fresh_) return set_error(TTT_ERR_STATE, "ttt_prefill needs a fresh context (call ttt_reset)");
   if (!tok || !losses || T_ < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: bad argument");
   fresh_ = false;
+  phase_ = "misc";
   TRY(timed(TTT_KC_OTHER, 0, [&] { return check_tokens(tok, T_, (int)V_, err_, st_); }));
   for (int64_t s0 = 0; s0 < T_; s0 += S_) {
     const int64_t S = std::min<int64_t>(S_, T_ - s0);

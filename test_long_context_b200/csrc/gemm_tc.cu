@@ -20,14 +20,20 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;
 
+// Warps: 0 = TMA producer, 1 = MMA issuer, 2 .. 9 = two epilogue groups of four
+// (one per TMEM accumulator buffer, so two units drain at the same time).
+constexpr int kEpiWarps = 8;
+constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
+
 template <int BN>
 struct TcCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int WBUF = 4 * 32 * 33 * 4;  // epilogue transpose tiles, one per epilogue warp
+  static constexpr int WBUF = kEpiWarps * 32 * 33 * 4;  // epilogue transpose tiles, one per epilogue warp
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + WBUF;
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.f + __expf(-g)) * u; }
@@ -78,8 +84,7 @@ __device__ __forceinline__ void ld32f(uint32_t taddr, float (&v)[32]) {
 // Epilogue of one accumulator row (thread) over the tile's BN columns.
 template <int BN, int EPI, typename TACT>
 __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool row_ok, int64_t n0, int64_t N,
-                                             const EpiArgs& ep, int tile_n, int split, float* wbuf, int64_t row0,
-                                             int64_t M) {
+                                             const EpiArgs& ep, int tile_n, int split) {
   float v[32];
   if constexpr (EPI == EPI_SWIGLU) {
 #pragma unroll 1
@@ -137,54 +142,6 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
       ep.part_sum[(int64_t)tile_n * ep.part_ld + row] = sm;
       if (found) ep.target_logit[row] = zt;
     }
-  } else if constexpr (EPI == EPI_ADD_F32 || EPI == EPI_SGD) {
-    // Read-modify-write epilogues: transpose each 32 x 32 chunk through this
-    // warp's padded smem tile so that global accesses walk rows with lane =
-    // column (coalesced 128-byte loads/stores, 8 rows in flight).
-    const int lane = threadIdx.x & 31;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      ld32f(t_row + c, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) wbuf[lane * 33 + i] = v[i];
-      __syncwarp();
-      const int64_t col = n0 + c + lane;
-      const bool col_ok = col < N;
-#pragma unroll 1
-      for (int r0 = 0; r0 < 32; r0 += 8) {
-        float cur[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int64_t rr = row0 + r0 + u;
-          cur[u] = 0.f;
-          if (col_ok && rr < M) {
-            if constexpr (EPI == EPI_ADD_F32)
-              cur[u] = ep.c2 ? reinterpret_cast<const float*>(ep.c2)[rr * ep.ldc2 + col]
-                             : reinterpret_cast<const float*>(ep.c)[rr * ep.ldc + col];
-            else
-              cur[u] = reinterpret_cast<const float*>(ep.c)[rr * ep.ldc + col];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int64_t rr = row0 + r0 + u;
-          if (!(col_ok && rr < M)) continue;
-          const float acc = wbuf[(r0 + u) * 33 + lane];
-          if constexpr (EPI == EPI_ADD_F32) {
-            reinterpret_cast<float*>(ep.c)[rr * ep.ldc + col] = cur[u] + acc;
-          } else {
-            const float w = cur[u] - ep.alpha * acc;
-            reinterpret_cast<float*>(ep.c)[rr * ep.ldc + col] = w;
-            if (ep.c2) {
-              const bf16 hi = __float2bfloat16_rn(w);
-              reinterpret_cast<bf16*>(ep.c2)[rr * ep.ldc2 + col] = hi;
-              if (ep.c3) reinterpret_cast<bf16*>(ep.c3)[rr * ep.ldc3 + col] = __float2bfloat16_rn(w - __bfloat162float(hi));
-            }
-          }
-        }
-      }
-      __syncwarp();
-    }
   } else {
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
@@ -192,16 +149,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
       const int64_t col0 = n0 + c;
       if (!row_ok || col0 >= N) continue;
       const int nval = (int)(N - col0 < 32 ? N - col0 : 32);
-      if constexpr (EPI == EPI_STORE_F32) {
-        store32<float>(reinterpret_cast<float*>(ep.c) + (int64_t)split * ep.split_stride + row * ep.ldc + col0, v,
-                       nval);
-      } else if constexpr (EPI == EPI_STORE_BF16) {
+      if constexpr (EPI == EPI_STORE_BF16) {
         store32<bf16>(reinterpret_cast<bf16*>(ep.c) + row * ep.ldc + col0, v, nval);
-      } else if constexpr (EPI == EPI_ADD_F32) {
-        float* dst = reinterpret_cast<float*>(ep.c) + row * ep.ldc + col0;
-        const float* src = ep.c2 ? reinterpret_cast<const float*>(ep.c2) + row * ep.ldc2 + col0 : dst;
-        for (int i = 0; i < nval; ++i) v[i] += src[i];
-        store32<float>(dst, v, nval);
       } else if constexpr (EPI == EPI_CE_BWD) {
         constexpr float LOG2E = 1.4426950408889634f;
         const float lse = ep.row_f[row], sc = ep.row_g[row];
@@ -212,13 +161,126 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
           v[i] = (p - (col0 + i == tgt ? 1.f : 0.f)) * sc;
         }
         store32<TACT>(reinterpret_cast<TACT*>(ep.c) + row * ep.ldc + col0, v, nval);
-      } else if constexpr (EPI == EPI_SGD) {
-        float* w = reinterpret_cast<float*>(ep.c) + row * ep.ldc + col0;
-        for (int i = 0; i < nval; ++i) v[i] = w[i] - ep.alpha * v[i];
-        store32<float>(w, v, nval);
-        if (ep.c2) store32<bf16>(reinterpret_cast<bf16*>(ep.c2) + row * ep.ldc2 + col0, v, nval);
       }
     }
+  }
+}
+
+// fp32 stores and read-modify-write epilogues (EPI_STORE_F32, EPI_ADD_F32,
+// EPI_SGD) go through a per-warp transpose so that global accesses run along
+// rows with lane = column (coalesced 128-byte lines).  The warp owns rows
+// row0 .. row0+31 of the tile.  Its read source (the residual or the master)
+// does not depend on the accumulator, so the first 32-column chunk is loaded
+// before the accumulator is ready and each later chunk one chunk ahead: with
+// 32 independent loads per lane in flight the epilogue is not bound by DRAM
+// latency.
+template <int EPI>
+constexpr bool kTransposedEpi = EPI == EPI_STORE_F32 || EPI == EPI_ADD_F32 || EPI == EPI_SGD;
+
+template <int EPI>
+__device__ __forceinline__ void epi_load_chunk(const EpiArgs& ep, int64_t row0, int64_t M, int64_t col, int64_t N,
+                                               float (&dst)[32]) {
+  if constexpr (EPI == EPI_ADD_F32 || EPI == EPI_SGD) {
+    const float* src = reinterpret_cast<const float*>(ep.c);
+    int64_t ld = ep.ldc;
+    if constexpr (EPI == EPI_ADD_F32) {
+      if (ep.c2) {
+        src = reinterpret_cast<const float*>(ep.c2);
+        ld = ep.ldc2;
+      }
+    }
+    const int nrows = (int)(M - row0 < 32 ? M - row0 : 32);
+    const float* p = src + row0 * ld + col;
+    if (col < N && nrows == 32) {
+#pragma unroll
+      for (int r = 0; r < 32; ++r, p += ld) dst[r] = *p;
+    } else {
+      const bool col_ok = col < N;
+#pragma unroll
+      for (int r = 0; r < 32; ++r, p += ld) dst[r] = (col_ok && r < nrows) ? *p : 0.f;
+    }
+  }
+}
+
+// Writes one 32 x 32 chunk (rows row0.., columns col - lane ..) from the
+// transposed accumulator in wbuf; `cur` holds the chunk's read source.
+template <int EPI, bool CHECK, bool HI, bool LO>
+__device__ __forceinline__ void epi_store_chunk(const EpiArgs& ep, int64_t row0, int64_t col, int split, int nrows,
+                                                const float* wbuf, const float (&cur)[32]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (EPI == EPI_STORE_F32) {
+    float* p = reinterpret_cast<float*>(ep.c) + (int64_t)split * ep.split_stride + row0 * ep.ldc + col;
+#pragma unroll
+    for (int r = 0; r < 32; ++r, p += ep.ldc)
+      if (!CHECK || r < nrows) *p = wbuf[r * 33 + lane];
+  } else if constexpr (EPI == EPI_ADD_F32) {
+    float* p = reinterpret_cast<float*>(ep.c) + row0 * ep.ldc + col;
+#pragma unroll
+    for (int r = 0; r < 32; ++r, p += ep.ldc)
+      if (!CHECK || r < nrows) *p = cur[r] + wbuf[r * 33 + lane];
+  } else {  // EPI_SGD
+    float* p = reinterpret_cast<float*>(ep.c) + row0 * ep.ldc + col;
+    bf16* ph = HI ? reinterpret_cast<bf16*>(ep.c2) + row0 * ep.ldc2 + col : nullptr;
+    bf16* pl = LO ? reinterpret_cast<bf16*>(ep.c3) + row0 * ep.ldc3 + col : nullptr;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      if (!CHECK || r < nrows) {
+        const float w = cur[r] - ep.alpha * wbuf[r * 33 + lane];
+        *p = w;
+        if constexpr (HI) {
+          const bf16 hi = __float2bfloat16_rn(w);
+          *ph = hi;
+          if constexpr (LO) *pl = __float2bfloat16_rn(w - __bfloat162float(hi));
+        }
+      }
+      p += ep.ldc;
+      if constexpr (HI) ph += ep.ldc2;
+      if constexpr (LO) pl += ep.ldc3;
+    }
+  }
+}
+
+template <int EPI, bool HI, bool LO>
+__device__ __forceinline__ void epi_store_dispatch_check(const EpiArgs& ep, int64_t row0, int64_t col, int split,
+                                                         int nrows, bool full, const float* wbuf,
+                                                         const float (&cur)[32]) {
+  if (full)
+    epi_store_chunk<EPI, false, HI, LO>(ep, row0, col, split, nrows, wbuf, cur);
+  else
+    epi_store_chunk<EPI, true, HI, LO>(ep, row0, col, split, nrows, wbuf, cur);
+}
+
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_transposed(uint32_t t_row, const EpiArgs& ep, int64_t n0, int64_t N,
+                                                    int split, float* wbuf, int64_t row0, int64_t M,
+                                                    float (&nxt)[32]) {
+  const int lane = threadIdx.x & 31;
+  const int nrows = (int)(M - row0 < 32 ? (M - row0 > 0 ? M - row0 : 0) : 32);
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    float cur[32], v[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) cur[r] = nxt[r];
+    if (c + 32 < BN) epi_load_chunk<EPI>(ep, row0, M, n0 + c + 32 + lane, N, nxt);
+    ld32f(t_row + c, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) wbuf[lane * 33 + i] = v[i];
+    __syncwarp();
+    const int64_t col = n0 + c + lane;
+    if (col < N && nrows > 0) {
+      const bool full = nrows == 32;
+      if constexpr (EPI == EPI_SGD) {
+        if (ep.c3)
+          epi_store_dispatch_check<EPI, true, true>(ep, row0, col, split, nrows, full, wbuf, cur);
+        else if (ep.c2)
+          epi_store_dispatch_check<EPI, true, false>(ep, row0, col, split, nrows, full, wbuf, cur);
+        else
+          epi_store_dispatch_check<EPI, false, false>(ep, row0, col, split, nrows, full, wbuf, cur);
+      } else {
+        epi_store_dispatch_check<EPI, false, false>(ep, row0, col, split, nrows, full, wbuf, cur);
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -233,7 +295,7 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
 // A B^T (k-blocks KB1 .. KB1+KB2-1 of the concatenated reduction; B2's row is
 // n0 - n_ext).  The k-splits cut the concatenated range.
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2, int64_t M,
                    int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt, int n_split, EpiArgs ep,
@@ -368,20 +430,27 @@ __global__ void __launch_bounds__(192, 1)
       ptx::mbar_drain(drain, 0);  // no MMA may still write TMEM when it is released
     }
   } else {
-    const int q = warp & 3;
+    // epilogue group eg drains accumulator buffer eg: the units with it = eg, eg + 2, ...
+    const int ew = warp - 2, eg = ew >> 2;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    uint32_t it = 0;
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+    uint32_t it = (uint32_t)eg;
+    for (int64_t u = blockIdx.x + (int64_t)eg * gridDim.x; u < units; u += 2 * (int64_t)gridDim.x, it += 2) {
       int64_t m0, n0;
       int split, nkb, kb_begin;
       decode(u, m0, n0, split, nkb, kb_begin);
       const uint32_t b = it & 1u, use = it >> 1;
+      float nxt[32];
+      if constexpr (kTransposedEpi<EPI>) epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, nxt);  // prefetch
       const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));  // warp-uniform
       if (!ok) break;
       ptx::tc_fence_after();
       const int64_t row = m0 + q * 32 + lane;
-      epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split,
-                                  wbufs + q * 32 * 33, m0 + q * 32, M);
+      if constexpr (kTransposedEpi<EPI>)
+        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * 33, m0 + q * 32,
+                                     M, nxt);
+      else
+        epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split);
       ptx::tc_fence_before();
       ptx::mbar_arrive(&acc_empty[b]);
     }
@@ -618,7 +687,7 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   const int KB1 = (int)((g.K + BK - 1) / BK), KB2 = (int)((g.K2 + BK - 1) / BK);
   const int64_t n_ext = g.K2 > 0 ? g.n_ext : INT64_MAX;
   if (g.ksplit <= 1) {
-    fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1,
+    fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1,
                                     g.args, dev_err);
     TTT_CUDA_TRY(cudaGetLastError());
     return TTT_OK;
@@ -628,7 +697,7 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   part.c = g.ws;
   part.ldc = g.N;
   part.split_stride = g.M * g.N;
-  fn<<<grid, 192, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, (int)(g.kps / BK), n_mt, n_nt,
+  fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, (int)(g.kps / BK), n_mt, n_nt,
                                   g.ksplit, part, dev_err);
   TTT_CUDA_TRY(cudaGetLastError());
   const unsigned blocks = ceil_div(g.M * ((g.N + 3) / 4), 256);

@@ -60,6 +60,8 @@ def make_ops(cfg):
     gemm("gemm_dgrad_gateup", b, d, 4 * f, 0, 1, L.EPI_STORE_F32, c=torch.empty(b, d, device=dev))
     gemm("gemm_wgrad_gateup_sgd", 2 * f, d, b, 1, 1, L.EPI_SGD, c=torch.zeros(2 * f, d, device=dev),
          c2=torch.empty(2 * f, d, device=dev, dtype=bf), alpha=1e-2)
+    gemm("gemm_wgrad_gateup_store", 2 * f, d, b, 1, 1, L.EPI_STORE_F32, c=torch.zeros(2 * f, d, device=dev))
+    gemm("gemm_wgrad_gateup_kmajor_store", 2 * f, d, b, 0, 0, L.EPI_STORE_F32, c=torch.zeros(2 * f, d, device=dev))
     nt = ops.gemm_ce_tiles(True, b, V)
     tgt = torch.randint(0, V, (b,), device=dev, dtype=torch.int32)
     gemm("gemm_lmhead_ce_fwd", b, V, d, 0, 0, L.EPI_CE_FWD, row_i=tgt, part_max=torch.empty(nt, b, device=dev),
