@@ -289,13 +289,12 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;  // warp-uniform: TMEM loads follow
       ptx::tc_fence_after();
       float s[64];  // raw scores; the scale is folded into the exponent
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        uint32_t rr[32];
-        ptx::tmem_ld32(t_s0 + (j & 1) * 128 + 64 * g + c + lane_off, rr);
+      {
+        uint32_t rr[64];  // one TMEM round trip for the warp's 64 columns
+        ptx::tmem_ld64(t_s0 + (j & 1) * 128 + 64 * g + lane_off, rr);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c + i] = __uint_as_float(rr[i]);
+        for (int i = 0; i < 64; ++i) s[i] = __uint_as_float(rr[i]);
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&s_empty[j & 1]);
@@ -414,7 +413,6 @@ __global__ void __launch_bounds__(384, 1)
     ptx::tmem_dealloc(tmem, 512);
   }
 }
-
 
 // ---------------------------------------------------------------------------------------------
 // Backward, dq part: dQ = scale * sum_j dS_j K_j over the band, with

@@ -25,6 +25,9 @@ enum : int {
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 // ... or after this many polls of the barrier (each poll may suspend briefly).
 constexpr uint32_t kWaitLimitIters = 1u << 26;
+// Suspend hint of one poll of a bounded mbarrier wait (the thread resumes
+// earlier when the phase completes).
+constexpr uint32_t kWaitSleepNs = 20000;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
