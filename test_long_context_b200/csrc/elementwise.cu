@@ -2,6 +2,8 @@
 // uses one 128-thread block per row with float4 access (one warp per row when
 // the layout is not vector-aligned); everything else is one thread per
 // element or one warp per row.
+#include <algorithm>
+
 #include "elementwise.cuh"
 
 namespace ttt {
@@ -175,9 +177,6 @@ __global__ void __launch_bounds__(VT) rmsnorm_bwd_vec_kernel(const float* x, int
 
 __host__ __forceinline__ bool al(const void* p, int b) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) % b) == 0; }
 
-// One warp per (token, head); lane t handles rotation pairs t and t + 32.
-constexpr int MAXP = 2;  // pairs per lane (head_dim <= 128)
-
 // Rotation table of positions p0 .. p0+n-1: tab[i * HD/2 + t] = (cos, sin) of
 // (p0 + i) * theta^(-2t/HD), angles in fp64, stored as fp32.
 __global__ void rope_table_kernel(float2* tab, int64_t p0, int64_t n, int HD, double theta) {
@@ -192,115 +191,121 @@ __global__ void rope_table_kernel(float2* tab, int64_t p0, int64_t n, int HD, do
   tab[idx] = make_float2((float)cd, (float)sd);
 }
 
+// QK-norm + RoPE forward, one token per block iteration: the token's q and k
+// rows are staged in smem with 16-byte loads, four threads share a head (a
+// quarter of its rotation pairs each, sums of squares combined by shuffles),
+// and the results leave with 16-byte stores; v is copied to the ring with
+// 16-byte accesses.  Needs H * HD a multiple of 16 bytes' worth of elements.
+constexpr int ROPE_THREADS = 256;
+
 template <typename T>
-__global__ void qknorm_rope_fwd_kernel(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n,
-                                       int64_t p0, int H, int HD, float eps, const float2* tab, int64_t tab_p0,
-                                       T* qout, int64_t ldq, T* kring, T* vring, int64_t ldkv, int64_t R, float* rq,
-                                       float* rk) {
-  // one block per token, the position's row of the rotation table shared by
-  // all heads; warp w handles heads w, w + 8, ...
-  const int64_t i = blockIdx.x;
-  const int lane = threadIdx.x % 32;
-  const int h2 = HD / 2;
-  if (i >= n) return;
-  const float2* cs = tab + (p0 + i - tab_p0) * h2;
-  for (int h = threadIdx.x / 32; h < H; h += blockDim.x / 32) {
-  const int D = H * HD;
-  const T* q = qkv + i * ldqkv + h * HD;
-  const T* k = q + D;
-  const T* v = q + 2 * D;
-  float q1[MAXP], q2[MAXP], k1[MAXP], k2[MAXP];
-  float sq = 0.f, sk = 0.f;
-#pragma unroll
-  for (int u = 0; u < MAXP; ++u) {
-    const int t = lane + 32 * u;
-    q1[u] = q2[u] = k1[u] = k2[u] = 0.f;
-    if (t < h2) {
-      q1[u] = to_f32(q[t]);
-      q2[u] = to_f32(q[t + h2]);
-      k1[u] = to_f32(k[t]);
-      k2[u] = to_f32(k[t + h2]);
-      sq += q1[u] * q1[u] + q2[u] * q2[u];
-      sk += k1[u] * k1[u] + k2[u] * k2[u];
+__global__ void __launch_bounds__(ROPE_THREADS) qknorm_rope_fwd_kernel(
+    const T* __restrict__ qkv, int64_t ldqkv, const float* __restrict__ gq, const float* __restrict__ gk, int64_t n,
+    int64_t p0, int H, int HD, float eps, const float2* __restrict__ tab, int64_t tab_p0, T* __restrict__ qout,
+    int64_t ldq, T* __restrict__ kring, T* __restrict__ vring, int64_t ldkv, int64_t R, float* __restrict__ rq,
+    float* __restrict__ rk) {
+  extern __shared__ __align__(16) unsigned char rope_smem[];
+  T* row = reinterpret_cast<T*>(rope_smem);  // [2 * D]: q | k of one token
+  constexpr int EV = 16 / sizeof(T);          // elements per 16-byte vector
+  const int D = H * HD, h2 = HD / 2;
+  const int per = (h2 + 3) / 4;               // rotation pairs per thread
+  const int tasks = ((8 * H + 31) / 32) * 32; // (q or k head, quarter), padded to whole warps
+  for (int64_t i = blockIdx.x; i < n; i += gridDim.x) {
+    const T* src = qkv + i * ldqkv;
+    const int64_t slot = (p0 + i) % R;
+    for (int c = threadIdx.x; c < 2 * D / EV; c += blockDim.x)
+      reinterpret_cast<uint4*>(row)[c] = reinterpret_cast<const uint4*>(src)[c];
+    for (int c = threadIdx.x; c < D / EV; c += blockDim.x)
+      reinterpret_cast<uint4*>(vring + slot * ldkv)[c] = reinterpret_cast<const uint4*>(src + 2 * D)[c];
+    __syncthreads();
+    const float2* cs = tab + (p0 + i - tab_p0) * h2;
+    for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
+      const int hh = task / 4, part = task % 4;  // hh < H: q head hh; else k head hh - H
+      const bool live = hh < 2 * H;
+      const int t0 = part * per, t1 = live ? min(t0 + per, h2) : t0;
+      T* x = row + hh * HD;
+      float ss = 0.f;
+      for (int t = t0; t < t1; ++t) {
+        const float a = to_f32(x[t]), b = to_f32(x[t + h2]);
+        ss += a * a + b * b;
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+      if (!live) continue;
+      const float r = 1.f / sqrtf(ss / (float)HD + eps);
+      const float* g = hh < H ? gq : gk;
+      for (int t = t0; t < t1; ++t) {
+        const float2 c = cs[t];
+        const float a = to_f32(x[t]) * r * g[t], b = to_f32(x[t + h2]) * r * g[t + h2];
+        x[t] = from_f32<T>(a * c.x - b * c.y);
+        x[t + h2] = from_f32<T>(b * c.x + a * c.y);
+      }
+      if (part == 0) (hh < H ? rq : rk)[i * H + (hh < H ? hh : hh - H)] = r;
     }
-  }
-  sq = warp_sum(sq);
-  sk = warp_sum(sk);
-  const float rqv = 1.f / sqrtf(sq / (float)HD + eps);
-  const float rkv = 1.f / sqrtf(sk / (float)HD + eps);
-  const int64_t pos = p0 + i;
-  const int64_t slot = pos % R;
-  T* qo = qout + i * ldq + h * HD;
-  T* ko = kring + slot * ldkv + h * HD;
-  T* vo = vring + slot * ldkv + h * HD;
-#pragma unroll
-  for (int u = 0; u < MAXP; ++u) {
-    const int t = lane + 32 * u;
-    if (t < h2) {
-      const float2 csv = cs[t];
-      const float c = csv.x, s = csv.y;
-      const float a1 = q1[u] * rqv * gq[t], a2 = q2[u] * rqv * gq[t + h2];
-      const float b1 = k1[u] * rkv * gk[t], b2 = k2[u] * rkv * gk[t + h2];
-      qo[t] = from_f32<T>(a1 * c - a2 * s);
-      qo[t + h2] = from_f32<T>(a2 * c + a1 * s);
-      ko[t] = from_f32<T>(b1 * c - b2 * s);
-      ko[t + h2] = from_f32<T>(b2 * c + b1 * s);
+    __syncthreads();
+    for (int c = threadIdx.x; c < D / EV; c += blockDim.x) {
+      reinterpret_cast<uint4*>(qout + i * ldq)[c] = reinterpret_cast<const uint4*>(row)[c];
+      reinterpret_cast<uint4*>(kring + slot * ldkv)[c] = reinterpret_cast<const uint4*>(row + D)[c];
     }
-  }
-  for (int c = lane; c < HD; c += 32) vo[c] = v[c];
-  if (lane == 0) {
-    rq[i * H + h] = rqv;
-    rk[i * H + h] = rkv;
-  }
+    __syncthreads();
   }
 }
 
+// Backward of QK-norm + RoPE, in place on the q and k parts of dqkv, with the
+// same staging as the forward: the token's dq|dk and raw q|k rows in smem,
+// four threads per head.
 template <typename T>
-__global__ void qknorm_rope_bwd_kernel(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq,
-                                       const float* gk, const float* rq, const float* rk, int64_t n, int64_t p0,
-                                       int H, int HD, const float2* tab, int64_t tab_p0) {
-  // one block per token, the position's table row shared by the 2H (q, k) heads
-  const int64_t i = blockIdx.x;
-  const int lane = threadIdx.x % 32;
-  const int h2 = HD / 2;
-  if (i >= n) return;
-  const float2* cs = tab + (p0 + i - tab_p0) * h2;
-  for (int w = threadIdx.x / 32; w < 2 * H; w += blockDim.x / 32) {
-  const int which = w % 2;  // 0: q, 1: k
-  const int h = w / 2;
-  const int D = H * HD;
-  T* dv = dqkv + i * ld + which * D + h * HD;
-  const T* xv = qkv + i * ldqkv + which * D + h * HD;
-  const float* g = which ? gk : gq;
-  const float r = (which ? rk : rq)[i * H + h];
-  const int64_t pos = p0 + i;
-  float u1[MAXP], u2[MAXP], x1[MAXP], x2[MAXP];
-  float dot = 0.f;
-#pragma unroll
-  for (int u = 0; u < MAXP; ++u) {
-    const int t = lane + 32 * u;
-    u1[u] = u2[u] = x1[u] = x2[u] = 0.f;
-    if (t < h2) {
-      const float2 csv = cs[t];
-      const float c = csv.x, s = csv.y;
-      const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
-      // transpose of the rotation, then the gain
-      u1[u] = (d1 * c + d2 * s) * g[t];
-      u2[u] = (d2 * c - d1 * s) * g[t + h2];
-      x1[u] = to_f32(xv[t]) * r;
-      x2[u] = to_f32(xv[t + h2]) * r;
-      dot += x1[u] * u1[u] + x2[u] * u2[u];
+__global__ void __launch_bounds__(ROPE_THREADS) qknorm_rope_bwd_kernel(
+    T* __restrict__ dqkv, int64_t ld, const T* __restrict__ qkv, int64_t ldqkv, const float* __restrict__ gq,
+    const float* __restrict__ gk, const float* __restrict__ rq, const float* __restrict__ rk, int64_t n, int64_t p0,
+    int H, int HD, const float2* __restrict__ tab, int64_t tab_p0) {
+  extern __shared__ __align__(16) unsigned char rope_smem[];
+  const int D = H * HD, h2 = HD / 2;
+  T* drow = reinterpret_cast<T*>(rope_smem);  // [2 * D]: dq | dk
+  T* xrow = drow + 2 * D;                     // [2 * D]: raw q | k
+  constexpr int EV = 16 / sizeof(T);
+  const int per = (h2 + 3) / 4;
+  const int tasks = ((8 * H + 31) / 32) * 32;
+  for (int64_t i = blockIdx.x; i < n; i += gridDim.x) {
+    for (int c = threadIdx.x; c < 2 * D / EV; c += blockDim.x) {
+      reinterpret_cast<uint4*>(drow)[c] = reinterpret_cast<const uint4*>(dqkv + i * ld)[c];
+      reinterpret_cast<uint4*>(xrow)[c] = reinterpret_cast<const uint4*>(qkv + i * ldqkv)[c];
     }
-  }
-  dot = warp_sum(dot) / (float)HD;
-#pragma unroll
-  for (int u = 0; u < MAXP; ++u) {
-    const int t = lane + 32 * u;
-    if (t < h2) {
-      dv[t] = from_f32<T>(r * (u1[u] - x1[u] * dot));
-      dv[t + h2] = from_f32<T>(r * (u2[u] - x2[u] * dot));
+    __syncthreads();
+    const float2* cs = tab + (p0 + i - tab_p0) * h2;
+    for (int task = threadIdx.x; task < tasks; task += blockDim.x) {
+      const int hh = task / 4, part = task % 4;
+      const bool live = hh < 2 * H;
+      const int t0 = part * per, t1 = live ? min(t0 + per, h2) : t0;
+      const int h = hh < H ? hh : hh - H;
+      const float* g = hh < H ? gq : gk;
+      const float r = live ? (hh < H ? rq : rk)[i * H + h] : 0.f;
+      T* dv = drow + hh * HD;
+      const T* xv = xrow + hh * HD;
+      float dot = 0.f;
+      for (int t = t0; t < t1; ++t) {
+        const float2 c = cs[t];
+        const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
+        // transpose of the rotation, then the gain
+        const float u1 = (d1 * c.x + d2 * c.y) * g[t], u2 = (d2 * c.x - d1 * c.y) * g[t + h2];
+        dot += to_f32(xv[t]) * r * u1 + to_f32(xv[t + h2]) * r * u2;
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+      if (!live) continue;
+      const float dm = dot / (float)HD;
+      for (int t = t0; t < t1; ++t) {
+        const float2 c = cs[t];
+        const float d1 = to_f32(dv[t]), d2 = to_f32(dv[t + h2]);
+        const float u1 = (d1 * c.x + d2 * c.y) * g[t], u2 = (d2 * c.x - d1 * c.y) * g[t + h2];
+        dv[t] = from_f32<T>(r * (u1 - to_f32(xv[t]) * r * dm));
+        dv[t + h2] = from_f32<T>(r * (u2 - to_f32(xv[t + h2]) * r * dm));
+      }
     }
-  }
+    __syncthreads();
+    for (int c = threadIdx.x; c < 2 * D / EV; c += blockDim.x)
+      reinterpret_cast<uint4*>(dqkv + i * ld)[c] = reinterpret_cast<const uint4*>(drow)[c];
+    __syncthreads();
   }
 }
 
@@ -496,10 +501,19 @@ template <typename T>
 int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* gk, int64_t n, int64_t p0, int H,
                     int HD, float eps, const float2* tab, int64_t tab_p0, T* qout, int64_t ldq, T* kring, T* vring,
                     int64_t ldkv, int64_t R, float* rq, float* rk, cudaStream_t s) {
-  if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
+  if (HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: odd head_dim");
   if (n <= 0) return TTT_OK;
-  qknorm_rope_fwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, tab, tab_p0,
-                                                                   qout, ldq, kring, vring, ldkv, R, rq, rk);
+  constexpr int EV = 16 / (int)sizeof(T);
+  const int64_t D = (int64_t)H * HD;
+  const bool vec_ok = D % EV == 0 && ldqkv % EV == 0 && ldq % EV == 0 && ldkv % EV == 0 &&
+                      reinterpret_cast<uintptr_t>(qkv) % 16 == 0 && reinterpret_cast<uintptr_t>(qout) % 16 == 0 &&
+                      reinterpret_cast<uintptr_t>(kring) % 16 == 0 && reinterpret_cast<uintptr_t>(vring) % 16 == 0;
+  if (!vec_ok) return set_error(TTT_ERR_INVALID_ARG, "qknorm_rope: rows must be 16-byte aligned");
+  const size_t smem = 2 * (size_t)D * sizeof(T);
+  if (smem > 48 * 1024) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: q and k rows exceed 48 KB");
+  const unsigned grid = (unsigned)std::min<int64_t>(n, 148 * 8);
+  qknorm_rope_fwd_kernel<T><<<grid, ROPE_THREADS, smem, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, tab, tab_p0,
+                                                             qout, ldq, kring, vring, ldkv, R, rq, rk);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -508,10 +522,17 @@ template <typename T>
 int qknorm_rope_bwd(T* dqkv, int64_t ld, const T* qkv, int64_t ldqkv, const float* gq, const float* gk,
                     const float* rq, const float* rk, int64_t n, int64_t p0, int H, int HD, const float2* tab,
                     int64_t tab_p0, cudaStream_t s) {
-  if (HD / 2 > 32 * MAXP || HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: head_dim too large");
+  if (HD % 2) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: odd head_dim");
   if (n <= 0) return TTT_OK;
-  qknorm_rope_bwd_kernel<T><<<(unsigned)n, 32 * ROW_WARPS, 0, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n, p0, H,
-                                                                   HD, tab, tab_p0);
+  constexpr int EV = 16 / (int)sizeof(T);
+  const int64_t D = (int64_t)H * HD;
+  if (D % EV || ld % EV || ldqkv % EV || reinterpret_cast<uintptr_t>(dqkv) % 16 || reinterpret_cast<uintptr_t>(qkv) % 16)
+    return set_error(TTT_ERR_INVALID_ARG, "qknorm_rope_bwd: rows must be 16-byte aligned");
+  const size_t smem = 4 * (size_t)D * sizeof(T);
+  if (smem > 48 * 1024) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope_bwd: rows exceed 48 KB of smem");
+  const unsigned grid = (unsigned)std::min<int64_t>(n, 148 * 8);
+  qknorm_rope_bwd_kernel<T><<<grid, ROPE_THREADS, smem, s>>>(dqkv, ld, qkv, ldqkv, gq, gk, rq, rk, n, p0, H, HD, tab,
+                                                             tab_p0);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
