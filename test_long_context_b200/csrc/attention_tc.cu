@@ -417,34 +417,46 @@ __global__ void __launch_bounds__(384, 1)
 // ---------------------------------------------------------------------------------------------
 // Backward, dq part: dQ = scale * sum_j dS_j K_j over the band, with
 // dS = P o (dP - D), P = exp(S*scale - lse), S = Q K^T, dP = dO V^T.
-// CTA = 128 queries x one head; key tiles of 64 keys (2 K/V stages).
-//   warp 0      TMA: Q and dO once, then K/V tiles
+// CTA = 128 queries x one head; key tiles of 64 keys.
+//   warp 0      TMA: K tiles (ring of BNK, released after dQ_j) one tile ahead
+//               of V tiles (ring of BNV, released after dP_j)
 //   warp 1      TMEM owner; lane 0 issues S_j = Q K_j^T and dP_j = dO V_j^T into
 //               one of two TMEM buffers (64 + 64 columns), then dQ += dS_j K_j
-//   warps 4..7  one query row per thread: P, dS in fp32 -> bf16 dS tile in
-//               128B-swizzled smem (K-major A operand of the dQ product)
-// The softmax statistics come from the forward (lse), so there is no online
-// rescaling and every TMEM access is warp-uniform.
+//               as one MMA of N = head_dim per 16 keys.  Q and dO, the A
+//               operands of every S_j and dP_j, sit in TMEM (written once by
+//               the softmax warps), so the tensor core reads only K and V
+//               from shared memory for them.
+//   warps 4..11 two warpgroups taking alternate key tiles (warpgroup j & 1
+//               owns tile j, TMEM buffer j & 1 and dS buffer j & 1): thread =
+//               query row; P, dS in fp32 -> bf16 dS in a 128B-swizzled smem
+//               tile (K-major A operand of the dQ product).  The two
+//               warpgroups run one tile apart, so one computes while the other
+//               waits for its scores.
+// K and V tiles are staged as whole 128B-swizzled atoms (the last one partly
+// past the head), so that a K tile is both the K-major B operand of S and the
+// MN-major B operand of dQ.  The softmax statistics come from the forward (lse), so there
+// is no online rescaling and the tiles of a row are independent.
 constexpr int BKT = 64;  // keys per tile in the backward
-constexpr int BNST = 3;  // K/V stages in the backward (also keeps one CTA per SM: each takes all of TMEM)
+constexpr int BNK = 4;   // K stages
+constexpr int BNV = 3;   // V stages
 
 template <int HD>
 struct BGeo {
   static constexpr int A = HD / 64;
   static constexpr int R = HD % 64;
   static constexpr int RB = R * 2;
-  static constexpr int QTILE = 128 * HD * 2;   // Q or dO tile (128 rows)
-  static constexpr int KTILE = BKT * HD * 2;   // K or V tile (64 rows)
-  static constexpr int KREM = A * 8192;        // remainder offset inside a 64-row tile
-  static constexpr int QREM = A * 16384;       // remainder offset inside a 128-row tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int DO_OFF = QTILE;
-  static constexpr int KV_OFF = 2 * QTILE;     // stage s: K at KV_OFF + s*2*KTILE, V after
-  static constexpr int DS_OFF = KV_OFF + BNST * 2 * KTILE;
+  static constexpr int KA = (HD + 63) / 64;     // whole atoms of a K or V tile
+  static constexpr int KTILE = BKT * 128 * KA;  // K or V tile (64 rows, KA atoms)
+  static constexpr int QTILE = 128 * HD * 2;    // 128-row tile (the dk/dv kernel's layout)
+  static constexpr int QREM = A * 16384;        // remainder offset inside a 128-row tile
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + BNK * KTILE;
+  static constexpr int DS_OFF = V_OFF + BNV * KTILE;
   static constexpr int DS_BYTES = 128 * BKT * 2;  // one 128B-swizzled atom column (64 keys)
   static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
   static constexpr int SMEM = BAR_OFF + 256 + 1024;
-  static_assert(KTILE % 1024 == 0 && QTILE % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(KTILE % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(SMEM <= 232448, "shared memory per block");
 };
 
 template <int HD>
@@ -457,24 +469,23 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m64, 
 }
 
 template <int HD>
-__global__ void __launch_bounds__(256, 1)
-    swa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tq_r,
-                         const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tdo_r,
-                         const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tk_r,
-                         const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tv_r, SwaArgs a,
+__global__ void __launch_bounds__(384, 1)
+    swa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, SwaArgs a,
                          int* err) {
   using G = BGeo<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
-  uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [BNST]
-  uint64_t* kv_empty = bars + 4;  // [BNST]
-  uint64_t* s_full = bars + 7;    // [2]  S_j, dP_j in TMEM buffer j&1
-  uint64_t* ds_full = bars + 9;   // [2]  dS_j written (and TMEM buffer j&1 read)
-  uint64_t* ds_free = bars + 11;  // [2]  dQ_j consumed dS buffer j&1
-  uint64_t* dq_full = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* q_full = bars + 0;        // Q and dO written to TMEM
+  uint64_t* k_full = bars + 1;        // [BNK]
+  uint64_t* k_empty = k_full + BNK;   // [BNK]
+  uint64_t* v_full = k_empty + BNK;   // [BNV]
+  uint64_t* v_empty = v_full + BNV;   // [BNV]
+  uint64_t* s_full = v_empty + BNV;   // [2]  S_j, dP_j in TMEM buffer j&1
+  uint64_t* ds_full = s_full + 2;     // [2]  dS_j written (and TMEM buffer j&1 read)
+  uint64_t* ds_free = ds_full + 2;    // [2]  dQ_j consumed dS buffer j&1
+  uint64_t* dq_full = ds_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_full + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -486,10 +497,14 @@ __global__ void __launch_bounds__(256, 1)
   const int col0 = h * HD;
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(q_full, 1);
-    for (int s = 0; s < BNST; ++s) {
-      ptx::mbar_init(&kv_full[s], 1);
-      ptx::mbar_init(&kv_empty[s], 1);
+    ptx::mbar_init(q_full, 256);
+    for (int s = 0; s < BNK; ++s) {
+      ptx::mbar_init(&k_full[s], 1);
+      ptx::mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < BNV; ++s) {
+      ptx::mbar_init(&v_full[s], 1);
+      ptx::mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&s_full[s], 1);
@@ -508,124 +523,129 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_dq = tmem + 256;  // S/dP buffers at columns [0,128) and [128,256)
+  // TMEM: S/dP buffers at columns [0,128) and [128,256), dQ at 256, Q and dO (bf16 pairs) from 384
+  const uint32_t t_dq = tmem + 256, t_q = tmem + 384, t_do = t_q + HD / 2;
 
   if (warp == 0) {
     if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(q_full, 2 * G::QTILE);
-      const int qrow = (int)(q0 - a.p0);
-      load_rows<HD>(sm + G::Q_OFF, &tq, &tq_r, q_full, col0, qrow, 16384, G::QREM);
-      load_rows<HD>(sm + G::DO_OFF, &tdo, &tdo_r, q_full, col0, qrow, 16384, G::QREM);
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j % BNST;
-        if (!ptx::mbar_wait(&kv_empty[s], ((j / BNST) & 1) ^ 1, err)) break;
-        ptx::mbar_arrive_expect_tx(&kv_full[s], 2 * G::KTILE);
+      auto load_k = [&](int j) {
+        const int s = j % BNK;
+        if (!ptx::mbar_wait(&k_empty[s], ((j / BNK) & 1) ^ 1, err)) return false;
+        ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
         const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
-        uint8_t* kd = sm + G::KV_OFF + s * 2 * G::KTILE;
-        load_rows<HD>(kd, &tk, &tk_r, &kv_full[s], col0, slot, 8192, G::KREM);
-        load_rows<HD>(kd + G::KTILE, &tv, &tv_r, &kv_full[s], col0, slot, 8192, G::KREM);
+        uint8_t* kd = sm + G::K_OFF + s * G::KTILE;
+#pragma unroll
+        for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(kd + at * 8192, &tk, &k_full[s], col0 + 64 * at, slot);
+        return true;
+      };
+      bool ok = ntiles > 0 ? load_k(0) : true;
+      for (int j = 0; ok && j < ntiles; ++j) {
+        if (j + 1 < ntiles && !(ok = load_k(j + 1))) break;
+        const int s = j % BNV;
+        if (!(ok = ptx::mbar_wait(&v_empty[s], ((j / BNV) & 1) ^ 1, err))) break;
+        ptx::mbar_arrive_expect_tx(&v_full[s], G::KTILE);
+        const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
+        uint8_t* vd = sm + G::V_OFF + s * G::KTILE;
+#pragma unroll
+        for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(vd + at * 8192, &tv, &v_full[s], col0 + 64 * at, slot);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, BKT, false, false);
-      constexpr uint32_t id_q64 = ptx::idesc_bf16_f32(128, 64, false, true);
-      constexpr uint32_t id_qr = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
-      const uint32_t q_addr = ptx::smem_u32(sm + G::Q_OFF), do_addr = ptx::smem_u32(sm + G::DO_OFF);
-      constexpr uint32_t rl = rem_swizzle_layout(G::R);
+      constexpr uint32_t id_dq = ptx::idesc_bf16_f32(128, HD, false, true);
       bool ok = ptx::mbar_wait(q_full, 0, err);
       // S_j = Q K_j^T and dP_j = dO V_j^T into TMEM buffer j&1
       auto issue_s = [&](int j) {
-        const int s = j % BNST;
-        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::KTILE);
-        const uint32_t v_addr = k_addr + G::KTILE;
+        const int sk = j % BNK, sv = j % BNV;
+        if (!ptx::mbar_wait(&k_full[sk], (j / BNK) & 1, err)) return false;
+        if (!ptx::mbar_wait(&v_full[sv], (j / BNV) & 1, err)) return false;
+        ptx::tc_fence_after();
+        const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
+        const uint32_t v_addr = ptx::smem_u32(sm + G::V_OFF + sv * G::KTILE);
         const uint32_t dS = tmem + (j & 1) * 128, dP = dS + 64;
-        int step = 0;
 #pragma unroll
-        for (int at = 0; at < G::A; ++at)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk, ++step) {
-            ptx::umma_bf16(dS, sdesc(q_addr + at * 16384 + kk * 32, 16, 1024, 2),
-                           sdesc(k_addr + at * 8192 + kk * 32, 16, 1024, 2), id_s, step > 0);
-            ptx::umma_bf16(dP, sdesc(do_addr + at * 16384 + kk * 32, 16, 1024, 2),
-                           sdesc(v_addr + at * 8192 + kk * 32, 16, 1024, 2), id_s, step > 0);
-          }
-        if constexpr (G::R > 0) {
-#pragma unroll
-          for (int kk = 0; kk < G::R / 16; ++kk, ++step) {
-            ptx::umma_bf16(dS, sdesc(q_addr + G::QREM + kk * 32, 16, 8 * G::RB, rl),
-                           sdesc(k_addr + G::KREM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
-            ptx::umma_bf16(dP, sdesc(do_addr + G::QREM + kk * 32, 16, 8 * G::RB, rl),
-                           sdesc(v_addr + G::KREM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
-          }
+        for (int ks = 0; ks < HD / 16; ++ks) {  // K-steps of 16 along head_dim: atom ks / 4, offset ks % 4
+          const uint32_t boff = (ks / 4) * 8192 + (ks % 4) * 32;
+          ptx::umma_bf16_ts(dS, t_q + ks * 8, sdesc(k_addr + boff, 16, 1024, 2), id_s, ks > 0);
+          ptx::umma_bf16_ts(dP, t_do + ks * 8, sdesc(v_addr + boff, 16, 1024, 2), id_s, ks > 0);
         }
         ptx::umma_commit(&s_full[j & 1]);
+        ptx::umma_commit(&v_empty[sv]);  // V_j is not read again
+        return true;
       };
-      if (ok && ntiles > 0 && (ok = ptx::mbar_wait(&kv_full[0], 0, err))) {
-        ptx::tc_fence_after();
-        issue_s(0);
-      }
+      if (ok && ntiles > 0) ok = issue_s(0);
       for (int j = 0; ok && j < ntiles; ++j) {
         // TMEM buffer (j+1)&1 was read by the softmax of tile j-1 (waited below in the previous iteration)
-        if (j + 1 < ntiles) {
-          if (!(ok = ptx::mbar_wait(&kv_full[(j + 1) % BNST], ((j + 1) / BNST) & 1, err))) break;
-          ptx::tc_fence_after();
-          issue_s(j + 1);
-        }
+        if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
         if (!(ok = ptx::mbar_wait(&ds_full[j & 1], (j / 2) & 1, err))) break;
         ptx::tc_fence_after();
-        const int s = j % BNST;
-        const uint32_t k_addr = ptx::smem_u32(sm + G::KV_OFF + s * 2 * G::KTILE);
+        const int sk = j % BNK;
+        const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
         const uint32_t ds_addr = ptx::smem_u32(sm + G::DS_OFF + (j & 1) * G::DS_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKT / 16; ++kk) {  // dQ += dS_j K_j, K over the 64 keys
-          const uint64_t ad = sdesc(ds_addr + kk * 32, 16, 1024, 2);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
-#pragma unroll
-          for (int at = 0; at < G::A; ++at)
-            ptx::umma_bf16(t_dq + 64 * at, ad, sdesc(k_addr + at * 8192 + kk * 2048, 16, 1024, 2), id_q64, acc);
-          if constexpr (G::R > 0)
-            ptx::umma_bf16(t_dq + 64 * G::A, ad, sdesc(k_addr + G::KREM + kk * 16 * G::RB, 16, 8 * G::RB, rl),
-                           id_qr, acc);
-        }
-        ptx::umma_commit(&kv_empty[s]);
+        for (int kk = 0; kk < BKT / 16; ++kk)  // dQ += dS_j K_j; K MN-major: atoms 8192 bytes apart (LBO)
+          ptx::umma_bf16(t_dq, sdesc(ds_addr + kk * 32, 16, 1024, 2), sdesc(k_addr + kk * 2048, 8192, 1024, 2),
+                         id_dq, (j > 0 || kk > 0) ? 1u : 0u);
+        ptx::umma_commit(&k_empty[sk]);
         ptx::umma_commit(&ds_free[j & 1]);
       }
       ptx::umma_commit(dq_full);
       ptx::mbar_drain(dq_full, 0);
     }
   } else if (warp >= 4) {
-    const int r = (warp - 4) * 32 + lane;
+    const int g = (warp - 4) >> 2;  // this warpgroup takes tiles g, g + 2, ...
+    const int q = warp & 3;         // TMEM lane quarter
+    const int r = q * 32 + lane;
     const int64_t p = q0 + r;
     const bool row_ok = p <= qlast;
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const float L2E = 1.4426950408889634f;
     const float sl2 = a.scale * L2E;
     const int64_t i = p - a.p0;
     const float lse2 = row_ok ? a.lse[(int64_t)h * a.ld_lse + i] * L2E : 0.f;
     const float Di = row_ok ? a.D[(int64_t)h * a.ld_lse + i] : 0.f;
+    {  // warpgroup 0 writes this row of Q, warpgroup 1 the row of dO, as packed bf16 pairs
+      const bf16* src = g == 0 ? reinterpret_cast<const bf16*>(a.q) + i * a.ldq + col0
+                               : reinterpret_cast<const bf16*>(a.dout) + i * a.lddo + col0;
+      const uint32_t dst = (g == 0 ? t_q : t_do) + lane_off;
+#pragma unroll
+      for (int c = 0; c < HD / 2; c += 8) {  // 8 columns = 16 bf16 = two 16-byte loads
+        uint32_t w[8];
+        uint4 u0 = make_uint4(0u, 0u, 0u, 0u), u1 = u0;
+        if (row_ok) {
+          u0 = *reinterpret_cast<const uint4*>(src + 2 * c);
+          u1 = *reinterpret_cast<const uint4*>(src + 2 * c + 8);
+        }
+        w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
+        w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+        ptx::tmem_st8(dst + c, w);
+      }
+      tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(q_full);
+    }
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    for (int j = g; j < ntiles; j += 2) {
       const int64_t j0 = j_begin + (int64_t)j * BKT;
-      ok = ptx::mbar_wait(&s_full[j & 1], (j / 2) & 1, err);
+      ok = ptx::mbar_wait(&s_full[g], (j / 2) & 1, err);
       if (!__all_sync(0xffffffffu, ok)) break;
       ptx::tc_fence_after();
       float sv[BKT], dp[BKT];
-#pragma unroll
-      for (int c = 0; c < BKT; c += 32) {
-        uint32_t rs[32], rd[32];
-        ptx::tmem_ld32(tmem + (j & 1) * 128 + c + lane_off, rs);
-        ptx::tmem_ld32(tmem + (j & 1) * 128 + 64 + c + lane_off, rd);
+      {
+        uint32_t rs[64], rd[64];
+        ptx::tmem_ld64(tmem + g * 128 + lane_off, rs);
+        ptx::tmem_ld64(tmem + g * 128 + 64 + lane_off, rd);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          sv[c + e] = __uint_as_float(rs[e]);
-          dp[c + e] = __uint_as_float(rd[e]);
+        for (int e = 0; e < BKT; ++e) {
+          sv[e] = __uint_as_float(rs[e]);
+          dp[e] = __uint_as_float(rd[e]);
         }
       }
       ptx::tc_fence_before();
-      if (j >= 2) {  // dS buffer j&1 is free once dQ_{j-2} consumed it
-        ok = ptx::mbar_wait(&ds_free[j & 1], ((j - 2) / 2) & 1, err);
+      if (j >= 2) {  // dS buffer g is free once dQ_{j-2} consumed it
+        ok = ptx::mbar_wait(&ds_free[g], ((j - 2) / 2) & 1, err);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
       const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
@@ -633,13 +653,13 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
         for (int c = 0; c < BKT; ++c) sv[c] = (row_ok && c >= lo && c <= hi) ? sv[c] : -INFINITY;
       }
-      uint8_t* drow = sm + G::DS_OFF + (j & 1) * G::DS_BYTES + r * 128;
+      uint8_t* drow = sm + G::DS_OFF + g * G::DS_BYTES + r * 128;
 #pragma unroll
-      for (int g = 0; g < BKT / 8; ++g) {
+      for (int gg = 0; gg < BKT / 8; ++gg) {  // granules of 8 keys
         float ds[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const int c = g * 8 + e;
+          const int c = gg * 8 + e;
           const float pr = ex2(fmaf(sv[c], sl2, -lse2));
           ds[e] = pr * (dp[c] - Di);
         }
@@ -650,18 +670,19 @@ __global__ void __launch_bounds__(256, 1)
         w.y = *reinterpret_cast<uint32_t*>(&b1);
         w.z = *reinterpret_cast<uint32_t*>(&b2);
         w.w = *reinterpret_cast<uint32_t*>(&b3);
-        *reinterpret_cast<uint4*>(drow + ((g ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4*>(drow + ((gg ^ (r & 7)) << 4)) = w;
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&ds_full[j & 1]);
+      ptx::mbar_arrive(&ds_full[g]);
     }
     if (ok) ok = ptx::mbar_wait(dq_full, 0, err);
     if (__all_sync(0xffffffffu, ok)) {
       ptx::tc_fence_after();
       bf16* out = reinterpret_cast<bf16*>(a.dq) + i * a.lddq + col0;
+      // warpgroup g writes the 16-column groups of parity g
 #pragma unroll
-      for (int c = 0; c < HD; c += 16) {
+      for (int c = 16 * g; c < HD; c += 32) {
         uint32_t o[16];
         tmem_ld16(t_dq + c + lane_off, o);
         ptx::tmem_ld_wait();
@@ -1042,7 +1063,7 @@ int launch_bwd_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* 
     }
   }
   dim3 grid(ceil_div(a.n, QT), a.heads);
-  fn<<<grid, 256, G::SMEM, s>>>(p.q128, p.qr, p.do128, p.dor, p.k64, p.kr, p.v64, p.vr, a, err);
+  fn<<<grid, 384, G::SMEM, s>>>(p.k64, p.v64, a, err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
