@@ -298,7 +298,8 @@ template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                    const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2, int64_t M,
-                   int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt, int n_split, EpiArgs ep,
+                   int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt, int n_split, int n_fast,
+                   EpiArgs ep,
                    int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -316,10 +317,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t units = (int64_t)n_mt * n_nt * n_split;
   // k-blocks [kb_begin, kb_begin + nkb) of this unit's concatenated reduction
+  // Raster: m-tile fastest (CTAs running together share B tiles: large weights,
+  // few rows) or n-tile fastest (they share A tiles: B small enough to stay in
+  // L2 while A streams through once).
   auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int& kb_begin) {
-    m0 = (u % n_mt) * BM;
-    const int64_t nt = (u / n_mt) % n_nt;
-    n0 = nt * BN;
+    const int64_t mn = u % ((int64_t)n_mt * n_nt);
+    m0 = (n_fast ? mn / n_nt : mn % n_mt) * BM;
+    n0 = (n_fast ? mn % n_nt : mn / n_mt) * BN;
     split = (int)(u / ((int64_t)n_mt * n_nt));
     const int total = KB1 + (n0 >= n_ext ? KB2 : 0);
     kb_begin = split * kpsb;
@@ -501,7 +505,7 @@ int make_tmap(CUtensorMap* tm, const MatView& v, int box_rows) {
 }
 
 using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, int64_t, int64_t, int, int, int64_t, int,
-                          int, int, int, EpiArgs, int*);
+                          int, int, int, int, EpiArgs, int*);
 
 // Sum of split-K partials in a fixed order (deterministic), then the epilogue.
 template <int EPI>
@@ -685,9 +689,12 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   }
   const dim3 grid((unsigned)std::min<int64_t>(units, n_sm));
   const int KB1 = (int)((g.K + BK - 1) / BK), KB2 = (int)((g.K2 + BK - 1) / BK);
+  // n-tile fastest when B (N x K, plus a second product) fits comfortably in L2 and A is the larger operand
+  const double a_bytes = 2.0 * (double)g.M * (double)(g.K + g.K2), b_bytes = 2.0 * (double)g.N * (double)(g.K + g.K2);
+  const int n_fast = (b_bytes <= 48e6 && a_bytes > b_bytes) ? 1 : 0;
   const int64_t n_ext = g.K2 > 0 ? g.n_ext : INT64_MAX;
   if (g.ksplit <= 1) {
-    fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1,
+    fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1, n_fast,
                                     g.args, dev_err);
     TTT_CUDA_TRY(cudaGetLastError());
     return TTT_OK;
@@ -698,7 +705,7 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   part.ldc = g.N;
   part.split_stride = g.M * g.N;
   fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, (int)(g.kps / BK), n_mt, n_nt,
-                                  g.ksplit, part, dev_err);
+                                  g.ksplit, n_fast, part, dev_err);
   TTT_CUDA_TRY(cudaGetLastError());
   const unsigned blocks = ceil_div(g.M * ((g.N + 3) / 4), 256);
   switch (g.epi) {
