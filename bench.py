@@ -104,6 +104,27 @@ def traffic_for(kc, workload):
     return e.get("dram_bytes_per_launch")
 
 
+def rank_tokens(cfg, T, rank):
+    """Replica `rank`'s synthetic sequence: an independent problem with its own seed."""
+    import synth
+    return synth.tokens(cfg, T, seed=cfg.seed + 7919 * rank)
+
+
+def max_over_ranks(x, dist, world, device):
+    """Largest value of x over the ranks (the job's time is its slowest rank's)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world, steps, T, ms):
+    """Whole-job throughput: every rank prefills `steps` sequences of T tokens."""
+    return world * steps * T / (ms / 1000.0)
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons while running."""
 
@@ -245,7 +266,7 @@ def main():
         gw.update(upload_weights([(name, arr, bits)], cfg.dtype))
         if want_cpu:
             keep[name] = arr
-    toks = synth.tokens(cfg, T, seed=cfg.seed + 7919 * rank)
+    toks = rank_tokens(cfg, T, rank)
     tok_dev = torch.from_numpy(toks).cuda()
     stream = torch.cuda.current_stream()
     ctx = Context(cfg, gw, stream=stream)
@@ -284,10 +305,7 @@ def main():
     launches = ctx.launch_count() - n0
     timing = ctx.timing_read()
     ctx.timing_enable(False)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist, world, "cuda")
 
     # end to end through the public API: pinned host tokens in, losses out
     e2e = None
@@ -307,18 +325,14 @@ def main():
         e1.record(stream)
         ctx.sync()
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": world * args.steps * T / (ems / 1000.0), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), dist, world, "cuda")
+        e2e = {"value": aggregate_tokens_per_s(world, args.steps, T, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(tok_host.numel() * 4), "d2h_bytes_per_step": int(loss_host.numel() * 4),
                "ms_per_step": ems / args.steps}
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        value = world * args.steps * T / (ms / 1000.0)
+        value = aggregate_tokens_per_s(world, args.steps, T, ms)
         flops_step = algorithmic_flops(cfg, T)
         tensor_peak = peaks["bf16_tflops_sustained"]
         classes = {}
@@ -330,9 +344,8 @@ def main():
         dom = max(KC_NAMES[:3], key=lambda n: timing[n][0])
         tms, tn, tfl = timing[dom]
         achieved = tfl / (tms / 1000.0) / 1e12
-        simt_attn = dom.startswith("attn")
-        if simt_attn:
-            # SIMT fp32 FMA kernels: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock
+        if cfg.dtype == "f32":
+            # fp32 mode runs SIMT FMA kernels: 148 SMs x 128 FP32 lanes x 2 flop x max SM clock
             peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
             bound, note = "alu", "fp32 FMA peak from unit counts and the max SM clock"
         else:
