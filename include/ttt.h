@@ -170,8 +170,11 @@ void ttt_free(ttt_ctx* ctx);
 int64_t ttt_launch_count(ttt_ctx* ctx);
 
 /* ---- optional per-kernel-class timing ----
- * When enabled, every launch is bracketed by CUDA events recorded on the
- * context's stream, and the launch's algorithmic work is accumulated:
+ * When enabled, a CUDA event is recorded on the context's stream after every
+ * launch (and before the first launch of each ttt_prefill / ttt_reset call);
+ * a launch's time runs from the event before it to the event after it, so
+ * back-to-back launches share one event per boundary.  The launch's
+ * algorithmic work is accumulated:
  *   GEMM: 2*M*N*K flops;  ATTN_FWD: 4 * d_model * (query-key pairs admitted by
  *   the window, eq. (1));  ATTN_BWD: 4 * d_model * (band pairs + causal pairs
  *   among the chunk's own positions).  OTHER: memory-bound kernels (no flops).

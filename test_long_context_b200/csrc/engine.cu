@@ -92,13 +92,18 @@ struct Gemm {
   const char* label = "gemm";
 };
 
-// Event-pair timing of launches, per kernel class (opt-in).
+// Event timing of launches, per kernel class (opt-in).  Back-to-back launches
+// share one event per boundary: a launch's start is the previous launch's end
+// event while nothing else was enqueued in between (`chain`), so a launch costs
+// one event record instead of two and the per-launch times add up to the
+// stream's elapsed time.
 struct LaunchTimer {
   struct Rec {
     int kc;
     cudaEvent_t a, b;
     double flops;
     std::string label;
+    bool own_a;  // `a` was recorded for this launch (else it is the previous launch's `b`)
   };
   struct Stat {
     double ms = 0, flops = 0;
@@ -109,15 +114,19 @@ struct LaunchTimer {
   bool on = false;
   std::vector<Rec> pending;
   std::vector<cudaEvent_t> pool;
+  cudaEvent_t chain = nullptr;  // end event of the last timed launch, if it is the stream's last operation
   double ms[TTT_KC_COUNT] = {}, flops[TTT_KC_COUNT] = {};
   int64_t n[TTT_KC_COUNT] = {};
   ~LaunchTimer() {
     for (auto& r : pending) {
-      cudaEventDestroy(r.a);
+      if (r.own_a) cudaEventDestroy(r.a);
       cudaEventDestroy(r.b);
     }
     for (auto e : pool) cudaEventDestroy(e);
   }
+  // Something other than a timed launch is about to be enqueued: the next
+  // timed launch records its own start event.
+  void cut() { chain = nullptr; }
   cudaEvent_t get() {
     if (!pool.empty()) {
       cudaEvent_t e = pool.back();
@@ -141,10 +150,11 @@ struct LaunchTimer {
         st.flops += r.flops;
         st.n += 1;
       }
-      pool.push_back(r.a);
+      if (r.own_a) pool.push_back(r.a);
       pool.push_back(r.b);
     }
     pending.clear();
+    chain = nullptr;  // its event is back in the pool
     return TTT_OK;
   }
   void clear() {
@@ -215,13 +225,19 @@ class Engine final : public ttt_ctx {
     if (trace_) return traced(kc, f);
     if (!timer_.on) return f();
     static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope"};
-    cudaEvent_t a = timer_.get(), b = timer_.get();
-    TTT_CUDA_TRY(cudaEventRecord(a, st_));
+    cudaEvent_t a = timer_.chain;
+    const bool own_a = a == nullptr;
+    if (own_a) {
+      a = timer_.get();
+      TTT_CUDA_TRY(cudaEventRecord(a, st_));
+    }
     const int rc = f();
+    cudaEvent_t b = timer_.get();
     TTT_CUDA_TRY(cudaEventRecord(b, st_));
+    timer_.chain = b;
     std::string lab;
     if (timer_.labels) lab = label ? std::string(label) : std::string(phase_) + "." + names[kc];
-    timer_.pending.push_back({kc, a, b, flops, std::move(lab)});
+    timer_.pending.push_back({kc, a, b, flops, std::move(lab), own_a});
     return rc;
   }
   // TTT_TRACE=1: synchronise after every launch and log it to stderr (debugging aid).
@@ -669,6 +685,7 @@ int Engine<T>::reset() {
   const int64_t d = d_, f = f_;
   for (int i = 0; i < nu_; ++i) {
     const int64_t l = nbot_ + i;
+    timer_.cut();
     TTT_CUDA_TRY(cudaMemcpyAsync(master_gu(i), init_gu_[i], 2 * f * d * sizeof(float), cudaMemcpyDeviceToDevice, st_));
     TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d<float>(init_d_[i], f, master_d(i), master_d_ld(), d, f, st_); }));
     if (BF) {
@@ -813,6 +830,7 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
   if (!tok || !losses || T_ < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_prefill: bad argument");
   fresh_ = false;
   phase_ = "misc";
+  timer_.cut();  // the caller may have enqueued work on the stream since the last call
   TRY(timed(TTT_KC_OTHER, 0, [&] { return check_tokens(tok, T_, (int)V_, err_, st_); }));
   for (int64_t s0 = 0; s0 < T_; s0 += S_) {
     const int64_t S = std::min<int64_t>(S_, T_ - s0);

@@ -170,25 +170,38 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
 // EPI_SGD) go through a per-warp transpose so that global accesses run along
 // rows with lane = column (coalesced 128-byte lines).  The warp owns rows
 // row0 .. row0+31 of the tile.  Its read source (the residual or the master)
-// does not depend on the accumulator, so the first 32-column chunk is loaded
-// before the accumulator is ready and each later chunk one chunk ahead: with
-// 32 independent loads per lane in flight the epilogue is not bound by DRAM
-// latency.
+// does not depend on the accumulator, so it is read ahead: two register
+// buffers of one 32 x 32 chunk each alternate between the even and the odd
+// chunks, the first two chunks are loaded before the accumulator is ready,
+// and each row's value for the chunk two steps ahead is loaded as soon as
+// that row's current value has been used.  Two chunks of loads (8 KB per
+// warp) stay in flight through the whole tile, which the HBM-bound SGD
+// epilogue needs to keep enough bytes in flight per SM.
 template <int EPI>
 constexpr bool kTransposedEpi = EPI == EPI_STORE_F32 || EPI == EPI_ADD_F32 || EPI == EPI_SGD;
 
 template <int EPI>
+constexpr bool kEpiReads = EPI == EPI_ADD_F32 || EPI == EPI_SGD;
+
+// Read source of a read-modify-write epilogue and its leading dimension.
+template <int EPI>
+__device__ __forceinline__ const float* epi_src(const EpiArgs& ep, int64_t& ld) {
+  ld = ep.ldc;
+  if constexpr (EPI == EPI_ADD_F32) {
+    if (ep.c2) {
+      ld = ep.ldc2;
+      return reinterpret_cast<const float*>(ep.c2);
+    }
+  }
+  return reinterpret_cast<const float*>(ep.c);
+}
+
+template <int EPI>
 __device__ __forceinline__ void epi_load_chunk(const EpiArgs& ep, int64_t row0, int64_t M, int64_t col, int64_t N,
                                                float (&dst)[32]) {
-  if constexpr (EPI == EPI_ADD_F32 || EPI == EPI_SGD) {
-    const float* src = reinterpret_cast<const float*>(ep.c);
-    int64_t ld = ep.ldc;
-    if constexpr (EPI == EPI_ADD_F32) {
-      if (ep.c2) {
-        src = reinterpret_cast<const float*>(ep.c2);
-        ld = ep.ldc2;
-      }
-    }
+  if constexpr (kEpiReads<EPI>) {
+    int64_t ld;
+    const float* src = epi_src<EPI>(ep, ld);
     const int nrows = (int)(M - row0 < 32 ? M - row0 : 32);
     const float* p = src + row0 * ld + col;
     if (col < N && nrows == 32) {
@@ -202,13 +215,17 @@ __device__ __forceinline__ void epi_load_chunk(const EpiArgs& ep, int64_t row0, 
   }
 }
 
-// Writes one 32 x 32 chunk (rows row0.., columns col - lane ..) from the
-// transposed accumulator in wbuf; `cur` holds the chunk's read source.
+// One 32 x 32 chunk (rows row0.., column col of this lane): writes it from the
+// transposed accumulator in wbuf when `store`, with buf[r] as row r's read
+// source; then, when `nsrc` is set (this lane's column two chunks ahead,
+// already offset to row0), refills buf[r] from it right after its use.
 template <int EPI, bool CHECK, bool HI, bool LO>
-__device__ __forceinline__ void epi_store_chunk(const EpiArgs& ep, int64_t row0, int64_t col, int split, int nrows,
-                                                const float* wbuf, const float (&cur)[32]) {
+__device__ __forceinline__ void epi_chunk(const EpiArgs& ep, int64_t row0, int64_t col, int split, int nrows,
+                                          bool store, const float* wbuf, float (&buf)[32], const float* nsrc,
+                                          int64_t nld) {
   const int lane = threadIdx.x & 31;
   if constexpr (EPI == EPI_STORE_F32) {
+    if (!store) return;
     float* p = reinterpret_cast<float*>(ep.c) + (int64_t)split * ep.split_stride + row0 * ep.ldc + col;
 #pragma unroll
     for (int r = 0; r < 32; ++r, p += ep.ldc)
@@ -216,16 +233,18 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs& ep, int64_t row0,
   } else if constexpr (EPI == EPI_ADD_F32) {
     float* p = reinterpret_cast<float*>(ep.c) + row0 * ep.ldc + col;
 #pragma unroll
-    for (int r = 0; r < 32; ++r, p += ep.ldc)
-      if (!CHECK || r < nrows) *p = cur[r] + wbuf[r * 33 + lane];
+    for (int r = 0; r < 32; ++r, p += ep.ldc) {
+      if (store && (!CHECK || r < nrows)) *p = buf[r] + wbuf[r * 33 + lane];
+      if (nsrc) buf[r] = (!CHECK || r < nrows) ? nsrc[r * nld] : 0.f;
+    }
   } else {  // EPI_SGD
     float* p = reinterpret_cast<float*>(ep.c) + row0 * ep.ldc + col;
     bf16* ph = HI ? reinterpret_cast<bf16*>(ep.c2) + row0 * ep.ldc2 + col : nullptr;
     bf16* pl = LO ? reinterpret_cast<bf16*>(ep.c3) + row0 * ep.ldc3 + col : nullptr;
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      if (!CHECK || r < nrows) {
-        const float w = cur[r] - ep.alpha * wbuf[r * 33 + lane];
+      if (store && (!CHECK || r < nrows)) {
+        const float w = buf[r] - ep.alpha * wbuf[r * 33 + lane];
         *p = w;
         if constexpr (HI) {
           const bf16 hi = __float2bfloat16_rn(w);
@@ -233,6 +252,7 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs& ep, int64_t row0,
           if constexpr (LO) *pl = __float2bfloat16_rn(w - __bfloat162float(hi));
         }
       }
+      if (nsrc) buf[r] = (!CHECK || r < nrows) ? nsrc[r * nld] : 0.f;
       p += ep.ldc;
       if constexpr (HI) ph += ep.ldc2;
       if constexpr (LO) pl += ep.ldc3;
@@ -241,46 +261,58 @@ __device__ __forceinline__ void epi_store_chunk(const EpiArgs& ep, int64_t row0,
 }
 
 template <int EPI, bool HI, bool LO>
-__device__ __forceinline__ void epi_store_dispatch_check(const EpiArgs& ep, int64_t row0, int64_t col, int split,
-                                                         int nrows, bool full, const float* wbuf,
-                                                         const float (&cur)[32]) {
-  if (full)
-    epi_store_chunk<EPI, false, HI, LO>(ep, row0, col, split, nrows, wbuf, cur);
+__device__ __forceinline__ void epi_chunk_check(const EpiArgs& ep, int64_t row0, int64_t col, int split, int nrows,
+                                                bool store, const float* wbuf, float (&buf)[32], const float* nsrc,
+                                                int64_t nld) {
+  if (nrows == 32)
+    epi_chunk<EPI, false, HI, LO>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, nld);
   else
-    epi_store_chunk<EPI, true, HI, LO>(ep, row0, col, split, nrows, wbuf, cur);
+    epi_chunk<EPI, true, HI, LO>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, nld);
 }
 
+// bufA / bufB hold the read source of chunks 0 and 1 on entry.
 template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_transposed(uint32_t t_row, const EpiArgs& ep, int64_t n0, int64_t N,
                                                     int split, float* wbuf, int64_t row0, int64_t M,
-                                                    float (&nxt)[32]) {
+                                                    float (&bufA)[32], float (&bufB)[32]) {
+  static_assert(BN % 64 == 0, "chunks come in pairs");
   const int lane = threadIdx.x & 31;
   const int nrows = (int)(M - row0 < 32 ? (M - row0 > 0 ? M - row0 : 0) : 32);
-#pragma unroll 1
-  for (int c = 0; c < BN; c += 32) {
-    float cur[32], v[32];
-#pragma unroll
-    for (int r = 0; r < 32; ++r) cur[r] = nxt[r];
-    if (c + 32 < BN) epi_load_chunk<EPI>(ep, row0, M, n0 + c + 32 + lane, N, nxt);
+  int64_t ld = 0;
+  const float* src = nullptr;
+  if constexpr (kEpiReads<EPI>) src = epi_src<EPI>(ep, ld);
+  auto step = [&](int c, float(&buf)[32]) {
+    float v[32];
     ld32f(t_row + c, v);
 #pragma unroll
     for (int i = 0; i < 32; ++i) wbuf[lane * 33 + i] = v[i];
     __syncwarp();
     const int64_t col = n0 + c + lane;
-    if (col < N && nrows > 0) {
-      const bool full = nrows == 32;
-      if constexpr (EPI == EPI_SGD) {
-        if (ep.c3)
-          epi_store_dispatch_check<EPI, true, true>(ep, row0, col, split, nrows, full, wbuf, cur);
-        else if (ep.c2)
-          epi_store_dispatch_check<EPI, true, false>(ep, row0, col, split, nrows, full, wbuf, cur);
-        else
-          epi_store_dispatch_check<EPI, false, false>(ep, row0, col, split, nrows, full, wbuf, cur);
-      } else {
-        epi_store_dispatch_check<EPI, false, false>(ep, row0, col, split, nrows, full, wbuf, cur);
-      }
+    const bool store = col < N && nrows > 0;
+    const float* nsrc = nullptr;
+    if constexpr (kEpiReads<EPI>) {
+      if (c + 64 < BN && col + 64 < N && nrows > 0) nsrc = src + row0 * ld + col + 64;
+    }
+    if constexpr (EPI == EPI_SGD) {
+      if (ep.c3)
+        epi_chunk_check<EPI, true, true>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, ld);
+      else if (ep.c2)
+        epi_chunk_check<EPI, true, false>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, ld);
+      else
+        epi_chunk_check<EPI, false, false>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, ld);
+    } else {
+      epi_chunk_check<EPI, false, false>(ep, row0, col, split, nrows, store, wbuf, buf, nsrc, ld);
     }
     __syncwarp();
+  };
+  // one chunk per iteration: the two buffers alternate by branch, so that the
+  // compiler cannot overlap two chunks' accumulator registers
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    if ((c & 32) == 0)
+      step(c, bufA);
+    else
+      step(c, bufB);
   }
 }
 
@@ -444,15 +476,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int split, nkb, kb_begin;
       decode(u, m0, n0, split, nkb, kb_begin);
       const uint32_t b = it & 1u, use = it >> 1;
-      float nxt[32];
-      if constexpr (kTransposedEpi<EPI>) epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, nxt);  // prefetch
+      float bufA[32], bufB[32];
+      if constexpr (kTransposedEpi<EPI>) {  // read source of the first two chunks, ahead of the accumulator
+        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
+        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+      }
       const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));  // warp-uniform
       if (!ok) break;
       ptx::tc_fence_after();
       const int64_t row = m0 + q * 32 + lane;
       if constexpr (kTransposedEpi<EPI>)
         epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * 33, m0 + q * 32,
-                                     M, nxt);
+                                     M, bufA, bufB);
       else
         epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split);
       ptx::tc_fence_before();
@@ -508,20 +543,31 @@ using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, in
                           int, int, int, int, EpiArgs, int*);
 
 // Sum of split-K partials in a fixed order (deterministic), then the epilogue.
+// A thread owns 4 consecutive columns of one row; when they are 16-byte aligned
+// and all inside the row, the S partials are read as float4, all loads issued
+// before the (in-order) sum so that up to 8 are in flight per thread.
 template <int EPI>
-__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int S, int64_t M, int64_t N, int64_t stride,
-                                     EpiArgs ep) {
-  const int64_t gpr = (N + 3) / 4;  // 4-column groups per row
-  const int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gi >= M * gpr) return;
-  const int64_t row = gi / gpr, col = (gi % gpr) * 4;
-  float v[4] = {0.f, 0.f, 0.f, 0.f};
-  const int cnt = (int)imin64(4, N - col);
-  for (int s = 0; s < S; ++s) {
-    const float* p = ws + s * stride + row * N + col;
-    for (int e = 0; e < cnt; ++e) v[e] += p[e];
+__device__ __forceinline__ void splitk_out(const EpiArgs& ep, int64_t row, int64_t col, const float* v, int cnt) {
+  if constexpr (EPI == EPI_STORE_F32 || EPI == EPI_ADD_F32) {
+    float* dst = reinterpret_cast<float*>(ep.c) + row * ep.ldc + col;
+    const float* res = nullptr;
+    if constexpr (EPI == EPI_ADD_F32)
+      res = ep.c2 ? reinterpret_cast<const float*>(ep.c2) + row * ep.ldc2 + col : dst;
+    const bool vec = cnt == 4 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0 &&
+                     (EPI != EPI_ADD_F32 || (reinterpret_cast<uintptr_t>(res) & 15) == 0);
+    if (vec) {
+      float4 o = make_float4(v[0], v[1], v[2], v[3]);
+      if constexpr (EPI == EPI_ADD_F32) {
+        const float4 r = *reinterpret_cast<const float4*>(res);
+        o = make_float4(r.x + v[0], r.y + v[1], r.z + v[2], r.w + v[3]);
+      }
+      *reinterpret_cast<float4*>(dst) = o;
+      return;
+    }
   }
-  for (int e = 0; e < cnt; ++e) {
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (e >= cnt) break;
     if constexpr (EPI == EPI_STORE_F32) {
       reinterpret_cast<float*>(ep.c)[row * ep.ldc + col + e] = v[e];
     } else if constexpr (EPI == EPI_STORE_BF16) {
@@ -532,6 +578,41 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ ws, int S, int64_
       reinterpret_cast<float*>(ep.c)[row * ep.ldc + col + e] = r + v[e];
     }
   }
+}
+
+template <int EPI>
+__global__ void splitk_reduce_kernel(const float* __restrict__ ws, int S, int64_t M, int64_t N, int64_t stride,
+                                     EpiArgs ep) {
+  const int64_t gpr = (N + 3) / 4;  // 4-column groups per row
+  const int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= M * gpr) return;
+  const int64_t row = gi / gpr, col = (gi % gpr) * 4;
+  float v[4] = {0.f, 0.f, 0.f, 0.f};
+  const int cnt = (int)imin64(4, N - col);
+  const float* p0 = ws + row * N + col;
+  if (cnt == 4 && (reinterpret_cast<uintptr_t>(p0) & 15) == 0 && (stride & 3) == 0 && S <= 8) {
+    float4 part[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s)
+      if (s < S) part[s] = *reinterpret_cast<const float4*>(p0 + s * stride);
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      if (s < S) {
+        v[0] += part[s].x;
+        v[1] += part[s].y;
+        v[2] += part[s].z;
+        v[3] += part[s].w;
+      }
+    }
+  } else {
+    for (int s = 0; s < S; ++s) {
+      const float* p = p0 + s * stride;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if (e < cnt) v[e] += p[e];
+    }
+  }
+  splitk_out<EPI>(ep, row, col, v, cnt);
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>

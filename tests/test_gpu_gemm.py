@@ -219,3 +219,49 @@ def test_sgd_two_term_bf16_shadow():
     assert (two - want).abs().max().item() <= 1e-2 * step.max().item()
     # a single bf16 copy would lose most of the step (half an ulp of 0.02 is ~6e-5)
     assert (hi.double() - W0.double()).abs().mean().item() < 0.5 * step.mean().item()
+
+
+def test_read_modify_write_epilogues_many_tiles():
+    """SGD (hi + lo shadows) and residual-add epilogues on shapes with more
+    work units than SMs (each persistent CTA drains several tiles in both
+    epilogue groups), ragged rows and a last n-tile that is only partly
+    inside N, so the read-ahead of the master / residual meets every edge."""
+    from test_long_context_b200 import ops
+    M, N, K = 2600, 2600, 192
+    Aw, Bw, G = _operands(M, N, K, 1, 1, torch.bfloat16, seed=5)
+    W = 0.02 * torch.randn(M, N, device="cuda")
+    W0 = W.clone()
+    hi = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+    lo = torch.full_like(hi, float("nan"))
+    ops.gemm(Aw, Bw, 1, 1, ops.L.EPI_SGD, c=W, c2=hi, c3=lo, alpha=1e-3)
+    ops.sync()
+    assert (W.double() - (W0.double() - 1e-3 * G)).abs().max().item() <= 1e-6
+    assert torch.equal(hi, W.to(torch.bfloat16))
+    assert torch.equal(lo, (W - hi.float()).to(torch.bfloat16))
+    # residual add into a separate output (c2 = residual), K-major operands
+    A, B, ref = _operands(M, N, K, 0, 0, torch.bfloat16, seed=6)
+    x0 = torch.randn(M, N, device="cuda")
+    x = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, 0, 0, ops.L.EPI_ADD_F32, c=x, c2=x0)
+    ops.sync()
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
+
+
+@pytest.mark.parametrize("N", [2600, 2602])
+def test_split_k_reduce_vector_and_scalar_paths(N):
+    """The ordered split-K sum reads float4 when a row's 4 columns are
+    16-byte aligned (N % 4 == 0) and falls back to scalars otherwise; both
+    give the same in-order sum."""
+    from test_long_context_b200 import ops
+    M, K, S = 260, 4096, 4
+    A, B, ref = _operands(M, N, K, 0, 0, torch.bfloat16, seed=7)
+    ws = torch.empty(S * M * N, device="cuda")
+    x0 = torch.randn(M, N, device="cuda")
+    x = x0.clone()
+    ops.gemm_split(A, B, 0, 0, ops.L.EPI_ADD_F32, S, ws, c=x)
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm_split(A, B, 0, 0, ops.L.EPI_STORE_F32, S, ws, c=c)
+    ops.sync()
+    tol = 1e-4 * ref.abs().max().item() + 1e-4
+    assert (c.double() - ref).abs().max().item() <= tol
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= tol
