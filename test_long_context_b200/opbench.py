@@ -57,9 +57,11 @@ def make_ops(cfg):
     gemm("gemm_gateup_top", b, 4 * f, d, 0, 0, L.EPI_SWIGLU, c=torch.empty(b, 2 * f, device=dev, dtype=bf),
          c2=torch.empty(b, 4 * f, device=dev, dtype=bf))
     gemm("gemm_down_top", b, d, 2 * f, 0, 0, L.EPI_ADD_F32, c=torch.zeros(b, d, device=dev))
+    gemm("gemm_o_top", b, d, d, 0, 0, L.EPI_ADD_F32, c=torch.zeros(b, d, device=dev),
+         c2=torch.zeros(b, d, device=dev))
     gemm("gemm_dgrad_gateup", b, d, 4 * f, 0, 1, L.EPI_STORE_F32, c=torch.empty(b, d, device=dev))
     gemm("gemm_wgrad_gateup_sgd", 2 * f, d, b, 1, 1, L.EPI_SGD, c=torch.zeros(2 * f, d, device=dev),
-         c2=torch.empty(2 * f, d, device=dev, dtype=bf), alpha=1e-2)
+         c2=torch.empty(2 * f, d, device=dev, dtype=bf), c3=torch.empty(2 * f, d, device=dev, dtype=bf), alpha=1e-2)
     gemm("gemm_wgrad_gateup_store", 2 * f, d, b, 1, 1, L.EPI_STORE_F32, c=torch.zeros(2 * f, d, device=dev))
     gemm("gemm_wgrad_gateup_kmajor_store", 2 * f, d, b, 0, 0, L.EPI_STORE_F32, c=torch.zeros(2 * f, d, device=dev))
     nt = ops.gemm_ce_tiles(True, b, V)
