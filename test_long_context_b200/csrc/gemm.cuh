@@ -69,6 +69,7 @@ struct TcGemm {
   alignas(64) CUtensorMap ta;
   alignas(64) CUtensorMap tb;
   int a_mn = 0, b_mn = 0, bn = 256, epi = 0;
+  int pair = 0;  // 256 x 256 tiles on CTA pairs (tcgen05 cta_group::2); B tensor maps then hold 128-row boxes
   int64_t M = 0, N = 0, K = 0;
   EpiArgs args;
   int act_bf16 = 1;  // activation dtype of EPI_SWIGLU / EPI_CE_BWD outputs

@@ -7,6 +7,7 @@
 // lanes 32*(w%4) .. +31, one accumulator row per thread).  Tile 128 x BN x 64,
 // BN in {128, 256}, a 4- or 6-stage smem ring between producer and MMA.
 #include <algorithm>
+#include <map>
 #include <mutex>
 #include <set>
 
@@ -503,6 +504,221 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// CTA-pair variant: a cluster of two CTAs (two SMs) computes one 256 x 256
+// output tile with tcgen05.mma.cta_group::2.  Each CTA loads its own 128 rows
+// of A and its half (128 rows) of the B tile, 32 KB per 64-deep k-block
+// instead of the 48 KB a single CTA needs for a 128 x 256 tile, so a CTA
+// streams 131 instead of 87 flop per operand byte and the ring holds six
+// stages instead of four.  Roles:
+//   even CTA, warp 0 lane 0   TMA for its halves; arrives on its own full
+//                             barrier with the bytes of both CTAs
+//   odd CTA,  warp 0 lane 0   TMA for its halves, counted on the even CTA's
+//                             full barrier
+//   even CTA, warp 1 lane 0   issues every MMA of the pair; each commit frees
+//                             the ring slot / fills the accumulator in both
+//                             CTAs at once
+//   warps 2..9 (both CTAs)    epilogue of the CTA's own 128 accumulator rows,
+//                             then an arrive on the even CTA's acc_empty
+//                             (256 arrivals: both CTAs' epilogue groups)
+// The units are (256-row pair tile, n-tile, k-split), walked by the pairs
+// like the single-CTA kernel walks its tiles.
+struct PairCfg {
+  static constexpr int BN = 256;
+  static constexpr int A_BYTES = BM * BK * 2;    // this CTA's 128 rows of A
+  static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of the B tile
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 6;
+  static constexpr int WBUF = kEpiWarps * 32 * 33 * 4;
+  static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + WBUF;
+  static_assert(SMEM <= 232448, "shared memory per block");
+};
+
+template <bool A_MN, bool B_MN, int EPI, typename TACT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
+                        const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2,
+                        int64_t M, int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt,
+                        int n_split, int n_fast, EpiArgs ep, int* err) {
+  using C = PairCfg;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* acc_full = empty + C::STAGES;   // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2], used in the even CTA
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  float* wbufs = reinterpret_cast<float*>(sB + C::STAGES * C::B_BYTES + 256);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();  // 0: issues the MMAs
+  const bool lead = rank == 0;
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int64_t units = (int64_t)n_mt * n_nt * n_split;
+  // n_mt counts 256-row pair tiles; m0 is the pair tile's first row
+  auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int& kb_begin) {
+    const int64_t mn = u % ((int64_t)n_mt * n_nt);
+    m0 = (n_fast ? mn / n_nt : mn % n_mt) * (2 * BM);
+    n0 = (n_fast ? mn % n_nt : mn / n_mt) * BN;
+    split = (int)(u / ((int64_t)n_mt * n_nt));
+    const int total = KB1 + (n0 >= n_ext ? KB2 : 0);
+    kb_begin = split * kpsb;
+    nkb = total - kb_begin < kpsb ? total - kb_begin : kpsb;
+    if (nkb < 0) nkb = 0;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_empty[b], 256);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tma);
+    ptx::prefetch_tmap(&tmb);
+    if (KB2 > 0) {
+      ptx::prefetch_tmap(&tma2);
+      ptx::prefetch_tmap(&tmb2);
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tmem_alloc_pair(tmem_slot, 2 * BN);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync_all();  // both CTAs' barriers are initialised before either signals the other
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t kbg = 0;
+      bool ok = true;
+      for (int64_t u = pair; ok && u < units; u += npairs) {
+        int64_t m0, n0;
+        int split, nkb, kb_begin;
+        decode(u, m0, n0, split, nkb, kb_begin);
+        const int mo = (int)(m0 + BM * rank);  // this CTA's A rows
+        for (int j = 0; j < nkb; ++j, ++kbg) {
+          const int s = (int)(kbg % C::STAGES);
+          const uint32_t ph = (kbg / C::STAGES) & 1u;
+          if (!(ok = ptx::mbar_wait(&empty[s], ph ^ 1u, err))) break;
+          if (lead) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
+          const uint32_t fb = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
+          uint8_t* a = sA + s * C::A_BYTES;
+          uint8_t* b = sB + s * C::B_BYTES;
+          const int kb = kb_begin + j;
+          const bool second = kb >= KB1;
+          const CUtensorMap* ta = second ? &tma2 : &tma;
+          const CUtensorMap* tb = second ? &tmb2 : &tmb;
+          const int k0 = (second ? kb - KB1 : kb) * BK;
+          const int nb = (int)(second ? n0 - n_ext : n0) + 128 * (int)rank;  // this CTA's half of B
+          if constexpr (!A_MN) {
+            ptx::tma_load_2d_pair(a, ta, fb, k0, mo);
+          } else {
+            ptx::tma_load_2d_pair(a, ta, fb, mo, k0);
+            ptx::tma_load_2d_pair(a + 8192, ta, fb, mo + 64, k0);
+          }
+          if constexpr (!B_MN) {
+            ptx::tma_load_2d_pair(b, tb, fb, k0, nb);
+          } else {
+            ptx::tma_load_2d_pair(b, tb, fb, nb, k0);
+            ptx::tma_load_2d_pair(b + 8192, tb, fb, nb + 64, k0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      if (lead) {
+        constexpr uint32_t idesc = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
+        uint32_t kbg = 0, it = 0;
+        bool ok = true;
+        for (int64_t u = pair; ok && u < units; u += npairs, ++it) {
+          int64_t m0, n0;
+          int split, nkb, kb_begin;
+          decode(u, m0, n0, split, nkb, kb_begin);
+          const uint32_t b = it & 1u, use = it >> 1;
+          // both CTAs' epilogues must have drained this accumulator buffer
+          if (!(ok = ptx::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem + b * BN;
+          for (int kb = 0; kb < nkb; ++kb, ++kbg) {
+            const int s = (int)(kbg % C::STAGES);
+            const uint32_t ph = (kbg / C::STAGES) & 1u;
+            if (!(ok = ptx::mbar_wait(&full[s], ph, err))) break;
+            ptx::tc_fence_after();
+            const uint32_t a_addr = ptx::smem_u32(sA + s * C::A_BYTES);
+            const uint32_t b_addr = ptx::smem_u32(sB + s * C::B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = A_MN ? ptx::smem_desc_sw128(a_addr + kk * 2048, 8192, 1024)
+                                       : ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+              const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
+                                       : ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+              ptx::umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            ptx::umma_commit_pair(&empty[s], 0x3);
+          }
+          if (!ok) break;
+          ptx::umma_commit_pair(&acc_full[b], 0x3);
+        }
+        ptx::umma_commit_pair(drain, 0x3);
+      }
+      // every MMA of the pair has completed (they read this CTA's shared
+      // memory and write its TMEM) before either CTA releases them
+      ptx::mbar_drain(drain, 0);
+    }
+  } else {
+    const int ew = warp - 2, eg = ew >> 2;
+    const int q = warp & 3;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t empty_lead0 = ptx::mapa_shared(ptx::smem_u32(&acc_empty[0]), 0);
+    const uint32_t empty_lead1 = ptx::mapa_shared(ptx::smem_u32(&acc_empty[1]), 0);
+    uint32_t it = (uint32_t)eg;
+    for (int64_t u = pair + (int64_t)eg * npairs; u < units; u += 2 * npairs, it += 2) {
+      int64_t m0, n0;
+      int split, nkb, kb_begin;
+      decode(u, m0, n0, split, nkb, kb_begin);
+      m0 += BM * rank;  // this CTA's 128 rows of the pair tile
+      const uint32_t b = it & 1u, use = it >> 1;
+      float bufA[32], bufB[32];
+      if constexpr (kTransposedEpi<EPI>) {
+        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
+        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+      }
+      const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int64_t row = m0 + q * 32 + lane;
+      if constexpr (kTransposedEpi<EPI>)
+        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * 33, m0 + q * 32,
+                                     M, bufA, bufB);
+      else
+        epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split);
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_cluster(b ? empty_lead1 : empty_lead0);
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::cluster_sync_all();  // neither CTA frees TMEM or exits while the pair still uses it
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem, 2 * BN);
+  }
+}
+
 // ---- host side -----------------------------------------------------------------
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -636,6 +852,42 @@ KernelFn pick_epi(int epi, int act_bf16) {
   return nullptr;
 }
 
+template <bool A_MN, bool B_MN, int EPI, typename TACT>
+KernelFn pair_ptr() {
+  return reinterpret_cast<KernelFn>(&tc_gemm_pair_kernel<A_MN, B_MN, EPI, TACT>);
+}
+
+template <bool A_MN, bool B_MN>
+KernelFn pick_pair_epi(int epi, int act_bf16) {
+  switch (epi) {
+    case EPI_STORE_F32: return pair_ptr<A_MN, B_MN, EPI_STORE_F32, bf16>();
+    case EPI_STORE_BF16: return pair_ptr<A_MN, B_MN, EPI_STORE_BF16, bf16>();
+    case EPI_ADD_F32: return pair_ptr<A_MN, B_MN, EPI_ADD_F32, bf16>();
+    case EPI_SWIGLU: return act_bf16 ? pair_ptr<A_MN, B_MN, EPI_SWIGLU, bf16>() : pair_ptr<A_MN, B_MN, EPI_SWIGLU, float>();
+    case EPI_CE_FWD: return pair_ptr<A_MN, B_MN, EPI_CE_FWD, bf16>();
+    case EPI_CE_BWD: return act_bf16 ? pair_ptr<A_MN, B_MN, EPI_CE_BWD, bf16>() : pair_ptr<A_MN, B_MN, EPI_CE_BWD, float>();
+    case EPI_SGD: return pair_ptr<A_MN, B_MN, EPI_SGD, bf16>();
+  }
+  return nullptr;
+}
+
+KernelFn pick_pair(int a_mn, int b_mn, int epi, int act_bf16) {
+  if (!a_mn && !b_mn) return pick_pair_epi<false, false>(epi, act_bf16);
+  if (!a_mn && b_mn) return pick_pair_epi<false, true>(epi, act_bf16);
+  if (a_mn && b_mn) return pick_pair_epi<true, true>(epi, act_bf16);
+  return pick_pair_epi<true, false>(epi, act_bf16);
+}
+
+// CTA pairs for 256-wide tiles of GEMMs with more than one 128-row tile;
+// TTT_GEMM_PAIR=0 keeps every GEMM on single CTAs.
+bool pair_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("TTT_GEMM_PAIR");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 template <int BN>
 KernelFn pick(int a_mn, int b_mn, int epi, int act_bf16) {
   if (!a_mn && !b_mn) return pick_epi<BN, false, false>(epi, act_bf16);
@@ -699,9 +951,10 @@ int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args,
   g->ws = nullptr;
   g->K2 = 0;
   g->n_ext = 0;
+  g->pair = (bn == 256 && M > BM && pair_enabled()) ? 1 : 0;
   int rc = make_tmap(&g->ta, s.a, s.a_mn ? 64 : BM);
   if (rc) return rc;
-  rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : bn);
+  rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : (g->pair ? 128 : bn));
   g->ta2 = g->ta;
   g->tb2 = g->tb;
   return rc;
@@ -716,7 +969,7 @@ int tc_gemm_set_ext(TcGemm* g, const MatView& a2, const MatView& b2, int64_t n_e
   if (g->epi == EPI_CE_FWD) return set_error(TTT_ERR_INVALID_ARG, "gemm: no second product with CE partials");
   int rc = make_tmap(&g->ta2, a2, g->a_mn ? 64 : BM);
   if (rc) return rc;
-  rc = make_tmap(&g->tb2, b2, g->b_mn ? 64 : g->bn);
+  rc = make_tmap(&g->tb2, b2, g->b_mn ? 64 : (g->pair ? 128 : g->bn));
   if (rc) return rc;
   g->K2 = K2;
   g->n_ext = n_ext;
@@ -745,9 +998,11 @@ int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws) {
 
 int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   const int kepi = g.ksplit > 1 ? EPI_STORE_F32 : g.epi;
-  KernelFn fn = g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, kepi, g.act_bf16) : pick<128>(g.a_mn, g.b_mn, kepi, g.act_bf16);
+  KernelFn fn = g.pair ? pick_pair(g.a_mn, g.b_mn, kepi, g.act_bf16)
+                       : (g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, kepi, g.act_bf16)
+                                      : pick<128>(g.a_mn, g.b_mn, kepi, g.act_bf16));
   if (!fn) return set_error(TTT_ERR_INVALID_ARG, "gemm: no kernel for this combination");
-  const int smem = g.bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM;
+  const int smem = g.pair ? PairCfg::SMEM : (g.bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM);
   {
     static std::mutex mu;
     static std::set<std::pair<int, KernelFn>> configured;
@@ -760,7 +1015,9 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
       configured.insert({dev, fn});
     }
   }
-  const int n_mt = (int)((g.M + BM - 1) / BM), n_nt = (int)((g.N + g.bn - 1) / g.bn);
+  // pairs: n_mt counts 256-row pair tiles and the grid is two CTAs per unit slot
+  const int mrows = g.pair ? 2 * BM : BM;
+  const int n_mt = (int)((g.M + mrows - 1) / mrows), n_nt = (int)((g.N + g.bn - 1) / g.bn);
   const int64_t units = (int64_t)n_mt * n_nt * g.ksplit;
   static int n_sm = 0;
   if (!n_sm) {
@@ -768,7 +1025,32 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
     TTT_CUDA_TRY(cudaGetDevice(&dev));
     TTT_CUDA_TRY(cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev));
   }
-  const dim3 grid((unsigned)std::min<int64_t>(units, n_sm));
+  int slots = n_sm;  // CTAs (or CTA pairs) that are resident at once
+  if (g.pair) {
+    // pairs that fit at the same time (a GPC with an odd number of free SMs
+    // leaves one idle); a grid of more would run a second, partial wave
+    static std::mutex mu;
+    static std::map<std::pair<int, KernelFn>, int> pairs_of;
+    int dev = 0;
+    TTT_CUDA_TRY(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = pairs_of.find({dev, fn});
+    if (it == pairs_of.end()) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2, 1, 1);
+      cfg.blockDim = dim3(kGemmThreads, 1, 1);
+      cfg.dynamicSmemBytes = (size_t)smem;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, reinterpret_cast<const void*>(fn), &cfg) != cudaSuccess || nc < 1) {
+        (void)cudaGetLastError();
+        nc = n_sm / 2;
+      }
+      it = pairs_of.emplace(std::make_pair(dev, fn), std::min(nc, n_sm / 2)).first;
+    }
+    slots = it->second;
+  }
+  const dim3 grid(g.pair ? (unsigned)(2 * std::min<int64_t>(units, slots))
+                         : (unsigned)std::min<int64_t>(units, slots));
   const int KB1 = (int)((g.K + BK - 1) / BK), KB2 = (int)((g.K2 + BK - 1) / BK);
   // n-tile fastest when B (N x K, plus a second product) fits comfortably in L2 and A is the larger operand
   const double a_bytes = 2.0 * (double)g.M * (double)(g.K + g.K2), b_bytes = 2.0 * (double)g.N * (double)(g.K + g.K2);

@@ -265,3 +265,90 @@ def test_split_k_reduce_vector_and_scalar_paths(N):
     tol = 1e-4 * ref.abs().max().item() + 1e-4
     assert (c.double() - ref).abs().max().item() <= tol
     assert (x.double() - (x0.double() + ref)).abs().max().item() <= tol
+
+
+@pytest.mark.parametrize("combo", COMBOS)
+def test_cta_pair_tiles_every_epilogue(combo):
+    """256-wide tiles run on CTA pairs (one 256 x 256 tile per pair, each CTA
+    loading its own 128 rows of A and half of the B tile): every epilogue
+    against the fp64 product and against single-CTA 128-wide tiles, with a
+    last pair tile whose odd CTA has no valid rows at all (M = 600)."""
+    from test_long_context_b200 import ops
+    M, N, K = 600, 768, 320
+    A, B, ref = _operands(M, N, K, *combo, torch.bfloat16, seed=31)
+    scale = ref.abs().max().item()
+    outs = {}
+    for bn in (128, 256):
+        c = torch.full((M, N), float("nan"), device="cuda")
+        ops.gemm(A, B, *combo, ops.L.EPI_STORE_F32, c=c, bn=bn)
+        cb = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+        ops.gemm(A, B, *combo, ops.L.EPI_STORE_BF16, c=cb, bn=bn)
+        x0 = torch.randn(M, N, device="cuda", generator=torch.Generator(device="cuda").manual_seed(1))
+        x = torch.full_like(x0, float("nan"))
+        ops.gemm(A, B, *combo, ops.L.EPI_ADD_F32, c=x, c2=x0, bn=bn)
+        a = torch.full((M, N // 2), float("nan"), device="cuda", dtype=torch.bfloat16)
+        raw = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+        ops.gemm(A, B, *combo, ops.L.EPI_SWIGLU, c=a, c2=raw, bn=bn)
+        W = (0.02 * torch.randn(M, N, device="cuda", generator=torch.Generator(device="cuda").manual_seed(2)))
+        W0 = W.clone()
+        hi = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+        lo = torch.full_like(hi, float("nan"))
+        ops.gemm(A, B, *combo, ops.L.EPI_SGD, c=W, c2=hi, c3=lo, alpha=1e-3, bn=bn)
+        ops.sync()
+        assert (c.double() - ref).abs().max().item() <= 1e-4 * scale + 1e-4, bn
+        assert (cb.double() - ref).abs().max().item() <= 1e-2 * scale, bn
+        assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * scale + 1e-4, bn
+        r = ref.view(M, N // 128, 2, 64)
+        want = (torch.nn.functional.silu(r[:, :, 0]) * r[:, :, 1]).reshape(M, N // 2)
+        assert (a.double() - want).abs().max().item() <= 2e-2 * want.abs().max().item(), bn
+        assert (W.double() - (W0.double() - 1e-3 * ref)).abs().max().item() <= 1e-6 * scale + 1e-6, bn
+        assert torch.equal(hi, W.to(torch.bfloat16)) and torch.equal(lo, (W - hi.float()).to(torch.bfloat16))
+        outs[bn] = c
+    assert (outs[128] - outs[256]).abs().max().item() <= 1e-5 * scale
+
+
+def test_cta_pair_tiles_cross_entropy_split_and_dual():
+    """CE partials / CE gradient, split-K partials and a second product on
+    256-wide pair tiles."""
+    from test_long_context_b200 import ops
+    M, V, K = 520, 1000, 192
+    h = (torch.randn(M, K, device="cuda") * 0.5).bfloat16()
+    W = (torch.randn(V, K, device="cuda") * 0.5).bfloat16()
+    z = h.double() @ W.double().T
+    tgt = torch.randint(0, V, (M,), device="cuda", dtype=torch.int32)
+    nt = ops.gemm_ce_tiles(True, M, V, 256)
+    pm, ps = torch.empty(nt, M, device="cuda"), torch.empty(nt, M, device="cuda")
+    zt = torch.full((M,), float("nan"), device="cuda")
+    ops.gemm(h, W, 0, 0, ops.L.EPI_CE_FWD, row_i=tgt, part_max=pm, part_sum=ps, target_logit=zt, part_ld=M, bn=256)
+    want_lse = torch.logsumexp(z, 1)
+    dz = torch.empty(M, V, device="cuda", dtype=torch.bfloat16)
+    scale = torch.full((M,), 1.0 / M, device="cuda")
+    ops.gemm(h, W, 0, 0, ops.L.EPI_CE_BWD, c=dz, row_f=want_lse.float(), row_g=scale, row_i=tgt, bn=256)
+    ops.sync()
+    gm = pm.max(0).values
+    lse = gm + torch.log((ps * torch.exp(pm - gm)).sum(0))
+    assert (lse.double() - want_lse).abs().max().item() <= 1e-4
+    assert (zt.double() - z.gather(1, tgt.long()[:, None])[:, 0]).abs().max().item() <= 1e-4
+    p = torch.softmax(z, 1)
+    oh = torch.nn.functional.one_hot(tgt.long(), V).double()
+    want = (p - oh) * scale.double()[:, None]
+    assert (dz.double() - want).abs().max().item() <= 1e-2 * want.abs().max().item()
+    # split-K partials on pair tiles, then the ordered sum
+    Ms, Ns, Ks, S = 300, 640, 4160, 3
+    A, B, ref = _operands(Ms, Ns, Ks, 0, 0, torch.bfloat16, seed=33)
+    ws = torch.empty(S * Ms * Ns, device="cuda")
+    c = torch.full((Ms, Ns), float("nan"), device="cuda")
+    ops.gemm_split(A, B, 0, 0, ops.L.EPI_STORE_F32, S, ws, c=c, bn=256)
+    # second product on the columns from n_ext on (a multiple of the 256-wide tile)
+    Md, Nd, Kd, K2, n_ext = 300, 1024, 192, 136, 512
+    g = torch.Generator(device="cuda").manual_seed(34)
+    Ad = torch.randn((Md, Kd), device="cuda", generator=g).bfloat16()
+    Bd = torch.randn((Nd, Kd), device="cuda", generator=g).bfloat16()
+    A2 = torch.randn((Md, K2), device="cuda", generator=g).bfloat16()
+    B2 = torch.randn((Nd - n_ext, K2), device="cuda", generator=g).bfloat16()
+    refd = _dual_ref(Ad, Bd, A2, B2, 0, 0, n_ext)
+    cd = torch.full((Md, Nd), float("nan"), device="cuda")
+    ops.gemm_dual(Ad, Bd, A2, B2, 0, 0, ops.L.EPI_STORE_F32, n_ext=n_ext, bn=256, c=cd)
+    ops.sync()
+    assert (c.double() - ref).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
+    assert (cd.double() - refd).abs().max().item() <= 1e-4 * refd.abs().max().item() + 1e-4
