@@ -20,12 +20,13 @@ reading notes by Zhongzhu Zhou, "算法 1：因果预填充与内层适应" and 
        keep the keys/values the window still needs (算法 1);
   3. return the per-token losses and the adapted W.
 
-Only the MLPs of the last n_u blocks carry fast weights ("只更新最后四分之一
-Transformer block 中的 MLP", reading notes §6); each such block keeps a static
-MLP beside the fast one and sums their outputs (reading notes §6 paragraph 2;
-reportify.cn "双MLP结构").  Everything else is frozen in the inner loop.
+Only the MLPs of the last n_u blocks carry fast weights (the reading notes,
+§6, restrict the inner-loop update to the MLPs of the final quarter of the
+blocks); each such block keeps a static MLP beside the fast one and sums
+their outputs (reading notes §6, second paragraph; reportify.cn, the section
+on the dual-MLP structure).  Everything else is frozen in the inner loop.
 
-Readings where the pages are silent (each one also listed in the design doc):
+Readings where the pages are silent:
   * position p (0-based) predicts tokens[p+1]; the last position has no
     target (loss NaN); A_c divides by the number n_c of targets in the chunk;
   * keys of earlier chunks are the values cached when those positions were
@@ -267,7 +268,8 @@ def forward_chunk(model, W, state, toks, p0, tgt, fast_on=True, count_pairs=Fals
 def backward_chunk(model, W, fwd, weights):
     """G = dA/dW for A = sum_p weights[p] * loss_p over valid positions p.
     Explicit backward through the top blocks only: below block L-n_u nothing
-    depends on W (reading notes §6; hyper.ai "梯度仅回传至更新层")."""
+    depends on W (reading notes §6; the hyper.ai summary: gradients reach
+    only the updated layers)."""
     cfg = model.cfg
     n, d, H, hd, eps = fwd["n"], cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.norm_eps
     valid, tgt = fwd["valid"], fwd["tgt"]
