@@ -55,8 +55,11 @@ typedef struct ttt_epilogue_args {
  * b_mn = 0: B stored [N, K] with row pitch ldb;  b_mn = 1: stored [K, N].
  * bf16 operands: 16-byte aligned base and row pitch.  (a_mn, b_mn) = (1, 0)
  * is not supported with TTT_BF16.  bn_hint: 0 (auto), 128 or 256 (tile
- * width; TTT_BF16 only).  CE_FWD writes ceil(N / tile) partial tiles:
- * query the tile count with ttt_op_gemm_ce_tiles.
+ * width; TTT_BF16 only).  256-wide tiles of a GEMM with M > 128 run on CTA
+ * pairs (clusters of two CTAs, one 256 x 256 tile per pair; environment
+ * TTT_GEMM_PAIR=0 keeps single CTAs); the results do not depend on it.
+ * CE_FWD writes ceil(N / tile) partial tiles: query the tile count with
+ * ttt_op_gemm_ce_tiles.
  */
 int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A,
                 int64_t lda, const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args,
