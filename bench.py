@@ -182,6 +182,24 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def latency_by_tokens(ctx, tok_dev, losses, T, stream, lengths=(8192, 16384, 32768, 65536)):
+    """Per-1K-token prefill latency (ms) of one prefill of each shorter prefix
+    of the same sequence and of the whole sequence, all without per-launch
+    timing events: the cost per token should stay flat once the window is
+    full."""
+    import torch
+    out = {}
+    for n in [m for m in lengths if m < T] + [T]:
+        ctx.reset()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        ctx.prefill(tok_dev[:n], losses[:n], sync=False)
+        e1.record(stream)
+        ctx.sync()
+        out[str(n)] = e0.elapsed_time(e1) / (n / 1000.0)
+    return out
+
+
 def workload_name(cfg, T):
     return (f"{cfg.name} TTT-E2E prefill: L={cfg.n_layers} d={cfg.d_model} H={cfg.n_heads}x{cfg.head_dim} "
             f"f={cfg.d_ff} V={cfg.vocab} n_u={cfg.n_updated} T={T} k={cfg.k} b={cfg.b} batch=1")
@@ -340,6 +358,8 @@ def main():
                "h2d_bytes_per_step": int(tok_host.numel() * 4), "d2h_bytes_per_step": int(loss_host.numel() * 4),
                "ms_per_step": ems / args.steps}
 
+    by_T = latency_by_tokens(ctx, tok_dev, losses, T, stream)
+
     if rank == 0:
         peaks, peak_src = load_peaks()
         value = aggregate_tokens_per_s(world, args.steps, T, ms)
@@ -371,6 +391,7 @@ def main():
                 "data": "synthetic (seeded Zipf(1.1) tokens + repeated 64-token spans; N(0,0.02) weights)",
                 "config": config_dict(cfg, T, world),
                 "ms_per_1k_tokens": (ms / args.steps) / (T / 1000.0),
+                "ms_per_1k_tokens_by_T": by_T,
                 "tensor_peak_frac": flops_step * world * args.steps / (ms / 1000.0) / 1e12 / tensor_peak,
                 "algorithmic_tflop_per_step": flops_step / 1e12,
                 "roofline": roof, "kernel_classes": classes, "gpu_launches": int(launches),

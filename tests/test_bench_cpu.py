@@ -46,3 +46,44 @@ def test_traffic_is_trusted_only_for_the_captured_source(tmp_path, monkeypatch):
     assert bench.traffic_for("gemm", "2.7b") == 123
     monkeypatch.setattr(bench, "kernel_source_hash", lambda kc: "changed")
     assert bench.traffic_for("gemm", "2.7b") is None
+
+
+def test_latency_sweep_covers_prefixes_and_the_whole_sequence(monkeypatch):
+    """latency_by_tokens prefills each shorter prefix once and the whole
+    sequence once, from a fresh state each time, and reports ms per 1K
+    tokens per length (fake context and events: no GPU)."""
+    import types
+
+    calls = []
+
+    class Ctx:
+        def reset(self):
+            calls.append("reset")
+
+        def prefill(self, tok, losses, sync=True):
+            calls.append(("prefill", len(tok), len(losses), sync))
+
+        def sync(self):
+            calls.append("sync")
+
+    class Event:
+        t = 0.0
+
+        def __init__(self, enable_timing=False):
+            self.at = None
+
+        def record(self, stream=None):
+            Event.t += 5.0
+            self.at = Event.t
+
+        def elapsed_time(self, other):
+            return other.at - self.at
+
+    fake_torch = types.SimpleNamespace(cuda=types.SimpleNamespace(Event=Event))
+    monkeypatch.setitem(sys.modules, "torch", fake_torch)
+    out = bench.latency_by_tokens(Ctx(), list(range(40000)), list(range(40000)), 40000, None)
+    assert list(out) == ["8192", "16384", "32768", "40000"]
+    assert [c[1] for c in calls if isinstance(c, tuple)] == [8192, 16384, 32768, 40000]
+    assert all(c[3] is False for c in calls if isinstance(c, tuple))
+    assert calls.count("reset") == 4 and calls.count("sync") == 4
+    assert abs(out["8192"] - 5.0 / 8.192) < 1e-12
