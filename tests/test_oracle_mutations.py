@@ -77,6 +77,18 @@ def _gradient_sign_flipped(orig):
     return f
 
 
+def _norm_gain_ignored(orig):
+    def f(x, g, eps):
+        return orig(x, np.ones_like(g), eps)
+    return f
+
+
+def _norm_bwd_gain_ignored(orig):
+    def f(x, r, g, dy):
+        return orig(x, r, np.ones_like(g), dy)
+    return f
+
+
 def _ce_target_shifted(orig):
     def f(z, targets):
         return orig(z, (np.asarray(targets) + 1) % z.shape[-1])
@@ -93,14 +105,18 @@ MUTATIONS = {
     "attention scale missing": ("swa", _attention_unscaled),
     "SGD step climbs the loss": ("backward_chunk", _gradient_sign_flipped),
     "cross-entropy scores the wrong target": ("log_softmax_ce", _ce_target_shifted),
+    "RMSNorm forward ignores its gain": ("rmsnorm", _norm_gain_ignored),
+    "RMSNorm backward ignores its gain": ("rmsnorm_bwd", _norm_bwd_gain_ignored),
 }
 
 PINS = {
     "forward vs Qwen3 (k = 12)": lambda: P.test_forward_matches_qwen3_sliding_window(CFG, 12),
-    "backward vs central differences (chunk 2)": lambda: P.test_backward_matches_central_differences(CFG, 2),
+    "backward vs central differences (chunk 2)": lambda: P.test_backward_matches_central_differences(CFG, 2, False),
     "eq. (3) toy, b = 1": lambda: P.test_toy_bigram_per_token_update_eq3(CFG),
     "eq. (9) chunk gradient": lambda: P.test_chunk_gradient_is_mean_of_token_gradients_eq9(CFG),
     "zero head: ln V": lambda: P.test_zero_head_gives_ln_V_and_zero_gradient(CFG),
+    "forward vs Qwen3, random norm gains": lambda: P.test_forward_matches_qwen3_with_random_norm_gains(CFG),
+    "central differences, random norm gains": lambda: P.test_backward_matches_central_differences(CFG, 2, True),
 }
 
 

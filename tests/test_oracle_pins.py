@@ -50,6 +50,25 @@ def test_forward_matches_qwen3_sliding_window(micro_cfg, k):
     assert np.isnan(ours[-1])
 
 
+def _random_gains(arrays, seed=5):
+    """Norm gains away from 1 (the synthetic weights start them at 1, where a
+    gain applied twice, to the wrong tensor or not at all is invisible)."""
+    rng = np.random.default_rng(seed)
+    for name in arrays:
+        if name.endswith("norm"):
+            arrays[name] = 1.0 + 0.3 * rng.standard_normal(arrays[name].shape)
+
+
+def test_forward_matches_qwen3_with_random_norm_gains(micro_cfg):
+    """The Qwen3 pin with every RMSNorm gain (block, QK-norm, final) drawn
+    away from 1: fixes which gain multiplies which normalised tensor."""
+    m, arrays = _model(micro_cfg, mutate=_random_gains)
+    toks = synth.tokens(micro_cfg)
+    ours = oracle.static_losses(m, toks)
+    ref = Q.losses(Q.build(micro_cfg, arrays, sliding=True), toks)
+    np.testing.assert_allclose(ours[:-1], ref[:-1], **QWEN_TOL)
+
+
 def test_window_ge_T_is_full_causal_attention(micro_cfg):
     """k >= T: sliding-window attention equals plain causal attention
     (reading notes §9.2: an 8K window over an 8K sequence is full attention)."""
@@ -124,13 +143,14 @@ def _run_to_chunk(m, toks, c_stop, eta):
     return W, st
 
 
-@pytest.mark.parametrize("chunk", [0, 2])
-def test_backward_matches_central_differences(micro_cfg, chunk):
+@pytest.mark.parametrize("chunk,gains", [(0, False), (2, False), (2, True)])
+def test_backward_matches_central_differences(micro_cfg, chunk, gains):
     """Hand-derived G = dA_c/dW agrees with fp64 central differences of A_c
     (relative error <= 1e-6), through two fast blocks, attention included,
-    with the keys of earlier chunks held as cached constants."""
+    with the keys of earlier chunks held as cached constants; once more with
+    every norm gain away from 1, which pins the gains in the backward."""
     cfg = micro_cfg.with_(n_updated=2, eta=0.3)
-    m, _ = _model(cfg)
+    m, _ = _model(cfg, mutate=_random_gains if gains else None)
     toks = synth.tokens(cfg)
     W, st = _run_to_chunk(m, toks, chunk, cfg.eta)
     b, p0 = cfg.b, chunk * cfg.b
