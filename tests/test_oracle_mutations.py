@@ -89,6 +89,37 @@ def _norm_bwd_gain_ignored(orig):
     return f
 
 
+def _rope_theta_doubled(orig):
+    def f(pos, hd, theta):
+        return orig(pos, hd, 2.0 * theta)
+    return f
+
+
+def _next_key_visible(orig):
+    def f(qpos, kpos, k):
+        qp = np.asarray(qpos)[:, None]
+        kp = np.asarray(kpos)[None, :]
+        return (kp <= qp + 1) & (kp > qp - k)
+    return f
+
+
+def _rope_adjacent_pairs(orig):
+    def f(x, cos, sin):
+        c, s = cos[:, None, :], sin[:, None, :]
+        x1, x2 = x[..., 0::2], x[..., 1::2]
+        y = np.empty_like(x)
+        y[..., 0::2] = x1 * c - x2 * s
+        y[..., 1::2] = x2 * c + x1 * s
+        return y
+    return f
+
+
+def _norm_eps_wrong(orig):
+    def f(x, g, eps):
+        return orig(x, g, 100.0 * eps)
+    return f
+
+
 def _ce_target_shifted(orig):
     def f(z, targets):
         return orig(z, (np.asarray(targets) + 1) % z.shape[-1])
@@ -107,6 +138,10 @@ MUTATIONS = {
     "cross-entropy scores the wrong target": ("log_softmax_ce", _ce_target_shifted),
     "RMSNorm forward ignores its gain": ("rmsnorm", _norm_gain_ignored),
     "RMSNorm backward ignores its gain": ("rmsnorm_bwd", _norm_bwd_gain_ignored),
+    "RoPE base theta doubled": ("rope_tables", _rope_theta_doubled),
+    "causal mask lets the next key in": ("window_mask", _next_key_visible),
+    "RoPE pairs adjacent elements": ("rope", _rope_adjacent_pairs),
+    "RMSNorm eps 100x too large": ("rmsnorm", _norm_eps_wrong),
 }
 
 PINS = {
