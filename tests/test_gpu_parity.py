@@ -71,3 +71,25 @@ def test_small_fp32_variants(over):
 def test_small_bf16_variants(over):
     cfg = SMALL.with_(dtype="bf16", **over)
     _check_bf16(cfg, synth.tokens(cfg))
+
+
+def _norm_gains_away_from_one(w, seed=5):
+    """The synthetic weights start every RMSNorm gain at 1, where a gain
+    applied to the wrong tensor (q vs k, attention vs MLP norm) or left out
+    of a backward changes nothing; draw them as 1 + 0.3 N(0, 1) instead.
+    Gains are fp32 on both sides in either dtype."""
+    rng = np.random.default_rng(seed)
+    for name in w.arrays:
+        if name.endswith("norm"):
+            w.arrays[name] = (1.0 + 0.3 * rng.standard_normal(w.arrays[name].shape)).astype(np.float32)
+    return w
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_small_with_norm_gains_away_from_one(dtype):
+    cfg = SMALL.with_(dtype=dtype)
+    w = _norm_gains_away_from_one(synth.make_weights(cfg))
+    if dtype == "f32":
+        _check_fp32(cfg, synth.tokens(cfg), w)
+    else:
+        _check_bf16(cfg, synth.tokens(cfg), w)
