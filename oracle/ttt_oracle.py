@@ -261,7 +261,7 @@ def forward_chunk(model, W, state, toks, p0, tgt, fast_on=True, count_pairs=Fals
     loss = np.full(n, np.nan)
     loss_v, probs, _ = log_softmax_ce(z[valid], tgt[valid])
     loss[valid] = loss_v
-    return loss, dict(saved=saved, x=x, rf=rf, hf=hf, probs=probs, valid=valid, tgt=tgt,
+    return loss, dict(saved=saved, x=x, rf=rf, hf=hf, probs=probs, valid=valid, tgt=tgt, z_last=z[n - 1].copy(),
                       cos=cos, sin=sin, n=n, p0=p0, kstart=kstart)
 
 
@@ -320,10 +320,12 @@ class Result:
     chunk_mean: list             # A_c per chunk (mean over its targets)
     pairs: int = 0               # window pairs of block 0 (eq. (1))
     grads: list = None           # per updated chunk G (when keep_grads)
+    state: object = None         # attention state after the last position (when keep_state)
+    z_last: np.ndarray = None    # logits of position T-1, scored before its chunk's update
 
 
 def prefill(model, toks, eta=None, b=None, k=None, keep_grads=False, count_pairs=False,
-            n_chunks=None):
+            n_chunks=None, keep_state=False, capacity=None):
     """The TTT prefill loop (算法 1).  ``toks`` int array of length T.
     Overrides of eta/b/k default to the config's.  ``n_chunks`` stops early
     (prefix runs).  Returns Result."""
@@ -335,9 +337,10 @@ def prefill(model, toks, eta=None, b=None, k=None, keep_grads=False, count_pairs
     T, b = len(toks), cfg.b
     toks = np.asarray(toks, dtype=np.int64)
     W = init_fast(model)
-    state = State(cfg, T)
+    state = State(cfg, max(T, capacity or 0))  # room for positions generated later (decode)
     losses = np.full(T, np.nan)
     means, grads = [], []
+    z_last = None
     nch = -(-T // b)
     if n_chunks is not None:
         nch = min(nch, n_chunks)
@@ -350,6 +353,7 @@ def prefill(model, toks, eta=None, b=None, k=None, keep_grads=False, count_pairs
             tgt[:nt] = toks[p0 + 1:p0 + 1 + nt]
         loss, fwd = forward_chunk(model, W, state, toks[p0:p0 + n], p0, tgt, count_pairs=count_pairs)
         losses[p0:p0 + n] = loss          # recorded before the update
+        z_last = fwd["z_last"]
         n_c = int((tgt >= 0).sum())
         means.append(float(np.nanmean(loss)) if n_c else float("nan"))
         if n == b and n_c > 0 and W:
@@ -360,7 +364,70 @@ def prefill(model, toks, eta=None, b=None, k=None, keep_grads=False, count_pairs
                     W[l][name] = W[l][name] - eta * G[l][name]   # eq. (9)
             if keep_grads:
                 grads.append(G)
-    return Result(losses, W, means, state.pairs, grads if keep_grads else None)
+    return Result(losses, W, means, state.pairs, grads if keep_grads else None,
+                  state if keep_state else None, z_last)
+
+
+@dataclass
+class DecodeResult:
+    tokens: np.ndarray           # [n_gen] generated token ids
+    losses: np.ndarray           # [n_gen] loss of the position before each generated token, against it
+    W: dict                      # fast weights after the last completed chunk
+    updates: list                # positions p after whose forward a chunk [p+1-b, p] updated W
+    prefill: Result              # the prefill of the prompt
+
+
+def decode(model, prompt, n_gen, eta=None):
+    """Greedy generation with periodic fast-weight updates (算法 3 of the
+    reading notes: generate causally from the state the prefill left, collect
+    the generated tokens until an inner chunk is full, take that chunk's
+    next-token loss, update the fast weights, continue from the new state).
+
+    Readings where the pages are silent:
+      * greedy: the next token is the argmax of the logits of the position
+        before it, ties to the lowest token id (np.argmax keeps the first);
+      * chunks keep the prefill's grid of absolute positions [cb, (c+1)b): a
+        trailing partial prompt chunk (scored but not applied by the
+        prefill) is completed by the first generated tokens and then
+        applied; the page names the half chunk as an open serving question;
+      * a position is scored with the fast weights of its chunk, before that
+        chunk's update: the token after position T-1 comes from the logits
+        the prefill computed for T-1, and the token after the last position
+        of a chunk from that position's pre-update logits;
+      * the chunk's update is the prefill's: the mean loss over its b
+        targets, the explicit backward, one SGD step (eq. (9))."""
+    cfg = model.cfg
+    b = cfg.b
+    eta = cfg.eta if eta is None else eta
+    prompt = np.asarray(prompt, dtype=np.int64)
+    T = len(prompt)
+    pre = prefill(model, prompt, eta=eta, keep_state=True, capacity=T + n_gen)
+    W, state = pre.W, pre.state
+    toks = [int(t) for t in prompt]
+    z = pre.z_last  # logits of position T-1
+    gen, losses, updates = [], [], []
+    none = np.full(1, -1, dtype=np.int64)
+    for p in range(T, T + n_gen):
+        x = int(np.argmax(z))
+        m = z.max()
+        losses.append(float(m + np.log(np.exp(z - m).sum()) - z[x]))
+        gen.append(x)
+        toks.append(x)
+        # forward of position p with the current fast weights (keys/values cached in `state`)
+        _, fwd = forward_chunk(model, W, state, np.asarray([x]), p, none)
+        z = fwd["z_last"]
+        if (p + 1) % b == 0:
+            # chunk [c0, p] is complete: every target is known once position p's argmax is
+            c0 = p + 1 - b
+            tgt = np.asarray(toks[c0 + 1:p + 1] + [int(np.argmax(z))], dtype=np.int64)
+            # its forward again, in one pass: the same W and cached keys give the same values
+            _, cf = forward_chunk(model, W, state, np.asarray(toks[c0:p + 1]), c0, tgt)
+            G = backward_chunk(model, W, cf, np.full(b, 1.0 / b))
+            for l in G:
+                for name in G[l]:
+                    W[l][name] = W[l][name] - eta * G[l][name]   # eq. (9)
+            updates.append(p)
+    return DecodeResult(np.asarray(gen, dtype=np.int64), np.asarray(losses), W, updates, pre)
 
 
 def static_losses(model, toks, k=None, fast=None):
