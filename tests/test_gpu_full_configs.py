@@ -1,23 +1,31 @@
 """Parity at the full workload sizes, in the launch configuration bench.py
 times (one sequence of T tokens through ttt_prefill).
 
-The oracle cannot run a whole 128K-token prefill, so it runs a prefix: by
-causality (算法 1 of the reading notes scores every position of a chunk
-before that chunk's labels update W), the losses of positions 0 .. T'-2 of the full GPU
-run equal those of a T'-token run, and W after the chunks that end before
-T'-1 is the same.  T' covers one full chunk (so an SGD update happens) and
-part of the next (scored with the updated weights).  At full size the GPU
-run is also checked for properties that hold at any size: run-to-run
+The oracle cannot run a whole 128K-token prefill in a test, so it runs a
+prefix: by causality (算法 1 of the reading notes scores every position of a
+chunk before that chunk's targets update W), the losses of positions
+0 .. T'-2 of the full GPU run equal those of a T'-token run.  T' covers one
+full chunk (so an SGD update happens) and part of the next (scored with the
+updated weights).  At 125M the oracle runs here; at 760M and 2.7B its losses
+were written once by tests/golden/make_prefix_losses.py (oracle only).  The
+760M prefix crosses the 16 384-position boundary where the GPU path starts
+the second super-chunk of its fast-weight-free blocks.  At full size the
+2.7B run is also checked for properties that hold at any size: run-to-run
 bit-identical losses, causality under a perturbed late token, finiteness.
 
-Tolerances: bf16 mean chunk loss 1e-2 absolute and per-token loss 5e-2
-absolute.  At 2.7B (32 blocks, d = 2560) the per-token bound is reached by
-the bf16 rounding of the activations alone: rounding the same tensors to
-bf16 in the fp64 CPU model (bf16_rounding_noise.py in this directory)
-gives the same error distribution as the GPU at 125M, and at 2.7B a few
-positions in a thousand land between 5e-2 and 6e-2 while the chunk means
-stay within 1e-3.  There the per-token check is on the 99.5th percentile
-(5e-2) plus a ceiling of 8e-2 on the maximum."""
+Tolerances (bf16): every chunk's mean loss within 1e-2 absolute, and the
+per-token loss within 5e-2 absolute at every compared position — unless the
+bf16 storage floor of the workload itself exceeds 5e-2.  The floor is the
+loss difference between the oracle's fp64 forward with and without the
+bf16 roundings of the stored activations (oracle/bf16_floor.py, stored for
+2.7B's first chunk in tests/golden/bf16_floor_2.7b.json); no bf16 pipeline
+with these storage points can beat it.  Where it reaches past 5e-2 (2.7B),
+the GPU's per-token errors must stay within the floor's distribution: the
+50th, 90th and 99th percentiles and the maximum at most 1.25 times the
+floor's, in each chunk compared."""
+import json
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -28,6 +36,8 @@ import synth
 from ._gpu_helpers import chunk_means
 
 pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
 
 
 def _gpu_run(cfg, toks, weights_dev, ctx_cache):
@@ -40,8 +50,33 @@ def _gpu_run(cfg, toks, weights_dev, ctx_cache):
     return losses.cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("name,prefix", [("125m", 1536), ("760m", 1536), ("2.7b", 1536)])
-def test_full_size_prefix_parity(name, prefix):
+def _stored_prefix(name):
+    with open(os.path.join(GOLDEN, f"prefix_losses_{name}.json")) as fh:
+        js = json.load(fh)
+    return [(a, b, np.asarray(v, dtype=np.float64)) for (a, b), v in zip(js["ranges"], js["losses"])]
+
+
+def _floor(name):
+    path = os.path.join(GOLDEN, f"bf16_floor_{name}.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        return np.asarray(json.load(fh)["abs_err"], dtype=np.float64)
+
+
+def _per_token_ok(d, floor, where):
+    """max |d| <= 5e-2, or (when the storage floor exceeds 5e-2) d within 1.25x the floor's distribution."""
+    if floor is None or floor.max() <= 5e-2:
+        assert d.max() <= 5e-2, (where, d.max())
+        return
+    for q in (50, 90, 99):
+        assert np.percentile(d, q) <= 1.25 * np.percentile(floor, q), (where, q, np.percentile(d, q),
+                                                                       np.percentile(floor, q))
+    assert d.max() <= 1.25 * floor.max(), (where, d.max(), floor.max())
+
+
+@pytest.mark.parametrize("name", ["125m", "760m", "2.7b"])
+def test_full_size_prefix_parity(name):
     from test_long_context_b200.context import upload_weights
     cfg = synth.get_config(name)
     w = synth.make_weights(cfg)
@@ -51,15 +86,22 @@ def test_full_size_prefix_parity(name, prefix):
     full = _gpu_run(cfg, toks, gw, cache)
     T = cfg.T
     assert np.isnan(full[T - 1]) and np.all(np.isfinite(full[:T - 1]))
-    ref = oracle.prefill(oracle.Model(cfg, w.arrays), toks[:prefix]).losses
-    d = np.abs(full[:prefix - 1] - ref[:prefix - 1])
-    if name == "2.7b":
-        assert np.percentile(d, 99.5) <= 5e-2, np.percentile(d, 99.5)
-        assert d.max() <= 8e-2, d.max()
+    if name == "125m":
+        prefix = 1536
+        ref = oracle.prefill(oracle.Model(cfg, w.arrays), toks[:prefix]).losses
+        spans = [(0, prefix - 1, ref[:prefix - 1])]
     else:
-        assert d.max() <= 5e-2, d.max()
-    cm = np.abs(chunk_means(full[:prefix - 1], cfg.b) - chunk_means(ref[:prefix - 1], cfg.b))
-    assert cm.max() <= 1e-2, cm.max()
+        spans = _stored_prefix(name)
+    floor = _floor(name)
+    B = cfg.b
+    for a, b, ref in spans:
+        d = np.abs(full[a:b] - ref)
+        # per chunk: positions before the first update and after it are compared separately
+        for c0 in range(a - a % B, b, B):
+            lo, hi = max(a, c0), min(b, c0 + B)
+            _per_token_ok(d[lo - a:hi - a], floor, (name, lo, hi))
+        cm = np.abs(chunk_means(full[a:b], B) - chunk_means(ref, B))
+        assert cm.max() <= 1e-2, (name, a, cm.max())
     if name == "2.7b":
         # properties at full size: determinism and causality
         again = _gpu_run(cfg, toks, gw, cache)
