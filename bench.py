@@ -15,9 +15,14 @@ sequence (the path does not shard: replicas only); value = tokens of all
 ranks / max over ranks of the device time.
 
 --impl reference times the CPU oracle (oracle/) on this machine's host cores on
-a bounded sample of the same workload: the first CPU_SAMPLE tokens of the
-sequence per step (at 2.7B that prefix is shorter than one chunk, so the
-sample is forward and loss only, which favours the CPU).
+a bounded sample of the same workload per step: the first CPU_SAMPLE tokens
+of the sequence as one chunk (the chunk length set to CPU_SAMPLE), so the
+sample runs the whole loop once: forward, loss, backward through the updated
+blocks and the SGD step.  The same sample gives cpu_baseline.
+
+After the headline workload, the other workloads (tiny fp32, 125M, 760M) get
+one short timing each under "per_config": tokens/s, per-1K-token latency and
+the achieved fraction of the roofline.
 """
 from __future__ import annotations
 
@@ -34,10 +39,16 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "prefill tokens/s (2.7B, SWA k=8K, TTT b=1K, T=128K) and % of bf16 tensor peak"
-# Tokens of the CPU oracle's bounded sample: about half a minute of fp64 work
-# per call at 2.7B on a 16-core host.
-CPU_SAMPLE = 256
-KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope")
+# Tokens of the CPU oracle's bounded sample, run as one chunk of that length
+# (forward, loss, backward, update): about ten seconds of fp64 work at 2.7B
+# on a 16-core host, most of it widening the weights to fp64.
+CPU_SAMPLE = 128
+# Workloads timed after the headline one (name -> timed steps)
+PER_CONFIG = ("tiny", "125m", "760m")
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope", "decode")
+# Greedy generation after the headline prefill (the 2.7B decode workload):
+# tokens generated, one SGD step on the fast MLPs after every chunk of them
+DECODE_TOKENS = 8192
 
 
 def parse_args():
@@ -50,6 +61,8 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=0, help="override T (testing only; not a bench line)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--decode-tokens", type=int, default=DECODE_TOKENS, help="0 skips the decode measurement")
     return ap.parse_args()
 
 
@@ -200,6 +213,15 @@ def latency_by_tokens(ctx, tok_dev, losses, T, stream, lengths=(8192, 16384, 327
     return out
 
 
+def marginal_latency(by_T):
+    """Per-1K-token cost of the tokens added between consecutive prefix
+    lengths, (t(T2) - t(T1)) / (T2 - T1): flat once the window is full
+    (reading notes, eq. (11)), while the average over a whole prefix still
+    carries the cheaper first k positions."""
+    pts = sorted((int(n), v * int(n) / 1000.0) for n, v in by_T.items())
+    return {f"{a}-{b}": (tb - ta) / ((b - a) / 1000.0) for (a, ta), (b, tb) in zip(pts, pts[1:])}
+
+
 def workload_name(cfg, T):
     return (f"{cfg.name} TTT-E2E prefill: L={cfg.n_layers} d={cfg.d_model} H={cfg.n_heads}x{cfg.head_dim} "
             f"f={cfg.d_ff} V={cfg.vocab} n_u={cfg.n_updated} T={T} k={cfg.k} b={cfg.b} batch=1")
@@ -212,25 +234,27 @@ def config_dict(cfg, T, n):
 
 
 def cpu_baseline(cfg, weights_arrays, toks, sample_tokens):
+    """The oracle as it stands on this host's cores: the first `sample_tokens`
+    tokens as one chunk of that length, so the sample runs forward, loss,
+    backward and the SGD update once."""
     import numpy as np
 
     import oracle
     m = oracle.Model(cfg, weights_arrays)
     t0 = time.perf_counter()
-    oracle.prefill(m, np.asarray(toks[:sample_tokens]))
+    oracle.prefill(m, np.asarray(toks[:sample_tokens]), b=sample_tokens)
     dt = time.perf_counter() - t0
     cores = os.cpu_count()
-    what = ("one full chunk with backward and SGD update" if sample_tokens >= cfg.b else
-            f"shorter than one chunk (b = {cfg.b}), so forward and loss only, no backward or update")
     return {"value": sample_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"oracle (fp64 numpy, BLAS threads = {cores}) prefill of the first {sample_tokens} tokens of "
-                       f"the same sequence: {what}; the window is not yet full either, so this favours the CPU"),
+            "sample": (f"oracle (fp64 numpy, BLAS threads = {cores}): the first {sample_tokens} tokens of the same "
+                       f"sequence as one chunk of {sample_tokens} (the workload's chunk is {cfg.b}): forward, loss, "
+                       f"backward through the {cfg.n_updated} updated blocks and the SGD step, including the "
+                       f"per-call widening of the weights to fp64; the window is not yet full"),
             "seconds": dt}
 
 
 def cpu_baseline_sample_text(cfg, sample):
-    return (f"first {sample} tokens" + (" (one full chunk with backward and update)" if sample >= cfg.b else
-                                        " (less than one chunk: forward and loss only)"))
+    return (f"first {sample} tokens as one chunk of {sample} (forward, loss, backward, SGD update)")
 
 
 def run_reference(args, cfg, T):
@@ -258,6 +282,110 @@ def run_reference(args, cfg, T):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def time_decode(ctx, cfg, tok_dev, T, n_tokens, stream):
+    """Greedy generation of n_tokens after a prefill of the T-token prompt
+    (the 2.7B decode workload): one ttt_decode call per chunk of b tokens,
+    each bracketed by CUDA events on the context's stream.  Reports tokens/s,
+    per-token latency, the time the chunk updates add (from the per-class
+    timing: the backward and SGD kernels run only at chunk ends), and the
+    HBM roofline of the per-position kernels (their algorithmic bytes: every
+    weight read once per position plus the window's keys and values)."""
+    import torch
+    peaks, src = load_peaks()
+    b = cfg.b
+    ctx.reset()
+    ctx.prefill(tok_dev, sync=False)
+    ctx.decode(64, sync=True)  # warm-up (kernels loaded, first pick taken)
+    ctx.reset()
+    ctx.prefill(tok_dev, sync=False)
+    ctx.sync()
+    toks = torch.empty(n_tokens, device="cuda", dtype=torch.int32)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_tokens // b + 2)]
+    evs[0].record(stream)
+    done, i = 0, 0
+    while done < n_tokens:
+        n = min(b - (T + done) % b, n_tokens - done)  # up to the next chunk end
+        ctx.decode(n, tokens=toks[done:done + n], sync=False)
+        done += n
+        i += 1
+        evs[i].record(stream)
+    ctx.sync()
+    total_ms = evs[0].elapsed_time(evs[i])
+    per_chunk = [evs[j].elapsed_time(evs[j + 1]) for j in range(i)]
+    # one more chunk with per-launch timing: bytes and time of the per-position
+    # kernels, and the time of the chunk's update (every other class)
+    ctx.timing_enable(True)
+    ctx.decode(b, sync=False)
+    timing = ctx.timing_read()
+    ctx.timing_enable(False)
+    dms, dn, dbytes = timing["decode"]
+    upd_ms = sum(v[0] for k, v in timing.items() if k != "decode")
+    n_upd = (T + n_tokens) // b - T // b
+    return {"workload": f"{cfg.name} greedy decode of {n_tokens} tokens after a {T}-token prefill, window {cfg.k}, "
+                        f"one SGD step on the fast MLPs after every {b} generated positions",
+            "tokens": n_tokens, "tokens_per_s": n_tokens / (total_ms / 1000.0), "ms_per_token": total_ms / n_tokens,
+            "updates": n_upd, "update_ms_each": upd_ms,
+            "ms_per_chunk_of_tokens": per_chunk,
+            "launches_per_token": dn / b,
+            "roofline": {"bound": "hbm", "kernel": "decode (per-position kernels)",
+                         "achieved": dbytes / (dms / 1000.0) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": dbytes / (dms / 1000.0) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_token": dbytes / b, "peak_source": src,
+                         "note": "per-launch events of one further chunk of b tokens"},
+            "first_tokens": toks[:8].cpu().tolist()}
+
+
+def time_config(name, steps=3, warmup=2):
+    """Short timing of one more workload (its own T, k, b, dtype) on this GPU:
+    tokens/s, per-1K-token latency and the achieved fraction of its roofline
+    (bf16: algorithmic flops against the sustained bf16 peak; fp32: against
+    the fp32 FMA peak of the SIMT kernels)."""
+    import torch
+
+    import synth
+    from test_long_context_b200.context import Context, upload_weights
+    cfg = synth.get_config(name)
+    T = cfg.T
+    gw = {}
+    for n, arr, bits in synth.iter_weights(cfg):
+        gw.update(upload_weights([(n, arr, bits)], cfg.dtype))
+    tok = torch.from_numpy(synth.tokens(cfg)).cuda()
+    stream = torch.cuda.current_stream()
+    ctx = Context(cfg, gw, stream=stream)
+    losses = torch.empty(T, device="cuda")
+    for _ in range(warmup):
+        ctx.reset()
+        ctx.prefill(tok, losses, sync=False)
+    ctx.sync()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        ctx.reset()
+        ctx.prefill(tok, losses, sync=False)
+    e1.record(stream)
+    ctx.sync()
+    ms = e0.elapsed_time(e1) / steps
+    ok = bool(torch.isfinite(losses[:-1]).all().item())
+    ctx.close()
+    del gw
+    torch.cuda.empty_cache()
+    peaks, src = load_peaks()
+    flops = algorithmic_flops(cfg, T)
+    if cfg.dtype == "f32":
+        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        bound = "alu"
+    else:
+        peak, bound = peaks["bf16_tflops_sustained"], "tensor"
+    achieved = flops / (ms / 1000.0) / 1e12
+    return {"workload": workload_name(cfg, T), "dtype": cfg.dtype, "tokens_per_s": T / (ms / 1000.0),
+            "ms_per_step": ms, "ms_per_1k_tokens": ms / (T / 1000.0), "steps": steps, "warmup": warmup,
+            "algorithmic_tflop_per_step": flops / 1e12,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "peak_source": src},
+            "finite_losses": ok}
 
 
 def main():
@@ -359,6 +487,9 @@ def main():
                "ms_per_step": ems / args.steps}
 
     by_T = latency_by_tokens(ctx, tok_dev, losses, T, stream)
+    dec = None
+    if args.decode_tokens > 0 and not args.tokens and args.config == "2.7b":
+        dec = time_decode(ctx, cfg, tok_dev, T, args.decode_tokens, stream)
 
     if rank == 0:
         peaks, peak_src = load_peaks()
@@ -392,15 +523,21 @@ def main():
                 "config": config_dict(cfg, T, world),
                 "ms_per_1k_tokens": (ms / args.steps) / (T / 1000.0),
                 "ms_per_1k_tokens_by_T": by_T,
+                "ms_per_1k_tokens_marginal": marginal_latency(by_T),
                 "tensor_peak_frac": flops_step * world * args.steps / (ms / 1000.0) / 1e12 / tensor_peak,
                 "algorithmic_tflop_per_step": flops_step / 1e12,
                 "roofline": roof, "kernel_classes": classes, "gpu_launches": int(launches),
-                "clocks": clk, "e2e": e2e}
+                "clocks": clk, "e2e": e2e, "decode": dec}
+    ctx.close()
+    del gw
+    torch.cuda.empty_cache()
+    if rank == 0:
+        if not args.no_per_config and world == 1 and args.config == "2.7b" and not args.tokens:
+            line["per_config"] = {name: time_config(name) for name in PER_CONFIG}
         if want_cpu:
             line["cpu_baseline"] = cpu_baseline(cfg, keep, toks, min(CPU_SAMPLE, T))
             line["cpu_baseline"].pop("seconds", None)
         print(json.dumps(line), flush=True)
-    ctx.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -146,10 +146,33 @@ int ttt_prefill(ttt_ctx* ctx, const int32_t* tokens_dev, int64_t T, float* losse
                 float* const* fast_out_dev);
 
 /*
- * Greedy generation with periodic updates (算法 3).  Not provided by this
- * build: returns TTT_ERR_UNSUPPORTED.
+ * Greedy generation with periodic fast-weight updates (算法 3 of the reading
+ * notes: generate causally from the state the prefill left, collect the new
+ * tokens until an inner chunk is full, update the fast weights on that
+ * chunk's next-token loss, continue from the new state).
+ * Each generated token is the argmax of the logits of the position before it
+ * (ties: the lowest token id).  The first one comes from the logits of the
+ * prompt's last position T-1, as the prefill scored it (with the fast weights
+ * of before its chunk's update).  Chunks keep the prefill's grid of absolute
+ * positions [c*b, (c+1)*b): when T % b != 0 the prompt's trailing partial
+ * chunk (scored, not applied, by the prefill) is completed by the first
+ * generated tokens.  After the forward of the last position of a chunk (its
+ * argmax gives that position's target), the chunk takes one SGD step on the
+ * mean loss of its b targets, exactly as in ttt_prefill, and generation
+ * continues with the updated weights.
+ * ttt_decode_step writes one token (int32) to next_token_dev and runs the
+ * forward of its position.  Requires a ttt_prefill since the last
+ * ttt_init / ttt_reset (TTT_ERR_STATE otherwise); asynchronous on the stream.
  */
 int ttt_decode_step(ttt_ctx* ctx, int32_t* next_token_dev);
+
+/*
+ * n_tokens steps of ttt_decode_step in one call: tokens_dev[i] (int32,
+ * device) receives the i-th generated token; losses_dev (fp32, device, may be
+ * NULL) receives, for each generated token, the loss of the position before
+ * it against it (log-sum-exp of that position's logits minus their maximum).
+ */
+int ttt_decode(ttt_ctx* ctx, int64_t n_tokens, int32_t* tokens_dev, float* losses_dev);
 
 /* Restore W_init (a fresh copy for a new document, as 算法 2 starts each document), empty the
  * attention state and set the position to 0.  Asynchronous on the stream. */
@@ -186,7 +209,9 @@ int64_t ttt_launch_count(ttt_ctx* ctx);
 #define TTT_KC_OTHER 3 /* embedding, SwiGLU backward, CE finalise, targets, copies */
 #define TTT_KC_NORM 4  /* RMSNorm forward and backward */
 #define TTT_KC_ROPE 5  /* QK-norm + RoPE forward (with the KV-ring write) and backward */
-#define TTT_KC_COUNT 6
+#define TTT_KC_DECODE 6 /* generation's per-position kernels; their third total counts algorithmic
+                           HBM bytes (weights and window keys/values read), not flops */
+#define TTT_KC_COUNT 7
 int ttt_timing_enable(ttt_ctx* ctx, int32_t enable);
 int ttt_timing_read(ttt_ctx* ctx, int32_t kernel_class, double* total_ms, int64_t* launches, double* flops);
 

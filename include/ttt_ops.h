@@ -155,6 +155,63 @@ int ttt_op_swa_backward_noalloc(int32_t dtype, int32_t n_heads, int32_t head_dim
                                 int64_t lddo, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv,
                                 void* stream);
 
+/*
+ * Memory-bound kernels of the loop, one launch each (bf16 only; they exist so
+ * that each can be timed and profiled on its own at the workload's shapes).
+ *
+ * RMSNorm (reading notes §6 block structure, pre-norm): for row i < n,
+ * r = 1/sqrt(mean_j x[i,j]^2 + eps), y[i,j] = bf16(x[i,j] * r * g[j]),
+ * rstd[i] = r.  x fp32 [n, ldx], g fp32 [d], y bf16 [n, ldy], rstd fp32 [n].
+ */
+int ttt_op_rmsnorm(int64_t n, int32_t d, const float* x, int64_t ldx, const float* g, float eps, void* y,
+                   int64_t ldy, float* rstd, void* stream);
+
+/*
+ * QK-norm + RoPE of n positions p0 .. p0+n-1 with the key/value ring write:
+ * qkv bf16 [n, ldqkv] holds (q | k | v) raw projections of n_heads heads of
+ * head_dim; per head q and k get RMSNorm over head_dim (gains gq, gk fp32
+ * [head_dim]) and the rotation of pairs (i, i + head_dim/2) by angle
+ * p * theta^(-2i/head_dim); q goes to qout [n, ldq], k and v to the rings
+ * [R, n_heads*head_dim] at slot p % R; rq, rk fp32 [n, n_heads] receive the
+ * RMS factors.  The angles are computed in fp64 into a table (scratch `tab`,
+ * fp32 pairs [n, head_dim/2], caller-owned) first.
+ */
+int ttt_op_qknorm_rope(int64_t n, int64_t p0, int32_t n_heads, int32_t head_dim, float eps, float theta,
+                       const void* qkv, int64_t ldqkv, const float* gq, const float* gk, void* qout, int64_t ldq,
+                       void* kring, void* vring, int64_t R, float* rq, float* rk, float* tab, void* stream);
+
+/*
+ * SwiGLU backward on (gate 64 | up 64) interleaved columns: for n rows and
+ * nfeat features j (pair j/64, lane j%64), with g, u from gu [n, ldgu] and
+ * da [n, ldda] (all bf16): dg = da * u * s(g) * (1 + g (1 - s(g))),
+ * du = da * g * s(g) (s = sigmoid), written interleaved to dgu [n, lddgu].
+ */
+int ttt_op_swiglu_bwd(int64_t n, int64_t nfeat, const void* da, int64_t ldda, const void* gu, int64_t ldgu,
+                      void* dgu, int64_t lddgu, void* stream);
+
+/*
+ * Matrix-vector product of generation (bf16 W [n, ldw], x [k]; fp32
+ * accumulation): epilogue 0 stores y (bf16 [n]) to out, 1 adds y to res
+ * (fp32 [n]) into out (fp32), 2 applies SwiGLU to (gate 64 | up 64) row
+ * blocks (out bf16 [n/2], raw bf16 [n] or NULL), 3 greedy-picks: out (int32
+ * [1]) = the row with the largest y (ties: the lowest row), lse_out (fp32 [1],
+ * may be NULL) = log sum exp y; part is scratch of 3 * 1184 floats.  Rows
+ * 16-byte aligned, k a multiple of 8.
+ */
+int ttt_op_gemv(int32_t epilogue, int64_t n, int64_t k, const void* w, int64_t ldw, const void* x, void* out,
+                const float* res, void* raw, float* lse_out, float* part, void* stream);
+
+/*
+ * One query per head at absolute position p over keys p-window+1 .. p of the
+ * rings (bf16 [R, n_heads*head_dim], slot = position % R, R >= window): o
+ * (bf16 [n_heads*head_dim]) and lse (fp32 [n_heads], natural log, may be
+ * NULL); scores scaled by 1/sqrt(head_dim).  ws: fp32 scratch of
+ * n_heads * (ceil(window / 128) + 1) * (head_dim + 2) floats.
+ */
+int ttt_op_attn_decode(int32_t n_heads, int32_t head_dim, int64_t p, int32_t window, const void* q,
+                       const void* kring, const void* vring, int64_t R, void* o, float* lse, float* ws,
+                       void* stream);
+
 /* Device watchdog self-test: launches one thread that waits on an mbarrier
  * nothing ever arrives at.  The bounded wait gives up (about 2 s) and records
  * a timeout, so the following ttt_op_sync returns TTT_ERR_TIMEOUT and the

@@ -20,8 +20,8 @@ TTT_ERR_UNSUPPORTED = -6
 TTT_F32 = 0
 TTT_BF16 = 1
 
-KC_GEMM, KC_ATTN_FWD, KC_ATTN_BWD, KC_OTHER, KC_NORM, KC_ROPE = range(6)
-KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope")
+KC_GEMM, KC_ATTN_FWD, KC_ATTN_BWD, KC_OTHER, KC_NORM, KC_ROPE, KC_DECODE = range(7)
+KC_NAMES = ("gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope", "decode")
 EPI_STORE_F32, EPI_STORE_BF16, EPI_ADD_F32, EPI_SWIGLU, EPI_CE_FWD, EPI_CE_BWD, EPI_SGD = range(7)
 
 c_i32, c_i64, c_f32, c_vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
@@ -67,6 +67,7 @@ def lib():
                                  c_i32, c_vp, ctypes.POINTER(c_vp)]),
             "ttt_prefill": (c_i32, [c_vp, c_vp, c_i64, c_vp, ctypes.POINTER(c_vp)]),
             "ttt_decode_step": (c_i32, [c_vp, c_vp]),
+            "ttt_decode": (c_i32, [c_vp, c_i64, c_vp, c_vp]),
             "ttt_reset": (c_i32, [c_vp]),
             "ttt_sync": (c_i32, [c_vp]),
             "ttt_last_error": (ctypes.c_char_p, [c_vp]),
@@ -93,6 +94,13 @@ def lib():
             "ttt_op_swa_backward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp,
                                             c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64,
                                             c_vp, c_i32, c_vp]),
+            "ttt_op_rmsnorm": (c_i32, [c_i64, c_i32, c_vp, c_i64, c_vp, c_f32, c_vp, c_i64, c_vp, c_vp]),
+            "ttt_op_qknorm_rope": (c_i32, [c_i64, c_i64, c_i32, c_i32, c_f32, c_f32, c_vp, c_i64, c_vp, c_vp, c_vp,
+                                           c_i64, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp]),
+            "ttt_op_swiglu_bwd": (c_i32, [c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp, c_i64, c_vp]),
+            "ttt_op_gemv": (c_i32, [c_i32, c_i64, c_i64, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+            "ttt_op_attn_decode": (c_i32, [c_i32, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp,
+                                           c_vp]),
         }
         for name, (res, args) in sig.items():
             if hasattr(L, name):
@@ -120,9 +128,10 @@ def exported_symbols():
     """Names of the ttt_* entry points the loaded library exports."""
     L = lib()
     names = []
-    for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
+    for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_decode", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
               "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_dual", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
-              "ttt_op_swa_backward", "ttt_op_watchdog_selftest",
+              "ttt_op_swa_backward", "ttt_op_watchdog_selftest", "ttt_op_rmsnorm", "ttt_op_qknorm_rope",
+              "ttt_op_swiglu_bwd", "ttt_op_gemv", "ttt_op_attn_decode",
               "ttt_op_swa_backward_noalloc"):
         if hasattr(L, n):
             names.append(n)

@@ -86,6 +86,25 @@ class Context:
             self.sync()
         return losses, fast_out
 
+    def decode_step(self, out=None, sync=True):
+        """ttt_decode_step: one greedy token (int32 CUDA tensor [1])."""
+        if out is None:
+            out = torch.empty(1, device="cuda", dtype=torch.int32)
+        L.check(L.lib().ttt_decode_step(self.h, _p(out)), self.h)
+        if sync:
+            self.sync()
+        return out
+
+    def decode(self, n, tokens=None, losses=None, sync=True):
+        """ttt_decode: n greedy tokens (int32 [n]) and, when `losses` is given
+        (fp32 [n]), the loss of the position before each token against it."""
+        if tokens is None:
+            tokens = torch.empty(n, device="cuda", dtype=torch.int32)
+        L.check(L.lib().ttt_decode(self.h, n, _p(tokens), _p(losses)), self.h)
+        if sync:
+            self.sync()
+        return tokens, losses
+
     def reset(self):
         L.check(L.lib().ttt_reset(self.h), self.h)
 

@@ -51,4 +51,15 @@ int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t
                    const void* v, int64_t ring, int64_t ldkv);
 int swa_tc_forward(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err);
 
+// Shared by the op-level entry points (ops.cu, noalloc.cu): the forward
+// arguments of one call (k/v ring pitch heads*head_dim, lse pitch n, scale
+// 1/sqrt(head_dim)), and the backward dispatch - tensor cores for bf16 with a
+// supported head_dim, a ring of whole 128-row tiles and q, dout sharing a
+// pitch, unless flags has TTT_SWA_FORCE_SIMT; SIMT otherwise.  a.D must point
+// to n*heads fp32 of work space.  Kernels report bounded-wait timeouts in the
+// op-level error word (ttt_op_sync).
+SwaArgs op_swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t window, const void* q, int64_t ldq,
+                    const void* k, const void* v, int64_t ring, void* o, int64_t ldo, const float* lse);
+int op_swa_backward_run(const SwaArgs& a, int32_t dtype, int32_t flags, cudaStream_t st);
+
 }  // namespace ttt

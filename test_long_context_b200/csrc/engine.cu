@@ -21,12 +21,14 @@
 #include "../../include/ttt.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "decode.cuh"
 #include "elementwise.cuh"
 #include "gemm.cuh"
 
 struct ttt_ctx {
   virtual ~ttt_ctx() = default;
   virtual int prefill(const int32_t* tok, int64_t T, float* losses, float* const* fast_out) = 0;
+  virtual int decode(int64_t count, int32_t* tokens, float* losses) = 0;
   virtual int reset() = 0;
   virtual int sync() = 0;
   virtual int timing_enable(bool on) = 0;
@@ -90,6 +92,9 @@ struct Gemm {
   bool bf = false;
   int64_t split = 1;  // deterministic split-K count (bf16 mode)
   const char* label = "gemm";
+  // the product recomputes values the forward already had (the LM-head
+  // logits of the backward): its flops are not algorithmic work
+  bool recompute = false;
 };
 
 // Event timing of launches, per kernel class (opt-in).  Back-to-back launches
@@ -185,6 +190,7 @@ class Engine final : public ttt_ctx {
 
   int init();
   int prefill(const int32_t* tok, int64_t T_, float* losses, float* const* fast_out) override;
+  int decode(int64_t count, int32_t* tokens, float* losses) override;
   int reset() override;
   int sync() override;
   ~Engine() override {
@@ -218,13 +224,25 @@ class Engine final : public ttt_ctx {
   int run(Gemm& g, int64_t rows);  // rows overrides the M extent (chunk/super-chunk length)
   int bottom_layers(const int32_t* tok, int64_t s0, int64_t S);
   int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
+  // backward through the updated blocks and the SGD steps of the chunk at p0
+  // (n rows of the per-chunk buffers, targets in tgt_, CE scale in scl_)
+  int chunk_backward(int64_t p0, int64_t n);
+  // generation: the forward of position p (token in dtok_) through every
+  // block, the greedy pick of the next token, and the chunk's update when p
+  // is its last position
+  int decode_position(int64_t p);
+  // greedy pick from the final-norm output row hf (the LM head as a
+  // matrix-vector product): next token -> dtok_, loss -> dloss_
+  int head_pick(const T* hf, int32_t* tgt_row, float* lse_row);
+  template <typename G>
+  int gemv_run(const GemvArgs<T>& a, int epi, G&& bytes_of);
   // Launch `f` (returns a status); bracket it with events when timing is on.
   template <typename F>
   int timed(int kc, double flops, F&& f, const char* label = nullptr) {
     ++launches;
     if (trace_) return traced(kc, f);
     if (!timer_.on) return f();
-    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope"};
+    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope", "decode"};
     cudaEvent_t a = timer_.chain;
     const bool own_a = a == nullptr;
     if (own_a) {
@@ -243,7 +261,7 @@ class Engine final : public ttt_ctx {
   // TTT_TRACE=1: synchronise after every launch and log it to stderr (debugging aid).
   template <typename F>
   int traced(int kc, F&& f) {
-    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope"};
+    static const char* names[TTT_KC_COUNT] = {"gemm", "attn_fwd", "attn_bwd", "other", "norm", "rope", "decode"};
     if (trace_verbose_) fprintf(stderr, "[ttt trace] launching %lld %s\n", (long long)launches, names[kc]);
     cudaEvent_t a = timer_.get(), b = timer_.get();
     TTT_CUDA_TRY(cudaEventRecord(a, st_));
@@ -315,6 +333,16 @@ class Engine final : public ttt_ctx {
   float trace_ms_ = 0.f;
   bool fresh_ = true;
   int* err_ = nullptr;
+  // generation state: the next position to process, whether dtok_ already
+  // holds its token, and the chunk start of the last processed position
+  bool prefilled_ = false, dec_ready_ = false;
+  int64_t dec_pos_ = 0;
+  int32_t* dtok_ = nullptr;
+  float* dloss_ = nullptr;
+  float* xd_ = nullptr;        // residual of the generated position through the blocks without fast weights
+  float* adws_ = nullptr;      // single-query attention work space
+  float* gvpart_ = nullptr;    // LM-head greedy-pick partials
+  int64_t gvparts_ = 0;
 
   int64_t d_ = 0, f_ = 0, H_ = 0, HD_ = 0, V_ = 0, L_ = 0, nbot_ = 0;
   int64_t S_ = 0, R1_ = 0, R_ = 0, Vc_ = 0, nvc_ = 0, ce_tiles_ = 0;
@@ -418,7 +446,7 @@ template <typename T>
 int Engine<T>::run(Gemm& g, int64_t rows) {
   GemmShape s = g.shape;
   if (rows > 0 && !s.a_mn) s.a.rows = rows;
-  const double flops = 2.0 * (double)s.M() * (double)s.N() * (double)s.K();
+  const double flops = g.recompute ? 0.0 : 2.0 * (double)s.M() * (double)s.N() * (double)s.K();
   if (BF) {
     TcGemm tc = g.tc;
     tc.args = g.args;
@@ -572,6 +600,13 @@ int Engine<T>::init() {
   TRY(arena_.alloc(&dgu_, b * 4 * f));
   TRY(arena_.alloc(&do_, b * d));
   TRY(arena_.alloc(&dqkv_, b * 3 * d));
+  // generation
+  TRY(arena_.alloc(&dtok_, 1));
+  TRY(arena_.alloc(&dloss_, 1));
+  TRY(arena_.alloc(&xd_, d));
+  TRY(arena_.alloc(&adws_, attn_decode_ws_floats((int)H_, (int)HD_, k_)));
+  gvparts_ = gemv_parts(V_);
+  TRY(arena_.alloc(&gvpart_, 3 * gvparts_));
 
   // ---- attention plans ----------------------------------------------------------------------
   tc_attn_ = BF && swa_tc_supported((int)HD_);
@@ -669,6 +704,7 @@ int Engine<T>::init() {
     e = EpiArgs{}; e.c = dz_; e.ldc = Vc_; e.row_f = lsef_; e.row_g = scl_; e.row_i = tgt_; e.col_offset = v0;
     TRY(prep(g_ce_dz_[c], 0, MatView{hf_, b, d, d}, 0, MatView{hv, vn, d, d}, EPI_CE_BWD, e));
     g_ce_dz_[c].label = "head.ce_dz";
+    g_ce_dz_[c].recompute = true;
     e = EpiArgs{}; e.c = dhf_; e.ldc = d;
     TRY(prep(g_ce_dh_[c], 0, MatView{dz_, b, vn, Vc_}, 1, MatView{hv, vn, d, d}, c == 0 ? EPI_STORE_F32 : EPI_ADD_F32,
              e));
@@ -696,6 +732,8 @@ int Engine<T>::reset() {
     }
   }
   fresh_ = true;
+  prefilled_ = dec_ready_ = false;
+  dec_pos_ = 0;
   return TTT_OK;
 }
 
@@ -773,7 +811,15 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
   TRY(timed(TTT_KC_OTHER, 0, [&] { return ce_finalize(pmax_, psum_, b, (int)ce_tiles_, zt_, n, n_valid, n_valid ? 1.f / (float)n_valid : 0.f,
                         losses + p0, lsef_, scl_, st_); }));
   if (n < b || n_valid == 0) return TTT_OK;  // a trailing partial chunk is scored only
+  // eta = 0: the step W -= 0 * G leaves every weight as it is, so the
+  // backward that would produce G is skipped (the L_static model of eq. (4))
+  if (eta_ == 0.f) return TTT_OK;
+  return chunk_backward(p0, n);
+}
 
+template <typename T>
+int Engine<T>::chunk_backward(int64_t p0, int64_t n) {
+  const int64_t d = d_, f = f_, b = b_;
   // ---- backward through the updated blocks, SGD on each fast MLP ----
   phase_ = "bwd";
   for (int64_t c = 0; c < nvc_; ++c) {
@@ -840,6 +886,9 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
       TRY(chunk(tok, T_, p0, n, xs_ + (p0 - s0) * d_, losses));
     }
   }
+  prefilled_ = true;
+  dec_ready_ = false;
+  dec_pos_ = T_;
   if (fast_out) {
     const int64_t d = d_, f = f_;
     for (int i = 0; i < nu_; ++i) {
@@ -850,6 +899,129 @@ int Engine<T>::prefill(const int32_t* tok, int64_t T_, float* losses, float* con
       TRY(timed(TTT_KC_OTHER, 0, [&] { return deinterleave_gate_up(master_gu(i), (int)f, (int)d, og, ou, st_); }));
       TRY(timed(TTT_KC_OTHER, 0, [&] { return copy2d<float>(master_d(i), master_d_ld(), od, f, d, f, st_); }));
     }
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+template <typename G>
+int Engine<T>::gemv_run(const GemvArgs<T>& a, int epi, G&& label) {
+  const double bytes = (double)sizeof(T) * ((double)a.n * (double)a.k + (a.w2 ? (double)(a.n - std::min<int64_t>(a.n, a.n_ext)) * (double)a.k2 : 0.0));
+  return timed(TTT_KC_DECODE, bytes, [&] { return gemv<T>(a, epi, st_); }, label);
+}
+
+template <typename T>
+int Engine<T>::head_pick(const T* hf, int32_t* tgt_row, float* lse_row) {
+  GemvArgs<T> g;
+  g.w = reinterpret_cast<const T*>(wt_.lm_head);
+  g.ldw = d_;
+  g.n = V_;
+  g.k = d_;
+  g.x = hf;
+  g.out = gvpart_;  // unused by the argmax epilogue, must be non-NULL
+  g.part = gvpart_;
+  TRY(gemv_run(g, GEMV_ARGMAX, "dec.head"));
+  return timed(TTT_KC_DECODE, 0, [&] { return argmax_finalize(gvpart_, gvparts_, dtok_, tgt_row, lse_row, dloss_, st_); },
+               "dec.pick");
+}
+
+template <typename T>
+int Engine<T>::decode_position(int64_t p) {
+  const int64_t d = d_, f = f_, b = b_;
+  const float eps = cfg_.norm_eps;
+  const int64_t c0 = p - p % b, r = p - c0;
+  phase_ = "dec";
+  if (tab_p0_ != c0) {  // rotation table of this chunk's positions (also read by its backward)
+    tab_p0_ = c0;
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return rope_table(rope_tab_, c0, b, (int)HD_, cfg_.rope_theta, st_); }, "dec.rope_table"));
+  }
+  TRY(timed(TTT_KC_DECODE, 0, [&] { return embed_gather<T>(dtok_, reinterpret_cast<const T*>(wt_.embed), 1, (int)d, (int)V_, xd_, err_, st_); }, "dec.embed"));
+  const double kv_bytes = 2.0 * (double)sizeof(T) * (double)d * (double)std::min<int64_t>(p + 1, k_);
+  // ---- blocks without fast weights: one row, scratch of the super-chunk buffers ----
+  for (int64_t l = 0; l < nbot_; ++l) {
+    const ttt_layer_weights& lw = wt_.layers[l];
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xd_, d, lw.attn_norm, eps, 1, (int)d, hs_, d, rs_, st_); }, "dec.norm"));
+    GemvArgs<T> g;
+    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.x = hs_; g.out = qkvs_;
+    TRY(gemv_run(g, GEMV_STORE, "dec.qkv"));
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, 1, p, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, qs_, d, kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }, "dec.qknorm_rope"));
+    TRY(timed(TTT_KC_DECODE, kv_bytes, [&] { return attn_decode<T>(qs_, kb_[l], vb_[l], d, R1_, (int)H_, (int)HD_, p, k_, scale_, os_, nullptr, 0, adws_, st_); }, "dec.attn"));
+    g = GemvArgs<T>();
+    g.w = reinterpret_cast<const T*>(lw.wo); g.ldw = d; g.n = d; g.k = d; g.x = os_; g.out = xd_; g.res = xd_;
+    TRY(gemv_run(g, GEMV_ADD_F32, "dec.o"));
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xd_, d, lw.mlp_norm, eps, 1, (int)d, hs_, d, rs_, st_); }, "dec.norm"));
+    g = GemvArgs<T>();
+    g.w = wgu_[l]; g.ldw = d; g.n = 2 * f; g.k = d; g.x = hs_; g.out = as_;
+    TRY(gemv_run(g, GEMV_SWIGLU, "dec.gateup"));
+    g = GemvArgs<T>();
+    g.w = wd_[l]; g.ldw = f; g.n = d; g.k = f; g.x = as_; g.out = xd_; g.res = xd_;
+    TRY(gemv_run(g, GEMV_ADD_F32, "dec.down"));
+  }
+  // ---- blocks with fast weights: row r of the chunk buffers (the chunk's backward reads them) ----
+  for (int i = 0; i < nu_; ++i) {
+    const int64_t l = nbot_ + i;
+    const ttt_layer_weights& lw = wt_.layers[l];
+    const float* xin = i == 0 ? xd_ : xin_[i] + r * d;
+    T* h = h_[i] + r * d;
+    T* qkv = qkv_[i] + r * 3 * d;
+    T* q = q_[i] + r * d;
+    T* o = o_[i] + r * d;
+    T* h2 = h2_[i] + r * d;
+    T* a = a_[i] + r * 2 * f;
+    float* xmid = xmid_[i] + r * d;
+    float* xout = (i + 1 < nu_ ? xin_[i + 1] : xf_) + r * d;
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, 1, (int)d, h, d, r1_[i] + r, st_); }, "dec.norm"));
+    GemvArgs<T> g;
+    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.x = h; g.out = qkv;
+    TRY(gemv_run(g, GEMV_STORE, "dec.qkv"));
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return qknorm_rope_fwd<T>(qkv, 3 * d, lw.q_norm, lw.k_norm, 1, p, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, q, d, kt_[i], vt_[i], d, R_, rq_[i] + r * H_, rk_[i] + r * H_, st_); }, "dec.qknorm_rope"));
+    TRY(timed(TTT_KC_DECODE, kv_bytes, [&] { return attn_decode<T>(q, kt_[i], vt_[i], d, R_, (int)H_, (int)HD_, p, k_, scale_, o, lse_[i] + r, b, adws_, st_); }, "dec.attn"));
+    g = GemvArgs<T>();
+    g.w = reinterpret_cast<const T*>(lw.wo); g.ldw = d; g.n = d; g.k = d; g.x = o; g.out = xmid; g.res = xin;
+    TRY(gemv_run(g, GEMV_ADD_F32, "dec.o"));
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xmid, d, lw.mlp_norm, eps, 1, (int)d, h2, d, r2_[i] + r, st_); }, "dec.norm"));
+    // [static | fast] gate/up with the SwiGLU epilogue; bf16: + h2 W_lo^T on the fast rows
+    g = GemvArgs<T>();
+    g.w = wgu_[l]; g.ldw = d; g.n = 4 * f; g.k = d; g.x = h2; g.out = a; g.raw = gu_[i] + r * 4 * f;
+    if (BF) { g.w2 = reinterpret_cast<const T*>(gu_lo_[i]); g.ldw2 = d; g.k2 = d; g.x2 = h2; g.n_ext = 2 * f; }
+    TRY(gemv_run(g, GEMV_SWIGLU, "dec.gateup"));
+    // [static | fast] down + residual; bf16: + a_fast W_down,lo^T
+    g = GemvArgs<T>();
+    g.w = wd_[l]; g.ldw = 2 * f; g.n = d; g.k = 2 * f; g.x = a; g.out = xout; g.res = xmid;
+    if (BF) { g.w2 = reinterpret_cast<const T*>(d_lo_[i]); g.ldw2 = f; g.k2 = f; g.x2 = a + f; g.n_ext = 0; }
+    TRY(gemv_run(g, GEMV_ADD_F32, "dec.down"));
+  }
+  TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xf_ + r * d, d, wt_.final_norm, eps, 1, (int)d, hf_ + r * d, d, rf_ + r, st_); }, "dec.norm"));
+  // next token = greedy pick of this position's logits; it is also this row's target
+  TRY(head_pick(hf_ + r * d, tgt_ + r, lsef_ + r));
+  if (r == b - 1 && eta_ != 0.f) {
+    // the chunk [c0, c0 + b) is complete: every position has its target
+    TRY(timed(TTT_KC_DECODE, 0, [&] { return fill_f32(scl_, b, 1.f / (float)b, st_); }, "dec.scale"));
+    TRY(chunk_backward(c0, b));
+  }
+  return TTT_OK;
+}
+
+template <typename T>
+int Engine<T>::decode(int64_t count, int32_t* tokens, float* losses) {
+  if (!prefilled_) return set_error(TTT_ERR_STATE, "ttt_decode needs a ttt_prefill of the prompt first");
+  if (count < 0 || (count > 0 && !tokens)) return set_error(TTT_ERR_INVALID_ARG, "ttt_decode: bad argument");
+  timer_.cut();
+  if (!dec_ready_) {
+    // the token after the prompt comes from the logits of its last position,
+    // scored with the weights of that position's chunk (the final-norm row
+    // the prefill left in hf_)
+    const int64_t p = dec_pos_ - 1, r = p % b_;
+    phase_ = "dec";
+    TRY(head_pick(hf_ + r * d_, tgt_ + r, nullptr));
+    dec_ready_ = true;
+  }
+  for (int64_t i = 0; i < count; ++i) {
+    timer_.cut();
+    TTT_CUDA_TRY(cudaMemcpyAsync(tokens + i, dtok_, sizeof(int32_t), cudaMemcpyDeviceToDevice, st_));
+    if (losses) TTT_CUDA_TRY(cudaMemcpyAsync(losses + i, dloss_, sizeof(float), cudaMemcpyDeviceToDevice, st_));
+    TRY(decode_position(dec_pos_));
+    ++dec_pos_;
   }
   return TTT_OK;
 }
@@ -914,8 +1086,13 @@ extern "C" int ttt_prefill(ttt_ctx* ctx, const int32_t* tokens_dev, int64_t T, f
 }
 
 extern "C" int ttt_decode_step(ttt_ctx* ctx, int32_t* next_token_dev) {
-  (void)next_token_dev;
-  return fail(ctx, set_error(TTT_ERR_UNSUPPORTED, "ttt_decode_step is not provided by this build"));
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_decode_step: NULL context");
+  return fail(ctx, ctx->decode(1, next_token_dev, nullptr));
+}
+
+extern "C" int ttt_decode(ttt_ctx* ctx, int64_t n_tokens, int32_t* tokens_dev, float* losses_dev) {
+  if (!ctx) return set_error(TTT_ERR_INVALID_ARG, "ttt_decode: NULL context");
+  return fail(ctx, ctx->decode(n_tokens, tokens_dev, losses_dev));
 }
 
 extern "C" int ttt_reset(ttt_ctx* ctx) {

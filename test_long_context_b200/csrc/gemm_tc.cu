@@ -26,13 +26,21 @@ constexpr int BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kGemmThreads = 64 + 32 * kEpiWarps;
 
-template <int BN>
+// Row pitch (floats) of an epilogue warp's 32 x 32 transpose tile: 33 for the
+// scalar column-per-lane reads, 36 for the SGD epilogue's float4 reads (rows
+// then start on 16-byte boundaries, and both the float4 writes of a row and
+// the float4 reads of four rows by eight lanes each hit 32 distinct banks).
+template <int EPI>
+constexpr int kWStride = EPI == EPI_SGD ? 36 : 33;
+
+template <int BN, int EPI>
 struct TcCfg {
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
-  static constexpr int WBUF = kEpiWarps * 32 * 33 * 4;  // epilogue transpose tiles, one per epilogue warp
+  // the SGD GEMMs reduce over one chunk (K = b): one stage fewer pays for the wider transpose tiles
+  static constexpr int STAGES = ((BN == 256) ? 4 : 6) - (EPI == EPI_SGD ? 1 : 0);
+  static constexpr int WBUF = kEpiWarps * 32 * kWStride<EPI> * 4;  // epilogue transpose tiles, one per epilogue warp
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + WBUF;
   static_assert(SMEM <= 232448, "shared memory per block");
 };
@@ -245,7 +253,7 @@ __device__ __forceinline__ void epi_chunk(const EpiArgs& ep, int64_t row0, int64
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
       if (store && (!CHECK || r < nrows)) {
-        const float w = buf[r] - ep.alpha * wbuf[r * 33 + lane];
+        const float w = __fmaf_rn(-ep.alpha, wbuf[r * 33 + lane], buf[r]);
         *p = w;
         if constexpr (HI) {
           const bf16 hi = __float2bfloat16_rn(w);
@@ -317,6 +325,112 @@ __device__ __forceinline__ void epilogue_transposed(uint32_t t_row, const EpiArg
   }
 }
 
+// Vectorised SGD epilogue of a warp's full 32 x BN tile (every row and
+// column inside the output; master rows 16-byte aligned, hi/lo rows 8-byte
+// aligned).  Per 32-column chunk, step it = 0..7 gives lane l row
+// 4*it + l/8 and columns 4*(l%8) .. +3: one float4 read of the transposed
+// accumulator, one float4 load (read ahead) and store of the master, one
+// 8-byte store each of hi and lo.  The arithmetic per element is that of
+// the scalar path: w = m - alpha*g, hi = bf16(w), lo = bf16(w - hi).
+template <int EPI>
+__device__ __forceinline__ bool sgd_vec_ok(const EpiArgs& ep, int64_t row0, int64_t M, int64_t n0, int64_t N,
+                                           int bn) {
+  if constexpr (EPI != EPI_SGD) {
+    return false;
+  } else {
+    const bool m_ok = (reinterpret_cast<uintptr_t>(ep.c) & 15) == 0 && (ep.ldc & 3) == 0;
+    const bool h_ok = !ep.c2 || ((reinterpret_cast<uintptr_t>(ep.c2) & 7) == 0 && (ep.ldc2 & 3) == 0);
+    const bool l_ok = !ep.c3 || ((reinterpret_cast<uintptr_t>(ep.c3) & 7) == 0 && (ep.ldc3 & 3) == 0);
+    return row0 + 32 <= M && n0 + bn <= N && m_ok && h_ok && l_ok;
+  }
+}
+
+// Master values of one 32-column chunk in the vectorised layout.
+__device__ __forceinline__ void sgd_load_vec(const EpiArgs& ep, int64_t row0, int64_t col0, float (&buf)[32]) {
+  const int lane = threadIdx.x & 31;
+  const float* p = reinterpret_cast<const float*>(ep.c) + (row0 + (lane >> 3)) * ep.ldc + col0 + 4 * (lane & 7);
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const float4 x = *reinterpret_cast<const float4*>(p + 4 * it * ep.ldc);
+    buf[4 * it] = x.x;
+    buf[4 * it + 1] = x.y;
+    buf[4 * it + 2] = x.z;
+    buf[4 * it + 3] = x.w;
+  }
+}
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float a, float b) {
+  __nv_bfloat162 t = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&t);
+}
+
+template <bool HI, bool LO>
+__device__ __forceinline__ void sgd_chunk_vec(const EpiArgs& ep, int64_t row0, int64_t col0, bool ahead,
+                                              const float* wbuf, float (&buf)[32]) {
+  const int lane = threadIdx.x & 31;
+  const int rs = lane >> 3, c4 = 4 * (lane & 7);
+  float* pm = reinterpret_cast<float*>(ep.c) + (row0 + rs) * ep.ldc + col0 + c4;
+  bf16* ph = HI ? reinterpret_cast<bf16*>(ep.c2) + (row0 + rs) * ep.ldc2 + col0 + c4 : nullptr;
+  bf16* pl = LO ? reinterpret_cast<bf16*>(ep.c3) + (row0 + rs) * ep.ldc3 + col0 + c4 : nullptr;
+  const float na = -ep.alpha;
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const float4 g = *reinterpret_cast<const float4*>(wbuf + (4 * it + rs) * 36 + c4);
+    const float w0 = __fmaf_rn(na, g.x, buf[4 * it]), w1 = __fmaf_rn(na, g.y, buf[4 * it + 1]);
+    const float w2 = __fmaf_rn(na, g.z, buf[4 * it + 2]), w3 = __fmaf_rn(na, g.w, buf[4 * it + 3]);
+    float* m = pm + (int64_t)(4 * it) * ep.ldc;
+    *reinterpret_cast<float4*>(m) = make_float4(w0, w1, w2, w3);
+    if constexpr (HI) {
+      const uint32_t h01 = bf16x2_bits(w0, w1), h23 = bf16x2_bits(w2, w3);
+      *reinterpret_cast<uint2*>(ph + (int64_t)(4 * it) * ep.ldc2) = make_uint2(h01, h23);
+      if constexpr (LO) {
+        const float f0 = __uint_as_float(h01 << 16), f1 = __uint_as_float(h01 & 0xFFFF0000u);
+        const float f2 = __uint_as_float(h23 << 16), f3 = __uint_as_float(h23 & 0xFFFF0000u);
+        *reinterpret_cast<uint2*>(pl + (int64_t)(4 * it) * ep.ldc3) =
+            make_uint2(bf16x2_bits(w0 - f0, w1 - f1), bf16x2_bits(w2 - f2, w3 - f3));
+      }
+    }
+    if (ahead) {  // the same rows, two chunks (64 columns) further on
+      const float4 x = *reinterpret_cast<const float4*>(m + 64);
+      buf[4 * it] = x.x;
+      buf[4 * it + 1] = x.y;
+      buf[4 * it + 2] = x.z;
+      buf[4 * it + 3] = x.w;
+    }
+  }
+}
+
+// bufA / bufB hold the master of chunks 0 and 1 (sgd_load_vec) on entry.
+template <int BN>
+__device__ __forceinline__ void epilogue_sgd_vec(uint32_t t_row, const EpiArgs& ep, int64_t n0, float* wbuf,
+                                                 int64_t row0, float (&bufA)[32], float (&bufB)[32]) {
+  const int lane = threadIdx.x & 31;
+  auto step = [&](int c, float(&buf)[32]) {
+    float v[32];
+    ld32f(t_row + c, v);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      *reinterpret_cast<float4*>(wbuf + lane * 36 + 4 * j) = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2],
+                                                                         v[4 * j + 3]);
+    __syncwarp();
+    const bool ahead = c + 64 < BN;
+    if (ep.c3)
+      sgd_chunk_vec<true, true>(ep, row0, n0 + c, ahead, wbuf, buf);
+    else if (ep.c2)
+      sgd_chunk_vec<true, false>(ep, row0, n0 + c, ahead, wbuf, buf);
+    else
+      sgd_chunk_vec<false, false>(ep, row0, n0 + c, ahead, wbuf, buf);
+    __syncwarp();
+  };
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 32) {
+    if ((c & 32) == 0)
+      step(c, bufA);
+    else
+      step(c, bufB);
+  }
+}
+
 // Persistent kernel: one CTA per SM walks the work units u = blockIdx.x,
 // blockIdx.x + gridDim.x, ...  A unit is (m-tile, n-tile, k-split) with the
 // m-tile fastest, so CTAs running at the same time share weight (B) tiles in
@@ -334,7 +448,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt, int n_split, int n_fast,
                    EpiArgs ep,
                    int* err) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, EPI>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -478,16 +592,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       decode(u, m0, n0, split, nkb, kb_begin);
       const uint32_t b = it & 1u, use = it >> 1;
       float bufA[32], bufB[32];
+      const bool vec = sgd_vec_ok<EPI>(ep, m0 + q * 32, M, n0, N, BN);  // warp-uniform
       if constexpr (kTransposedEpi<EPI>) {  // read source of the first two chunks, ahead of the accumulator
-        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
-        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+        if (vec) {
+          sgd_load_vec(ep, m0 + q * 32, n0, bufA);
+          sgd_load_vec(ep, m0 + q * 32, n0 + 32, bufB);
+        } else {
+          epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
+          epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+        }
       }
       const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));  // warp-uniform
       if (!ok) break;
       ptx::tc_fence_after();
       const int64_t row = m0 + q * 32 + lane;
-      if constexpr (kTransposedEpi<EPI>)
-        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * 33, m0 + q * 32,
+      if constexpr (EPI == EPI_SGD) {
+        if (vec)
+          epilogue_sgd_vec<BN>(tmem + b * BN + lane_off, ep, n0, wbufs + ew * 32 * kWStride<EPI>, m0 + q * 32, bufA,
+                               bufB);
+        else
+          epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * kWStride<EPI>,
+                                       m0 + q * 32, M, bufA, bufB);
+      } else if constexpr (kTransposedEpi<EPI>)
+        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * kWStride<EPI>, m0 + q * 32,
                                      M, bufA, bufB);
       else
         epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split);
@@ -522,13 +649,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //                             (256 arrivals: both CTAs' epilogue groups)
 // The units are (256-row pair tile, n-tile, k-split), walked by the pairs
 // like the single-CTA kernel walks its tiles.
+template <int EPI>
 struct PairCfg {
   static constexpr int BN = 256;
   static constexpr int A_BYTES = BM * BK * 2;    // this CTA's 128 rows of A
   static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of the B tile
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = 6;
-  static constexpr int WBUF = kEpiWarps * 32 * 33 * 4;
+  static constexpr int STAGES = EPI == EPI_SGD ? 5 : 6;
+  static constexpr int WBUF = kEpiWarps * 32 * kWStride<EPI> * 4;
   static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + WBUF;
   static_assert(SMEM <= 232448, "shared memory per block");
 };
@@ -539,7 +667,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                         const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2,
                         int64_t M, int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt,
                         int n_split, int n_fast, EpiArgs ep, int* err) {
-  using C = PairCfg;
+  using C = PairCfg<EPI>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -692,16 +820,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       m0 += BM * rank;  // this CTA's 128 rows of the pair tile
       const uint32_t b = it & 1u, use = it >> 1;
       float bufA[32], bufB[32];
+      const bool vec = sgd_vec_ok<EPI>(ep, m0 + q * 32, M, n0, N, BN);  // warp-uniform
       if constexpr (kTransposedEpi<EPI>) {
-        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
-        epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+        if (vec) {
+          sgd_load_vec(ep, m0 + q * 32, n0, bufA);
+          sgd_load_vec(ep, m0 + q * 32, n0 + 32, bufB);
+        } else {
+          epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + lane, N, bufA);
+          epi_load_chunk<EPI>(ep, m0 + q * 32, M, n0 + 32 + lane, N, bufB);
+        }
       }
       const bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[b], use & 1u, err));
       if (!ok) break;
       ptx::tc_fence_after();
       const int64_t row = m0 + q * 32 + lane;
-      if constexpr (kTransposedEpi<EPI>)
-        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * 33, m0 + q * 32,
+      if constexpr (EPI == EPI_SGD) {
+        if (vec)
+          epilogue_sgd_vec<BN>(tmem + b * BN + lane_off, ep, n0, wbufs + ew * 32 * kWStride<EPI>, m0 + q * 32, bufA,
+                               bufB);
+        else
+          epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * kWStride<EPI>,
+                                       m0 + q * 32, M, bufA, bufB);
+      } else if constexpr (kTransposedEpi<EPI>)
+        epilogue_transposed<BN, EPI>(tmem + b * BN + lane_off, ep, n0, N, split, wbufs + ew * 32 * kWStride<EPI>, m0 + q * 32,
                                      M, bufA, bufB);
       else
         epilogue_row<BN, EPI, TACT>(tmem + b * BN + lane_off, row, row < M, n0, N, ep, (int)(n0 / BN), split);
@@ -896,6 +1037,15 @@ KernelFn pick(int a_mn, int b_mn, int epi, int act_bf16) {
   return pick_epi<BN, true, false>(epi, act_bf16);
 }
 
+template <int EPI>
+int smem_bytes_epi(int pair, int bn) {
+  return pair ? PairCfg<EPI>::SMEM : (bn == 256 ? TcCfg<256, EPI>::SMEM : TcCfg<128, EPI>::SMEM);
+}
+
+int smem_bytes(int pair, int bn, int epi) {
+  return epi == EPI_SGD ? smem_bytes_epi<EPI_SGD>(pair, bn) : smem_bytes_epi<EPI_STORE_F32>(pair, bn);
+}
+
 }  // namespace
 
 int64_t tc_ce_tiles(int64_t N, int bn) { return (N + bn - 1) / bn; }
@@ -1002,7 +1152,7 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
                        : (g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, kepi, g.act_bf16)
                                       : pick<128>(g.a_mn, g.b_mn, kepi, g.act_bf16));
   if (!fn) return set_error(TTT_ERR_INVALID_ARG, "gemm: no kernel for this combination");
-  const int smem = g.pair ? PairCfg::SMEM : (g.bn == 256 ? TcCfg<256>::SMEM : TcCfg<128>::SMEM);
+  const int smem = smem_bytes(g.pair, g.bn, kepi);
   {
     static std::mutex mu;
     static std::set<std::pair<int, KernelFn>> configured;

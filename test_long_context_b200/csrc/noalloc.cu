@@ -14,6 +14,7 @@
 
 #include "../../include/ttt_ops.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 
 namespace ttt {
 namespace {
@@ -66,23 +67,8 @@ extern "C" int ttt_op_swa_backward_noalloc(int32_t dtype, int32_t n_heads, int32
   float* work = nullptr;
   int rc = work_address(&work);
   if (rc) return rc;
-  SwaArgs a;
-  a.heads = n_heads;
-  a.head_dim = head_dim;
-  a.n = n_q;
-  a.p0 = q_pos0;
-  a.window = window;
-  a.scale = 1.f / sqrtf((float)head_dim);
-  a.q = q;
-  a.ldq = ldq;
-  a.k = k_ring;
-  a.v = v_ring;
-  a.ldkv = (int64_t)n_heads * head_dim;
-  a.ring = ring_slots;
-  a.o = const_cast<void*>(o);
-  a.ldo = ldo;
-  a.lse = const_cast<float*>(lse);
-  a.ld_lse = n_q;
+  SwaArgs a = op_swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots,
+                          const_cast<void*>(o), ldo, lse);
   a.dout = dout;
   a.lddo = lddo;
   a.dq = dq;
@@ -91,5 +77,6 @@ extern "C" int ttt_op_swa_backward_noalloc(int32_t dtype, int32_t n_heads, int32
   a.dv = dv;
   a.lddkv = lddkv;
   a.D = work;  // every entry is written before it is read: no clearing needed
-  return swa_backward(a, dtype == TTT_BF16, reinterpret_cast<cudaStream_t>(stream));
+  // the same kernels as ttt_op_swa_backward with default flags (tensor cores where it uses them)
+  return op_swa_backward_run(a, dtype, 0, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -3,6 +3,8 @@
 #include "../../include/ttt_ops.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "decode.cuh"
+#include "elementwise.cuh"
 #include "gemm.cuh"
 #include "ptx.cuh"
 
@@ -132,8 +134,10 @@ extern "C" int ttt_op_sync(void* stream) {
   return TTT_OK;
 }
 
-static SwaArgs swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t window, const void* q, int64_t ldq,
-                        const void* k, const void* v, int64_t ring, void* o, int64_t ldo, const float* lse) {
+namespace ttt {
+
+SwaArgs op_swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t window, const void* q, int64_t ldq,
+                    const void* k, const void* v, int64_t ring, void* o, int64_t ldo, const float* lse) {
   SwaArgs a;
   a.heads = H;
   a.head_dim = HD;
@@ -154,13 +158,30 @@ static SwaArgs swa_args(int32_t H, int32_t HD, int64_t n, int64_t p0, int32_t wi
   return a;
 }
 
+int op_swa_backward_run(const SwaArgs& a, int32_t dtype, int32_t flags, cudaStream_t st) {
+  if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(a.head_dim) && a.ring % 128 == 0 &&
+      a.ldq == a.lddo) {
+    SwaTcBwdPlan plan;
+    int rc = swa_tc_bwd_prepare(&plan, a.heads, a.head_dim, a.q, a.dout, a.n, a.ldq, a.k, a.v, a.ring, a.ldkv);
+    if (rc) return rc;
+    int* err = op_err_word();
+    if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_swa_backward: no device error word");
+    std::function<int()> dkdv;
+    if (swa_tc_dkdv_supported(a) && a.lddkv == a.ldq) dkdv = [&] { return swa_tc_backward_dkdv(plan, a, st, err); };
+    return swa_backward_with_dq(a, true, st, [&] { return swa_tc_backward_dq(plan, a, st, err); }, dkdv);
+  }
+  return swa_backward(a, dtype == TTT_BF16, st);
+}
+
+}  // namespace ttt
+
 extern "C" int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
                                   int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
                                   int64_t ring_slots, void* o, int64_t ldo, float* lse, int32_t flags, void* stream) {
   if (!q || !k_ring || !v_ring || !o || !lse || n_q < 1 || q_pos0 < 0 || window < 1 || ring_slots < 1 ||
       n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
     return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_forward: bad argument");
-  SwaArgs a = swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots, o, ldo, lse);
+  SwaArgs a = op_swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots, o, ldo, lse);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0) {
     SwaTcPlan plan;
@@ -182,8 +203,8 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
   if (!q || !k_ring || !v_ring || !o || !lse || !dout || !dq || !dk || !dv || !D_scratch || n_q < 1 || q_pos0 < 0 ||
       window < 1 || ring_slots < 1 || n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
     return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_backward: bad argument");
-  SwaArgs a = swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots,
-                       const_cast<void*>(o), ldo, lse);
+  SwaArgs a = op_swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots,
+                          const_cast<void*>(o), ldo, lse);
   a.dout = dout;
   a.lddo = lddo;
   a.dq = dq;
@@ -192,20 +213,7 @@ extern "C" int ttt_op_swa_backward(int32_t dtype, int32_t n_heads, int32_t head_
   a.dv = dv;
   a.lddkv = lddkv;
   a.D = D_scratch;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0 &&
-      ldq == lddo) {
-    SwaTcBwdPlan plan;
-    int rc = swa_tc_bwd_prepare(&plan, n_heads, head_dim, q, dout, n_q, ldq, k_ring, v_ring, ring_slots,
-                                (int64_t)n_heads * head_dim);
-    if (rc) return rc;
-    int* err = op_err_word();
-    if (!err) return set_error(TTT_ERR_CUDA, "ttt_op_swa_backward: no device error word");
-    std::function<int()> dkdv;
-    if (swa_tc_dkdv_supported(a) && lddkv == ldq) dkdv = [&] { return swa_tc_backward_dkdv(plan, a, st, err); };
-    return swa_backward_with_dq(a, true, st, [&] { return swa_tc_backward_dq(plan, a, st, err); }, dkdv);
-  }
-  return swa_backward(a, dtype == TTT_BF16, st);
+  return op_swa_backward_run(a, dtype, flags, reinterpret_cast<cudaStream_t>(stream));
 }
 
 namespace ttt {
@@ -225,4 +233,67 @@ extern "C" int ttt_op_watchdog_selftest(void* stream) {
   watchdog_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
+}
+
+extern "C" int ttt_op_rmsnorm(int64_t n, int32_t d, const float* x, int64_t ldx, const float* g, float eps, void* y,
+                              int64_t ldy, float* rstd, void* stream) {
+  if (!x || !g || !y || !rstd || n < 1 || d < 1) return set_error(TTT_ERR_INVALID_ARG, "ttt_op_rmsnorm: bad argument");
+  return rmsnorm_fwd<bf16>(x, ldx, g, eps, n, d, reinterpret_cast<bf16*>(y), ldy, rstd,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ttt_op_qknorm_rope(int64_t n, int64_t p0, int32_t n_heads, int32_t head_dim, float eps, float theta,
+                                  const void* qkv, int64_t ldqkv, const float* gq, const float* gk, void* qout,
+                                  int64_t ldq, void* kring, void* vring, int64_t R, float* rq, float* rk, float* tab,
+                                  void* stream) {
+  if (!qkv || !gq || !gk || !qout || !kring || !vring || !rq || !rk || !tab || n < 1 || p0 < 0 || R < 1 ||
+      n_heads < 1 || head_dim < 2)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_qknorm_rope: bad argument");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float2* t2 = reinterpret_cast<float2*>(tab);
+  int rc = rope_table(t2, p0, n, head_dim, (double)theta, st);
+  if (rc) return rc;
+  return qknorm_rope_fwd<bf16>(reinterpret_cast<const bf16*>(qkv), ldqkv, gq, gk, n, p0, n_heads, head_dim, eps, t2,
+                               p0, reinterpret_cast<bf16*>(qout), ldq, reinterpret_cast<bf16*>(kring),
+                               reinterpret_cast<bf16*>(vring), (int64_t)n_heads * head_dim, R, rq, rk, st);
+}
+
+extern "C" int ttt_op_swiglu_bwd(int64_t n, int64_t nfeat, const void* da, int64_t ldda, const void* gu, int64_t ldgu,
+                                 void* dgu, int64_t lddgu, void* stream) {
+  if (!da || !gu || !dgu || n < 1 || nfeat < 1 || nfeat % 64)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swiglu_bwd: bad argument");
+  return swiglu_bwd<bf16>(reinterpret_cast<const bf16*>(da), ldda, reinterpret_cast<const bf16*>(gu), ldgu, n, nfeat,
+                          reinterpret_cast<bf16*>(dgu), lddgu, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int ttt_op_gemv(int32_t epilogue, int64_t n, int64_t k, const void* w, int64_t ldw, const void* x,
+                           void* out, const float* res, void* raw, float* lse_out, float* part, void* stream) {
+  if (!w || !x || !out || n < 1 || k < 1 || epilogue < 0 || epilogue > 3 || (epilogue == GEMV_ADD_F32 && !res) ||
+      (epilogue == GEMV_ARGMAX && !part))
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_gemv: bad argument");
+  GemvArgs<bf16> g;
+  g.w = reinterpret_cast<const bf16*>(w);
+  g.ldw = ldw;
+  g.n = n;
+  g.k = k;
+  g.x = reinterpret_cast<const bf16*>(x);
+  g.out = epilogue == GEMV_ARGMAX ? static_cast<void*>(part) : out;
+  g.res = res;
+  g.raw = reinterpret_cast<bf16*>(raw);
+  g.part = part;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int rc = gemv<bf16>(g, epilogue, st);
+  if (rc || epilogue != GEMV_ARGMAX) return rc;
+  return argmax_finalize(part, gemv_parts(n), reinterpret_cast<int32_t*>(out), nullptr, lse_out, nullptr, st);
+}
+
+extern "C" int ttt_op_attn_decode(int32_t n_heads, int32_t head_dim, int64_t p, int32_t window, const void* q,
+                                  const void* kring, const void* vring, int64_t R, void* o, float* lse, float* ws,
+                                  void* stream) {
+  if (!q || !kring || !vring || !o || !ws || n_heads < 1 || p < 0 || window < 1 || R < window)
+    return set_error(TTT_ERR_INVALID_ARG, "ttt_op_attn_decode: bad argument");
+  return attn_decode<bf16>(reinterpret_cast<const bf16*>(q), reinterpret_cast<const bf16*>(kring),
+                           reinterpret_cast<const bf16*>(vring), (int64_t)n_heads * head_dim, R, n_heads, head_dim, p,
+                           window, 1.f / sqrtf((float)head_dim), reinterpret_cast<bf16*>(o), lse, 1, ws,
+                           reinterpret_cast<cudaStream_t>(stream));
 }

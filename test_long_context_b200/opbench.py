@@ -5,7 +5,9 @@
 Each op runs through the op-level C ABI (include/ttt_ops.h) on random
 inputs of the exact shapes the engine uses for the named config, timed
 with CUDA events after warm-up; one JSON line per op with the average
-launch time and the algorithmic TFLOP/s.  With --iters 1 --warmup 0 it is
+launch time and the algorithmic TFLOP/s (contractions) or GB/s (the
+memory-bound kernels: algorithmic bytes = every operand read and every
+result written once).  With --iters 1 --warmup 0 it is
 also the small, self-contained command that ncu captures (a few hundred MB
 on the device instead of the whole model).
 """
@@ -49,7 +51,7 @@ def make_ops(cfg):
 
         def run():
             ops.gemm(A, B, a_mn, b_mn, epi, **args)
-        out[name] = (run, 2.0 * M * N * K)
+        out[name] = (run, 2.0 * M * N * K, 0.0)
 
     gemm("gemm_qkv_bottom", S, 3 * d, d, 0, 0, L.EPI_STORE_BF16, c=torch.empty(S, 3 * d, device=dev, dtype=bf))
     gemm("gemm_gateup_bottom", S, 2 * f, d, 0, 0, L.EPI_SWIGLU, c=torch.empty(S, f, device=dev, dtype=bf))
@@ -77,13 +79,59 @@ def make_ops(cfg):
         ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse)
         pairs = band_pairs(p0, n, k)
         if not backward:
-            out[name] = (lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse), 4.0 * d * pairs)
+            out[name] = (lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse), 4.0 * d * pairs, 0.0)
         else:
             dout = rn(n, H * hd)
             dq, dk, dv = (torch.empty_like(q) for _ in range(3))
             D = torch.empty(H * n, device=dev)
             out[name] = (lambda: ops.swa_backward(q, kr, vr, H, hd, p0, k, o, lse, dout, dq, dk, dv, D),
-                         4.0 * d * (pairs + n * (n + 1) // 2))
+                         4.0 * d * (pairs + n * (n + 1) // 2), 0.0)
+
+    gemm("gemm_o_bottom", S, d, d, 0, 0, L.EPI_ADD_F32, c=torch.zeros(S, d, device=dev),
+         c2=torch.zeros(S, d, device=dev))
+    gemm("gemm_qkv_top", b, 3 * d, d, 0, 0, L.EPI_STORE_BF16, c=torch.empty(b, 3 * d, device=dev, dtype=bf))
+    gemm("gemm_da_top", b, 2 * f, d, 0, 1, L.EPI_STORE_BF16, c=torch.empty(b, 2 * f, device=dev, dtype=bf))
+    gemm("gemm_dgrad_o", b, d, d, 0, 1, L.EPI_STORE_BF16, c=torch.empty(b, d, device=dev, dtype=bf))
+    gemm("gemm_dgrad_qkv", b, d, 3 * d, 0, 1, L.EPI_STORE_F32, c=torch.empty(b, d, device=dev))
+    gemm("gemm_wgrad_down_sgd", d, f, b, 1, 1, L.EPI_SGD, c=torch.zeros(d, f, device=dev),
+         c2=torch.empty(d, f, device=dev, dtype=bf), c3=torch.empty(d, f, device=dev, dtype=bf), alpha=1e-2)
+
+    # memory-bound kernels (algorithmic bytes)
+    x = torch.randn(S, d, device=dev)
+    g1 = torch.ones(d, device=dev)
+    y = torch.empty(S, d, device=dev, dtype=bf)
+    rs = torch.empty(S, device=dev)
+    out["rmsnorm_bottom"] = (lambda: ops.rmsnorm(x, g1, 1e-5, y, rs), 0.0, S * (4.0 * d + 2.0 * d + 4.0))
+    qkv = rn(S, 3 * d)
+    gq, gk = torch.ones(hd, device=dev), torch.ones(hd, device=dev)
+    qo = torch.empty(S, d, device=dev, dtype=bf)
+    kring, vring = torch.empty(R1, d, device=dev, dtype=bf), torch.empty(R1, d, device=dev, dtype=bf)
+    rq, rk = torch.empty(S, H, device=dev), torch.empty(S, H, device=dev)
+    tab = torch.empty(S * hd, device=dev)
+    out["qknorm_rope_bottom"] = (lambda: ops.qknorm_rope(qkv, S, H, hd, 1e-5, 1e4, gq, gk, qo, kring, vring, rq, rk,
+                                                         tab), 0.0, S * (2.0 * 3 * d * 2 + 8.0 * H + 4.0 * hd))
+    da = rn(b, 2 * f)
+    gu = rn(b, 4 * f)
+    dgu = torch.empty(b, 4 * f, device=dev, dtype=bf)
+    out["swiglu_bwd_top"] = (lambda: ops.swiglu_bwd(da, gu, dgu), 0.0, b * (2.0 * 2 * f + 2.0 * 4 * f * 2))
+    # generation: one position
+    wgu = rn(4 * f, d)
+    hv = rn(d)
+    av = torch.empty(2 * f, device=dev, dtype=bf)
+    rawv = torch.empty(4 * f, device=dev, dtype=bf)
+    out["gemv_gateup_top"] = (lambda: ops.gemv(2, wgu, hv, av, raw=rawv), 0.0, 2.0 * 4 * f * d)
+    whead = rn(V, d)
+    part = torch.empty(3 * 1184, device=dev)
+    tok = torch.empty(1, device=dev, dtype=torch.int32)
+    out["gemv_lmhead_pick"] = (lambda: ops.gemv(3, whead, hv, tok, part=part), 0.0, 2.0 * V * d)
+    qd = rn(d)
+    od = torch.empty(d, device=dev, dtype=bf)
+    lsed = torch.empty(H, device=dev)
+    wsd = torch.empty(H * ((k + 127) // 128 + 1) * (hd + 2), device=dev)
+    kdec, vdec = rn(R, d), rn(R, d)
+    pdec = 16 * k + 5
+    out["attn_decode_top"] = (lambda: ops.attn_decode(qd, kdec, vdec, H, hd, pdec, k, od, lsed, wsd), 0.0,
+                              2.0 * 2 * d * k)
 
     swa("swa_fwd_bottom", S, S, R1)
     swa("swa_fwd_top", b, 8 * b + 64 * 1024 // b * b, R)
@@ -102,7 +150,7 @@ def main():
     table = make_ops(cfg)
     names = args.op or list(table)
     for name in names:
-        run, flops = table[name]
+        run, flops, nbytes = table[name]
         for _ in range(args.warmup):
             run()
         torch.cuda.synchronize()
@@ -113,8 +161,12 @@ def main():
         e1.record()
         ops.sync()
         ms = e0.elapsed_time(e1) / args.iters
-        print(json.dumps({"op": name, "config": args.config, "ms": ms, "tflops": flops / (ms / 1e3) / 1e12,
-                          "algorithmic_flops": flops}), flush=True)
+        rec = {"op": name, "config": args.config, "ms": ms}
+        if flops:
+            rec.update(tflops=flops / (ms / 1e3) / 1e12, algorithmic_flops=flops)
+        if nbytes:
+            rec.update(gbps=nbytes / (ms / 1e3) / 1e9, algorithmic_bytes=nbytes)
+        print(json.dumps(rec), flush=True)
 
 
 if __name__ == "__main__":

@@ -112,3 +112,38 @@ def swa_backward_noalloc(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o
                                              o.stride(0), _p(lse), _p(dout), dout.stride(0), _p(dq), dq.stride(0),
                                              _p(dk), _p(dv), dk.stride(0), _stream(stream))
     L.check(rc)
+
+
+def rmsnorm(x, g, eps, y, rstd, stream=None):
+    """ttt_op_rmsnorm: x fp32 [n, d] -> y bf16 [n, d], rstd fp32 [n]."""
+    n, d = x.shape
+    L.check(L.lib().ttt_op_rmsnorm(n, d, _p(x), x.stride(0), _p(g), eps, _p(y), y.stride(0), _p(rstd),
+                                   _stream(stream)))
+
+
+def qknorm_rope(qkv, p0, n_heads, head_dim, eps, theta, gq, gk, qout, kring, vring, rq, rk, tab, stream=None):
+    """ttt_op_qknorm_rope: qkv bf16 [n, 3*H*hd] at positions p0.. -> qout, ring slots, rq/rk [n, H]."""
+    n = qkv.shape[0]
+    L.check(L.lib().ttt_op_qknorm_rope(n, p0, n_heads, head_dim, eps, theta, _p(qkv), qkv.stride(0), _p(gq), _p(gk),
+                                       _p(qout), qout.stride(0), _p(kring), _p(vring), kring.shape[0], _p(rq),
+                                       _p(rk), _p(tab), _stream(stream)))
+
+
+def swiglu_bwd(da, gu, dgu, stream=None):
+    """ttt_op_swiglu_bwd: da [n, F], gu/dgu [n, 2F] interleaved in (gate 64 | up 64) blocks (bf16)."""
+    n, nfeat = da.shape
+    L.check(L.lib().ttt_op_swiglu_bwd(n, nfeat, _p(da), da.stride(0), _p(gu), gu.stride(0), _p(dgu), dgu.stride(0),
+                                      _stream(stream)))
+
+
+def gemv(epi, w, x, out, res=None, raw=None, lse=None, part=None, stream=None):
+    """ttt_op_gemv: y = w x (bf16 w [n, k], x [k]) with epilogue 0 store, 1 add, 2 SwiGLU, 3 greedy pick."""
+    n, k = w.shape
+    L.check(L.lib().ttt_op_gemv(epi, n, k, _p(w), w.stride(0), _p(x), _p(out), _p(res), _p(raw), _p(lse), _p(part),
+                                _stream(stream)))
+
+
+def attn_decode(q, kring, vring, n_heads, head_dim, p, window, o, lse, ws, stream=None):
+    """ttt_op_attn_decode: one query per head (bf16 [H*hd]) over the window of the rings."""
+    L.check(L.lib().ttt_op_attn_decode(n_heads, head_dim, p, window, _p(q), _p(kring), _p(vring), kring.shape[0],
+                                       _p(o), _p(lse), _p(ws), _stream(stream)))
