@@ -375,6 +375,7 @@ class DecodeResult:
     W: dict                      # fast weights after the last completed chunk
     updates: list                # positions p after whose forward a chunk [p+1-b, p] updated W
     prefill: Result              # the prefill of the prompt
+    gaps: np.ndarray = None      # [n_gen] largest minus second-largest logit at each pick
 
 
 def decode(model, prompt, n_gen, eta=None):
@@ -405,10 +406,11 @@ def decode(model, prompt, n_gen, eta=None):
     W, state = pre.W, pre.state
     toks = [int(t) for t in prompt]
     z = pre.z_last  # logits of position T-1
-    gen, losses, updates = [], [], []
+    gen, losses, updates, gaps = [], [], [], []
     none = np.full(1, -1, dtype=np.int64)
     for p in range(T, T + n_gen):
         x = int(np.argmax(z))
+        gaps.append(float(z[x] - np.max(np.delete(z, x))) if len(z) > 1 else float("inf"))
         m = z.max()
         losses.append(float(m + np.log(np.exp(z - m).sum()) - z[x]))
         gen.append(x)
@@ -427,7 +429,7 @@ def decode(model, prompt, n_gen, eta=None):
                 for name in G[l]:
                     W[l][name] = W[l][name] - eta * G[l][name]   # eq. (9)
             updates.append(p)
-    return DecodeResult(np.asarray(gen, dtype=np.int64), np.asarray(losses), W, updates, pre)
+    return DecodeResult(np.asarray(gen, dtype=np.int64), np.asarray(losses), W, updates, pre, np.asarray(gaps))
 
 
 def static_losses(model, toks, k=None, fast=None):
