@@ -58,6 +58,23 @@ __device__ __forceinline__ float dot16(const uint4& w, const uint4& x, float acc
   return acc;
 }
 
+// o[e] += w * x[e] over the elements of 16 bytes of x
+__device__ __forceinline__ void axpy16(float w, const uint4& x, float (&o)[8], bf16) {
+  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(a[i]);
+    o[2 * i] = fmaf(w, f.x, o[2 * i]);
+    o[2 * i + 1] = fmaf(w, f.y, o[2 * i + 1]);
+  }
+}
+__device__ __forceinline__ void axpy16(float w, const uint4& x, float (&o)[4], float) {
+  o[0] = fmaf(w, __uint_as_float(x.x), o[0]);
+  o[1] = fmaf(w, __uint_as_float(x.y), o[1]);
+  o[2] = fmaf(w, __uint_as_float(x.z), o[2]);
+  o[3] = fmaf(w, __uint_as_float(x.w), o[3]);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -124,19 +141,52 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_kernel(GemvArgs<T> a) {
   extern __shared__ __align__(16) uint8_t gv_smem[];
   constexpr int V = VecOf<T>::N;
   T* xs = reinterpret_cast<T*>(gv_smem);
-  T* xs2 = xs + a.k;
-  {
+  T* xs2 = a.x2 ? xs + a.k : xs;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (a.xres) {
+    // RMSNorm of the residual row, in every block (the same order everywhere)
+    __shared__ float nred[GV_WARPS];
+    const float4* x4 = reinterpret_cast<const float4*>(a.xres);
+    float ss = 0.f;
+    for (int64_t i = threadIdx.x; i < a.k / 4; i += GV_THREADS) {
+      const float4 v = x4[i];
+      ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) nred[warp] = ss;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < GV_WARPS; ++w) tot += nred[w];
+    const float r = 1.f / sqrtf(tot / (float)a.k + a.eps);
+    const float4* g4 = reinterpret_cast<const float4*>(a.gain);
+    for (int64_t i = threadIdx.x; i < a.k / 4; i += GV_THREADS) {
+      const float4 v = x4[i], gg = g4[i];
+      const T y0 = from_f32<T>(v.x * r * gg.x), y1 = from_f32<T>(v.y * r * gg.y);
+      const T y2 = from_f32<T>(v.z * r * gg.z), y3 = from_f32<T>(v.w * r * gg.w);
+      xs[4 * i] = y0;
+      xs[4 * i + 1] = y1;
+      xs[4 * i + 2] = y2;
+      xs[4 * i + 3] = y3;
+      if (blockIdx.x == 0 && a.h_out) {
+        a.h_out[4 * i] = y0;
+        a.h_out[4 * i + 1] = y1;
+        a.h_out[4 * i + 2] = y2;
+        a.h_out[4 * i + 3] = y3;
+      }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0 && a.r_out) *a.r_out = r;
+  } else {
     const uint4* src = reinterpret_cast<const uint4*>(a.x);
     uint4* dst = reinterpret_cast<uint4*>(xs);
     for (int64_t i = threadIdx.x; i < a.k / V; i += GV_THREADS) dst[i] = src[i];
-    if (a.w2) {
-      const uint4* src2 = reinterpret_cast<const uint4*>(a.x2);
-      uint4* dst2 = reinterpret_cast<uint4*>(xs2);
-      for (int64_t i = threadIdx.x; i < a.k2 / V; i += GV_THREADS) dst2[i] = src2[i];
-    }
+  }
+  if (a.w2 && a.x2) {
+    const uint4* src2 = reinterpret_cast<const uint4*>(a.x2);
+    uint4* dst2 = reinterpret_cast<uint4*>(xs2);
+    for (int64_t i = threadIdx.x; i < a.k2 / V; i += GV_THREADS) dst2[i] = src2[i];
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t units = EPI == GEMV_SWIGLU ? a.n / 2 : a.n;
   ArgMax am;
   for (int64_t u = (int64_t)blockIdx.x * GV_WARPS + warp; u < units; u += (int64_t)gridDim.x * GV_WARPS) {
@@ -230,7 +280,8 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
                                                               int64_t R, int64_t p, int64_t jlo, float scale,
                                                               float* ws, int nsplit) {
   constexpr int V = VecOf<T>::N;
-  constexpr int PAIRS = HD / 2, GROUPS = AD_KEYS / PAIRS;
+  constexpr int CV = HD / V;             // 16-byte column vectors of a head row
+  constexpr int GROUPS = AD_KEYS / CV;   // key groups of the P V phase
   const int h = blockIdx.x, sp = blockIdx.y, t = threadIdx.x;
   __shared__ __align__(16) T qs[HD];
   __shared__ float ps[AD_KEYS];
@@ -244,9 +295,12 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
   if (t < nk) {
     const uint4* kv = reinterpret_cast<const uint4*>(kr + ((j0 + t) % R) * ldkv + (int64_t)h * HD);
     const uint4* qv = reinterpret_cast<const uint4*>(qs);
+    uint4 kk[CV];
+#pragma unroll
+    for (int i = 0; i < CV; ++i) kk[i] = __ldcs(kv + i);  // all loads of the row in flight
     float acc = 0.f;
 #pragma unroll
-    for (int i = 0; i < HD / V; ++i) acc = dot16(kv[i], qv[i], acc, T());
+    for (int i = 0; i < CV; ++i) acc = dot16(kk[i], qv[i], acc, T());
     s = acc * scale;
   }
   // block max
@@ -267,18 +321,30 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
   l = 0.f;
 #pragma unroll
   for (int w = 0; w < AD_KEYS / 32; ++w) l += red[w];
-  // P V: thread (g, c) sums column pair c over keys g, g + GROUPS, ...
-  const int g = t / PAIRS, c = t % PAIRS;
-  float o0 = 0.f, o1 = 0.f;
+  // P V: thread (g, c) sums column vector c (16 bytes) over keys g, g + GROUPS, ...;
+  // the keys of one step are independent, four value rows in flight per thread
+  const int g = t / CV, c = t % CV;
+  float o[V];
+#pragma unroll
+  for (int e = 0; e < V; ++e) o[e] = 0.f;
   if (g < GROUPS) {
-    for (int kk = g; kk < nk; kk += GROUPS) {
-      const T* vrow = vr + ((j0 + kk) % R) * ldkv + (int64_t)h * HD + 2 * c;
-      const float w = ps[kk];
-      o0 = fmaf(w, to_f32(vrow[0]), o0);
-      o1 = fmaf(w, to_f32(vrow[1]), o1);
+    const T* vbase = vr + (int64_t)h * HD + c * V;
+    int kk = g;
+    for (; kk + 3 * GROUPS < nk; kk += 4 * GROUPS) {
+      uint4 v4[4];
+      float w4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v4[u] = __ldcs(reinterpret_cast<const uint4*>(vbase + ((j0 + kk + u * GROUPS) % R) * ldkv));
+        w4[u] = ps[kk + u * GROUPS];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) axpy16(w4[u], v4[u], o, T());
     }
-    oacc[g][2 * c] = o0;
-    oacc[g][2 * c + 1] = o1;
+    for (; kk < nk; kk += GROUPS)
+      axpy16(ps[kk], __ldcs(reinterpret_cast<const uint4*>(vbase + ((j0 + kk) % R) * ldkv)), o, T());
+#pragma unroll
+    for (int e = 0; e < V; ++e) oacc[g][c * V + e] = o[e];
   }
   __syncthreads();
   float* out = ws + ((int64_t)h * nsplit + sp) * (HD + 2);
@@ -337,9 +403,12 @@ template <typename T>
 int gemv(const GemvArgs<T>& a, int epi, cudaStream_t s) {
   constexpr int V = VecOf<T>::N;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-  if (a.n < 1 || a.k < 1 || a.k % V || !al16(a.w) || (a.ldw * (int64_t)sizeof(T)) % 16 || !al16(a.x) || !a.out)
+  if (a.n < 1 || a.k < 1 || a.k % V || !al16(a.w) || (a.ldw * (int64_t)sizeof(T)) % 16 || !a.out)
     return set_error(TTT_ERR_INVALID_ARG, "gemv: rows must be 16-byte aligned and k a multiple of 16 bytes");
-  if (a.w2 && (a.k2 < 1 || a.k2 % V || !al16(a.w2) || (a.ldw2 * (int64_t)sizeof(T)) % 16 || !al16(a.x2)))
+  if (a.xres ? (!al16(a.xres) || !al16(a.gain) || a.k % 4) : !al16(a.x))
+    return set_error(TTT_ERR_INVALID_ARG, "gemv: input vector misaligned");
+  if (a.w2 && (a.k2 < 1 || a.k2 % V || !al16(a.w2) || (a.ldw2 * (int64_t)sizeof(T)) % 16 || (a.x2 && !al16(a.x2)) ||
+               (!a.x2 && a.k2 != a.k)))
     return set_error(TTT_ERR_INVALID_ARG, "gemv: second product misaligned");
   if (epi == GEMV_SWIGLU && (a.n % 128 || (a.w2 && a.n_ext % 128)))
     return set_error(TTT_ERR_INVALID_ARG, "gemv: SwiGLU rows come in blocks of 128");
@@ -349,7 +418,7 @@ int gemv(const GemvArgs<T>& a, int epi, cudaStream_t s) {
   const int64_t units = epi == GEMV_SWIGLU ? a.n / 2 : a.n;
   const unsigned blocks = (unsigned)(epi == GEMV_ARGMAX ? gemv_parts(a.n)
                                                         : std::min<int64_t>(GV_MAX_BLOCKS, (units + GV_WARPS - 1) / GV_WARPS));
-  const size_t smem = (size_t)(a.k + b.k2) * sizeof(T);
+  const size_t smem = (size_t)(a.k + (b.x2 ? b.k2 : 0)) * sizeof(T);
   if (smem > 200 * 1024) return set_error(TTT_ERR_INVALID_ARG, "gemv: input vector too long for shared memory");
   auto go = [&](auto kern) -> int {
     if (smem > 48 * 1024) TTT_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

@@ -30,6 +30,15 @@ struct GemvArgs {
   const float* res = nullptr;
   T* raw = nullptr;
   float* part = nullptr;  // GEMV_ARGMAX: [gemv_parts(n)] x 3 floats
+  // RMSNorm prologue (when xres is set, x is not read): x = T(xres * r * gain)
+  // with r = 1/sqrt(mean(xres^2) + eps), computed by every block; block 0
+  // also writes x to h_out and r to r_out (either may be NULL).  x2 == NULL
+  // with w2 set means the second product reads the same normalised x.
+  const float* xres = nullptr;
+  const float* gain = nullptr;
+  float eps = 0.f;
+  T* h_out = nullptr;
+  float* r_out = nullptr;
 };
 
 // Blocks a GEMV_ARGMAX launch writes partials for.

@@ -408,6 +408,32 @@ __global__ void __launch_bounds__(32 * CE_SLICES) ce_finalize_kernel(const float
   scale[i] = ok ? inv_nc : 0.f;
 }
 
+// One thread per 4 columns of a row (float4 logits, 8-byte bf16 stores when aligned).
+template <typename T>
+__global__ void ce_grad_kernel(const float* z, int64_t ldz, const float* lse, const float* scale, const int32_t* tgt,
+                               int64_t col0, int64_t n, int64_t ncols, T* dz, int64_t lddz) {
+  constexpr float LOG2E = 1.4426950408889634f;
+  const int64_t g4 = (ncols + 3) / 4;
+  const int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (gi >= n * g4) return;
+  const int64_t row = gi / g4, c = (gi % g4) * 4;
+  const float l = lse[row], sc = scale[row];
+  const int64_t t = (int64_t)tgt[row] - col0;
+  const float* zr = z + row * ldz + col0 + c;
+  T* out = dz + row * lddz + c;
+  const int cnt = (int)(ncols - c < 4 ? ncols - c : 4);
+  float v[4];
+  if (cnt == 4 && (reinterpret_cast<uintptr_t>(zr) & 15) == 0) {
+    const float4 x = *reinterpret_cast<const float4*>(zr);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    for (int e = 0; e < 4; ++e) v[e] = e < cnt ? zr[e] : 0.f;
+  }
+#pragma unroll
+  for (int e = 0; e < 4; ++e) v[e] = (exp2f((v[e] - l) * LOG2E) - (c + e == t ? 1.f : 0.f)) * sc;
+  for (int e = 0; e < cnt; ++e) out[e] = from_f32<T>(v[e]);
+}
+
 __global__ void check_tokens_kernel(const int32_t* tok, int64_t T, int V, int* err) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T) return;
@@ -563,6 +589,20 @@ int ce_finalize(const float* pmax, const float* psum, int64_t part_ld, int tiles
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
+
+template <typename T>
+int ce_grad_from_logits(const float* z, int64_t ldz, const float* lse, const float* scale, const int32_t* tgt,
+                        int64_t col0, int64_t n, int64_t ncols, T* dz, int64_t lddz, cudaStream_t s) {
+  if (n <= 0 || ncols <= 0) return TTT_OK;
+  ce_grad_kernel<T><<<ceil_div(n * ((ncols + 3) / 4), 256), 256, 0, s>>>(z, ldz, lse, scale, tgt, col0, n, ncols, dz,
+                                                                          lddz);
+  TTT_CUDA_TRY(cudaGetLastError());
+  return TTT_OK;
+}
+template int ce_grad_from_logits<float>(const float*, int64_t, const float*, const float*, const int32_t*, int64_t,
+                                        int64_t, int64_t, float*, int64_t, cudaStream_t);
+template int ce_grad_from_logits<bf16>(const float*, int64_t, const float*, const float*, const int32_t*, int64_t,
+                                       int64_t, int64_t, bf16*, int64_t, cudaStream_t);
 
 int check_tokens(const int32_t* tok, int64_t T, int V, int* err, cudaStream_t s) {
   check_tokens_kernel<<<ceil_div(T, 256), 256, 0, s>>>(tok, T, V, err);

@@ -55,6 +55,13 @@ int swiglu_bwd(const T* da, int64_t ldda, const T* gu, int64_t ldgu, int64_t n, 
 int ce_finalize(const float* pmax, const float* psum, int64_t part_ld, int tiles, const float* zt, int64_t n,
                 int64_t n_valid, float inv_nc, float* loss_out, float* lse, float* scale, cudaStream_t s);
 
+// Softmax-CE gradient of n rows over logit columns col0 .. col0+ncols-1
+// from stored fp32 logits z [n, ldz] (column index = vocab id):
+//   dz[i, c] = (exp(z[i, col0+c] - lse[i]) - [col0+c == tgt[i]]) * scale[i]  (T, [n, lddz]).
+template <typename T>
+int ce_grad_from_logits(const float* z, int64_t ldz, const float* lse, const float* scale, const int32_t* tgt,
+                        int64_t col0, int64_t n, int64_t ncols, T* dz, int64_t lddz, cudaStream_t s);
+
 // Flags (DEV_ERR_BAD_TOKEN) any id outside [0, V) among tok[0 .. T-1].
 int check_tokens(const int32_t* tok, int64_t T, int V, int* err, cudaStream_t s);
 // targets[i] = tok[p0+i+1] when p0+i+1 < T, else -1 (no target), i < n.

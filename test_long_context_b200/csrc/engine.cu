@@ -226,14 +226,18 @@ class Engine final : public ttt_ctx {
   int chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, const float* x0, float* losses);
   // backward through the updated blocks and the SGD steps of the chunk at p0
   // (n rows of the per-chunk buffers, targets in tgt_, CE scale in scl_)
-  int chunk_backward(int64_t p0, int64_t n);
+  // logits_stored: the forward kept this chunk's LM-head logits in logits_
+  // (the prefill in bf16 mode); else they are recomputed per vocab chunk
+  int chunk_backward(int64_t p0, int64_t n, bool logits_stored);
   // generation: the forward of position p (token in dtok_) through every
   // block, the greedy pick of the next token, and the chunk's update when p
   // is its last position
   int decode_position(int64_t p);
   // greedy pick from the final-norm output row hf (the LM head as a
   // matrix-vector product): next token -> dtok_, loss -> dloss_
-  int head_pick(const T* hf, int32_t* tgt_row, float* lse_row);
+  // hf: a final-norm output row; or (hf NULL) xres: the residual row, normalised
+  // in the product's prologue and stored to h_out, its factor to r_out
+  int head_pick(const T* hf, const float* xres, T* h_out, float* r_out, int32_t* tgt_row, float* lse_row);
   template <typename G>
   int gemv_run(const GemvArgs<T>& a, int epi, G&& bytes_of);
   // Launch `f` (returns a status); bracket it with events when timing is on.
@@ -371,6 +375,7 @@ class Engine final : public ttt_ctx {
   float *xf_ = nullptr, *rf_ = nullptr;
   T* hf_ = nullptr;
   float *pmax_ = nullptr, *psum_ = nullptr, *zt_ = nullptr, *lsef_ = nullptr, *scl_ = nullptr;
+  float* logits_ = nullptr;  // bf16 mode: the chunk's LM-head logits [b, V] (fp32), kept for the backward
   int32_t* tgt_ = nullptr;
   // backward
   float *dx_ = nullptr, *dxm_ = nullptr, *dhf_ = nullptr, *dh2_ = nullptr, *dh_ = nullptr, *Dbuf_ = nullptr;
@@ -596,6 +601,7 @@ int Engine<T>::init() {
     nvc_ = (V_ + Vc_ - 1) / Vc_;
   }
   TRY(arena_.alloc(&dz_, b * Vc_));
+  if (BF) TRY(arena_.alloc(&logits_, b * V_));
   TRY(arena_.alloc(&da_, b * 2 * f));
   TRY(arena_.alloc(&dgu_, b * 4 * f));
   TRY(arena_.alloc(&do_, b * d));
@@ -694,6 +700,7 @@ int Engine<T>::init() {
     }
   }
   e = EpiArgs{}; e.row_i = tgt_; e.part_max = pmax_; e.part_sum = psum_; e.target_logit = zt_; e.part_ld = b;
+  if (BF) { e.c = logits_; e.ldc = V_; }  // the logits stay for the backward
   TRY(prep(g_head_, 0, MatView{hf_, b, d, d}, 0, MatView{wt_.lm_head, V_, d, d}, EPI_CE_FWD, e));
   g_head_.label = "head.ce_fwd";
   g_ce_dz_.resize(nvc_);
@@ -814,16 +821,20 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
   // eta = 0: the step W -= 0 * G leaves every weight as it is, so the
   // backward that would produce G is skipped (the L_static model of eq. (4))
   if (eta_ == 0.f) return TTT_OK;
-  return chunk_backward(p0, n);
+  return chunk_backward(p0, n, BF);
 }
 
 template <typename T>
-int Engine<T>::chunk_backward(int64_t p0, int64_t n) {
+int Engine<T>::chunk_backward(int64_t p0, int64_t n, bool logits_stored) {
   const int64_t d = d_, f = f_, b = b_;
   // ---- backward through the updated blocks, SGD on each fast MLP ----
   phase_ = "bwd";
   for (int64_t c = 0; c < nvc_; ++c) {
-    TRY(run(g_ce_dz_[c], n));
+    const int64_t v0 = c * Vc_, vn = std::min<int64_t>(Vc_, V_ - v0);
+    if (logits_stored)  // dz of this vocab chunk from the forward's logits (L2-sized, read by the next product)
+      TRY(timed(TTT_KC_OTHER, 0, [&] { return ce_grad_from_logits<T>(logits_, V_, lsef_, scl_, tgt_, v0, n, vn, dz_, Vc_, st_); }, "head.ce_grad"));
+    else
+      TRY(run(g_ce_dz_[c], n));
     TRY(run(g_ce_dh_[c], n));
   }
   TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xf_, d, rf_, wt_.final_norm, dhf_, d, nullptr, 0, n, (int)d, dx_, d, dx16_, d, st_); }));
@@ -911,13 +922,20 @@ int Engine<T>::gemv_run(const GemvArgs<T>& a, int epi, G&& label) {
 }
 
 template <typename T>
-int Engine<T>::head_pick(const T* hf, int32_t* tgt_row, float* lse_row) {
+int Engine<T>::head_pick(const T* hf, const float* xres, T* h_out, float* r_out, int32_t* tgt_row, float* lse_row) {
   GemvArgs<T> g;
   g.w = reinterpret_cast<const T*>(wt_.lm_head);
   g.ldw = d_;
   g.n = V_;
   g.k = d_;
   g.x = hf;
+  if (!hf) {
+    g.xres = xres;
+    g.gain = wt_.final_norm;
+    g.eps = cfg_.norm_eps;
+    g.h_out = h_out;
+    g.r_out = r_out;
+  }
   g.out = gvpart_;  // unused by the argmax epilogue, must be non-NULL
   g.part = gvpart_;
   TRY(gemv_run(g, GEMV_ARGMAX, "dec.head"));
@@ -938,20 +956,21 @@ int Engine<T>::decode_position(int64_t p) {
   TRY(timed(TTT_KC_DECODE, 0, [&] { return embed_gather<T>(dtok_, reinterpret_cast<const T*>(wt_.embed), 1, (int)d, (int)V_, xd_, err_, st_); }, "dec.embed"));
   const double kv_bytes = 2.0 * (double)sizeof(T) * (double)d * (double)std::min<int64_t>(p + 1, k_);
   // ---- blocks without fast weights: one row, scratch of the super-chunk buffers ----
+  // (the RMSNorms run as the prologue of the product that reads them)
   for (int64_t l = 0; l < nbot_; ++l) {
     const ttt_layer_weights& lw = wt_.layers[l];
-    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xd_, d, lw.attn_norm, eps, 1, (int)d, hs_, d, rs_, st_); }, "dec.norm"));
     GemvArgs<T> g;
-    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.x = hs_; g.out = qkvs_;
+    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.out = qkvs_;
+    g.xres = xd_; g.gain = lw.attn_norm; g.eps = eps;
     TRY(gemv_run(g, GEMV_STORE, "dec.qkv"));
     TRY(timed(TTT_KC_DECODE, 0, [&] { return qknorm_rope_fwd<T>(qkvs_, 3 * d, lw.q_norm, lw.k_norm, 1, p, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, qs_, d, kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }, "dec.qknorm_rope"));
     TRY(timed(TTT_KC_DECODE, kv_bytes, [&] { return attn_decode<T>(qs_, kb_[l], vb_[l], d, R1_, (int)H_, (int)HD_, p, k_, scale_, os_, nullptr, 0, adws_, st_); }, "dec.attn"));
     g = GemvArgs<T>();
     g.w = reinterpret_cast<const T*>(lw.wo); g.ldw = d; g.n = d; g.k = d; g.x = os_; g.out = xd_; g.res = xd_;
     TRY(gemv_run(g, GEMV_ADD_F32, "dec.o"));
-    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xd_, d, lw.mlp_norm, eps, 1, (int)d, hs_, d, rs_, st_); }, "dec.norm"));
     g = GemvArgs<T>();
-    g.w = wgu_[l]; g.ldw = d; g.n = 2 * f; g.k = d; g.x = hs_; g.out = as_;
+    g.w = wgu_[l]; g.ldw = d; g.n = 2 * f; g.k = d; g.out = as_;
+    g.xres = xd_; g.gain = lw.mlp_norm; g.eps = eps;
     TRY(gemv_run(g, GEMV_SWIGLU, "dec.gateup"));
     g = GemvArgs<T>();
     g.w = wd_[l]; g.ldw = f; g.n = d; g.k = f; g.x = as_; g.out = xd_; g.res = xd_;
@@ -970,20 +989,20 @@ int Engine<T>::decode_position(int64_t p) {
     T* a = a_[i] + r * 2 * f;
     float* xmid = xmid_[i] + r * d;
     float* xout = (i + 1 < nu_ ? xin_[i + 1] : xf_) + r * d;
-    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xin, d, lw.attn_norm, eps, 1, (int)d, h, d, r1_[i] + r, st_); }, "dec.norm"));
     GemvArgs<T> g;
-    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.x = h; g.out = qkv;
+    g.w = wqkv_[l]; g.ldw = d; g.n = 3 * d; g.k = d; g.out = qkv;
+    g.xres = xin; g.gain = lw.attn_norm; g.eps = eps; g.h_out = h; g.r_out = r1_[i] + r;
     TRY(gemv_run(g, GEMV_STORE, "dec.qkv"));
     TRY(timed(TTT_KC_DECODE, 0, [&] { return qknorm_rope_fwd<T>(qkv, 3 * d, lw.q_norm, lw.k_norm, 1, p, (int)H_, (int)HD_, eps, rope_tab_, tab_p0_, q, d, kt_[i], vt_[i], d, R_, rq_[i] + r * H_, rk_[i] + r * H_, st_); }, "dec.qknorm_rope"));
     TRY(timed(TTT_KC_DECODE, kv_bytes, [&] { return attn_decode<T>(q, kt_[i], vt_[i], d, R_, (int)H_, (int)HD_, p, k_, scale_, o, lse_[i] + r, b, adws_, st_); }, "dec.attn"));
     g = GemvArgs<T>();
     g.w = reinterpret_cast<const T*>(lw.wo); g.ldw = d; g.n = d; g.k = d; g.x = o; g.out = xmid; g.res = xin;
     TRY(gemv_run(g, GEMV_ADD_F32, "dec.o"));
-    TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xmid, d, lw.mlp_norm, eps, 1, (int)d, h2, d, r2_[i] + r, st_); }, "dec.norm"));
     // [static | fast] gate/up with the SwiGLU epilogue; bf16: + h2 W_lo^T on the fast rows
     g = GemvArgs<T>();
-    g.w = wgu_[l]; g.ldw = d; g.n = 4 * f; g.k = d; g.x = h2; g.out = a; g.raw = gu_[i] + r * 4 * f;
-    if (BF) { g.w2 = reinterpret_cast<const T*>(gu_lo_[i]); g.ldw2 = d; g.k2 = d; g.x2 = h2; g.n_ext = 2 * f; }
+    g.w = wgu_[l]; g.ldw = d; g.n = 4 * f; g.k = d; g.out = a; g.raw = gu_[i] + r * 4 * f;
+    g.xres = xmid; g.gain = lw.mlp_norm; g.eps = eps; g.h_out = h2; g.r_out = r2_[i] + r;
+    if (BF) { g.w2 = reinterpret_cast<const T*>(gu_lo_[i]); g.ldw2 = d; g.k2 = d; g.n_ext = 2 * f; }
     TRY(gemv_run(g, GEMV_SWIGLU, "dec.gateup"));
     // [static | fast] down + residual; bf16: + a_fast W_down,lo^T
     g = GemvArgs<T>();
@@ -991,13 +1010,13 @@ int Engine<T>::decode_position(int64_t p) {
     if (BF) { g.w2 = reinterpret_cast<const T*>(d_lo_[i]); g.ldw2 = f; g.k2 = f; g.x2 = a + f; g.n_ext = 0; }
     TRY(gemv_run(g, GEMV_ADD_F32, "dec.down"));
   }
-  TRY(timed(TTT_KC_DECODE, 0, [&] { return rmsnorm_fwd<T>(xf_ + r * d, d, wt_.final_norm, eps, 1, (int)d, hf_ + r * d, d, rf_ + r, st_); }, "dec.norm"));
-  // next token = greedy pick of this position's logits; it is also this row's target
-  TRY(head_pick(hf_ + r * d, tgt_ + r, lsef_ + r));
+  // next token = greedy pick of this position's logits (final RMSNorm in the
+  // product's prologue); it is also this row's target
+  TRY(head_pick(nullptr, xf_ + r * d, hf_ + r * d, rf_ + r, tgt_ + r, lsef_ + r));
   if (r == b - 1 && eta_ != 0.f) {
     // the chunk [c0, c0 + b) is complete: every position has its target
     TRY(timed(TTT_KC_DECODE, 0, [&] { return fill_f32(scl_, b, 1.f / (float)b, st_); }, "dec.scale"));
-    TRY(chunk_backward(c0, b));
+    TRY(chunk_backward(c0, b, false));  // decode positions kept no logits: recompute them
   }
   return TTT_OK;
 }
@@ -1013,7 +1032,7 @@ int Engine<T>::decode(int64_t count, int32_t* tokens, float* losses) {
     // the prefill left in hf_)
     const int64_t p = dec_pos_ - 1, r = p % b_;
     phase_ = "dec";
-    TRY(head_pick(hf_ + r * d_, tgt_ + r, nullptr));
+    TRY(head_pick(hf_ + r * d_, nullptr, nullptr, nullptr, tgt_ + r, nullptr));
     dec_ready_ = true;
   }
   for (int64_t i = 0; i < count; ++i) {

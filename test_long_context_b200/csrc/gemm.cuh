@@ -21,7 +21,8 @@ enum Epi : int {
   EPI_SWIGLU = 3,      // columns come in (gate 64 | up 64) pairs: C[:, pair*64 + i] = silu(g) * u
                        // (activation dtype); C2 (optional) = raw acc (activation dtype)
   EPI_CE_FWD = 4,      // per row and N tile: part_max, part_sum of exp; target_logit[row] if the
-                       // target column (row_i[row] - col_offset) is in this GEMM's columns
+                       // target column (row_i[row] - col_offset) is in this GEMM's columns;
+                       // C (fp32, optional, tensor-core path) = acc (the logits)
   EPI_CE_BWD = 5,      // C (activation dtype) = (exp(acc - row_f[row]) - [col + col_offset ==
                        // row_i[row]]) * row_g[row]
   EPI_SGD = 6,         // C (fp32 master) -= alpha * acc; C2 (optional, bf16) = hi = bf16(new master);

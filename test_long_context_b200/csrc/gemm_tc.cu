@@ -127,6 +127,8 @@ __device__ __forceinline__ void epilogue_row(uint32_t t_row, int64_t row, bool r
       ld32f(t_row + c, v);
       const int64_t col0 = n0 + c;
       const int nval = (int)(N - col0 < 32 ? N - col0 : 32);
+      if (ep.c && row_ok && nval > 0)  // keep the logits for the backward (instead of recomputing them)
+        store32<float>(reinterpret_cast<float*>(ep.c) + row * ep.ldc + col0, v, nval);
       float cm = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i)
@@ -343,6 +345,16 @@ __device__ __forceinline__ bool sgd_vec_ok(const EpiArgs& ep, int64_t row0, int6
     const bool l_ok = !ep.c3 || ((reinterpret_cast<uintptr_t>(ep.c3) & 7) == 0 && (ep.ldc3 & 3) == 0);
     return row0 + 32 <= M && n0 + bn <= N && m_ok && h_ok && l_ok;
   }
+}
+
+// L2 prefetch of the warp tile's master rows (lane l: row row0 + l, all bn
+// columns, one request per 128-byte line), issued before the accumulator is
+// ready: the tile's loads then find the master in L2 instead of waiting out a
+// DRAM round trip two chunks at a time.
+__device__ __forceinline__ void sgd_prefetch_tile(const EpiArgs& ep, int64_t row0, int64_t n0, int bn) {
+  const int lane = threadIdx.x & 31;
+  const float* p = reinterpret_cast<const float*>(ep.c) + (row0 + lane) * ep.ldc + n0;
+  for (int c = 0; c < bn; c += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + c));
 }
 
 // Master values of one 32-column chunk in the vectorised layout.
@@ -595,6 +607,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const bool vec = sgd_vec_ok<EPI>(ep, m0 + q * 32, M, n0, N, BN);  // warp-uniform
       if constexpr (kTransposedEpi<EPI>) {  // read source of the first two chunks, ahead of the accumulator
         if (vec) {
+          sgd_prefetch_tile(ep, m0 + q * 32, n0, BN);
           sgd_load_vec(ep, m0 + q * 32, n0, bufA);
           sgd_load_vec(ep, m0 + q * 32, n0 + 32, bufB);
         } else {
@@ -823,6 +836,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       const bool vec = sgd_vec_ok<EPI>(ep, m0 + q * 32, M, n0, N, BN);  // warp-uniform
       if constexpr (kTransposedEpi<EPI>) {
         if (vec) {
+          sgd_prefetch_tile(ep, m0 + q * 32, n0, BN);
           sgd_load_vec(ep, m0 + q * 32, n0, bufA);
           sgd_load_vec(ep, m0 + q * 32, n0 + 32, bufB);
         } else {

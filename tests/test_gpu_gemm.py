@@ -319,7 +319,11 @@ def test_cta_pair_tiles_cross_entropy_split_and_dual():
     nt = ops.gemm_ce_tiles(True, M, V, 256)
     pm, ps = torch.empty(nt, M, device="cuda"), torch.empty(nt, M, device="cuda")
     zt = torch.full((M,), float("nan"), device="cuda")
-    ops.gemm(h, W, 0, 0, ops.L.EPI_CE_FWD, row_i=tgt, part_max=pm, part_sum=ps, target_logit=zt, part_ld=M, bn=256)
+    logits = torch.full((M, V), float("nan"), device="cuda")
+    ops.gemm(h, W, 0, 0, ops.L.EPI_CE_FWD, c=logits, row_i=tgt, part_max=pm, part_sum=ps, target_logit=zt,
+             part_ld=M, bn=256)
+    plain = torch.full((M, V), float("nan"), device="cuda")
+    ops.gemm(h, W, 0, 0, ops.L.EPI_STORE_F32, c=plain, bn=256)
     want_lse = torch.logsumexp(z, 1)
     dz = torch.empty(M, V, device="cuda", dtype=torch.bfloat16)
     scale = torch.full((M,), 1.0 / M, device="cuda")
@@ -329,6 +333,8 @@ def test_cta_pair_tiles_cross_entropy_split_and_dual():
     lse = gm + torch.log((ps * torch.exp(pm - gm)).sum(0))
     assert (lse.double() - want_lse).abs().max().item() <= 1e-4
     assert (zt.double() - z.gather(1, tgt.long()[:, None])[:, 0]).abs().max().item() <= 1e-4
+    # the kept logits are the accumulator itself: the plain product's values, bit for bit
+    assert torch.equal(logits, plain)
     p = torch.softmax(z, 1)
     oh = torch.nn.functional.one_hot(tgt.long(), V).double()
     want = (p - oh) * scale.double()[:, None]
