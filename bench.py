@@ -63,6 +63,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--decode-tokens", type=int, default=DECODE_TOKENS, help="0 skips the decode measurement")
+    ap.add_argument("--no-full-attention", action="store_true")
+    ap.add_argument("--no-multi-sequence", action="store_true")
     return ap.parse_args()
 
 
@@ -337,6 +339,78 @@ def time_decode(ctx, cfg, tok_dev, T, n_tokens, stream):
             "first_tokens": toks[:8].cpu().tolist()}
 
 
+def time_full_attention(cfg, gw, tok_dev, T, stream, ttt_ms):
+    """The same model as a plain full-attention Transformer prefill: window
+    k = T (every query sees all earlier positions) and eta = 0, so no chunk
+    is updated and the engine runs no backward.  One prefill of the whole
+    sequence after a short warm-up, timed with CUDA events; the ratio to the
+    TTT prefill's time is the comparison the pages make at 128K (reading
+    notes §11.1)."""
+    import torch
+
+    from test_long_context_b200.context import Context
+    ctx = Context(cfg, gw, k=T, eta=0.0, stream=stream)
+    losses = torch.empty(T, device="cuda")
+    ctx.prefill(tok_dev[:4096], losses[:4096], sync=True)  # warm-up
+    ctx.reset()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    ctx.prefill(tok_dev, losses, sync=False)
+    e1.record(stream)
+    ctx.sync()
+    ms = e0.elapsed_time(e1)
+    ok = bool(torch.isfinite(losses[:-1]).all().item())
+    ctx.close()
+    torch.cuda.empty_cache()
+    return {"workload": f"{cfg.name} full-attention prefill (window k = T = {T}, eta = 0: no update, no backward), "
+                        "same model and tokens", "tokens_per_s": T / (ms / 1000.0), "ms": ms,
+            "ms_per_1k_tokens": ms / (T / 1000.0), "ttt_prefill_speedup": ms / ttt_ms, "finite_losses": ok}
+
+
+def time_multi_sequence(cfg, gw, n_seq, T_seq, ttt_tokens_per_s):
+    """The batch the pages measure with: 128K tokens per batch as n_seq
+    independent sequences of T_seq tokens (4 x 32K), each with its own fast
+    weights, attention state and context, prefilled at the same time on its
+    own CUDA stream (static weights shared).  Time from an event before the
+    first launch to the last stream's end; throughput = all tokens / that."""
+    import torch
+
+    import synth
+    from test_long_context_b200.context import Context
+    streams = [torch.cuda.Stream() for _ in range(n_seq)]
+    ctxs = [Context(cfg, gw, stream=st) for st in streams]
+    toks = [torch.from_numpy(synth.tokens(cfg, T_seq, seed=cfg.seed + 101 * (i + 1))).cuda() for i in range(n_seq)]
+    losses = [torch.empty(T_seq, device="cuda") for _ in range(n_seq)]
+
+    def run():
+        start = torch.cuda.Event(enable_timing=True)
+        start.record(torch.cuda.current_stream())
+        ends = []
+        for c, t, l, st in zip(ctxs, toks, losses, streams):
+            st.wait_event(start)
+            c.reset()
+            c.prefill(t, l, sync=False)
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(st)
+            ends.append(e)
+        for c in ctxs:
+            c.sync()
+        return max(start.elapsed_time(e) for e in ends)
+
+    run()  # warm-up
+    ms = run()
+    ok = all(bool(torch.isfinite(l[:-1]).all().item()) for l in losses)
+    for c in ctxs:
+        c.close()
+    torch.cuda.empty_cache()
+    tps = n_seq * T_seq / (ms / 1000.0)
+    return {"workload": f"{cfg.name} prefill of {n_seq} independent sequences x {T_seq} tokens (window {cfg.k}, chunk "
+                        f"{cfg.b}), one context and CUDA stream per sequence, prefilled concurrently",
+            "tokens_per_s": tps, "ms": ms, "ms_per_1k_tokens": ms / (n_seq * T_seq / 1000.0),
+            "vs_one_sequence_of_the_same_tokens": tps / ttt_tokens_per_s, "finite_losses": ok}
+
+
 def time_config(name, steps=3, warmup=2):
     """Short timing of one more workload (its own T, k, b, dtype) on this GPU:
     tokens/s, per-1K-token latency and the achieved fraction of its roofline
@@ -529,9 +603,17 @@ def main():
                 "roofline": roof, "kernel_classes": classes, "gpu_launches": int(launches),
                 "clocks": clk, "e2e": e2e, "decode": dec}
     ctx.close()
+    torch.cuda.empty_cache()
+    full = multi = None
+    if rank == 0 and not args.no_full_attention and world == 1 and args.config == "2.7b" and not args.tokens:
+        full = time_full_attention(cfg, gw, tok_dev, T, stream, ms / args.steps)
+    if rank == 0 and not args.no_multi_sequence and world == 1 and args.config == "2.7b" and not args.tokens:
+        multi = time_multi_sequence(cfg, gw, 4, T // 4, aggregate_tokens_per_s(1, args.steps, T, ms))
     del gw
     torch.cuda.empty_cache()
     if rank == 0:
+        line["full_attention"] = full
+        line["multi_sequence"] = multi
         if not args.no_per_config and world == 1 and args.config == "2.7b" and not args.tokens:
             line["per_config"] = {name: time_config(name) for name in PER_CONFIG}
         if want_cpu:

@@ -206,7 +206,9 @@ int ttt_op_gemv(int32_t epilogue, int64_t n, int64_t k, const void* w, int64_t l
  * rings (bf16 [R, n_heads*head_dim], slot = position % R, R >= window): o
  * (bf16 [n_heads*head_dim]) and lse (fp32 [n_heads], natural log, may be
  * NULL); scores scaled by 1/sqrt(head_dim).  ws: fp32 scratch of
- * n_heads * (ceil(window / 128) + 1) * (head_dim + 2) floats.
+ * n_heads * ((ceil(window / 128) + 1) * (head_dim + 2) + 1) floats whose last
+ * n_heads words are zero before the first call (each call leaves them zero:
+ * they count the finished splits of each head).  window <= 16384.
  */
 int ttt_op_attn_decode(int32_t n_heads, int32_t head_dim, int64_t p, int32_t window, const void* q,
                        const void* kring, const void* vring, int64_t R, void* o, float* lse, float* ws,

@@ -15,8 +15,9 @@
 // of the split against the query (16-byte loads of its key row), the block
 // forms exp(s - m) for its keys, then threads in (group, column pair) layout
 // accumulate P V over the split's value rows (each value row read as one
-// coalesced line per group).  attn_combine_kernel merges the splits with
-// their maxima into o and the log-sum-exp.
+// coalesced line per group).  The last split of a head to finish (a counter
+// per head in the work space) merges the splits' (max, sum, o) into o and the
+// log-sum-exp, so one launch does the whole product.
 #include <algorithm>
 
 #include "decode.cuh"
@@ -278,10 +279,13 @@ constexpr int AD_KEYS = 128;  // keys per split = threads per block
 template <typename T, int HD>
 __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const T* kr, const T* vr, int64_t ldkv,
                                                               int64_t R, int64_t p, int64_t jlo, float scale,
-                                                              float* ws, int nsplit) {
+                                                              float* ws, unsigned* counters, int nsplit, T* o_out,
+                                                              float* lse_out, int64_t ld_lse) {
   constexpr int V = VecOf<T>::N;
   constexpr int CV = HD / V;             // 16-byte column vectors of a head row
   constexpr int GROUPS = AD_KEYS / CV;   // key groups of the P V phase
+  constexpr int NKT = (AD_KEYS + GROUPS - 1) / GROUPS;  // keys per thread in the P V phase
+  constexpr int NKT_PRE = NKT <= 16 ? NKT : 0;          // prefetched into registers when few
   const int h = blockIdx.x, sp = blockIdx.y, t = threadIdx.x;
   __shared__ __align__(16) T qs[HD];
   __shared__ float ps[AD_KEYS];
@@ -291,13 +295,29 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
   __syncthreads();
   const int64_t j0 = jlo + (int64_t)sp * AD_KEYS;
   const int nk = (int)imin64(AD_KEYS, p - j0 + 1);
+  // P V layout: thread (g, c) sums column vector c (16 bytes) over keys g, g + GROUPS, ...
+  const int g = t / CV, c = t % CV;
+  const T* vbase = vr + (int64_t)h * HD + c * V;
   float s = -INFINITY;
+  uint4 kk[CV];
   if (t < nk) {
     const uint4* kv = reinterpret_cast<const uint4*>(kr + ((j0 + t) % R) * ldkv + (int64_t)h * HD);
-    const uint4* qv = reinterpret_cast<const uint4*>(qs);
-    uint4 kk[CV];
 #pragma unroll
-    for (int i = 0; i < CV; ++i) kk[i] = __ldcs(kv + i);  // all loads of the row in flight
+    for (int i = 0; i < CV; ++i) kk[i] = __ldcs(kv + i);  // all loads of the key row in flight
+  }
+  // the value rows of this thread's keys, requested together with the key rows
+  uint4 vpre[NKT_PRE > 0 ? NKT_PRE : 1];
+  if constexpr (NKT_PRE > 0) {
+    if (g < GROUPS) {
+#pragma unroll
+      for (int u = 0; u < NKT_PRE; ++u) {
+        const int kv2 = g + u * GROUPS;
+        if (kv2 < nk) vpre[u] = __ldcs(reinterpret_cast<const uint4*>(vbase + ((j0 + kv2) % R) * ldkv));
+      }
+    }
+  }
+  if (t < nk) {
+    const uint4* qv = reinterpret_cast<const uint4*>(qs);
     float acc = 0.f;
 #pragma unroll
     for (int i = 0; i < CV; ++i) acc = dot16(kk[i], qv[i], acc, T());
@@ -321,14 +341,22 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
   l = 0.f;
 #pragma unroll
   for (int w = 0; w < AD_KEYS / 32; ++w) l += red[w];
-  // P V: thread (g, c) sums column vector c (16 bytes) over keys g, g + GROUPS, ...;
-  // the keys of one step are independent, four value rows in flight per thread
-  const int g = t / CV, c = t % CV;
+  // P V over this thread's keys: from the prefetched value rows, or (long rows
+  // of fp32 heads) four value rows in flight at a time
   float o[V];
 #pragma unroll
   for (int e = 0; e < V; ++e) o[e] = 0.f;
-  if (g < GROUPS) {
-    const T* vbase = vr + (int64_t)h * HD + c * V;
+  if constexpr (NKT_PRE > 0) {
+    if (g < GROUPS) {
+#pragma unroll
+      for (int u = 0; u < NKT_PRE; ++u) {
+        const int kv2 = g + u * GROUPS;
+        if (kv2 < nk) axpy16(ps[kv2], vpre[u], o, T());
+      }
+#pragma unroll
+      for (int e = 0; e < V; ++e) oacc[g][c * V + e] = o[e];
+    }
+  } else if (g < GROUPS) {
     int kk = g;
     for (; kk + 3 * GROUPS < nk; kk += 4 * GROUPS) {
       uint4 v4[4];
@@ -358,24 +386,51 @@ __global__ void __launch_bounds__(AD_KEYS) attn_decode_kernel(const T* q, const 
     out[0] = m;
     out[1] = l;
   }
-}
-
-template <typename T, int HD>
-__global__ void __launch_bounds__(128) attn_combine_kernel(const float* ws, int nsplit, T* o, float* lse,
-                                                           int64_t ld_lse) {
-  const int h = blockIdx.x, t = threadIdx.x;
+  // the last split of this head to finish merges all of them (its counter
+  // then returns to zero for the next call)
+  __shared__ unsigned last;
+  __threadfence();
+  __syncthreads();
+  if (t == 0) last = atomicAdd(&counters[h], 1u) == (unsigned)(nsplit - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
   const float* base = ws + (int64_t)h * nsplit * (HD + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[(int64_t)s * (HD + 2)]);
-  float L = 0.f, acc = 0.f;
-  for (int s = 0; s < nsplit; ++s) {
-    const float* e = base + (int64_t)s * (HD + 2);
-    const float f = expf(e[0] - M);
-    L = fmaf(e[1], f, L);
-    if (t < HD) acc = fmaf(e[2 + t], f, acc);
+  __shared__ float sf[AD_KEYS + 1];  // per-split factor exp(m_s - M); [AD_KEYS] = L
+  float ms = -INFINITY;
+  if (t < nsplit) ms = __ldcg(base + (int64_t)t * (HD + 2));
+  float M = ms;
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+  if ((t & 31) == 0) red[t >> 5] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < AD_KEYS / 32; ++w) M = fmaxf(M, red[w]);
+  const float fct = t < nsplit ? expf(ms - M) : 0.f;
+  sf[t] = fct;
+  float lsum = warp_sum(t < nsplit ? __ldcg(base + (int64_t)t * (HD + 2) + 1) * fct : 0.f);
+  __syncthreads();
+  if ((t & 31) == 0) red[t >> 5] = lsum;
+  __syncthreads();
+  if (t == 0) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < AD_KEYS / 32; ++w) L += red[w];
+    sf[AD_KEYS] = L;
   }
-  if (t < HD) o[(int64_t)h * HD + t] = from_f32<T>(acc / L);
-  if (t == 0 && lse) lse[(int64_t)h * ld_lse] = M + logf(L);
+  __syncthreads();
+  const float L = sf[AD_KEYS];
+  if (t < HD) {
+    float acc = 0.f;
+#pragma unroll 8
+    for (int s2 = 0; s2 < nsplit; ++s2) acc = fmaf(__ldcg(base + (int64_t)s2 * (HD + 2) + 2 + t), sf[s2], acc);
+    o_out[(int64_t)h * HD + t] = from_f32<T>(acc / L);
+  }
+  if (t == 0) {
+    if (lse_out) lse_out[(int64_t)h * ld_lse] = M + logf(L);
+    counters[h] = 0u;
+  }
 }
 
 __global__ void fill_kernel(float* dst, int64_t n, float v) {
@@ -388,9 +443,11 @@ int launch_attn(const T* q, const T* kr, const T* vr, int64_t ldkv, int64_t R, i
                 float scale, T* o, float* lse, int64_t ld_lse, float* ws, cudaStream_t s) {
   const int64_t jlo = p - window + 1 > 0 ? p - window + 1 : 0;
   const int nsplit = (int)((p - jlo + AD_KEYS) / AD_KEYS);
-  attn_decode_kernel<T, HD><<<dim3(H, nsplit), AD_KEYS, 0, s>>>(q, kr, vr, ldkv, R, p, jlo, scale, ws, nsplit);
-  TTT_CUDA_TRY(cudaGetLastError());
-  attn_combine_kernel<T, HD><<<H, 128, 0, s>>>(ws, nsplit, o, lse, ld_lse);
+  if (nsplit > AD_KEYS) return set_error(TTT_ERR_UNSUPPORTED, "attn_decode: window above 16 384 keys");
+  // per-head split counters after the partials (zero between calls)
+  unsigned* counters = reinterpret_cast<unsigned*>(ws + (int64_t)H * ((window + AD_KEYS - 1) / AD_KEYS + 1) * (HD + 2));
+  attn_decode_kernel<T, HD><<<dim3(H, nsplit), AD_KEYS, 0, s>>>(q, kr, vr, ldkv, R, p, jlo, scale, ws, counters,
+                                                                 nsplit, o, lse, ld_lse);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
@@ -443,7 +500,7 @@ int argmax_finalize(const float* part, int64_t nparts, int32_t* tok_out, int32_t
 }
 
 int64_t attn_decode_ws_floats(int H, int HD, int64_t window) {
-  return (int64_t)H * ((window + AD_KEYS - 1) / AD_KEYS + 1) * (HD + 2);
+  return (int64_t)H * ((window + AD_KEYS - 1) / AD_KEYS + 1) * (HD + 2) + H;
 }
 
 template <typename T>

@@ -56,7 +56,9 @@ int argmax_finalize(const float* part, int64_t nparts, int32_t* tok_out, int32_t
 // One query per head at absolute position p over the keys p-window+1 .. p
 // in the rings (slot = position % R): o (T) [H*HD], lse[h * ld_lse] (natural
 // log of the scaled scores' sum of exponentials; skipped when lse is NULL).
-// ws: fp32 work space of attn_decode_ws_floats(H, HD, window) floats.
+// ws: fp32 work space of attn_decode_ws_floats(H, HD, window) floats, its
+// last H words zero before the first call (every call leaves them zero);
+// window <= 16 384.
 int64_t attn_decode_ws_floats(int H, int HD, int64_t window);
 template <typename T>
 int attn_decode(const T* q, const T* kring, const T* vring, int64_t ldkv, int64_t R, int H, int HD, int64_t p,

@@ -251,6 +251,100 @@ __global__ void __launch_bounds__(ROPE_THREADS) qknorm_rope_fwd_kernel(
   }
 }
 
+// QK-norm + RoPE forward without shared memory: a group of 8 lanes per q or
+// k head (4 heads per warp, warps walk (token, head group) tasks); lane l of a
+// group holds the 16-byte vectors l, l + 8 of both halves of the head
+// (elements t and t + hd/2 are rotated together), the head's sum of squares
+// is reduced over the group with shuffles, and the rotated halves go straight
+// to q or the key ring.  Every access is a 16-byte vector and no block-wide
+// barrier separates the loads of one token from the stores of another.
+// Needs (hd/2) a multiple of 16 bytes of elements and at most 16 vectors per
+// half (head_dim <= 128 in bf16, <= 64 in fp32 - larger heads take the
+// kernel above).  The v rows are copied to the value ring by the same grid.
+template <typename T>
+__global__ void __launch_bounds__(256) qknorm_rope_fwd_warp_kernel(
+    const T* __restrict__ qkv, int64_t ldqkv, const float* __restrict__ gq, const float* __restrict__ gk, int64_t n,
+    int64_t p0, int H, int HD, float eps, const float2* __restrict__ tab, int64_t tab_p0, T* __restrict__ qout,
+    int64_t ldq, T* __restrict__ kring, T* __restrict__ vring, int64_t ldkv, int64_t R, float* __restrict__ rq,
+    float* __restrict__ rk) {
+  constexpr int EV = 16 / sizeof(T);
+  const int lane = threadIdx.x & 31, sub = lane & 7, hw = lane >> 3;
+  const int h2 = HD / 2, NV = h2 / EV;
+  const int hg = (2 * H + 3) / 4;  // groups of 4 among the 2H q and k heads
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < n * hg; w += nwarps) {
+    const int64_t i = w / hg;
+    const int hh = (int)(w % hg) * 4 + hw;  // q head hh < H, else k head hh - H
+    const bool live = hh < 2 * H;
+    const T* x = qkv + i * ldqkv + (int64_t)hh * HD;
+    uint4 va[2], vb[2];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = sub + 8 * u;
+      if (live && v < NV) {
+        va[u] = *reinterpret_cast<const uint4*>(x + v * EV);
+        vb[u] = *reinterpret_cast<const uint4*>(x + h2 + v * EV);
+        const T* ea = reinterpret_cast<const T*>(&va[u]);
+        const T* eb = reinterpret_cast<const T*>(&vb[u]);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+          const float fa = to_f32(ea[e]), fb = to_f32(eb[e]);
+          ss = fmaf(fa, fa, fmaf(fb, fb, ss));
+        }
+      }
+    }
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    if (!live) continue;
+    const float r = 1.f / sqrtf(ss / (float)HD + eps);
+    const bool is_q = hh < H;
+    const float* g = is_q ? gq : gk;
+    const float2* cs = tab + (p0 + i - tab_p0) * h2;
+    T* dst = is_q ? qout + i * ldq + (int64_t)hh * HD : kring + ((p0 + i) % R) * ldkv + (int64_t)(hh - H) * HD;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = sub + 8 * u;
+      if (v < NV) {
+        const T* ea = reinterpret_cast<const T*>(&va[u]);
+        const T* eb = reinterpret_cast<const T*>(&vb[u]);
+        // the vector's gains and (cos, sin) pairs as 16-byte loads
+        float ga[EV], gb[EV], cc[2 * EV];
+#pragma unroll
+        for (int e = 0; e < EV; e += 4) {
+          *reinterpret_cast<float4*>(ga + e) = *reinterpret_cast<const float4*>(g + v * EV + e);
+          *reinterpret_cast<float4*>(gb + e) = *reinterpret_cast<const float4*>(g + h2 + v * EV + e);
+        }
+#pragma unroll
+        for (int e = 0; e < 2 * EV; e += 4)
+          *reinterpret_cast<float4*>(cc + e) = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(cs + v * EV) + e);
+        uint4 oa, ob;
+        T* pa = reinterpret_cast<T*>(&oa);
+        T* pb = reinterpret_cast<T*>(&ob);
+#pragma unroll
+        for (int e = 0; e < EV; ++e) {
+          const float a = to_f32(ea[e]) * r * ga[e], b = to_f32(eb[e]) * r * gb[e];
+          const float cx = cc[2 * e], sy = cc[2 * e + 1];
+          pa[e] = from_f32<T>(a * cx - b * sy);
+          pb[e] = from_f32<T>(b * cx + a * sy);
+        }
+        *reinterpret_cast<uint4*>(dst + v * EV) = oa;
+        *reinterpret_cast<uint4*>(dst + h2 + v * EV) = ob;
+      }
+    }
+    if (sub == 0) (is_q ? rq : rk)[i * H + (is_q ? hh : hh - H)] = r;
+  }
+  // v rows into the value ring
+  const int64_t D = (int64_t)H * HD, dv = D / EV;
+  const int64_t nthreads = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; k < n * dv; k += nthreads) {
+    const int64_t i = k / dv, c = k % dv;
+    reinterpret_cast<uint4*>(vring + ((p0 + i) % R) * ldkv)[c] =
+        reinterpret_cast<const uint4*>(qkv + i * ldqkv + 2 * D)[c];
+  }
+}
+
 // Backward of QK-norm + RoPE, in place on the q and k parts of dqkv, with the
 // same staging as the forward: the token's dq|dk and raw q|k rows in smem,
 // four threads per head.
@@ -408,30 +502,44 @@ __global__ void __launch_bounds__(32 * CE_SLICES) ce_finalize_kernel(const float
   scale[i] = ok ? inv_nc : 0.f;
 }
 
-// One thread per 4 columns of a row (float4 logits, 8-byte bf16 stores when aligned).
+// One thread per 8 columns of a row: two float4 loads of the logits and one
+// 16-byte store of the bf16 gradient when the row segment is whole and
+// aligned (the vocab chunks used here always are); element by element at a
+// ragged end.
 template <typename T>
 __global__ void ce_grad_kernel(const float* z, int64_t ldz, const float* lse, const float* scale, const int32_t* tgt,
                                int64_t col0, int64_t n, int64_t ncols, T* dz, int64_t lddz) {
   constexpr float LOG2E = 1.4426950408889634f;
-  const int64_t g4 = (ncols + 3) / 4;
+  const int64_t g8 = (ncols + 7) / 8;
   const int64_t gi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (gi >= n * g4) return;
-  const int64_t row = gi / g4, c = (gi % g4) * 4;
+  if (gi >= n * g8) return;
+  const int64_t row = gi / g8, c = (gi % g8) * 8;
   const float l = lse[row], sc = scale[row];
   const int64_t t = (int64_t)tgt[row] - col0;
   const float* zr = z + row * ldz + col0 + c;
   T* out = dz + row * lddz + c;
-  const int cnt = (int)(ncols - c < 4 ? ncols - c : 4);
-  float v[4];
-  if (cnt == 4 && (reinterpret_cast<uintptr_t>(zr) & 15) == 0) {
-    const float4 x = *reinterpret_cast<const float4*>(zr);
-    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  const int cnt = (int)(ncols - c < 8 ? ncols - c : 8);
+  const bool vec = cnt == 8 && (reinterpret_cast<uintptr_t>(zr) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(out) & 15) == 0 && sizeof(T) == 2;
+  float v[8];
+  if (vec) {
+    const float4 x0 = *reinterpret_cast<const float4*>(zr), x1 = *reinterpret_cast<const float4*>(zr + 4);
+    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
   } else {
-    for (int e = 0; e < 4; ++e) v[e] = e < cnt ? zr[e] : 0.f;
+    for (int e = 0; e < 8; ++e) v[e] = e < cnt ? zr[e] : 0.f;
   }
 #pragma unroll
-  for (int e = 0; e < 4; ++e) v[e] = (exp2f((v[e] - l) * LOG2E) - (c + e == t ? 1.f : 0.f)) * sc;
-  for (int e = 0; e < cnt; ++e) out[e] = from_f32<T>(v[e]);
+  for (int e = 0; e < 8; ++e) v[e] = (exp2f((v[e] - l) * LOG2E) - (c + e == t ? 1.f : 0.f)) * sc;
+  if (vec) {
+    uint4 w;
+    T* pw = reinterpret_cast<T*>(&w);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) pw[e] = from_f32<T>(v[e]);
+    *reinterpret_cast<uint4*>(out) = w;
+  } else {
+    for (int e = 0; e < cnt; ++e) out[e] = from_f32<T>(v[e]);
+  }
 }
 
 __global__ void check_tokens_kernel(const int32_t* tok, int64_t T, int V, int* err) {
@@ -535,6 +643,16 @@ int qknorm_rope_fwd(const T* qkv, int64_t ldqkv, const float* gq, const float* g
                       reinterpret_cast<uintptr_t>(qkv) % 16 == 0 && reinterpret_cast<uintptr_t>(qout) % 16 == 0 &&
                       reinterpret_cast<uintptr_t>(kring) % 16 == 0 && reinterpret_cast<uintptr_t>(vring) % 16 == 0;
   if (!vec_ok) return set_error(TTT_ERR_INVALID_ARG, "qknorm_rope: rows must be 16-byte aligned");
+  const bool al = reinterpret_cast<uintptr_t>(gq) % 16 == 0 && reinterpret_cast<uintptr_t>(gk) % 16 == 0 &&
+                  reinterpret_cast<uintptr_t>(tab) % 16 == 0 && (HD / 2) % 4 == 0;
+  if (al && (HD / 2) % EV == 0 && (HD / 2) / EV <= 16) {
+    const int64_t tasks = n * ((2 * H + 3) / 4);  // warps of work
+    const unsigned grid = (unsigned)std::min<int64_t>((tasks + 7) / 8, 148 * 16);
+    qknorm_rope_fwd_warp_kernel<T><<<grid, 256, 0, s>>>(qkv, ldqkv, gq, gk, n, p0, H, HD, eps, tab, tab_p0, qout, ldq,
+                                                        kring, vring, ldkv, R, rq, rk);
+    TTT_CUDA_TRY(cudaGetLastError());
+    return TTT_OK;
+  }
   const size_t smem = 2 * (size_t)D * sizeof(T);
   if (smem > 48 * 1024) return set_error(TTT_ERR_UNSUPPORTED, "qknorm_rope: q and k rows exceed 48 KB");
   const unsigned grid = (unsigned)std::min<int64_t>(n, 148 * 8);
@@ -594,7 +712,7 @@ template <typename T>
 int ce_grad_from_logits(const float* z, int64_t ldz, const float* lse, const float* scale, const int32_t* tgt,
                         int64_t col0, int64_t n, int64_t ncols, T* dz, int64_t lddz, cudaStream_t s) {
   if (n <= 0 || ncols <= 0) return TTT_OK;
-  ce_grad_kernel<T><<<ceil_div(n * ((ncols + 3) / 4), 256), 256, 0, s>>>(z, ldz, lse, scale, tgt, col0, n, ncols, dz,
+  ce_grad_kernel<T><<<ceil_div(n * ((ncols + 7) / 8), 256), 256, 0, s>>>(z, ldz, lse, scale, tgt, col0, n, ncols, dz,
                                                                           lddz);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;

@@ -138,9 +138,14 @@ def test_attn_decode(hd, p, window, R):
     vr = torch.randn(R, d, device="cuda", generator=gen).to(bf)
     o = torch.empty(d, device="cuda", dtype=bf)
     lse = torch.empty(H, device="cuda")
-    ws = torch.empty(H * ((window + 127) // 128 + 1) * (hd + 2), device="cuda")
+    # the last H words count finished splits: zero before the first call, left zero by every call
+    ws = torch.zeros(H * (((window + 127) // 128 + 1) * (hd + 2) + 1), device="cuda")
     ops.attn_decode(q, kr, vr, H, hd, p, window, o, lse, ws)
+    o2 = torch.empty_like(o)
+    ops.attn_decode(q, kr, vr, H, hd, p, window, o2, None, ws)  # a second call on the same work space
     ops.sync()
+    assert torch.equal(o, o2)
+    assert (ws[-H:] == 0).all()
     lo = max(0, p - window + 1)
     pos = np.arange(lo, p + 1)
     K = kr.double().cpu().numpy()[pos % R].reshape(-1, H, hd)
