@@ -54,12 +54,13 @@ typedef struct ttt_epilogue_args {
  * a_mn = 0: A stored [M, K] with row pitch lda;  a_mn = 1: stored [K, M].
  * b_mn = 0: B stored [N, K] with row pitch ldb;  b_mn = 1: stored [K, N].
  * bf16 operands: 16-byte aligned base and row pitch.  (a_mn, b_mn) = (1, 0)
- * is not supported with TTT_BF16.  bn_hint: 0 (auto), 128 or 256 (tile
- * width; TTT_BF16 only).  256-wide tiles of a GEMM with M > 128 run on CTA
- * pairs (clusters of two CTAs, one 256 x 256 tile per pair; environment
- * TTT_GEMM_PAIR=0 keeps single CTAs); the results do not depend on it.
- * CE_FWD writes ceil(N / tile) partial tiles: query the tile count with
- * ttt_op_gemm_ce_tiles.
+ * is not supported with TTT_BF16.  bn_hint: 0 (auto), 128, 160 or 256
+ * (tile width; TTT_BF16 only; 160 only with M > 128 and the STORE_F32,
+ * STORE_BF16 or ADD_F32 epilogue).  A GEMM with M > 128 runs on CTA pairs
+ * (clusters of two CTAs, one 256 x tile-width output tile per pair;
+ * environment TTT_GEMM_PAIR=0 keeps single CTAs); the results do not depend
+ * on it.  CE_FWD writes ceil(N / tile) partial tiles: query the tile count
+ * with ttt_op_gemm_ce_tiles.
  */
 int ttt_op_gemm(int32_t dtype, int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t K, const void* A,
                 int64_t lda, const void* B, int64_t ldb, int32_t epilogue, const ttt_epilogue_args* args,
@@ -97,6 +98,15 @@ int ttt_op_gemm_split(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N, int64_t 
 int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint);
 
 /*
+ * The launch plan the prefill uses for a bf16 M x N x K product with this
+ * epilogue: returns the split-K count (1 = none) and writes the tile width
+ * to *bn_out (0 = the automatic choice of ttt_op_gemm).  Pass both to
+ * ttt_op_gemm_split (workspace: split * M * N floats) to run the product as
+ * the prefill does.  No device work.
+ */
+int64_t ttt_op_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t epilogue, int32_t* bn_out);
+
+/*
  * Sliding-window causal attention, eq. (1) of the reading notes: query at
  * absolute position p = q_pos0 + i attends to keys p-window+1 .. p.
  *   q, o: [n_q, ldq] / [n_q, ldo] rows, head h in columns h*head_dim ...
@@ -108,11 +118,29 @@ int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hin
  * head_dim in {64, 80, 96, 128}, ring_slots a multiple of 128 and flags bit 0
  * clear, the tcgen05 tensor-core kernel runs (fp32 softmax, bf16 P); otherwise
  * the SIMT kernel (fp32 math).  Scores are scaled by 1/sqrt(head_dim).
+ *
+ * q_norm_max, k_norm_max (0 = unknown): upper bounds on the Euclidean norm
+ * of every query row and every key row of a head, e.g. max|gain| *
+ * sqrt(head_dim) after an RMSNorm with that gain (the model's QK-norm).  With
+ * both given and log2(e) q_norm_max k_norm_max / sqrt(head_dim) <= 48 (about
+ * 47.5 with the 1% allowance for bf16 rounding), the tensor-core path shifts
+ * each query row's softmax by the Cauchy-Schwarz bound of its scores instead
+ * of a running maximum (the same result: softmax is shift-invariant), which
+ * lets it skip the max reduction and the rescaling of o.  The bounds are the
+ * caller's promise; keys up to 3.5x longer than k_norm_max still give exact
+ * results.
+ * flags bits 4..7, TTT_SWA_EXP_POLY(n): on that path n of every 8 groups of
+ * 8 keys (n in 0, 2, 4) take 2^x from an FMA-pipe polynomial (relative error
+ * 7.5e-5) instead of the MUFU unit; flags bits 8..11, TTT_SWA_SOFTMAX_GROUPS
+ * (2 or 4): softmax warpgroups per CTA.  0 in these bits = library default.
  */
 #define TTT_SWA_FORCE_SIMT 1
+#define TTT_SWA_EXP_POLY(n) ((((n) + 1) & 15) << 4)
+#define TTT_SWA_SOFTMAX_GROUPS(n) (((n) & 15) << 8)
 int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
                        const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
-                       void* o, int64_t ldo, float* lse, int32_t flags, void* stream);
+                       void* o, int64_t ldo, float* lse, float q_norm_max, float k_norm_max, int32_t flags,
+                       void* stream);
 
 /*
  * Backward of ttt_op_swa_forward given dout = dL/do: dq for every query (over

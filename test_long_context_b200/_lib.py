@@ -85,12 +85,13 @@ def lib():
             "ttt_op_gemm_split": (c_i32, [c_i32, c_i32, c_i64, c_i64, c_i64, c_vp, c_i64, c_vp, c_i64, c_i32,
                                           ctypes.POINTER(ttt_epilogue_args), c_i32, c_i32, c_vp, c_vp]),
             "ttt_op_sync": (c_i32, [c_vp]),
+            "ttt_op_gemm_plan": (c_i64, [c_i64, c_i64, c_i64, c_i32, ctypes.POINTER(c_i32)]),
             "ttt_op_watchdog_selftest": (c_i32, [c_vp]),
             "ttt_op_swa_backward_noalloc": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp,
                                                     c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
                                                     c_vp, c_i64, c_vp]),
             "ttt_op_swa_forward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp, c_i64,
-                                           c_vp, c_i64, c_vp, c_i32, c_vp]),
+                                           c_vp, c_i64, c_vp, c_f32, c_f32, c_i32, c_vp]),
             "ttt_op_swa_backward": (c_i32, [c_i32, c_i32, c_i32, c_i64, c_i64, c_i32, c_vp, c_i64, c_vp, c_vp,
                                             c_i64, c_vp, c_i64, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp, c_vp, c_i64,
                                             c_vp, c_i32, c_vp]),
@@ -129,7 +130,7 @@ def exported_symbols():
     L = lib()
     names = []
     for n in ("ttt_init", "ttt_prefill", "ttt_decode_step", "ttt_decode", "ttt_reset", "ttt_sync", "ttt_last_error", "ttt_free",
-              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_dual", "ttt_op_gemm_ce_tiles", "ttt_op_sync", "ttt_op_swa_forward",
+              "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_dual", "ttt_op_gemm_ce_tiles", "ttt_op_gemm_plan", "ttt_op_sync", "ttt_op_swa_forward",
               "ttt_op_swa_backward", "ttt_op_watchdog_selftest", "ttt_op_rmsnorm", "ttt_op_qknorm_rope",
               "ttt_op_swiglu_bwd", "ttt_op_gemv", "ttt_op_attn_decode",
               "ttt_op_swa_backward_noalloc"):

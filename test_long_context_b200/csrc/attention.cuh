@@ -20,6 +20,16 @@ struct SwaArgs {
   const void* k = nullptr;
   const void* v = nullptr;
   int64_t ldkv = 0, ring = 1;
+  // Upper bounds on the Euclidean norm of every query row and key row of a
+  // head (0 = unknown): with both known and scale log2(e) q_norm_max
+  // k_norm_max <= 48, the tensor-core forward shifts each row's softmax by
+  // the Cauchy-Schwarz bound of its scores instead of a running maximum.
+  float q_norm_max = 0.f, k_norm_max = 0.f;
+  // Fixed-shift forward tuning: how many of every 8 groups of 8 keys take
+  // 2^x from an FMA-pipe polynomial instead of the MUFU unit (0, 2, 4), and
+  // the number of softmax warpgroups (2, 4); -1 / 0 = library defaults.
+  int exp_poly = -1;
+  int softmax_groups = 0;
   void* o = nullptr;
   int64_t ldo = 0;
   float* lse = nullptr;

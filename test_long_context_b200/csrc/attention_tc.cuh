@@ -50,6 +50,8 @@ int swa_tc_backward_dkdv(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s
 int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t q_rows, int64_t ldq, const void* k,
                    const void* v, int64_t ring, int64_t ldkv);
 int swa_tc_forward(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err);
+// True when swa_tc_forward takes the fixed-shift kernel for these arguments.
+bool swa_fixed_shift_ok(const SwaArgs& a);
 
 // Shared by the op-level entry points (ops.cu, noalloc.cu): the forward
 // arguments of one call (k/v ring pitch heads*head_dim, lse pitch n, scale

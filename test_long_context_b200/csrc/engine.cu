@@ -299,8 +299,10 @@ class Engine final : public ttt_ctx {
     return s;
   }
   SwaArgs swa_args(const T* q, int64_t n, int64_t p0, const T* kr, const T* vr, int64_t ring, T* o, float* lse,
-                   int64_t ld_lse) const {
+                   int64_t ld_lse, int64_t layer) const {
     SwaArgs a;
+    a.q_norm_max = qn_max_[layer];  // bounds from the block's QK-norm gains
+    a.k_norm_max = kn_max_[layer];
     a.heads = (int)H_;
     a.head_dim = (int)HD_;
     a.n = n;
@@ -402,6 +404,9 @@ class Engine final : public ttt_ctx {
   }
   // tensor-core attention plans (bf16, supported head_dim)
   bool tc_attn_ = false;
+  // per block: max|g| sqrt(head_dim) of the QK-norm gains, bounds on the norms
+  // of the normalised query and key rows (read once, at init)
+  std::vector<float> qn_max_, kn_max_;
   std::vector<SwaTcPlan> att_bot_, att_top_;
   std::vector<SwaTcBwdPlan> att_bwd_;
   int attn_fwd(const SwaTcPlan* plan, const SwaArgs& a) {
@@ -616,6 +621,26 @@ int Engine<T>::init() {
 
   // ---- attention plans ----------------------------------------------------------------------
   tc_attn_ = BF && swa_tc_supported((int)HD_);
+  qn_max_.assign(L_, 0.f);
+  kn_max_.assign(L_, 0.f);
+  if (tc_attn_) {
+    std::vector<float> gq(HD_), gk(HD_);
+    for (int64_t l = 0; l < L_; ++l) {
+      TTT_CUDA_TRY(cudaMemcpyAsync(gq.data(), wt_.layers[l].q_norm, HD_ * sizeof(float), cudaMemcpyDeviceToHost, st_));
+      TTT_CUDA_TRY(cudaMemcpyAsync(gk.data(), wt_.layers[l].k_norm, HD_ * sizeof(float), cudaMemcpyDeviceToHost, st_));
+      TTT_CUDA_TRY(cudaStreamSynchronize(st_));
+      float mq = 0.f, mk = 0.f;
+      for (int64_t c = 0; c < HD_; ++c) {
+        mq = std::max(mq, std::fabs(gq[c]));
+        mk = std::max(mk, std::fabs(gk[c]));
+      }
+      // RMSNorm output rows have norm <= sqrt(head_dim) before the gain; RoPE keeps the norm
+      if (std::isfinite(mq) && std::isfinite(mk)) {
+        qn_max_[l] = mq * std::sqrt((float)HD_);
+        kn_max_[l] = mk * std::sqrt((float)HD_);
+      }
+    }
+  }
   if (tc_attn_) {
     att_bot_.resize(nbot_);
     att_top_.resize(nu_);
@@ -777,7 +802,7 @@ int Engine<T>::bottom_layers(const int32_t* tok, int64_t s0, int64_t S) {
                                  kb_[l], vb_[l], d, R1_, rqs_, rks_, st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(s0, S),
               [&] { return attn_fwd(tc_attn_ ? &att_bot_[l] : nullptr,
-                                    swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_)); }));
+                                    swa_args(qs_, S, s0, kb_[l], vb_[l], R1_, os_, lses_, S_, l)); }));
     TRY(run(g[1], S));
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xs_, d, lw.mlp_norm, eps, S, (int)d, hs_, d, rs_, st_); }));
     TRY(run(g[2], S));
@@ -806,7 +831,7 @@ int Engine<T>::chunk(const int32_t* tok, int64_t T_, int64_t p0, int64_t n, cons
                                  kt_[i], vt_[i], d, R_, rq_[i], rk_[i], st_); }));
     TRY(timed(TTT_KC_ATTN_FWD, 4.0 * d * band_pairs(p0, n),
               [&] { return attn_fwd(tc_attn_ ? &att_top_[i] : nullptr,
-                                    swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b)); }));
+                                    swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b, l)); }));
     g[1].args.c2 = const_cast<float*>(xin);
     TRY(run(g[1], n));
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_fwd<T>(xmid_[i], d, lw.mlp_norm, eps, n, (int)d, h2_[i], d, r2_[i], st_); }));
@@ -854,7 +879,7 @@ int Engine<T>::chunk_backward(int64_t p0, int64_t n, bool logits_stored) {
     if (i == 0) break;  // nothing below the lowest fast block depends on W
     TRY(timed(TTT_KC_NORM, 0, [&] { return rmsnorm_bwd<T>(xmid_[i], d, r2_[i], lw.mlp_norm, dh2_, d, dx_, d, n, (int)d, dxm_, d, dxm16_, d, st_); }));
     TRY(run(g[8], n));
-    SwaArgs a = swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b);
+    SwaArgs a = swa_args(q_[i], n, p0, kt_[i], vt_[i], R_, o_[i], lse_[i], b, l);
     a.dout = do_;
     a.lddo = d;
     a.dq = dqkv_;

@@ -286,7 +286,7 @@ template <int BN, int EPI>
 __device__ __forceinline__ void epilogue_transposed(uint32_t t_row, const EpiArgs& ep, int64_t n0, int64_t N,
                                                     int split, float* wbuf, int64_t row0, int64_t M,
                                                     float (&bufA)[32], float (&bufB)[32]) {
-  static_assert(BN % 64 == 0, "chunks come in pairs");
+  static_assert(BN % 32 == 0, "32-column chunks");
   const int lane = threadIdx.x & 31;
   const int nrows = (int)(M - row0 < 32 ? (M - row0 > 0 ? M - row0 : 0) : 32);
   int64_t ld = 0;
@@ -644,12 +644,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-// CTA-pair variant: a cluster of two CTAs (two SMs) computes one 256 x 256
-// output tile with tcgen05.mma.cta_group::2.  Each CTA loads its own 128 rows
-// of A and its half (128 rows) of the B tile, 32 KB per 64-deep k-block
-// instead of the 48 KB a single CTA needs for a 128 x 256 tile, so a CTA
-// streams 131 instead of 87 flop per operand byte and the ring holds six
-// stages instead of four.  Roles:
+// CTA-pair variant: a cluster of two CTAs (two SMs) computes one 256 x BN
+// output tile (BN = 256 or 128) with tcgen05.mma.cta_group::2.  Each CTA
+// loads its own 128 rows of A and its half (BN/2 rows) of the B tile: for
+// BN = 256, 32 KB per 64-deep k-block instead of the 48 KB a single CTA needs
+// for a 128 x 256 tile, so a CTA streams 131 instead of 87 flop per operand
+// byte.  A pair MMA also runs at the tensor cores' rate for N = 128 (about 65
+// cycles per 16-deep step, measured), where a single-CTA M = 128 MMA costs
+// about 100 cycles whatever its N up to 128: the narrow tiles of the
+// M = b products therefore run on pairs as well.  Roles:
 //   even CTA, warp 0 lane 0   TMA for its halves; arrives on its own full
 //                             barrier with the bytes of both CTAs
 //   odd CTA,  warp 0 lane 0   TMA for its halves, counted on the even CTA's
@@ -662,25 +665,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //                             (256 arrivals: both CTAs' epilogue groups)
 // The units are (256-row pair tile, n-tile, k-split), walked by the pairs
 // like the single-CTA kernel walks its tiles.
-template <int EPI>
+template <int EPI, int BN_, bool B_MN>
 struct PairCfg {
-  static constexpr int BN = 256;
-  static constexpr int A_BYTES = BM * BK * 2;    // this CTA's 128 rows of A
-  static constexpr int B_BYTES = 128 * BK * 2;   // this CTA's half of the B tile
+  static constexpr int BN = BN_;
+  static constexpr int A_BYTES = BM * BK * 2;  // this CTA's 128 rows of A
+  // this CTA's half of the B tile: BN/2 rows (K-major), or BN/2 columns in
+  // whole 64-column boxes (MN-major)
+  static constexpr int NBOX = (BN / 2 + 63) / 64;
+  static constexpr int B_BYTES = B_MN ? NBOX * 64 * BK * 2 : (BN / 2) * BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = EPI == EPI_SGD ? 5 : 6;
   static constexpr int WBUF = kEpiWarps * 32 * kWStride<EPI> * 4;
+  static constexpr int STAGES_FIT = (232448 - 1024 - 256 - WBUF) / STAGE;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int SMEM = STAGES * STAGE + 1024 + 256 + WBUF;
+  // TMEM: two accumulator buffers of BN columns, allocated as a power of two
+  static constexpr int TMEM_COLS = 2 * BN <= 256 ? 256 : 512;
+  static_assert(B_BYTES % 1024 == 0, "1024-byte aligned B stages");
   static_assert(SMEM <= 232448, "shared memory per block");
 };
 
-template <bool A_MN, bool B_MN, int EPI, typename TACT>
+template <int BN_, bool A_MN, bool B_MN, int EPI, typename TACT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
                         const __grid_constant__ CUtensorMap tma2, const __grid_constant__ CUtensorMap tmb2,
                         int64_t M, int64_t N, int KB1, int KB2, int64_t n_ext, int kpsb, int n_mt, int n_nt,
                         int n_split, int n_fast, EpiArgs ep, int* err) {
-  using C = PairCfg<EPI>;
+  using C = PairCfg<EPI, BN_, B_MN>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -731,7 +741,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
   if (warp == 1) {
     __syncwarp();
-    ptx::tmem_alloc_pair(tmem_slot, 2 * BN);
+    ptx::tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
@@ -762,7 +772,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const CUtensorMap* ta = second ? &tma2 : &tma;
           const CUtensorMap* tb = second ? &tmb2 : &tmb;
           const int k0 = (second ? kb - KB1 : kb) * BK;
-          const int nb = (int)(second ? n0 - n_ext : n0) + 128 * (int)rank;  // this CTA's half of B
+          const int nb = (int)(second ? n0 - n_ext : n0) + (BN / 2) * (int)rank;  // this CTA's half of B
           if constexpr (!A_MN) {
             ptx::tma_load_2d_pair(a, ta, fb, k0, mo);
           } else {
@@ -772,8 +782,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           if constexpr (!B_MN) {
             ptx::tma_load_2d_pair(b, tb, fb, k0, nb);
           } else {
-            ptx::tma_load_2d_pair(b, tb, fb, nb, k0);
-            ptx::tma_load_2d_pair(b + 8192, tb, fb, nb + 64, k0);
+#pragma unroll
+            for (int i = 0; i < C::NBOX; ++i) ptx::tma_load_2d_pair(b + 8192 * i, tb, fb, nb + 64 * i, k0);
           }
         }
       }
@@ -870,7 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   if (warp == 1) {
     __syncwarp();
     ptx::tc_fence_after();
-    ptx::tmem_dealloc_pair(tmem, 2 * BN);
+    ptx::tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
 }
 
@@ -1007,33 +1017,53 @@ KernelFn pick_epi(int epi, int act_bf16) {
   return nullptr;
 }
 
-template <bool A_MN, bool B_MN, int EPI, typename TACT>
+template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 KernelFn pair_ptr() {
-  return reinterpret_cast<KernelFn>(&tc_gemm_pair_kernel<A_MN, B_MN, EPI, TACT>);
+  return reinterpret_cast<KernelFn>(&tc_gemm_pair_kernel<BN, A_MN, B_MN, EPI, TACT>);
 }
 
-template <bool A_MN, bool B_MN>
+template <int BN, bool A_MN, bool B_MN>
 KernelFn pick_pair_epi(int epi, int act_bf16) {
+  if constexpr (BN == 160) {  // 160-wide tiles: plain stores and the residual add only
+    switch (epi) {
+      case EPI_STORE_F32: return pair_ptr<BN, A_MN, B_MN, EPI_STORE_F32, bf16>();
+      case EPI_STORE_BF16: return pair_ptr<BN, A_MN, B_MN, EPI_STORE_BF16, bf16>();
+      case EPI_ADD_F32: return pair_ptr<BN, A_MN, B_MN, EPI_ADD_F32, bf16>();
+    }
+    return nullptr;
+  }
   switch (epi) {
-    case EPI_STORE_F32: return pair_ptr<A_MN, B_MN, EPI_STORE_F32, bf16>();
-    case EPI_STORE_BF16: return pair_ptr<A_MN, B_MN, EPI_STORE_BF16, bf16>();
-    case EPI_ADD_F32: return pair_ptr<A_MN, B_MN, EPI_ADD_F32, bf16>();
-    case EPI_SWIGLU: return act_bf16 ? pair_ptr<A_MN, B_MN, EPI_SWIGLU, bf16>() : pair_ptr<A_MN, B_MN, EPI_SWIGLU, float>();
-    case EPI_CE_FWD: return pair_ptr<A_MN, B_MN, EPI_CE_FWD, bf16>();
-    case EPI_CE_BWD: return act_bf16 ? pair_ptr<A_MN, B_MN, EPI_CE_BWD, bf16>() : pair_ptr<A_MN, B_MN, EPI_CE_BWD, float>();
-    case EPI_SGD: return pair_ptr<A_MN, B_MN, EPI_SGD, bf16>();
+    case EPI_STORE_F32: return pair_ptr<BN, A_MN, B_MN, EPI_STORE_F32, bf16>();
+    case EPI_STORE_BF16: return pair_ptr<BN, A_MN, B_MN, EPI_STORE_BF16, bf16>();
+    case EPI_ADD_F32: return pair_ptr<BN, A_MN, B_MN, EPI_ADD_F32, bf16>();
+    case EPI_SWIGLU:
+      return act_bf16 ? pair_ptr<BN, A_MN, B_MN, EPI_SWIGLU, bf16>() : pair_ptr<BN, A_MN, B_MN, EPI_SWIGLU, float>();
+    case EPI_CE_FWD: return pair_ptr<BN, A_MN, B_MN, EPI_CE_FWD, bf16>();
+    case EPI_CE_BWD:
+      return act_bf16 ? pair_ptr<BN, A_MN, B_MN, EPI_CE_BWD, bf16>() : pair_ptr<BN, A_MN, B_MN, EPI_CE_BWD, float>();
+    case EPI_SGD: return pair_ptr<BN, A_MN, B_MN, EPI_SGD, bf16>();
   }
   return nullptr;
 }
 
-KernelFn pick_pair(int a_mn, int b_mn, int epi, int act_bf16) {
-  if (!a_mn && !b_mn) return pick_pair_epi<false, false>(epi, act_bf16);
-  if (!a_mn && b_mn) return pick_pair_epi<false, true>(epi, act_bf16);
-  if (a_mn && b_mn) return pick_pair_epi<true, true>(epi, act_bf16);
-  return pick_pair_epi<true, false>(epi, act_bf16);
+template <int BN>
+KernelFn pick_pair_bn(int a_mn, int b_mn, int epi, int act_bf16) {
+  if (!a_mn && !b_mn) return pick_pair_epi<BN, false, false>(epi, act_bf16);
+  if (!a_mn && b_mn) return pick_pair_epi<BN, false, true>(epi, act_bf16);
+  if (a_mn && b_mn) return pick_pair_epi<BN, true, true>(epi, act_bf16);
+  return pick_pair_epi<BN, true, false>(epi, act_bf16);
 }
 
-// CTA pairs for 256-wide tiles of GEMMs with more than one 128-row tile;
+KernelFn pick_pair(int bn, int a_mn, int b_mn, int epi, int act_bf16) {
+  switch (bn) {
+    case 256: return pick_pair_bn<256>(a_mn, b_mn, epi, act_bf16);
+    case 160: return pick_pair_bn<160>(a_mn, b_mn, epi, act_bf16);
+    case 128: return pick_pair_bn<128>(a_mn, b_mn, epi, act_bf16);
+  }
+  return nullptr;
+}
+
+// CTA pairs for every GEMM with more than one 128-row tile;
 // TTT_GEMM_PAIR=0 keeps every GEMM on single CTAs.
 bool pair_enabled() {
   static const bool on = [] {
@@ -1051,13 +1081,20 @@ KernelFn pick(int a_mn, int b_mn, int epi, int act_bf16) {
   return pick_epi<BN, true, false>(epi, act_bf16);
 }
 
-template <int EPI>
-int smem_bytes_epi(int pair, int bn) {
-  return pair ? PairCfg<EPI>::SMEM : (bn == 256 ? TcCfg<256, EPI>::SMEM : TcCfg<128, EPI>::SMEM);
+template <int EPI, bool B_MN>
+int pair_smem(int bn) {
+  return bn == 256 ? PairCfg<EPI, 256, B_MN>::SMEM
+                   : (bn == 160 ? PairCfg<EPI, 160, B_MN>::SMEM : PairCfg<EPI, 128, B_MN>::SMEM);
 }
 
-int smem_bytes(int pair, int bn, int epi) {
-  return epi == EPI_SGD ? smem_bytes_epi<EPI_SGD>(pair, bn) : smem_bytes_epi<EPI_STORE_F32>(pair, bn);
+template <int EPI>
+int smem_bytes_epi(int pair, int bn, int b_mn) {
+  if (pair) return b_mn ? pair_smem<EPI, true>(bn) : pair_smem<EPI, false>(bn);
+  return bn == 256 ? TcCfg<256, EPI>::SMEM : TcCfg<128, EPI>::SMEM;
+}
+
+int smem_bytes(int pair, int bn, int epi, int b_mn) {
+  return epi == EPI_SGD ? smem_bytes_epi<EPI_SGD>(pair, bn, b_mn) : smem_bytes_epi<EPI_STORE_F32>(pair, bn, b_mn);
 }
 
 }  // namespace
@@ -1065,18 +1102,63 @@ int smem_bytes(int pair, int bn, int epi) {
 int64_t tc_ce_tiles(int64_t N, int bn) { return (N + bn - 1) / bn; }
 
 int tc_pick_bn(int64_t M, int64_t N, int hint) {
-  if (hint == 128 || hint == 256) return hint;
+  if (hint == 128 || hint == 160 || hint == 256) return hint;
   // Prefer 256-wide tiles when that still gives every SM a tile.
   const int64_t tiles256 = ((N + 255) / 256) * ((M + BM - 1) / BM);
   return (tiles256 >= 148 || N > 4096) ? 256 : 128;
 }
 
+namespace {
+// Cost (cycles) of a store/add GEMM on CTA pairs with bn-wide tiles and S
+// splits of K, fitted to measured b-row products (M = 1024, N = 2560, K from
+// 2560 to 27648, tile widths 128 to 256, 1 to 6 splits): every pair slot
+// runs ceil(units / slots) work units one after the other; a unit costs
+// about 13000 cycles of start, pipeline fill and epilogue plus about 760
+// cycles per 64-deep k-block (whatever the tile width: the operand pipeline,
+// not the tensor core, sets that pace), or its four pair MMAs if slower;
+// split-K adds about 30000 cycles for the partials' round trip through HBM
+// and the reduction launch.  Only the ranking matters.
+double pair_cost(int64_t M, int64_t N, int64_t K, int bn, int64_t S) {
+  const int64_t slots = 74;
+  const int64_t tiles = ((M + 2 * BM - 1) / (2 * BM)) * ((N + bn - 1) / bn);
+  const int64_t units = tiles * S;
+  const int64_t waves = (units + slots - 1) / slots;
+  const int64_t kb = ((K + BK - 1) / BK + S - 1) / S;
+  const double per_kb = std::max(4.0 * (bn / 2 + 1), 760.0);
+  double t = (double)waves * ((double)kb * per_kb + 13000.0);
+  if (S > 1) t += 30000.0 + (double)(S + 1) * (double)M * (double)N * 4.0 / 3600.0;
+  return t;
+}
+}  // namespace
+
 int64_t tc_split_plan(int64_t M, int64_t N, int64_t K, int epi, int* bn_out) {
-  // Split K when the output alone gives fewer than two waves of 256-wide tiles
-  // and the reduction is long: pick the split count (2..8, >= 1024 of K each)
-  // whose work units fill the 148 SMs best.
   *bn_out = 0;
   if (epi != EPI_STORE_F32 && epi != EPI_STORE_BF16 && epi != EPI_ADD_F32) return 1;
+  if (M > BM && pair_enabled()) {
+    // CTA pairs: the tile width (160, 256 or 128) and split count (1..8, at
+    // least 16 k-blocks each) of least modelled cost; an earlier width or
+    // fewer splits must lose by more than 3% to be passed over.
+    const int64_t kb = (K + BK - 1) / BK;
+    double best = 0.0;
+    int best_bn = 0;
+    int64_t best_s = 1;
+    for (int bn : {160, 256, 128}) {
+      for (int64_t S = 1; S <= 8; ++S) {
+        if (S > 1 && kb / S < 16) break;
+        const double c = pair_cost(M, N, K, bn, S);
+        if (best_bn == 0 || c < 0.97 * best) {
+          best = c;
+          best_bn = bn;
+          best_s = S;
+        }
+      }
+    }
+    *bn_out = best_bn;
+    return best_s;
+  }
+  // Single CTAs: split K when the output alone gives fewer than two waves of
+  // 256-wide tiles and the reduction is long: pick the split count (2..8,
+  // >= 1024 of K each) whose work units fill the 148 SMs best.
   const int64_t tiles = ((N + 255) / 256) * ((M + BM - 1) / BM);
   if (tiles >= 2 * 148 || K < 2048) return 1;
   auto fill = [](int64_t units) { return (double)units / (double)(((units + 147) / 148) * 148); };
@@ -1102,6 +1184,8 @@ int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args,
   if (epi < 0 || epi >= EPI_COUNT) return set_error(TTT_ERR_INVALID_ARG, "gemm: bad epilogue");
   const int bn = tc_pick_bn(M, N, bn_hint);
   if (epi == EPI_SWIGLU && (N % 128) != 0) return set_error(TTT_ERR_INVALID_ARG, "gemm: SwiGLU needs N % 128 == 0");
+  if (bn == 160 && !(M > BM && pair_enabled() && (epi == EPI_STORE_F32 || epi == EPI_STORE_BF16 || epi == EPI_ADD_F32)))
+    return set_error(TTT_ERR_INVALID_ARG, "gemm: 160-wide tiles need more than 128 rows and a store/add epilogue");
   g->a_mn = s.a_mn;
   g->b_mn = s.b_mn;
   g->bn = bn;
@@ -1115,10 +1199,10 @@ int tc_gemm_prepare(TcGemm* g, const GemmShape& s, int epi, const EpiArgs& args,
   g->ws = nullptr;
   g->K2 = 0;
   g->n_ext = 0;
-  g->pair = (bn == 256 && M > BM && pair_enabled()) ? 1 : 0;
+  g->pair = (M > BM && pair_enabled()) ? 1 : 0;
   int rc = make_tmap(&g->ta, s.a, s.a_mn ? 64 : BM);
   if (rc) return rc;
-  rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : (g->pair ? 128 : bn));
+  rc = make_tmap(&g->tb, s.b, s.b_mn ? 64 : (g->pair ? bn / 2 : bn));
   g->ta2 = g->ta;
   g->tb2 = g->tb;
   return rc;
@@ -1133,7 +1217,7 @@ int tc_gemm_set_ext(TcGemm* g, const MatView& a2, const MatView& b2, int64_t n_e
   if (g->epi == EPI_CE_FWD) return set_error(TTT_ERR_INVALID_ARG, "gemm: no second product with CE partials");
   int rc = make_tmap(&g->ta2, a2, g->a_mn ? 64 : BM);
   if (rc) return rc;
-  rc = make_tmap(&g->tb2, b2, g->b_mn ? 64 : (g->pair ? 128 : g->bn));
+  rc = make_tmap(&g->tb2, b2, g->b_mn ? 64 : (g->pair ? g->bn / 2 : g->bn));
   if (rc) return rc;
   g->K2 = K2;
   g->n_ext = n_ext;
@@ -1162,11 +1246,11 @@ int tc_gemm_set_split(TcGemm* g, int64_t ksplit, float* ws) {
 
 int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   const int kepi = g.ksplit > 1 ? EPI_STORE_F32 : g.epi;
-  KernelFn fn = g.pair ? pick_pair(g.a_mn, g.b_mn, kepi, g.act_bf16)
+  KernelFn fn = g.pair ? pick_pair(g.bn, g.a_mn, g.b_mn, kepi, g.act_bf16)
                        : (g.bn == 256 ? pick<256>(g.a_mn, g.b_mn, kepi, g.act_bf16)
                                       : pick<128>(g.a_mn, g.b_mn, kepi, g.act_bf16));
   if (!fn) return set_error(TTT_ERR_INVALID_ARG, "gemm: no kernel for this combination");
-  const int smem = smem_bytes(g.pair, g.bn, kepi);
+  const int smem = smem_bytes(g.pair, g.bn, kepi, g.b_mn);
   {
     static std::mutex mu;
     static std::set<std::pair<int, KernelFn>> configured;

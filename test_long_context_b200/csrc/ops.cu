@@ -1,5 +1,6 @@
 // Op-level entry points (include/ttt_ops.h): thin wrappers that validate the
 // arguments and launch one kernel family each.
+#include <cmath>
 #include "../../include/ttt_ops.h"
 #include "attention.cuh"
 #include "attention_tc.cuh"
@@ -114,6 +115,13 @@ extern "C" int ttt_op_gemm_dual(int32_t a_mn, int32_t b_mn, int64_t M, int64_t N
   return tc_gemm_launch(g, reinterpret_cast<cudaStream_t>(stream), err);
 }
 
+extern "C" int64_t ttt_op_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t epilogue, int32_t* bn_out) {
+  int bn = 0;
+  const int64_t S = (M < 1 || N < 1 || K < 1) ? 1 : tc_split_plan(M, N, K, epilogue, &bn);
+  if (bn_out) *bn_out = bn;
+  return S;
+}
+
 extern "C" int64_t ttt_op_gemm_ce_tiles(int32_t dtype, int64_t M, int64_t N, int32_t bn_hint) {
   if (dtype == TTT_F32) return (N + 127) / 128;
   return tc_ce_tiles(N, tc_pick_bn(M, N, bn_hint));
@@ -177,11 +185,16 @@ int op_swa_backward_run(const SwaArgs& a, int32_t dtype, int32_t flags, cudaStre
 
 extern "C" int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0,
                                   int32_t window, const void* q, int64_t ldq, const void* k_ring, const void* v_ring,
-                                  int64_t ring_slots, void* o, int64_t ldo, float* lse, int32_t flags, void* stream) {
+                                  int64_t ring_slots, void* o, int64_t ldo, float* lse, float q_norm_max,
+                                  float k_norm_max, int32_t flags, void* stream) {
   if (!q || !k_ring || !v_ring || !o || !lse || n_q < 1 || q_pos0 < 0 || window < 1 || ring_slots < 1 ||
       n_heads < 1 || (dtype != TTT_F32 && dtype != TTT_BF16))
     return set_error(TTT_ERR_INVALID_ARG, "ttt_op_swa_forward: bad argument");
   SwaArgs a = op_swa_args(n_heads, head_dim, n_q, q_pos0, window, q, ldq, k_ring, v_ring, ring_slots, o, ldo, lse);
+  a.q_norm_max = std::isfinite(q_norm_max) ? q_norm_max : 0.f;
+  a.k_norm_max = std::isfinite(k_norm_max) ? k_norm_max : 0.f;
+  a.exp_poly = ((flags >> 4) & 15) - 1;
+  a.softmax_groups = (flags >> 8) & 15;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0) {
     SwaTcPlan plan;

@@ -34,9 +34,10 @@ def band_pairs(p0, n, k):
     return s
 
 
-def op_builders(cfg):
+def op_builders(cfg, exp_poly=None, softmax_groups=None):
     """{name: builder}; a builder allocates the op's inputs and returns
-    (run, algorithmic flops, algorithmic bytes)."""
+    (run, algorithmic flops, algorithmic bytes).  exp_poly, softmax_groups:
+    tuning of the fixed-shift attention forward (None = defaults)."""
     d, f, V, b, k, H, hd = cfg.d_model, cfg.d_ff, cfg.vocab, cfg.b, cfg.k, cfg.n_heads, cfg.head_dim
     S = max(1, 16384 // b) * b
     bf = torch.bfloat16
@@ -52,7 +53,11 @@ def op_builders(cfg):
             A = rn(K, M) if a_mn else rn(M, K)
             Bm = rn(K, N) if b_mn else rn(N, K)
             args = {key: (v() if callable(v) else v) for key, v in outs.items()}
-            return (lambda: ops.gemm(A, Bm, a_mn, b_mn, epi, **args)), 2.0 * M * N * K, 0.0
+            S, bn = ops.gemm_plan(M, N, K, epi)  # the prefill's tile width and split-K count
+            if S > 1:
+                ws = torch.empty(S * M * N, device=dev)
+                return (lambda: ops.gemm_split(A, Bm, a_mn, b_mn, epi, S, ws, bn=bn, **args)), 2.0 * M * N * K, 0.0
+            return (lambda: ops.gemm(A, Bm, a_mn, b_mn, epi, bn=bn, **args)), 2.0 * M * N * K, 0.0
         B[name] = build
 
     f32 = torch.float32
@@ -105,10 +110,13 @@ def op_builders(cfg):
             kr, vr = rn(ring, H * hd), rn(ring, H * hd)
             o = emp(n, H * hd)
             lse = emp(H, n, dt=f32)
+            # the engine passes the bounds of the QK-norm (unit gains: sqrt(head_dim))
+            nb = dict(q_norm_max=hd ** 0.5, k_norm_max=hd ** 0.5)
             pairs = band_pairs(p0, n, k)
             if not backward:
-                return (lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse)), 4.0 * d * pairs, 0.0
-            ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse)
+                return ((lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse, exp_poly=exp_poly,
+                                                 softmax_groups=softmax_groups, **nb)), 4.0 * d * pairs, 0.0)
+            ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse, **nb)
             dout = rn(n, H * hd)
             dq, dk, dv = (torch.empty_like(q) for _ in range(3))
             D = emp(H * n, dt=f32)
@@ -153,7 +161,7 @@ def op_builders(cfg):
 
     def attn_dec():
         qd, od, lsed = rn(d), emp(d), emp(H, dt=f32)
-        wsd = emp(H * ((k + 127) // 128 + 1) * (hd + 2), dt=f32)
+        wsd = torch.zeros(H * (((k + 127) // 128 + 1) * (hd + 2) + 1), device=dev)
         kdec, vdec = rn(R, d), rn(R, d)
         pdec = 16 * k + 5
         return (lambda: ops.attn_decode(qd, kdec, vdec, H, hd, pdec, k, od, lsed, wsd)), 0.0, 2.0 * 2 * d * k
@@ -167,9 +175,11 @@ def main():
     ap.add_argument("--op", nargs="*", default=None)
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--exp-poly", type=int, default=None, choices=[0, 2, 4])
+    ap.add_argument("--softmax-groups", type=int, default=None, choices=[2, 4])
     args = ap.parse_args()
     cfg = get_config(args.config)
-    builders = op_builders(cfg)
+    builders = op_builders(cfg, args.exp_poly, args.softmax_groups)
     for name in args.op or list(builders):
         run, flops, nbytes = builders[name]()
         for _ in range(args.warmup):
@@ -183,6 +193,8 @@ def main():
         ops.sync()
         ms = e0.elapsed_time(e1) / args.iters
         rec = {"op": name, "config": args.config, "ms": ms}
+        if name.startswith("swa_fwd"):
+            rec.update(exp_poly=args.exp_poly, softmax_groups=args.softmax_groups)
         if flops:
             rec.update(tflops=flops / (ms / 1e3) / 1e12, algorithmic_flops=flops)
         if nbytes:

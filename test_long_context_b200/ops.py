@@ -72,6 +72,13 @@ def gemm_dual(A, B, A2, B2, a_mn, b_mn, epi, n_ext=0, ksplit=1, workspace=None, 
     L.check(rc)
 
 
+def gemm_plan(M, N, K, epi):
+    """ttt_op_gemm_plan: (split count, tile width) the prefill uses."""
+    bn = ctypes.c_int32(0)
+    S = int(L.lib().ttt_op_gemm_plan(M, N, K, epi, ctypes.byref(bn)))
+    return S, int(bn.value)
+
+
 def gemm_ce_tiles(dtype_is_bf16, M, N, bn=0):
     return int(L.lib().ttt_op_gemm_ce_tiles(L.TTT_BF16 if dtype_is_bf16 else L.TTT_F32, M, N, bn))
 
@@ -80,11 +87,21 @@ def sync(stream=None):
     L.check(L.lib().ttt_op_sync(_stream(stream)))
 
 
-def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, force_simt=False, stream=None):
-    """ttt_op_swa_forward; q/o [n, H*hd], rings [R, H*hd], lse [H, n]."""
+def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, force_simt=False, stream=None,
+                q_norm_max=0.0, k_norm_max=0.0, exp_poly=None, softmax_groups=None):
+    """ttt_op_swa_forward; q/o [n, H*hd], rings [R, H*hd], lse [H, n].
+    q_norm_max, k_norm_max: bounds on the row norms of q and k (0 = unknown;
+    both known: the fixed-shift tensor-core forward); exp_poly: its
+    polynomial share of the exponentials (0, 2 or 4 of 8), softmax_groups: its
+    softmax warpgroups (2 or 4); None = library defaults."""
+    flags = 1 if force_simt else 0
+    if exp_poly is not None:
+        flags |= ((exp_poly + 1) & 15) << 4
+    if softmax_groups is not None:
+        flags |= (softmax_groups & 15) << 8
     rc = L.lib().ttt_op_swa_forward(_dtype(q), n_heads, head_dim, q.shape[0], q_pos0, window, _p(q), q.stride(0),
                                     _p(k_ring), _p(v_ring), k_ring.shape[0], _p(o), o.stride(0), _p(lse),
-                                    1 if force_simt else 0, _stream(stream))
+                                    float(q_norm_max), float(k_norm_max), flags, _stream(stream))
     L.check(rc)
 
 

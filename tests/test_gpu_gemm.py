@@ -269,10 +269,11 @@ def test_split_k_reduce_vector_and_scalar_paths(N):
 
 @pytest.mark.parametrize("combo", COMBOS)
 def test_cta_pair_tiles_every_epilogue(combo):
-    """256-wide tiles run on CTA pairs (one 256 x 256 tile per pair, each CTA
-    loading its own 128 rows of A and half of the B tile): every epilogue
-    against the fp64 product and against single-CTA 128-wide tiles, with a
-    last pair tile whose odd CTA has no valid rows at all (M = 600)."""
+    """GEMMs with more than 128 rows run on CTA pairs (one 256 x BN tile per
+    pair, each CTA loading its own 128 rows of A and half of the B tile):
+    every epilogue on 128- and 256-wide pair tiles against the fp64 product
+    and against each other, with a last pair tile whose odd CTA has no valid
+    rows at all (M = 600)."""
     from test_long_context_b200 import ops
     M, N, K = 600, 768, 320
     A, B, ref = _operands(M, N, K, *combo, torch.bfloat16, seed=31)
@@ -358,3 +359,60 @@ def test_cta_pair_tiles_cross_entropy_split_and_dual():
     ops.sync()
     assert (c.double() - ref).abs().max().item() <= 1e-4 * ref.abs().max().item() + 1e-4
     assert (cd.double() - refd).abs().max().item() <= 1e-4 * refd.abs().max().item() + 1e-4
+
+
+@pytest.mark.parametrize("combo", [(0, 0), (0, 1), (1, 1)])
+def test_pair_tiles_160_wide(combo):
+    """160-wide pair tiles (the M = b products of the prefill: a single wave
+    of 256 x 160 tiles): plain stores, the residual add and split-K partials
+    against the fp64 product, on a ragged N (1000: the last tile holds 40
+    columns) and a last pair tile whose odd CTA has no rows (M = 600)."""
+    from test_long_context_b200 import ops
+    M, N, K = 600, 1000, 704
+    A, B, ref = _operands(M, N, K, *combo, torch.bfloat16, seed=37)
+    scale = ref.abs().max().item()
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, *combo, ops.L.EPI_STORE_F32, c=c, bn=160)
+    cb = torch.full((M, N), float("nan"), device="cuda", dtype=torch.bfloat16)
+    ops.gemm(A, B, *combo, ops.L.EPI_STORE_BF16, c=cb, bn=160)
+    x0 = torch.randn(M, N, device="cuda", generator=torch.Generator(device="cuda").manual_seed(3))
+    x = torch.full_like(x0, float("nan"))
+    ops.gemm(A, B, *combo, ops.L.EPI_ADD_F32, c=x, c2=x0, bn=160)
+    ws = torch.empty(3 * M * N, device="cuda")
+    cs = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm_split(A, B, *combo, ops.L.EPI_STORE_F32, 3, ws, c=cs, bn=160)
+    c128 = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, *combo, ops.L.EPI_STORE_F32, c=c128, bn=128)
+    ops.sync()
+    assert (c.double() - ref).abs().max().item() <= 1e-4 * scale + 1e-4
+    assert (cb.double() - ref).abs().max().item() <= 1e-2 * scale
+    assert (x.double() - (x0.double() + ref)).abs().max().item() <= 1e-4 * scale + 1e-4
+    assert (cs.double() - ref).abs().max().item() <= 1e-4 * scale + 1e-4
+    assert (c - c128).abs().max().item() <= 1e-5 * scale
+
+
+def test_pair_tiles_160_wide_refused_where_unsupported():
+    """160-wide tiles are refused for epilogues that need 128-column groups
+    (SwiGLU, CE, SGD) and for single-CTA products (M <= 128)."""
+    from test_long_context_b200 import _lib as L
+    from test_long_context_b200 import ops
+    A = torch.randn(600, 256, device="cuda").bfloat16()
+    B = torch.randn(512, 256, device="cuda").bfloat16()
+    a = torch.empty(600, 256, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(L.TTTError):
+        ops.gemm(A, B, 0, 0, ops.L.EPI_SWIGLU, c=a, bn=160)
+    c = torch.empty(100, 512, device="cuda")
+    with pytest.raises(L.TTTError):
+        ops.gemm(A[:100], B, 0, 0, ops.L.EPI_STORE_F32, c=c, bn=160)
+
+
+def test_gemm_plan_of_the_prefill_products():
+    """The plan picks one wave of 160-wide pair tiles for the b x d outputs
+    of the blocks with fast weights, and 256-wide tiles for the large ones."""
+    from test_long_context_b200 import ops
+    S, bn = ops.gemm_plan(1024, 2560, 2560, ops.L.EPI_ADD_F32)
+    assert (S, bn) == (1, 160)
+    S, bn = ops.gemm_plan(16384, 2560, 2560, ops.L.EPI_ADD_F32)
+    assert (S, bn) == (1, 256)
+    S, bn = ops.gemm_plan(1024, 2560, 2560, ops.L.EPI_SWIGLU)
+    assert (S, bn) == (1, 0)
