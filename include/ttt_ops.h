@@ -131,12 +131,10 @@ int64_t ttt_op_gemm_plan(int64_t M, int64_t N, int64_t K, int32_t epilogue, int3
  * results.
  * flags bits 4..7, TTT_SWA_EXP_POLY(n): on that path n of every 8 groups of
  * 8 keys (n in 0, 2, 4) take 2^x from an FMA-pipe polynomial (relative error
- * 7.5e-5) instead of the MUFU unit; flags bits 8..11, TTT_SWA_SOFTMAX_GROUPS
- * (2 or 4): softmax warpgroups per CTA.  0 in these bits = library default.
+ * 7.5e-5) instead of the MUFU unit; 0 in these bits = library default.
  */
 #define TTT_SWA_FORCE_SIMT 1
 #define TTT_SWA_EXP_POLY(n) ((((n) + 1) & 15) << 4)
-#define TTT_SWA_SOFTMAX_GROUPS(n) (((n) & 15) << 8)
 int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_dim, int64_t n_q, int64_t q_pos0, int32_t window,
                        const void* q, int64_t ldq, const void* k_ring, const void* v_ring, int64_t ring_slots,
                        void* o, int64_t ldo, float* lse, float q_norm_max, float k_norm_max, int32_t flags,

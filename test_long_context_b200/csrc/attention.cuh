@@ -25,11 +25,9 @@ struct SwaArgs {
   // k_norm_max <= 48, the tensor-core forward shifts each row's softmax by
   // the Cauchy-Schwarz bound of its scores instead of a running maximum.
   float q_norm_max = 0.f, k_norm_max = 0.f;
-  // Fixed-shift forward tuning: how many of every 8 groups of 8 keys take
-  // 2^x from an FMA-pipe polynomial instead of the MUFU unit (0, 2, 4), and
-  // the number of softmax warpgroups (2, 4); -1 / 0 = library defaults.
+  // Fixed-shift forward: how many of every 8 groups of 8 keys take 2^x from
+  // an FMA-pipe polynomial instead of the MUFU unit (0, 2, 4); -1 = default.
   int exp_poly = -1;
-  int softmax_groups = 0;
   void* o = nullptr;
   int64_t ldo = 0;
   float* lse = nullptr;

@@ -1,8 +1,9 @@
 // Tensor-core (tcgen05) flash attention forward for the banded causal window
 // of eq. (1) (query p sees keys p-k+1 .. p), bf16 operands, fp32 softmax.
-// Two forwards: the one below keeps a running row maximum (any inputs); the
-// fixed-shift forward further down serves queries and keys of bounded norm
-// (the model's QK-norm) and needs neither the maximum nor O rescaling.
+// Two forwards: the one below keeps a running row maximum and serves any
+// inputs; the fixed-shift forward further down serves queries and keys of
+// bounded norm (the model's QK-norm) and needs neither the maximum nor the
+// rescaling of O.
 //
 // CTA = one tile of 128 queries x one head; 12 warps:
 //   warp 0       TMA producer: Q once, then K/V tiles of 128 keys (2 stages)
@@ -630,14 +631,14 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, KT, false, false);
       constexpr uint32_t id_pv = ptx::idesc_bf16_f32(128, HD, false, true);
-      bool ok = ptx::mbar_wait(q_full, 0, err);
+      bool ok = ptx::mbar_wait_warp(q_full, 0, err);
       auto issue_s = [&](int j) {
         const int s = j % NS;
-        if (!ptx::mbar_wait(&k_full[s], (j / NS) & 1, err)) return false;
-        if (j >= 2 && !ptx::mbar_wait(&s_free[j & 1], ((j - 2) / 2) & 1, err)) return false;
+        if (!ptx::mbar_wait_warp(&k_full[s], (j / NS) & 1, err)) return false;
+        if (j >= 2 && !ptx::mbar_wait_warp(&s_free[j & 1], ((j - 2) / 2) & 1, err)) return false;
         ptx::tc_fence_after();
         const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + s * G::KTILE);
         const uint32_t d = t_s + (j & 1) * 128;
@@ -646,25 +647,25 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
         for (int at = 0; at < G::A; ++at)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk, ++step)
-            ptx::umma_bf16_ts(d, t_q + (at * 64 + kk * 16) / 2, sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2),
+            ptx::umma_bf16_ts_elect(d, t_q + (at * 64 + kk * 16) / 2, sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2),
                               id_s, step > 0);
         if constexpr (G::R > 0) {
 #pragma unroll
           for (int kk = 0; kk < G::R / 16; ++kk, ++step)
-            ptx::umma_bf16_ts(d, t_q + (G::A * 64 + kk * 16) / 2,
+            ptx::umma_bf16_ts_elect(d, t_q + (G::A * 64 + kk * 16) / 2,
                               sdesc(k_addr + G::REM_OFF + kk * 32, 16, 8 * G::R * 2, rem_swizzle_layout(G::R)), id_s,
                               step > 0);
         }
-        ptx::umma_commit(&s_full[j & 1]);
-        ptx::umma_commit(&k_empty[s]);
+        ptx::umma_commit_elect(&s_full[j & 1]);
+        ptx::umma_commit_elect(&k_empty[s]);
         return true;
       };
       if (ok && ntiles > 0) ok = issue_s(0);
       if (ok && ntiles > 1) ok = issue_s(1);
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % NS;
-        if (!(ok = ptx::mbar_wait(&p_full[j & 1], (j / 2) & 1, err))) break;
-        if (!(ok = ptx::mbar_wait(&v_full[s], (j / NS) & 1, err))) break;
+        if (!(ok = ptx::mbar_wait_warp(&p_full[j & 1], (j / 2) & 1, err))) break;
+        if (!(ok = ptx::mbar_wait_warp(&v_full[s], (j / NS) & 1, err))) break;
         ptx::tc_fence_after();
         const uint32_t v_addr = ptx::smem_u32(sm + G::V_OFF + s * G::VTILE);
         const uint32_t pbuf = t_s + (j & 1) * 128;
@@ -673,13 +674,13 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
           const int gk = (kk * 16) / W;
           const uint32_t pa = pbuf + gk * W + (kk * 16 - gk * W) / 2;
           // V: MN-major, VA atoms 16384 bytes apart along head_dim (LBO), 8-key groups 1024 apart (SBO)
-          ptx::umma_bf16_ts(t_o, pa, sdesc(v_addr + kk * 2048, 16384, 1024, 2), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_bf16_ts_elect(t_o, pa, sdesc(v_addr + kk * 2048, 16384, 1024, 2), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::umma_commit(&v_empty[s]);
-        ptx::umma_commit(&s_free[j & 1]);
+        ptx::umma_commit_elect(&v_empty[s]);
+        ptx::umma_commit_elect(&s_free[j & 1]);
         if (j + 2 < ntiles && !(ok = issue_s(j + 2))) break;
       }
-      ptx::umma_commit(o_full);
+      ptx::umma_commit_elect(o_full);
       ptx::mbar_drain(o_full, 0);  // no MMA may still write TMEM when it is released
     }
   } else if (warp >= 4) {
@@ -929,15 +930,15 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, BKT, false, false);
       constexpr uint32_t id_dq = ptx::idesc_bf16_f32(128, HD, false, true);
-      bool ok = ptx::mbar_wait(q_full, 0, err);
+      bool ok = ptx::mbar_wait_warp(q_full, 0, err);
       // S_j = Q K_j^T and dP_j = dO V_j^T into TMEM buffer j&1
       auto issue_s = [&](int j) {
         const int sk = j % BNK, sv = j % BNV;
-        if (!ptx::mbar_wait(&k_full[sk], (j / BNK) & 1, err)) return false;
-        if (!ptx::mbar_wait(&v_full[sv], (j / BNV) & 1, err)) return false;
+        if (!ptx::mbar_wait_warp(&k_full[sk], (j / BNK) & 1, err)) return false;
+        if (!ptx::mbar_wait_warp(&v_full[sv], (j / BNV) & 1, err)) return false;
         ptx::tc_fence_after();
         const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
         const uint32_t v_addr = ptx::smem_u32(sm + G::V_OFF + sv * G::KTILE);
@@ -945,30 +946,30 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {  // K-steps of 16 along head_dim: atom ks / 4, offset ks % 4
           const uint32_t boff = (ks / 4) * 8192 + (ks % 4) * 32;
-          ptx::umma_bf16_ts(dS, t_q + ks * 8, sdesc(k_addr + boff, 16, 1024, 2), id_s, ks > 0);
-          ptx::umma_bf16_ts(dP, t_do + ks * 8, sdesc(v_addr + boff, 16, 1024, 2), id_s, ks > 0);
+          ptx::umma_bf16_ts_elect(dS, t_q + ks * 8, sdesc(k_addr + boff, 16, 1024, 2), id_s, ks > 0);
+          ptx::umma_bf16_ts_elect(dP, t_do + ks * 8, sdesc(v_addr + boff, 16, 1024, 2), id_s, ks > 0);
         }
-        ptx::umma_commit(&s_full[j & 1]);
-        ptx::umma_commit(&v_empty[sv]);  // V_j is not read again
+        ptx::umma_commit_elect(&s_full[j & 1]);
+        ptx::umma_commit_elect(&v_empty[sv]);  // V_j is not read again
         return true;
       };
       if (ok && ntiles > 0) ok = issue_s(0);
       for (int j = 0; ok && j < ntiles; ++j) {
         // TMEM buffer (j+1)&1 was read by the softmax of tile j-1 (waited below in the previous iteration)
         if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
-        if (!(ok = ptx::mbar_wait(&ds_full[j & 1], (j / 2) & 1, err))) break;
+        if (!(ok = ptx::mbar_wait_warp(&ds_full[j & 1], (j / 2) & 1, err))) break;
         ptx::tc_fence_after();
         const int sk = j % BNK;
         const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
         const uint32_t ds_addr = ptx::smem_u32(sm + G::DS_OFF + (j & 1) * G::DS_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKT / 16; ++kk)  // dQ += dS_j K_j; K MN-major: atoms 8192 bytes apart (LBO)
-          ptx::umma_bf16(t_dq, sdesc(ds_addr + kk * 32, 16, 1024, 2), sdesc(k_addr + kk * 2048, 8192, 1024, 2),
+          ptx::umma_bf16_elect(t_dq, sdesc(ds_addr + kk * 32, 16, 1024, 2), sdesc(k_addr + kk * 2048, 8192, 1024, 2),
                          id_dq, (j > 0 || kk > 0) ? 1u : 0u);
-        ptx::umma_commit(&k_empty[sk]);
-        ptx::umma_commit(&ds_free[j & 1]);
+        ptx::umma_commit_elect(&k_empty[sk]);
+        ptx::umma_commit_elect(&ds_free[j & 1]);
       }
-      ptx::umma_commit(dq_full);
+      ptx::umma_commit_elect(dq_full);
       ptx::mbar_drain(dq_full, 0);
     }
   } else if (warp >= 4) {
@@ -1190,17 +1191,17 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t id_o64 = ptx::idesc_bf16_f32(128, 64, false, true);
       constexpr uint32_t id_or = ptx::idesc_bf16_f32(128, G::R > 0 ? G::R : 16, false, true);
       constexpr uint32_t rl = rem_swizzle_layout(G::R);
       const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF), v_addr = ptx::smem_u32(sm + G::V_OFF);
       const uint32_t pt_addr = ptx::smem_u32(sm + G::PT_OFF), dst_addr = ptx::smem_u32(sm + G::DST_OFF);
-      bool ok = ptx::mbar_wait(kv_full, 0, err);
+      bool ok = ptx::mbar_wait_warp(kv_full, 0, err);
       for (int t = 0; ok && t < ntiles; ++t) {
         const int s = t % G::QDST;
-        if (!(ok = ptx::mbar_wait(&qd_full[s], (t / G::QDST) & 1, err))) break;
+        if (!(ok = ptx::mbar_wait_warp(&qd_full[s], (t / G::QDST) & 1, err))) break;
         ptx::tc_fence_after();
         const uint32_t q_addr = ptx::smem_u32(sm + G::QD_OFF + s * 2 * G::TILE), do_addr = q_addr + G::TILE;
         // S^T = K Q^T and dP^T = V dO^T (K over head_dim)
@@ -1209,22 +1210,22 @@ __global__ void __launch_bounds__(256, 1)
         for (int at = 0; at < G::A; ++at)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk, ++step) {
-            ptx::umma_bf16(t_s, sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2),
+            ptx::umma_bf16_elect(t_s, sdesc(k_addr + at * 16384 + kk * 32, 16, 1024, 2),
                            sdesc(q_addr + at * 16384 + kk * 32, 16, 1024, 2), id_s, step > 0);
-            ptx::umma_bf16(t_dp, sdesc(v_addr + at * 16384 + kk * 32, 16, 1024, 2),
+            ptx::umma_bf16_elect(t_dp, sdesc(v_addr + at * 16384 + kk * 32, 16, 1024, 2),
                            sdesc(do_addr + at * 16384 + kk * 32, 16, 1024, 2), id_s, step > 0);
           }
         if constexpr (G::R > 0) {
 #pragma unroll
           for (int kk = 0; kk < G::R / 16; ++kk, ++step) {
-            ptx::umma_bf16(t_s, sdesc(k_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
+            ptx::umma_bf16_elect(t_s, sdesc(k_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
                            sdesc(q_addr + G::REM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
-            ptx::umma_bf16(t_dp, sdesc(v_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
+            ptx::umma_bf16_elect(t_dp, sdesc(v_addr + G::REM + kk * 32, 16, 8 * G::RB, rl),
                            sdesc(do_addr + G::REM + kk * 32, 16, 8 * G::RB, rl), id_s, step > 0);
           }
         }
-        ptx::umma_commit(s_full);
-        if (!(ok = ptx::mbar_wait(s_read, t & 1, err))) break;
+        ptx::umma_commit_elect(s_full);
+        if (!(ok = ptx::mbar_wait_warp(s_read, t & 1, err))) break;
         ptx::tc_fence_after();
         // dV += P^T dO and dK += dS^T Q (K over the tile's 128 queries)
 #pragma unroll
@@ -1234,20 +1235,20 @@ __global__ void __launch_bounds__(256, 1)
           const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
 #pragma unroll
           for (int at = 0; at < G::A; ++at) {
-            ptx::umma_bf16(t_dv + 64 * at, pd, sdesc(do_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
-            ptx::umma_bf16(t_dk + 64 * at, dd, sdesc(q_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
+            ptx::umma_bf16_elect(t_dv + 64 * at, pd, sdesc(do_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
+            ptx::umma_bf16_elect(t_dk + 64 * at, dd, sdesc(q_addr + at * 16384 + kk * 2048, 16, 1024, 2), id_o64, acc);
           }
           if constexpr (G::R > 0) {
-            ptx::umma_bf16(t_dv + 64 * G::A, pd, sdesc(do_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
+            ptx::umma_bf16_elect(t_dv + 64 * G::A, pd, sdesc(do_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
                            acc);
-            ptx::umma_bf16(t_dk + 64 * G::A, dd, sdesc(q_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
+            ptx::umma_bf16_elect(t_dk + 64 * G::A, dd, sdesc(q_addr + G::REM + kk * 16 * G::RB, 16, 8 * G::RB, rl), id_or,
                            acc);
           }
         }
-        ptx::umma_commit(&qd_empty[s]);
-        ptx::umma_commit(pv_done);
+        ptx::umma_commit_elect(&qd_empty[s]);
+        ptx::umma_commit_elect(pv_done);
       }
-      ptx::umma_commit(o_full);
+      ptx::umma_commit_elect(o_full);
       ptx::mbar_drain(o_full, 0);
     }
   } else if (warp >= 4) {
@@ -1544,28 +1545,28 @@ int swa_tc_prepare(SwaTcPlan* p, int heads, int head_dim, const void* q, int64_t
   const int rem = head_dim % 64;
   int rc = tmap(&p->q128, q, q_rows, cols, ldq, 64);
   if (!rc) rc = tmap(&p->k128, k, ring, cols, ldkv, 64);
+  if (!rc) rc = tmap(&p->k64, k, ring, cols, ldkv, 64, 64);
   if (!rc) rc = tmap(&p->v128, v, ring, cols, ldkv, 64);
   if (rc) return rc;
   if (rem) {
     rc = tmap(&p->qr, q, q_rows, cols, ldq, rem);
     if (!rc) rc = tmap(&p->kr, k, ring, cols, ldkv, rem);
-    if (!rc) rc = tmap(&p->vr, v, ring, cols, ldkv, rem);
+    if (!rc) rc = tmap(&p->kr64, k, ring, cols, ldkv, rem, 64);
   } else {
     p->qr = p->q128;
     p->kr = p->k128;
-    p->vr = p->v128;
+    p->kr64 = p->k64;
   }
   return rc;
 }
 
 namespace {
-constexpr int kExpPolyDefault = 2;  // of every 8 groups of 8 keys (fixed-shift forward)
-constexpr int kSoftmaxGroupsDefault = 2;
+constexpr int kExpPolyDefault = 2;  // of every 8 groups of 8 keys (fixed-shift path)
 
-template <int HD, int EMU, int NWG>
+template <int HD, int EMU>
 int launch_fx(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
   using G = FxGeo<HD>;
-  auto fn = &swa_fwd_fx_kernel<HD, EMU, NWG>;
+  auto fn = &swa_fwd_fx_kernel<HD, EMU, 2>;
   {
     static std::mutex mu;
     static std::set<int> done;
@@ -1578,28 +1579,20 @@ int launch_fx(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
     }
   }
   dim3 grid(ceil_div(a.n, QT), a.heads);
-  fn<<<grid, 128 + 128 * NWG, G::SMEM, s>>>(p.k128, p.kr, p.v128, a, err);
+  fn<<<grid, 384, G::SMEM, s>>>(p.k128, p.kr, p.v128, a, err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
 
-template <int HD, int NWG>
-int launch_fx_emu(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
+template <int HD>
+int launch_emu(const SwaTcPlan& p, const SwaArgs& a, int fixed, cudaStream_t s, int* err) {
+  if (!fixed) return launch<HD>(p, a, s, err);
   switch (a.exp_poly < 0 ? kExpPolyDefault : a.exp_poly) {
-    case 0: return launch_fx<HD, 0, NWG>(p, a, s, err);
-    case 2: return launch_fx<HD, 2, NWG>(p, a, s, err);
-    case 4: return launch_fx<HD, 4, NWG>(p, a, s, err);
+    case 0: return launch_fx<HD, 0>(p, a, s, err);
+    case 2: return launch_fx<HD, 2>(p, a, s, err);
+    case 4: return launch_fx<HD, 4>(p, a, s, err);
   }
   return set_error(TTT_ERR_INVALID_ARG, "attention: polynomial share must be 0, 2 or 4 of 8");
-}
-
-template <int HD>
-int launch_fixed(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
-  switch (a.softmax_groups <= 0 ? kSoftmaxGroupsDefault : a.softmax_groups) {
-    case 2: return launch_fx_emu<HD, 2>(p, a, s, err);
-    case 4: return launch_fx_emu<HD, 4>(p, a, s, err);
-  }
-  return set_error(TTT_ERR_INVALID_ARG, "attention: softmax warpgroups must be 2 or 4");
 }
 }  // namespace
 
@@ -1610,12 +1603,12 @@ bool swa_fixed_shift_ok(const SwaArgs& a) {
 
 int swa_tc_forward(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
   if (a.ring != p.ring || a.head_dim != p.head_dim) return set_error(TTT_ERR_INVALID_ARG, "attention: plan mismatch");
-  const bool fx = swa_fixed_shift_ok(a);
+  const int fx = swa_fixed_shift_ok(a) ? 1 : 0;
   switch (a.head_dim) {
-    case 64: return fx ? launch_fixed<64>(p, a, s, err) : launch<64>(p, a, s, err);
-    case 80: return fx ? launch_fixed<80>(p, a, s, err) : launch<80>(p, a, s, err);
-    case 96: return fx ? launch_fixed<96>(p, a, s, err) : launch<96>(p, a, s, err);
-    case 128: return fx ? launch_fixed<128>(p, a, s, err) : launch<128>(p, a, s, err);
+    case 64: return launch_emu<64>(p, a, fx, s, err);
+    case 80: return launch_emu<80>(p, a, fx, s, err);
+    case 96: return launch_emu<96>(p, a, fx, s, err);
+    case 128: return launch_emu<128>(p, a, fx, s, err);
   }
   return set_error(TTT_ERR_UNSUPPORTED, "attention (tensor cores): head_dim must be 64, 80, 96 or 128");
 }

@@ -10,8 +10,9 @@ struct SwaTcPlan {
   alignas(64) CUtensorMap qr;
   alignas(64) CUtensorMap k128;
   alignas(64) CUtensorMap kr;
+  alignas(64) CUtensorMap k64;   // 64-row boxes: one CTA's half of a key tile (CTA-pair forward)
+  alignas(64) CUtensorMap kr64;
   alignas(64) CUtensorMap v128;
-  alignas(64) CUtensorMap vr;
   int head_dim = 0;
   int64_t ring = 0;
 };

@@ -194,7 +194,6 @@ extern "C" int ttt_op_swa_forward(int32_t dtype, int32_t n_heads, int32_t head_d
   a.q_norm_max = std::isfinite(q_norm_max) ? q_norm_max : 0.f;
   a.k_norm_max = std::isfinite(k_norm_max) ? k_norm_max : 0.f;
   a.exp_poly = ((flags >> 4) & 15) - 1;
-  a.softmax_groups = (flags >> 8) & 15;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == TTT_BF16 && !(flags & TTT_SWA_FORCE_SIMT) && swa_tc_supported(head_dim) && ring_slots % 128 == 0) {
     SwaTcPlan plan;

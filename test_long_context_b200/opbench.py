@@ -34,10 +34,10 @@ def band_pairs(p0, n, k):
     return s
 
 
-def op_builders(cfg, exp_poly=None, softmax_groups=None):
+def op_builders(cfg, exp_poly=None):
     """{name: builder}; a builder allocates the op's inputs and returns
-    (run, algorithmic flops, algorithmic bytes).  exp_poly, softmax_groups:
-    tuning of the fixed-shift attention forward (None = defaults)."""
+    (run, algorithmic flops, algorithmic bytes).  exp_poly: polynomial share
+    of the fixed-shift attention forward's exponentials (None = default)."""
     d, f, V, b, k, H, hd = cfg.d_model, cfg.d_ff, cfg.vocab, cfg.b, cfg.k, cfg.n_heads, cfg.head_dim
     S = max(1, 16384 // b) * b
     bf = torch.bfloat16
@@ -114,8 +114,8 @@ def op_builders(cfg, exp_poly=None, softmax_groups=None):
             nb = dict(q_norm_max=hd ** 0.5, k_norm_max=hd ** 0.5)
             pairs = band_pairs(p0, n, k)
             if not backward:
-                return ((lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse, exp_poly=exp_poly,
-                                                 softmax_groups=softmax_groups, **nb)), 4.0 * d * pairs, 0.0)
+                return ((lambda: ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse, exp_poly=exp_poly, **nb)),
+                        4.0 * d * pairs, 0.0)
             ops.swa_forward(q, kr, vr, H, hd, p0, k, o, lse, **nb)
             dout = rn(n, H * hd)
             dq, dk, dv = (torch.empty_like(q) for _ in range(3))
@@ -176,10 +176,9 @@ def main():
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--exp-poly", type=int, default=None, choices=[0, 2, 4])
-    ap.add_argument("--softmax-groups", type=int, default=None, choices=[2, 4])
     args = ap.parse_args()
     cfg = get_config(args.config)
-    builders = op_builders(cfg, args.exp_poly, args.softmax_groups)
+    builders = op_builders(cfg, args.exp_poly)
     for name in args.op or list(builders):
         run, flops, nbytes = builders[name]()
         for _ in range(args.warmup):
@@ -194,7 +193,7 @@ def main():
         ms = e0.elapsed_time(e1) / args.iters
         rec = {"op": name, "config": args.config, "ms": ms}
         if name.startswith("swa_fwd"):
-            rec.update(exp_poly=args.exp_poly, softmax_groups=args.softmax_groups)
+            rec.update(exp_poly=args.exp_poly)
         if flops:
             rec.update(tflops=flops / (ms / 1e3) / 1e12, algorithmic_flops=flops)
         if nbytes:

@@ -88,17 +88,14 @@ def sync(stream=None):
 
 
 def swa_forward(q, k_ring, v_ring, n_heads, head_dim, q_pos0, window, o, lse, force_simt=False, stream=None,
-                q_norm_max=0.0, k_norm_max=0.0, exp_poly=None, softmax_groups=None):
+                q_norm_max=0.0, k_norm_max=0.0, exp_poly=None):
     """ttt_op_swa_forward; q/o [n, H*hd], rings [R, H*hd], lse [H, n].
     q_norm_max, k_norm_max: bounds on the row norms of q and k (0 = unknown;
     both known: the fixed-shift tensor-core forward); exp_poly: its
-    polynomial share of the exponentials (0, 2 or 4 of 8), softmax_groups: its
-    softmax warpgroups (2 or 4); None = library defaults."""
+    polynomial share of the exponentials (0, 2 or 4 of 8; None = default)."""
     flags = 1 if force_simt else 0
     if exp_poly is not None:
         flags |= ((exp_poly + 1) & 15) << 4
-    if softmax_groups is not None:
-        flags |= (softmax_groups & 15) << 8
     rc = L.lib().ttt_op_swa_forward(_dtype(q), n_heads, head_dim, q.shape[0], q_pos0, window, _p(q), q.stride(0),
                                     _p(k_ring), _p(v_ring), k_ring.shape[0], _p(o), o.stride(0), _p(lse),
                                     float(q_norm_max), float(k_norm_max), flags, _stream(stream))
