@@ -614,20 +614,25 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
   const uint32_t t_s = tmem, t_o = tmem + 256, t_q = tmem + 384;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {  // the converged warp polls the rings; lane 0 issues the loads
       bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
         const int s = j % NS;
         const uint32_t ph = ((j / NS) & 1) ^ 1;
         const int slot = (int)((j_begin + (int64_t)j * KT) % a.ring);
-        if (!(ok = ptx::mbar_wait(&k_empty[s], ph, err))) break;
-        ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
-        load_tile<HD>(sm + G::K_OFF + s * G::KTILE, &tk, &tk_r, &k_full[s], col0, slot);
-        if (!(ok = ptx::mbar_wait(&v_empty[s], ph, err))) break;
-        ptx::mbar_arrive_expect_tx(&v_full[s], G::VTILE);
-        uint8_t* vd = sm + G::V_OFF + s * G::VTILE;
+        if (!(ok = ptx::mbar_wait_warp(&k_empty[s], ph, err))) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
+          load_tile<HD>(sm + G::K_OFF + s * G::KTILE, &tk, &tk_r, &k_full[s], col0, slot);
+        }
+        if (!(ok = ptx::mbar_wait_warp(&v_empty[s], ph, err))) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&v_full[s], G::VTILE);
+          uint8_t* vd = sm + G::V_OFF + s * G::VTILE;
 #pragma unroll
-        for (int at = 0; at < G::VA; ++at) ptx::tma_load_2d(vd + at * 16384, &tv, &v_full[s], col0 + 64 * at, slot);
+          for (int at = 0; at < G::VA; ++at)
+            ptx::tma_load_2d(vd + at * 16384, &tv, &v_full[s], col0 + 64 * at, slot);
+        }
       }
     }
   } else if (warp == 1) {
@@ -906,27 +911,31 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t t_dq = tmem + 256, t_q = tmem + 384, t_do = t_q + HD / 2;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {  // the converged warp polls the rings; lane 0 issues the loads
       auto load_k = [&](int j) {
         const int s = j % BNK;
-        if (!ptx::mbar_wait(&k_empty[s], ((j / BNK) & 1) ^ 1, err)) return false;
-        ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
-        const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
-        uint8_t* kd = sm + G::K_OFF + s * G::KTILE;
+        if (!ptx::mbar_wait_warp(&k_empty[s], ((j / BNK) & 1) ^ 1, err)) return false;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
+          const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
+          uint8_t* kd = sm + G::K_OFF + s * G::KTILE;
 #pragma unroll
-        for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(kd + at * 8192, &tk, &k_full[s], col0 + 64 * at, slot);
+          for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(kd + at * 8192, &tk, &k_full[s], col0 + 64 * at, slot);
+        }
         return true;
       };
       bool ok = ntiles > 0 ? load_k(0) : true;
       for (int j = 0; ok && j < ntiles; ++j) {
         if (j + 1 < ntiles && !(ok = load_k(j + 1))) break;
         const int s = j % BNV;
-        if (!(ok = ptx::mbar_wait(&v_empty[s], ((j / BNV) & 1) ^ 1, err))) break;
-        ptx::mbar_arrive_expect_tx(&v_full[s], G::KTILE);
-        const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
-        uint8_t* vd = sm + G::V_OFF + s * G::KTILE;
+        if (!(ok = ptx::mbar_wait_warp(&v_empty[s], ((j / BNV) & 1) ^ 1, err))) break;
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&v_full[s], G::KTILE);
+          const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
+          uint8_t* vd = sm + G::V_OFF + s * G::KTILE;
 #pragma unroll
-        for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(vd + at * 8192, &tv, &v_full[s], col0 + 64 * at, slot);
+          for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(vd + at * 8192, &tv, &v_full[s], col0 + 64 * at, slot);
+        }
       }
     }
   } else if (warp == 1) {

@@ -519,7 +519,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {  // the converged warp polls the ring; lane 0 issues the loads
       uint32_t kbg = 0;  // k-blocks issued by this CTA so far (ring position)
       bool ok = true;
       for (int64_t u = blockIdx.x; ok && u < units; u += gridDim.x) {
@@ -529,7 +529,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int j = 0; j < nkb; ++j, ++kbg) {
           const int s = (int)(kbg % C::STAGES);
           const uint32_t ph = (kbg / C::STAGES) & 1u;
-          if (!(ok = ptx::mbar_wait(&empty[s], ph ^ 1u, err))) break;
+          if (!(ok = ptx::mbar_wait_warp(&empty[s], ph ^ 1u, err))) break;
+          if (lane != 0) continue;
           ptx::mbar_arrive_expect_tx(&full[s], C::STAGE);
           uint8_t* a = sA + s * C::A_BYTES;
           uint8_t* b = sB + s * C::B_BYTES;
@@ -555,7 +556,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(BM, BN, A_MN, B_MN);
       uint32_t kbg = 0, it = 0;
       bool ok = true;
@@ -565,13 +566,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         decode(u, m0, n0, split, nkb, kb_begin);
         const uint32_t b = it & 1u, use = it >> 1;
         // the epilogue must have drained this accumulator buffer's previous unit
-        if (!(ok = ptx::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
+        if (!(ok = ptx::mbar_wait_warp(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem + b * BN;
         for (int kb = 0; kb < nkb; ++kb, ++kbg) {
           const int s = (int)(kbg % C::STAGES);
           const uint32_t ph = (kbg / C::STAGES) & 1u;
-          if (!(ok = ptx::mbar_wait(&full[s], ph, err))) break;
+          if (!(ok = ptx::mbar_wait_warp(&full[s], ph, err))) break;
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(sA + s * C::A_BYTES);
           const uint32_t b_addr = ptx::smem_u32(sB + s * C::B_BYTES);
@@ -581,15 +582,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                      : ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                      : ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-            ptx::umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            ptx::umma_bf16_elect(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          ptx::umma_commit(&empty[s]);
+          ptx::umma_commit_elect(&empty[s]);
         }
         if (!ok) break;
-        ptx::umma_commit(&acc_full[b]);
+        ptx::umma_commit_elect(&acc_full[b]);
       }
       // Arrives once every MMA issued above has completed (also on a bail-out).
-      ptx::umma_commit(drain);
+      ptx::umma_commit_elect(drain);
       ptx::mbar_drain(drain, 0);  // no MMA may still write TMEM when it is released
     }
   } else {
@@ -751,7 +752,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    if (lane == 0) {
+    {  // the converged warp polls the ring; lane 0 issues the loads
       uint32_t kbg = 0;
       bool ok = true;
       for (int64_t u = pair; ok && u < units; u += npairs) {
@@ -762,7 +763,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         for (int j = 0; j < nkb; ++j, ++kbg) {
           const int s = (int)(kbg % C::STAGES);
           const uint32_t ph = (kbg / C::STAGES) & 1u;
-          if (!(ok = ptx::mbar_wait(&empty[s], ph ^ 1u, err))) break;
+          if (!(ok = ptx::mbar_wait_warp(&empty[s], ph ^ 1u, err))) break;
+          if (lane != 0) continue;
           if (lead) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
           const uint32_t fb = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
           uint8_t* a = sA + s * C::A_BYTES;
@@ -789,7 +791,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
       if (lead) {
         constexpr uint32_t idesc = ptx::idesc_bf16_f32(2 * BM, BN, A_MN, B_MN);
         uint32_t kbg = 0, it = 0;
@@ -800,13 +802,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           decode(u, m0, n0, split, nkb, kb_begin);
           const uint32_t b = it & 1u, use = it >> 1;
           // both CTAs' epilogues must have drained this accumulator buffer
-          if (!(ok = ptx::mbar_wait(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
+          if (!(ok = ptx::mbar_wait_warp(&acc_empty[b], (use & 1u) ^ 1u, err))) break;
           ptx::tc_fence_after();
           const uint32_t d_tmem = tmem + b * BN;
           for (int kb = 0; kb < nkb; ++kb, ++kbg) {
             const int s = (int)(kbg % C::STAGES);
             const uint32_t ph = (kbg / C::STAGES) & 1u;
-            if (!(ok = ptx::mbar_wait(&full[s], ph, err))) break;
+            if (!(ok = ptx::mbar_wait_warp(&full[s], ph, err))) break;
             ptx::tc_fence_after();
             const uint32_t a_addr = ptx::smem_u32(sA + s * C::A_BYTES);
             const uint32_t b_addr = ptx::smem_u32(sB + s * C::B_BYTES);
@@ -816,14 +818,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
                                        : ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
               const uint64_t bd = B_MN ? ptx::smem_desc_sw128(b_addr + kk * 2048, 8192, 1024)
                                        : ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
-              ptx::umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              ptx::umma_bf16_pair_elect(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             }
-            ptx::umma_commit_pair(&empty[s], 0x3);
+            ptx::umma_commit_pair_elect(&empty[s], 0x3);
           }
           if (!ok) break;
-          ptx::umma_commit_pair(&acc_full[b], 0x3);
+          ptx::umma_commit_pair_elect(&acc_full[b], 0x3);
         }
-        ptx::umma_commit_pair(drain, 0x3);
+        ptx::umma_commit_pair_elect(drain, 0x3);
       }
       // every MMA of the pair has completed (they read this CTA's shared
       // memory and write its TMEM) before either CTA releases them
