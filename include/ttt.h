@@ -122,6 +122,11 @@ typedef struct ttt_ctx ttt_ctx;
  *   1 <= n_updated_blocks <= n_layers: the last n_updated_blocks blocks carry
  *   a fast MLP beside their static one (outputs summed).
  *   stream: a cudaStream_t (may be NULL for the legacy default stream).
+ * In TTT_BF16 mode ttt_init also reads each block's QK-norm gains (q_norm,
+ * k_norm) once, synchronously: max|gain| * sqrt(head_dim) bounds the norm of
+ * every normalised query and key row, which lets the attention forward use a
+ * fixed softmax shift (include/ttt_ops.h, ttt_op_swa_forward).  Static
+ * weights are therefore fixed for the context's life, like the copies above.
  * Errors: TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_OOM, TTT_ERR_CUDA.
  * On error *out is set to NULL.
  */
