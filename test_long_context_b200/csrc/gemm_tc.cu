@@ -752,7 +752,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    {  // the converged warp polls the ring; lane 0 issues the loads
+    {  // the converged warp polls the ring; lanes 0 .. NLOADS-1 issue the stage's boxes together
+      constexpr int NA = A_MN ? 2 : 1;
+      constexpr int NLOADS = NA + (B_MN ? C::NBOX : 1);
+      const uint32_t fb0 = ptx::mapa_shared(ptx::smem_u32(&full[0]), 0);
       uint32_t kbg = 0;
       bool ok = true;
       for (int64_t u = pair; ok && u < units; u += npairs) {
@@ -764,29 +767,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
           const int s = (int)(kbg % C::STAGES);
           const uint32_t ph = (kbg / C::STAGES) & 1u;
           if (!(ok = ptx::mbar_wait_warp(&empty[s], ph ^ 1u, err))) break;
-          if (lane != 0) continue;
-          if (lead) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
-          const uint32_t fb = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
-          uint8_t* a = sA + s * C::A_BYTES;
-          uint8_t* b = sB + s * C::B_BYTES;
+          // one lane per box, all boxes of the stage in one TMA instruction of the warp: a
+          // TMA instruction costs its issuing thread about 125 cycles (measured), so issuing
+          // the boxes one after another from lane 0 made the producer, not the MMAs, set the
+          // pace of the narrow-tile products
+          if (lane >= NLOADS) continue;
+          if (lane == 0 && lead) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::STAGE);
+          const uint32_t fb = fb0 + 8u * (uint32_t)s;  // &full[s] in the even CTA
           const int kb = kb_begin + j;
           const bool second = kb >= KB1;
-          const CUtensorMap* ta = second ? &tma2 : &tma;
-          const CUtensorMap* tb = second ? &tmb2 : &tmb;
           const int k0 = (second ? kb - KB1 : kb) * BK;
           const int nb = (int)(second ? n0 - n_ext : n0) + (BN / 2) * (int)rank;  // this CTA's half of B
-          if constexpr (!A_MN) {
-            ptx::tma_load_2d_pair(a, ta, fb, k0, mo);
-          } else {
-            ptx::tma_load_2d_pair(a, ta, fb, mo, k0);
-            ptx::tma_load_2d_pair(a + 8192, ta, fb, mo + 64, k0);
+          uint8_t* dst;
+          const CUtensorMap* tm;
+          int c0, c1;
+          if (lane < NA) {  // A: this CTA's 128 rows (K-major: one box; MN-major: two 64-row boxes)
+            dst = sA + s * C::A_BYTES + 8192 * lane;
+            tm = second ? &tma2 : &tma;
+            c0 = A_MN ? mo + 64 * lane : k0;
+            c1 = A_MN ? k0 : mo;
+          } else {  // B: this CTA's half (K-major: one box; MN-major: NBOX 64-column boxes)
+            const int i = lane - NA;
+            dst = sB + s * C::B_BYTES + 8192 * i;
+            tm = second ? &tmb2 : &tmb;
+            c0 = B_MN ? nb + 64 * i : k0;
+            c1 = B_MN ? k0 : nb;
           }
-          if constexpr (!B_MN) {
-            ptx::tma_load_2d_pair(b, tb, fb, k0, nb);
-          } else {
-#pragma unroll
-            for (int i = 0; i < C::NBOX; ++i) ptx::tma_load_2d_pair(b + 8192 * i, tb, fb, nb + 64 * i, k0);
-          }
+          ptx::tma_load_2d_pair(dst, tm, fb, c0, c1);
         }
       }
     }
