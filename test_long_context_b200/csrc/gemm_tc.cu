@@ -453,6 +453,27 @@ __device__ __forceinline__ void epilogue_sgd_vec(uint32_t t_row, const EpiArgs& 
 // Second product: output tiles with n0 >= n_ext accumulate A2 B2^T after
 // A B^T (k-blocks KB1 .. KB1+KB2-1 of the concatenated reduction; B2's row is
 // n0 - n_ext).  The k-splits cut the concatenated range.
+// Output tile (m-tile, n-tile) of linear index mn.  raster 0: m-tile fastest;
+// 1: n-tile fastest; raster >= 2: groups of `raster` m-tiles walked m-tile
+// fastest, one n-tile after the other, so that while the resident units
+// cover a group, its rows of A and the current columns of B both stay in L2
+// (for products whose A and B are each larger than a third of L2).
+__device__ __forceinline__ void tile_of(int64_t mn, int n_mt, int n_nt, int raster, int64_t& mt, int64_t& nt) {
+  if (raster == 0) {
+    mt = mn % n_mt;
+    nt = mn / n_mt;
+  } else if (raster == 1) {
+    mt = mn / n_nt;
+    nt = mn % n_nt;
+  } else {
+    const int64_t per_group = (int64_t)raster * n_nt;
+    const int64_t m_first = (mn / per_group) * raster, r = mn % per_group;
+    const int64_t gm = imin64(raster, n_mt - m_first);  // the last group may hold fewer m-tiles
+    mt = m_first + r % gm;
+    nt = r / gm;
+  }
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI, typename TACT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tma, const __grid_constant__ CUtensorMap tmb,
@@ -481,8 +502,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // L2 while A streams through once).
   auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int& kb_begin) {
     const int64_t mn = u % ((int64_t)n_mt * n_nt);
-    m0 = (n_fast ? mn / n_nt : mn % n_mt) * BM;
-    n0 = (n_fast ? mn % n_nt : mn / n_mt) * BN;
+    int64_t mt, nt;
+    tile_of(mn, n_mt, n_nt, n_fast, mt, nt);
+    m0 = mt * BM;
+    n0 = nt * BN;
     split = (int)(u / ((int64_t)n_mt * n_nt));
     const int total = KB1 + (n0 >= n_ext ? KB2 : 0);
     kb_begin = split * kpsb;
@@ -713,8 +736,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   // n_mt counts 256-row pair tiles; m0 is the pair tile's first row
   auto decode = [&](int64_t u, int64_t& m0, int64_t& n0, int& split, int& nkb, int& kb_begin) {
     const int64_t mn = u % ((int64_t)n_mt * n_nt);
-    m0 = (n_fast ? mn / n_nt : mn % n_mt) * (2 * BM);
-    n0 = (n_fast ? mn % n_nt : mn / n_mt) * BN;
+    int64_t mt, nt;
+    tile_of(mn, n_mt, n_nt, n_fast, mt, nt);
+    m0 = mt * (2 * BM);
+    n0 = nt * BN;
     split = (int)(u / ((int64_t)n_mt * n_nt));
     const int total = KB1 + (n0 >= n_ext ? KB2 : 0);
     kb_begin = split * kpsb;
@@ -1309,9 +1334,14 @@ int tc_gemm_launch(const TcGemm& g, cudaStream_t stream, int* dev_err) {
   const dim3 grid(g.pair ? (unsigned)(2 * std::min<int64_t>(units, slots))
                          : (unsigned)std::min<int64_t>(units, slots));
   const int KB1 = (int)((g.K + BK - 1) / BK), KB2 = (int)((g.K2 + BK - 1) / BK);
-  // n-tile fastest when B (N x K, plus a second product) fits comfortably in L2 and A is the larger operand
+  // n-tile fastest when B (N x K, plus a second product) fits comfortably in L2 and A is the larger
+  // operand; when A and B are both larger than that, groups of m-tiles whose rows of A take about 24 MB
   const double a_bytes = 2.0 * (double)g.M * (double)(g.K + g.K2), b_bytes = 2.0 * (double)g.N * (double)(g.K + g.K2);
-  const int n_fast = (b_bytes <= 48e6 && a_bytes > b_bytes) ? 1 : 0;
+  int n_fast = (b_bytes <= 48e6 && a_bytes > b_bytes) ? 1 : 0;
+  if (a_bytes > 48e6 && b_bytes > 48e6 && n_mt > 2) {
+    const double tile_a = a_bytes / (double)n_mt;  // bytes of A per m-tile
+    n_fast = (int)std::max(2.0, std::min(16.0, std::floor(24e6 / tile_a)));
+  }
   const int64_t n_ext = g.K2 > 0 ? g.n_ext : INT64_MAX;
   if (g.ksplit <= 1) {
     fn<<<grid, kGemmThreads, smem, stream>>>(g.ta, g.tb, g.ta2, g.tb2, g.M, g.N, KB1, KB2, n_ext, KB1 + KB2, n_mt, n_nt, 1, n_fast,

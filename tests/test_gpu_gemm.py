@@ -416,3 +416,30 @@ def test_gemm_plan_of_the_prefill_products():
     assert (S, bn) == (1, 256)
     S, bn = ops.gemm_plan(1024, 2560, 2560, ops.L.EPI_SWIGLU)
     assert (S, bn) == (1, 0)
+
+
+def test_grouped_raster_large_operands():
+    """A and B both larger than a third of L2 (here 52 MB each): the tiles
+    are walked in groups of m-tiles (m fastest inside a group, one n-tile
+    after the other).  Every output row block and column block is checked
+    against the fp64 product, with the plain store and with SwiGLU."""
+    from test_long_context_b200 import ops
+    M, N, K = 12800, 12800, 2048
+    g = torch.Generator(device="cuda").manual_seed(41)
+    A = torch.randn(M, K, device="cuda", generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, device="cuda", generator=g).to(torch.bfloat16)
+    c = torch.full((M, N), float("nan"), device="cuda")
+    ops.gemm(A, B, 0, 0, ops.L.EPI_STORE_F32, c=c)
+    a = torch.full((M, N // 2), float("nan"), device="cuda", dtype=torch.bfloat16)
+    ops.gemm(A, B, 0, 0, ops.L.EPI_SWIGLU, c=a)
+    ops.sync()
+    Bd = B.double()
+    for r0 in range(0, M, 1600):  # one 128-row block per group-sized stride, every column
+        rows = slice(r0, r0 + 128)
+        ref = A[rows].double() @ Bd.T
+        scale = ref.abs().max().item()
+        assert (c[rows].double() - ref).abs().max().item() <= 1e-4 * scale + 1e-4, r0
+        r = ref.view(128, N // 128, 2, 64)
+        want = (torch.nn.functional.silu(r[:, :, 0]) * r[:, :, 1]).reshape(128, N // 2)
+        assert (a[rows].double() - want).abs().max().item() <= 2e-2 * want.abs().max().item(), r0
+    assert not torch.isnan(c).any() and not torch.isnan(a.float()).any()
