@@ -798,51 +798,6 @@ __global__ void __launch_bounds__(128 + 128 * NWG, 1)
   }
 }
 
-// ---------------------------------------------------------------------------------------------
-// Backward, dq part: dQ = scale * sum_j dS_j K_j over the band, with
-// dS = P o (dP - D), P = exp(S*scale - lse), S = Q K^T, dP = dO V^T.
-// CTA = 128 queries x one head; key tiles of 64 keys.
-//   warp 0      TMA: K tiles (ring of BNK, released after dQ_j) one tile ahead
-//               of V tiles (ring of BNV, released after dP_j)
-//   warp 1      TMEM owner; lane 0 issues S_j = Q K_j^T and dP_j = dO V_j^T into
-//               one of two TMEM buffers (64 + 64 columns), then dQ += dS_j K_j
-//               as one MMA of N = head_dim per 16 keys.  Q and dO, the A
-//               operands of every S_j and dP_j, sit in TMEM (written once by
-//               the softmax warps), so the tensor core reads only K and V
-//               from shared memory for them.
-//   warps 4..11 two warpgroups taking alternate key tiles (warpgroup j & 1
-//               owns tile j, TMEM buffer j & 1 and dS buffer j & 1): thread =
-//               query row; P, dS in fp32 -> bf16 dS in a 128B-swizzled smem
-//               tile (K-major A operand of the dQ product).  The two
-//               warpgroups run one tile apart, so one computes while the other
-//               waits for its scores.
-// K and V tiles are staged as whole 128B-swizzled atoms (the last one partly
-// past the head), so that a K tile is both the K-major B operand of S and the
-// MN-major B operand of dQ.  The softmax statistics come from the forward (lse), so there
-// is no online rescaling and the tiles of a row are independent.
-constexpr int BKT = 64;  // keys per tile in the backward
-constexpr int BNK = 4;   // K stages
-constexpr int BNV = 3;   // V stages
-
-template <int HD>
-struct BGeo {
-  static constexpr int A = HD / 64;
-  static constexpr int R = HD % 64;
-  static constexpr int RB = R * 2;
-  static constexpr int KA = (HD + 63) / 64;     // whole atoms of a K or V tile
-  static constexpr int KTILE = BKT * 128 * KA;  // K or V tile (64 rows, KA atoms)
-  static constexpr int QTILE = 128 * HD * 2;    // 128-row tile (the dk/dv kernel's layout)
-  static constexpr int QREM = A * 16384;        // remainder offset inside a 128-row tile
-  static constexpr int K_OFF = 0;
-  static constexpr int V_OFF = K_OFF + BNK * KTILE;
-  static constexpr int DS_OFF = V_OFF + BNV * KTILE;
-  static constexpr int DS_BYTES = 128 * BKT * 2;  // one 128B-swizzled atom column (64 keys)
-  static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;
-  static_assert(KTILE % 1024 == 0, "1024-byte aligned tiles");
-  static_assert(SMEM <= 232448, "shared memory per block");
-};
-
 template <int HD>
 __device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m64, const CUtensorMap* mrem,
                                           uint64_t* bar, int col0, int row0, int atom_bytes, int rem_off) {
@@ -852,22 +807,63 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* m64, 
   if constexpr (R > 0) ptx::tma_load_2d(dst + rem_off, mrem, bar, col0 + 64 * A, row0);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Backward, dq part: dQ = scale * sum_j dS_j K_j over the band, with
+// dS = P o (dP - D), P = exp(S*scale - lse), S = Q K^T, dP = dO V^T; the
+// softmax statistics come from the forward (lse), so the tiles of a row are
+// independent.  Tiles of 128 keys: 18 MMAs per 128 keys (S and dP of
+// N = 128, then dQ += dS K as 8 MMAs of N = head_dim) where 64-key tiles
+// need 28, and a single-CTA MMA costs about 100 cycles whatever its N.
+// CTA = 128 queries x one head; 12 warps:
+//   warp 0      TMA: K tiles (ring of NK, released after dQ_j) and V tiles
+//               (ring of NV, released after dP_j), 128 keys as whole
+//               128B-swizzled atoms; one lane per atom
+//   warp 1      TMEM owner; the converged warp issues S_j = Q K_j^T and
+//               dP_j = dO V_j^T (A operands Q and dO from TMEM) into one TMEM
+//               buffer, then dQ += dS_j K_j once both warpgroups wrote dS_j
+//   warps 4..11 two warpgroups owning key columns 64g .. 64g+63 of every tile:
+//               thread = query row; P = 2^(S scale log2e - lse log2e),
+//               dS = P o (dP - D) -> bf16 into the 128B-swizzled dS tile (one
+//               64-key atom per warpgroup, double-buffered)
+// TMEM: S at columns 0..127, dP at 128..255, dQ at 256, Q and dO (bf16 pairs)
+// from 384.  S and dP of tile j+1 are issued as soon as both warpgroups have
+// read tile j's, so they run under tile j's dS arithmetic.
+constexpr int DKT = 128;
+
+template <int HD>
+struct DGeo {
+  static constexpr int KA = (HD + 63) / 64;         // whole atoms of a K or V tile
+  static constexpr int KTILE = DKT * 128 * KA;      // 128 keys x KA atoms of 128 B per row
+  static constexpr int NK = KA == 1 ? 4 : 3;        // K stages (released after dQ_j)
+  static constexpr int NV = KA == 1 ? 3 : 2;        // V stages (released after dP_j)
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + NK * KTILE;
+  static constexpr int DS_OFF = V_OFF + NV * KTILE;
+  static constexpr int DS_BYTES = 128 * DKT * 2;    // two 64-key atoms
+  static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;
+  static_assert(KTILE % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(SMEM <= 232448, "shared memory per block");
+};
+
 template <int HD>
 __global__ void __launch_bounds__(384, 1)
-    swa_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, SwaArgs a,
+    swa_bwd_dq128_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv, SwaArgs a,
                          int* err) {
-  using G = BGeo<HD>;
+  using G = DGeo<HD>;
+  constexpr int NK = G::NK, NV = G::NV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + G::BAR_OFF);
   uint64_t* q_full = bars + 0;        // Q and dO written to TMEM
-  uint64_t* k_full = bars + 1;        // [BNK]
-  uint64_t* k_empty = k_full + BNK;   // [BNK]
-  uint64_t* v_full = k_empty + BNK;   // [BNV]
-  uint64_t* v_empty = v_full + BNV;   // [BNV]
-  uint64_t* s_full = v_empty + BNV;   // [2]  S_j, dP_j in TMEM buffer j&1
-  uint64_t* ds_full = s_full + 2;     // [2]  dS_j written (and TMEM buffer j&1 read)
-  uint64_t* ds_free = ds_full + 2;    // [2]  dQ_j consumed dS buffer j&1
+  uint64_t* k_full = bars + 1;        // [NK]
+  uint64_t* k_empty = k_full + NK;    // [NK]
+  uint64_t* v_full = k_empty + NK;    // [NV]
+  uint64_t* v_empty = v_full + NV;    // [NV]
+  uint64_t* s_full = v_empty + NV;    // S_j and dP_j in TMEM
+  uint64_t* s_empty = s_full + 1;     // both warpgroups read S_j and dP_j
+  uint64_t* ds_full = s_empty + 1;    // [2] dS_j written
+  uint64_t* ds_free = ds_full + 2;    // [2] dQ_j consumed dS buffer j&1
   uint64_t* dq_full = ds_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(dq_full + 1);
 
@@ -876,23 +872,24 @@ __global__ void __launch_bounds__(384, 1)
   const int64_t q0 = a.p0 + (int64_t)blockIdx.x * QT;
   const int64_t qlast = imin64(q0 + QT, a.p0 + a.n) - 1;
   const int64_t kfirst = imax64(0, q0 - a.window + 1);
-  const int64_t j_begin = (kfirst / BKT) * BKT;
-  const int ntiles = (int)((qlast - j_begin) / BKT + 1);
+  const int64_t j_begin = (kfirst / DKT) * DKT;
+  const int ntiles = (int)((qlast - j_begin) / DKT + 1);
   const int col0 = h * HD;
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(q_full, 256);
-    for (int s = 0; s < BNK; ++s) {
+    for (int s = 0; s < NK; ++s) {
       ptx::mbar_init(&k_full[s], 1);
       ptx::mbar_init(&k_empty[s], 1);
     }
-    for (int s = 0; s < BNV; ++s) {
+    for (int s = 0; s < NV; ++s) {
       ptx::mbar_init(&v_full[s], 1);
       ptx::mbar_init(&v_empty[s], 1);
     }
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(s_empty, 256);
     for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&s_full[s], 1);
-      ptx::mbar_init(&ds_full[s], 128);
+      ptx::mbar_init(&ds_full[s], 256);
       ptx::mbar_init(&ds_free[s], 1);
     }
     ptx::mbar_init(dq_full, 1);
@@ -907,74 +904,62 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // TMEM: S/dP buffers at columns [0,128) and [128,256), dQ at 256, Q and dO (bf16 pairs) from 384
-  const uint32_t t_dq = tmem + 256, t_q = tmem + 384, t_do = t_q + HD / 2;
+  const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256, t_q = tmem + 384, t_do = t_q + HD / 2;
 
   if (warp == 0) {
-    {  // the converged warp polls the rings; lane 0 issues the loads
-      auto load_k = [&](int j) {
-        const int s = j % BNK;
-        if (!ptx::mbar_wait_warp(&k_empty[s], ((j / BNK) & 1) ^ 1, err)) return false;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&k_full[s], G::KTILE);
-          const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
-          uint8_t* kd = sm + G::K_OFF + s * G::KTILE;
-#pragma unroll
-          for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(kd + at * 8192, &tk, &k_full[s], col0 + 64 * at, slot);
-        }
-        return true;
-      };
-      bool ok = ntiles > 0 ? load_k(0) : true;
+    {  // the converged warp polls the rings; one lane per atom issues the loads
+      bool ok = true;
       for (int j = 0; ok && j < ntiles; ++j) {
-        if (j + 1 < ntiles && !(ok = load_k(j + 1))) break;
-        const int s = j % BNV;
-        if (!(ok = ptx::mbar_wait_warp(&v_empty[s], ((j / BNV) & 1) ^ 1, err))) break;
-        if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(&v_full[s], G::KTILE);
-          const int slot = (int)((j_begin + (int64_t)j * BKT) % a.ring);
-          uint8_t* vd = sm + G::V_OFF + s * G::KTILE;
-#pragma unroll
-          for (int at = 0; at < G::KA; ++at) ptx::tma_load_2d(vd + at * 8192, &tv, &v_full[s], col0 + 64 * at, slot);
-        }
+        const int slot = (int)((j_begin + (int64_t)j * DKT) % a.ring);
+        const int sk = j % NK, sv = j % NV;
+        if (!(ok = ptx::mbar_wait_warp(&k_empty[sk], ((j / NK) & 1) ^ 1, err))) break;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&k_full[sk], G::KTILE);
+        __syncwarp();
+        if (lane < G::KA)
+          ptx::tma_load_2d(sm + G::K_OFF + sk * G::KTILE + lane * 16384, &tk, &k_full[sk], col0 + 64 * lane, slot);
+        if (!(ok = ptx::mbar_wait_warp(&v_empty[sv], ((j / NV) & 1) ^ 1, err))) break;
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&v_full[sv], G::KTILE);
+        __syncwarp();
+        if (lane < G::KA)
+          ptx::tma_load_2d(sm + G::V_OFF + sv * G::KTILE + lane * 16384, &tv, &v_full[sv], col0 + 64 * lane, slot);
       }
     }
   } else if (warp == 1) {
     {  // the converged warp runs the issue loop; one elected lane issues each MMA and commit
-      constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, BKT, false, false);
+      constexpr uint32_t id_s = ptx::idesc_bf16_f32(128, DKT, false, false);
       constexpr uint32_t id_dq = ptx::idesc_bf16_f32(128, HD, false, true);
       bool ok = ptx::mbar_wait_warp(q_full, 0, err);
-      // S_j = Q K_j^T and dP_j = dO V_j^T into TMEM buffer j&1
+      // S_j = Q K_j^T and dP_j = dO V_j^T into the TMEM buffer, once both warpgroups read tile j-1's
       auto issue_s = [&](int j) {
-        const int sk = j % BNK, sv = j % BNV;
-        if (!ptx::mbar_wait_warp(&k_full[sk], (j / BNK) & 1, err)) return false;
-        if (!ptx::mbar_wait_warp(&v_full[sv], (j / BNV) & 1, err)) return false;
+        const int sk = j % NK, sv = j % NV;
+        if (!ptx::mbar_wait_warp(&k_full[sk], (j / NK) & 1, err)) return false;
+        if (!ptx::mbar_wait_warp(&v_full[sv], (j / NV) & 1, err)) return false;
+        if (j >= 1 && !ptx::mbar_wait_warp(s_empty, (j - 1) & 1, err)) return false;
         ptx::tc_fence_after();
         const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
         const uint32_t v_addr = ptx::smem_u32(sm + G::V_OFF + sv * G::KTILE);
-        const uint32_t dS = tmem + (j & 1) * 128, dP = dS + 64;
 #pragma unroll
         for (int ks = 0; ks < HD / 16; ++ks) {  // K-steps of 16 along head_dim: atom ks / 4, offset ks % 4
-          const uint32_t boff = (ks / 4) * 8192 + (ks % 4) * 32;
-          ptx::umma_bf16_ts_elect(dS, t_q + ks * 8, sdesc(k_addr + boff, 16, 1024, 2), id_s, ks > 0);
-          ptx::umma_bf16_ts_elect(dP, t_do + ks * 8, sdesc(v_addr + boff, 16, 1024, 2), id_s, ks > 0);
+          const uint32_t boff = (ks / 4) * 16384 + (ks % 4) * 32;
+          ptx::umma_bf16_ts_elect(t_s, t_q + ks * 8, sdesc(k_addr + boff, 16, 1024, 2), id_s, ks > 0);
+          ptx::umma_bf16_ts_elect(t_dp, t_do + ks * 8, sdesc(v_addr + boff, 16, 1024, 2), id_s, ks > 0);
         }
-        ptx::umma_commit_elect(&s_full[j & 1]);
+        ptx::umma_commit_elect(s_full);
         ptx::umma_commit_elect(&v_empty[sv]);  // V_j is not read again
         return true;
       };
       if (ok && ntiles > 0) ok = issue_s(0);
       for (int j = 0; ok && j < ntiles; ++j) {
-        // TMEM buffer (j+1)&1 was read by the softmax of tile j-1 (waited below in the previous iteration)
         if (j + 1 < ntiles && !(ok = issue_s(j + 1))) break;
         if (!(ok = ptx::mbar_wait_warp(&ds_full[j & 1], (j / 2) & 1, err))) break;
         ptx::tc_fence_after();
-        const int sk = j % BNK;
+        const int sk = j % NK;
         const uint32_t k_addr = ptx::smem_u32(sm + G::K_OFF + sk * G::KTILE);
         const uint32_t ds_addr = ptx::smem_u32(sm + G::DS_OFF + (j & 1) * G::DS_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKT / 16; ++kk)  // dQ += dS_j K_j; K MN-major: atoms 8192 bytes apart (LBO)
-          ptx::umma_bf16_elect(t_dq, sdesc(ds_addr + kk * 32, 16, 1024, 2), sdesc(k_addr + kk * 2048, 8192, 1024, 2),
-                         id_dq, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < DKT / 16; ++kk)  // dQ += dS_j K_j; K MN-major: atoms 16384 bytes apart (LBO)
+          ptx::umma_bf16_elect(t_dq, sdesc(ds_addr + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024, 2),
+                               sdesc(k_addr + kk * 2048, 16384, 1024, 2), id_dq, (j > 0 || kk > 0) ? 1u : 0u);
         ptx::umma_commit_elect(&k_empty[sk]);
         ptx::umma_commit_elect(&ds_free[j & 1]);
       }
@@ -982,7 +967,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_drain(dq_full, 0);
     }
   } else if (warp >= 4) {
-    const int g = (warp - 4) >> 2;  // this warpgroup takes tiles g, g + 2, ...
+    const int g = (warp - 4) >> 2;  // this warpgroup owns key columns 64g .. 64g+63
     const int q = warp & 3;         // TMEM lane quarter
     const int r = q * 32 + lane;
     const int64_t p = q0 + r;
@@ -999,14 +984,12 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t dst = (g == 0 ? t_q : t_do) + lane_off;
 #pragma unroll
       for (int c = 0; c < HD / 2; c += 8) {  // 8 columns = 16 bf16 = two 16-byte loads
-        uint32_t w[8];
         uint4 u0 = make_uint4(0u, 0u, 0u, 0u), u1 = u0;
         if (row_ok) {
           u0 = *reinterpret_cast<const uint4*>(src + 2 * c);
           u1 = *reinterpret_cast<const uint4*>(src + 2 * c + 8);
         }
-        w[0] = u0.x; w[1] = u0.y; w[2] = u0.z; w[3] = u0.w;
-        w[4] = u1.x; w[5] = u1.y; w[6] = u1.z; w[7] = u1.w;
+        const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
         ptx::tmem_st8(dst + c, w);
       }
       tmem_st_wait();
@@ -1014,36 +997,37 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_arrive(q_full);
     }
     bool ok = true;
-    for (int j = g; j < ntiles; j += 2) {
-      const int64_t j0 = j_begin + (int64_t)j * BKT;
-      ok = ptx::mbar_wait(&s_full[g], (j / 2) & 1, err);
-      if (!__all_sync(0xffffffffu, ok)) break;
+    for (int j = 0; j < ntiles; ++j) {
+      const int64_t j0 = j_begin + (int64_t)j * DKT + 64 * g;  // position of this warpgroup's first key
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(s_full, j & 1, err));
+      if (!ok) break;
       ptx::tc_fence_after();
-      float sv[BKT], dp[BKT];
+      float sv[64], dp[64];
       {
         uint32_t rs[64], rd[64];
-        ptx::tmem_ld64(tmem + g * 128 + lane_off, rs);
-        ptx::tmem_ld64(tmem + g * 128 + 64 + lane_off, rd);
+        ptx::tmem_ld64(t_s + 64 * g + lane_off, rs);
+        ptx::tmem_ld64(t_dp + 64 * g + lane_off, rd);
         ptx::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < BKT; ++e) {
+        for (int e = 0; e < 64; ++e) {
           sv[e] = __uint_as_float(rs[e]);
           dp[e] = __uint_as_float(rd[e]);
         }
       }
       ptx::tc_fence_before();
-      if (j >= 2) {  // dS buffer g is free once dQ_{j-2} consumed it
-        ok = ptx::mbar_wait(&ds_free[g], ((j - 2) / 2) & 1, err);
-        if (!__all_sync(0xffffffffu, ok)) break;
+      ptx::mbar_arrive(s_empty);
+      if (j >= 2) {  // dS buffer j&1 is free once dQ_{j-2} consumed it
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&ds_free[j & 1], ((j - 2) / 2) & 1, err));
+        if (!ok) break;
       }
       const int64_t lo = p - a.window + 1 - j0, hi = p - j0;
-      if (!(row_ok && lo <= 0 && hi >= BKT - 1)) {  // edge tile: masked scores give P = 0
+      if (!(row_ok && lo <= 0 && hi >= 63)) {  // edge tile: masked scores give P = 0
 #pragma unroll
-        for (int c = 0; c < BKT; ++c) sv[c] = (row_ok && c >= lo && c <= hi) ? sv[c] : -INFINITY;
+        for (int c = 0; c < 64; ++c) sv[c] = (row_ok && c >= lo && c <= hi) ? sv[c] : -INFINITY;
       }
-      uint8_t* drow = sm + G::DS_OFF + g * G::DS_BYTES + r * 128;
+      uint8_t* drow = sm + G::DS_OFF + (j & 1) * G::DS_BYTES + g * 16384 + r * 128;
 #pragma unroll
-      for (int gg = 0; gg < BKT / 8; ++gg) {  // granules of 8 keys
+      for (int gg = 0; gg < 8; ++gg) {  // granules of 8 keys
         float ds[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -1051,18 +1035,15 @@ __global__ void __launch_bounds__(384, 1)
           const float pr = ex2(fmaf(sv[c], sl2, -lse2));
           ds[e] = pr * (dp[c] - Di);
         }
-        uint4 w;
         __nv_bfloat162 b0 = __floats2bfloat162_rn(ds[0], ds[1]), b1 = __floats2bfloat162_rn(ds[2], ds[3]);
         __nv_bfloat162 b2 = __floats2bfloat162_rn(ds[4], ds[5]), b3 = __floats2bfloat162_rn(ds[6], ds[7]);
-        w.x = *reinterpret_cast<uint32_t*>(&b0);
-        w.y = *reinterpret_cast<uint32_t*>(&b1);
-        w.z = *reinterpret_cast<uint32_t*>(&b2);
-        w.w = *reinterpret_cast<uint32_t*>(&b3);
-        *reinterpret_cast<uint4*>(drow + ((gg ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4*>(drow + ((gg ^ (r & 7)) << 4)) =
+            make_uint4(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1),
+                       *reinterpret_cast<uint32_t*>(&b2), *reinterpret_cast<uint32_t*>(&b3));
       }
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&ds_full[g]);
+      ptx::mbar_arrive(&ds_full[j & 1]);
     }
     if (ok) ok = ptx::mbar_wait(dq_full, 0, err);
     if (__all_sync(0xffffffffu, ok)) {
@@ -1075,20 +1056,15 @@ __global__ void __launch_bounds__(384, 1)
         tmem_ld16(t_dq + c + lane_off, o);
         ptx::tmem_ld_wait();
         if (row_ok) {
-          uint4 w0, w1;
-          uint32_t* pw = &w0.x;
-          uint32_t* pw1 = &w1.x;
+          uint32_t pk[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 t0 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * a.scale,
+          for (int e = 0; e < 8; ++e) {
+            __nv_bfloat162 t2 = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * a.scale,
                                                       __uint_as_float(o[2 * e + 1]) * a.scale);
-            __nv_bfloat162 t1 = __floats2bfloat162_rn(__uint_as_float(o[8 + 2 * e]) * a.scale,
-                                                      __uint_as_float(o[9 + 2 * e]) * a.scale);
-            pw[e] = *reinterpret_cast<uint32_t*>(&t0);
-            pw1[e] = *reinterpret_cast<uint32_t*>(&t1);
+            pk[e] = *reinterpret_cast<uint32_t*>(&t2);
           }
-          *reinterpret_cast<uint4*>(out + c) = w0;
-          *reinterpret_cast<uint4*>(out + c + 8) = w1;
+          *reinterpret_cast<uint4*>(out + c) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          *reinterpret_cast<uint4*>(out + c + 8) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
     }
@@ -1437,8 +1413,8 @@ int launch(const SwaTcPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
 
 template <int HD>
 int launch_bwd_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* err) {
-  using G = BGeo<HD>;
-  auto fn = &swa_bwd_dq_tc_kernel<HD>;
+  using G = DGeo<HD>;
+  auto fn = &swa_bwd_dq128_kernel<HD>;
   {
     static std::mutex mu;
     static std::set<int> done;
@@ -1451,7 +1427,7 @@ int launch_bwd_dq(const SwaTcBwdPlan& p, const SwaArgs& a, cudaStream_t s, int* 
     }
   }
   dim3 grid(ceil_div(a.n, QT), a.heads);
-  fn<<<grid, 384, G::SMEM, s>>>(p.k64, p.v64, a, err);
+  fn<<<grid, 384, G::SMEM, s>>>(p.k128, p.v128, a, err);
   TTT_CUDA_TRY(cudaGetLastError());
   return TTT_OK;
 }
