@@ -65,6 +65,7 @@ def parse_args():
     ap.add_argument("--decode-tokens", type=int, default=DECODE_TOKENS, help="0 skips the decode measurement")
     ap.add_argument("--no-full-attention", action="store_true")
     ap.add_argument("--no-multi-sequence", action="store_true")
+    ap.add_argument("--no-meta-grad", action="store_true")
     return ap.parse_args()
 
 
@@ -411,6 +412,47 @@ def time_multi_sequence(cfg, gw, n_seq, T_seq, ttt_tokens_per_s):
             "vs_one_sequence_of_the_same_tokens": tps / ttt_tokens_per_s, "finite_losses": ok}
 
 
+def time_meta_grad(cfg, n_chunks=2, steps=2, warmup=1):
+    """The outer loop's meta-gradient (eq. (7) of the reading notes, §4) for a
+    fast MLP in the last block at the model's shapes: n_chunks chunks of b
+    rows through ttt_op_meta_grad (fp32), inputs seeded and resident, timed
+    with CUDA events; achieved = its GEMM flops / time against the fp32 FMA
+    peak of the SIMT kernels."""
+    import torch
+
+    from test_long_context_b200 import ops
+    from test_long_context_b200.opbench import meta_grad_flops, meta_grad_inputs
+    b, d, f, V = cfg.b, cfg.d_model, cfg.d_ff, cfg.vocab
+    h, r, tgt, W, gf, head = meta_grad_inputs(n_chunks, b, d, f, V)
+    outs = [torch.empty_like(w) for w in W]
+    losses = torch.empty(n_chunks * b, device="cuda")
+    work = torch.empty(ops.meta_grad_work(n_chunks, b, d, f, V), device="cuda")
+    run = lambda: ops.meta_grad(h, r, tgt, *W, gf, head, cfg.norm_eps, cfg.eta, b, *outs, losses=losses, work=work)
+    for _ in range(warmup):
+        run()
+    ops.sync()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        run()
+    e1.record(stream)
+    ops.sync()
+    ms = e0.elapsed_time(e1) / steps
+    ok = all(bool(torch.isfinite(o).all().item()) for o in outs)
+    flops = meta_grad_flops(n_chunks, b, d, f, V)
+    peaks, src = load_peaks()
+    peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    del h, r, W, head, work, outs
+    torch.cuda.empty_cache()
+    return {"workload": f"{cfg.name} fast-MLP meta-gradient, eq. (7): {n_chunks} chunks x {b} rows, d={d} f={f} "
+                        f"V={V}, eta={cfg.eta}, fp32", "ms": ms, "steps": steps, "warmup": warmup,
+            "algorithmic_tflop": flops / 1e12,
+            "roofline": {"bound": "alu", "achieved": flops / (ms / 1000.0) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                         "frac": flops / (ms / 1000.0) / 1e12 / peak, "peak_source": src},
+            "finite": ok}
+
+
 def time_config(name, steps=3, warmup=2):
     """Short timing of one more workload (its own T, k, b, dtype) on this GPU:
     tokens/s, per-1K-token latency and the achieved fraction of its roofline
@@ -604,7 +646,12 @@ def main():
                 "clocks": clk, "e2e": e2e, "decode": dec}
     ctx.close()
     torch.cuda.empty_cache()
-    full = multi = None
+    full = multi = meta = None
+    if rank == 0 and not args.no_meta_grad and world == 1 and args.config == "2.7b" and not args.tokens:
+        try:
+            meta = time_meta_grad(cfg)
+        except Exception as e:  # an optional arm must not cost the headline line
+            meta = {"unavailable": f"{type(e).__name__}: {e}"}
     if rank == 0 and not args.no_full_attention and world == 1 and args.config == "2.7b" and not args.tokens:
         full = time_full_attention(cfg, gw, tok_dev, T, stream, ms / args.steps)
     if rank == 0 and not args.no_multi_sequence and world == 1 and args.config == "2.7b" and not args.tokens:
@@ -614,6 +661,7 @@ def main():
     if rank == 0:
         line["full_attention"] = full
         line["multi_sequence"] = multi
+        line["meta_grad"] = meta
         if not args.no_per_config and world == 1 and args.config == "2.7b" and not args.tokens:
             line["per_config"] = {name: time_config(name) for name in PER_CONFIG}
         if want_cpu:

@@ -240,6 +240,41 @@ int ttt_op_attn_decode(int32_t n_heads, int32_t head_dim, int64_t p, int32_t win
                        const void* kring, const void* vring, int64_t R, void* o, float* lse, float* ws,
                        void* stream);
 
+/*
+ * Outer-loop meta-gradient (End-to-End Test-Time Training for Long Context;
+ * reading notes by Zhongzhu Zhou, §4, eqs. (5)-(7)) for a fast SwiGLU MLP in
+ * the model's last block, the only block with fast weights.  Per chunk c of
+ * b rows, with W = (w_gate, w_up, w_down):
+ *   A_c(W) = mean over the chunk's rows with a target of
+ *            CE(RMSNorm(r + (silu(h w_gate^T) * (h w_up^T)) w_down^T; g_final) w_head^T, target),
+ * where h (the block's MLP-norm output) and r (the residual plus the static
+ * MLP's output) do not depend on W, so eq. (7) is exact for this loss.
+ * Inner loop W^(c+1) = W^(c) - eta grad A_c(W^(c)) from W^(0) = the given
+ * weights (eq. (5)); outer loss L = (1/N) sum_c A_c(W^(c)); outputs
+ * d_* = dL/dW^(0) = (1/N) sum_c J_c^T grad A_c(W^(c)), J_(c+1) = (I - eta H_c) J_c
+ * (eq. (7)), evaluated from the last chunk backwards with Hessian-vector
+ * products (eq. (6)).  All fp32, row-major:
+ *   h, r      [n_chunks * b, d];  targets int32 [n_chunks * b], -1 = no target
+ *             (another id outside [0, vocab) counts as none and makes
+ *             ttt_op_sync return TTT_ERR_INVALID_ARG);
+ *   w_gate, w_up, d_gate, d_up [f, d];  w_down, d_down [d, f];
+ *   g_final [d];  w_head [vocab, d];  eps > 0 (RMSNorm);  eta finite;
+ *   losses    (optional, [n_chunks * b]) the per-row losses along the inner
+ *             loop, each scored with the W before its chunk's step (NaN
+ *             without a target);
+ *   work      scratch of at least ttt_op_meta_grad_work(...) floats, owned by
+ *             the caller, not read before it is written.
+ * The inputs are not modified.  Logits are materialised per chunk ([b, vocab]
+ * three times in work).  Errors: TTT_ERR_INVALID_ARG (sizes < 1, NULL
+ * pointers, work too small, eta or eps not finite or eps <= 0), TTT_ERR_CUDA.
+ */
+int64_t ttt_op_meta_grad_work(int64_t n_chunks, int64_t b, int32_t d, int32_t f, int64_t vocab);
+int ttt_op_meta_grad(int64_t n_chunks, int64_t b, int32_t d, int32_t f, int64_t vocab, const float* h,
+                     const float* r, const int32_t* targets, const float* w_gate, const float* w_up,
+                     const float* w_down, const float* g_final, const float* w_head, float eps, float eta,
+                     float* d_gate, float* d_up, float* d_down, float* losses, float* work, int64_t work_floats,
+                     void* stream);
+
 /* Device watchdog self-test: launches one thread that waits on an mbarrier
  * nothing ever arrives at.  The bounded wait gives up (about 2 s) and records
  * a timeout, so the following ttt_op_sync returns TTT_ERR_TIMEOUT and the
@@ -247,7 +282,8 @@ int ttt_op_attn_decode(int32_t n_heads, int32_t head_dim, int64_t p, int32_t win
 int ttt_op_watchdog_selftest(void* stream);
 
 /* Wait for `stream`; return TTT_ERR_TIMEOUT if a kernel launched through this
- * header recorded a bounded-wait timeout since the last call (then clears it). */
+ * header recorded a bounded-wait timeout since the last call, TTT_ERR_INVALID_ARG
+ * if one met a target id outside its range (then clears the record). */
 int ttt_op_sync(void* stream);
 
 #ifdef __cplusplus

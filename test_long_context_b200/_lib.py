@@ -102,6 +102,9 @@ def lib():
             "ttt_op_gemv": (c_i32, [c_i32, c_i64, c_i64, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
             "ttt_op_attn_decode": (c_i32, [c_i32, c_i32, c_i64, c_i32, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp,
                                            c_vp]),
+            "ttt_op_meta_grad_work": (c_i64, [c_i64, c_i64, c_i32, c_i32, c_i64]),
+            "ttt_op_meta_grad": (c_i32, [c_i64, c_i64, c_i32, c_i32, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                         c_vp, c_f32, c_f32, c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp]),
         }
         for name, (res, args) in sig.items():
             if hasattr(L, name):
@@ -133,7 +136,7 @@ def exported_symbols():
               "ttt_launch_count", "ttt_timing_enable", "ttt_timing_read", "ttt_op_gemm", "ttt_op_gemm_split", "ttt_op_gemm_dual", "ttt_op_gemm_ce_tiles", "ttt_op_gemm_plan", "ttt_op_sync", "ttt_op_swa_forward",
               "ttt_op_swa_backward", "ttt_op_watchdog_selftest", "ttt_op_rmsnorm", "ttt_op_qknorm_rope",
               "ttt_op_swiglu_bwd", "ttt_op_gemv", "ttt_op_attn_decode",
-              "ttt_op_swa_backward_noalloc"):
+              "ttt_op_swa_backward_noalloc", "ttt_op_meta_grad_work", "ttt_op_meta_grad"):
         if hasattr(L, n):
             names.append(n)
     return names

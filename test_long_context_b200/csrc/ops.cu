@@ -137,6 +137,7 @@ extern "C" int ttt_op_sync(void* stream) {
     int zero = 0;
     TTT_CUDA_TRY(cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice));
     if (h & DEV_ERR_TIMEOUT) return set_error(TTT_ERR_TIMEOUT, "a kernel's bounded wait timed out");
+    if (h & DEV_ERR_BAD_TOKEN) return set_error(TTT_ERR_INVALID_ARG, "a token or target id outside its range");
     return set_error(TTT_ERR_CUDA, "kernel error word " + std::to_string(h));
   }
   return TTT_OK;

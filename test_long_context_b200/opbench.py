@@ -34,6 +34,38 @@ def band_pairs(p0, n, k):
     return s
 
 
+def meta_grad_flops(n_chunks, b, d, f, V):
+    """GEMM flops of ttt_op_meta_grad: the inner loop runs every chunk's
+    forward and backward (9 products: 7 of b x d x f, 2 of b x d x V); the
+    reverse sweep runs them again for chunks N-2 .. 0 plus their tangents (14
+    products: 10 of b x d x f, 2 of b x d x V)."""
+    fb = 2.0 * b * (7 * d * f + 2 * d * V)
+    hv = 2.0 * b * (10 * d * f + 2 * d * V)
+    return n_chunks * fb + (n_chunks - 1) * (fb + hv)
+
+
+def meta_grad_inputs(n_chunks, b, d, f, V, seed=0):
+    """Seeded synthetic inputs of the meta-gradient at a model's shapes:
+    h, r ~ N(0, 1); fast and head weights ~ N(0, 0.02) (the weights' init);
+    unit final-norm gain; targets uniform over the vocabulary, the last one
+    absent."""
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    rows = n_chunks * b
+    h = torch.randn(rows, d, device="cuda", generator=g)
+    r = torch.randn(rows, d, device="cuda", generator=g)
+    tgt = torch.randint(0, V, (rows,), device="cuda", generator=g, dtype=torch.int32)
+    tgt[-1] = -1
+    W = [0.02 * torch.randn(f, d, device="cuda", generator=g), 0.02 * torch.randn(f, d, device="cuda", generator=g),
+         0.02 * torch.randn(d, f, device="cuda", generator=g)]
+    gf = torch.ones(d, device="cuda")
+    head = 0.02 * torch.randn(V, d, device="cuda", generator=g)
+    return h, r, tgt, W, gf, head
+
+
+# ops that run only when named with --op (not part of the default list)
+OPT_IN = {"meta_grad_top"}
+
+
 def op_builders(cfg, exp_poly=None):
     """{name: builder}; a builder allocates the op's inputs and returns
     (run, algorithmic flops, algorithmic bytes).  exp_poly: polynomial share
@@ -166,6 +198,15 @@ def op_builders(cfg, exp_poly=None):
         pdec = 16 * k + 5
         return (lambda: ops.attn_decode(qd, kdec, vdec, H, hd, pdec, k, od, lsed, wsd)), 0.0, 2.0 * 2 * d * k
     B["attn_decode_top"] = attn_dec
+
+    # outer loop: meta-gradient of a fast MLP in the last block over two chunks
+    def meta_grad():
+        h, r, tgt, W, gf, head = meta_grad_inputs(2, b, d, f, V)
+        outs = [torch.empty_like(w) for w in W]
+        work = torch.empty(ops.meta_grad_work(2, b, d, f, V), device=dev)
+        run = lambda: ops.meta_grad(h, r, tgt, *W, gf, head, 1e-5, 0.5, b, *outs, work=work)
+        return run, meta_grad_flops(2, b, d, f, V), 0.0
+    B["meta_grad_top"] = meta_grad
     return B
 
 
@@ -179,7 +220,7 @@ def main():
     args = ap.parse_args()
     cfg = get_config(args.config)
     builders = op_builders(cfg, args.exp_poly)
-    for name in args.op or list(builders):
+    for name in args.op or [n for n in builders if n not in OPT_IN]:
         run, flops, nbytes = builders[name]()
         for _ in range(args.warmup):
             run()

@@ -161,3 +161,30 @@ def attn_decode(q, kring, vring, n_heads, head_dim, p, window, o, lse, ws, strea
     """ttt_op_attn_decode: one query per head (bf16 [H*hd]) over the window of the rings."""
     L.check(L.lib().ttt_op_attn_decode(n_heads, head_dim, p, window, _p(q), _p(kring), _p(vring), kring.shape[0],
                                        _p(o), _p(lse), _p(ws), _stream(stream)))
+
+
+def meta_grad_work(n_chunks, b, d, f, vocab):
+    """ttt_op_meta_grad_work: floats of scratch ttt_op_meta_grad needs."""
+    n = L.lib().ttt_op_meta_grad_work(n_chunks, b, d, f, vocab)
+    if n < 0:
+        raise ValueError("meta_grad_work: sizes must be >= 1")
+    return n
+
+
+def meta_grad(h, r, targets, w_gate, w_up, w_down, g_final, w_head, eps, eta, b, d_gate, d_up, d_down,
+              losses=None, work=None, stream=None):
+    """ttt_op_meta_grad: dL/dW^(0) of the adapted loss over len(targets) / b
+    chunks into d_gate, d_up, d_down (fp32, shaped like the weights); the
+    per-row losses along the inner loop into ``losses`` when given.  ``work``
+    (fp32) is allocated here when not given."""
+    rows, d = h.shape
+    f = w_gate.shape[0]
+    V = w_head.shape[0]
+    n_chunks = rows // b
+    need = meta_grad_work(n_chunks, b, d, f, V)
+    if work is None:
+        work = torch.empty(need, dtype=torch.float32, device=h.device)
+    L.check(L.lib().ttt_op_meta_grad(n_chunks, b, d, f, V, _p(h), _p(r), _p(targets), _p(w_gate), _p(w_up),
+                                     _p(w_down), _p(g_final), _p(w_head), eps, eta, _p(d_gate), _p(d_up),
+                                     _p(d_down), _p(losses), _p(work), work.numel(), _stream(stream)))
+    return work

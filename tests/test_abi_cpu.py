@@ -55,3 +55,25 @@ def test_python_binding_has_no_compute():
         with open(os.path.join(ROOT, "test_long_context_b200", f)) as fh:
             src = fh.read()
         assert "import oracle" not in src and "from oracle" not in src
+
+
+def test_meta_grad_validates_on_the_host():
+    """ttt_op_meta_grad checks its arguments before any device call; its
+    scratch size follows from the shapes alone."""
+    from test_long_context_b200 import _lib as L
+    lib = L.lib()
+    N, b, d, f, V = 3, 40, 64, 96, 500
+    P = 3 * d * f
+    assert lib.ttt_op_meta_grad_work(N, b, d, f, V) == N * P + 3 * P + 12 * b * f + 8 * b * d + 3 * b + 3 * b * V + 1
+    assert lib.ttt_op_meta_grad_work(0, b, d, f, V) == -1
+    fake = 256  # never dereferenced: every call below fails validation first
+    args = [fake] * 8
+    rc = lib.ttt_op_meta_grad(N, b, d, f, V, *args, 1e-5, 0.5, fake, fake, fake, None, None, 0, None)
+    assert rc == L.TTT_ERR_INVALID_ARG  # no work array
+    rc = lib.ttt_op_meta_grad(N, b, d, f, V, *args, 1e-5, 0.5, fake, fake, fake, None, fake,
+                              lib.ttt_op_meta_grad_work(N, b, d, f, V) - 1, None)
+    assert rc == L.TTT_ERR_INVALID_ARG and b"work" in lib.ttt_last_error(None)
+    rc = lib.ttt_op_meta_grad(N, b, d, f, V, *args, 1e-5, float("nan"), fake, fake, fake, None, fake, 1 << 40, None)
+    assert rc == L.TTT_ERR_INVALID_ARG
+    rc = lib.ttt_op_meta_grad(N, b, d, f, V, *args, 0.0, 0.5, fake, fake, fake, None, fake, 1 << 40, None)
+    assert rc == L.TTT_ERR_INVALID_ARG
