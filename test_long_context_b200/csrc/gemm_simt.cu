@@ -2,20 +2,25 @@
 // at 1e-4 relative holds).  Same operand conventions and epilogues as the
 // tensor-core GEMM; tile 64 x 128 x 16, 256 threads, 4 x 8 outputs each:
 // rows ty*4+i, columns tx*4+j and 64+tx*4+j (so a SwiGLU gate column and its
-// up column land in the same thread).
+// up column land in the same thread).  The k-slices of both tiles sit in
+// shared memory with the row (m or n) contiguous, each row padded by 4
+// floats: a thread reads its 4 A values and its two groups of 4 B values as
+// three 16-byte loads, and the transposing stores of K-major operands (16
+// lanes on one m or n) spread over banks instead of piling onto one.
 #include "gemm.cuh"
 
 namespace ttt {
 namespace {
 
 constexpr int SBM = 64, SBN = 128, SBK = 16;
+constexpr int SPAD = 4;  // row padding (floats): keeps 16-byte alignment, breaks the stores' bank pile-up
 
 template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict__ A, int64_t lda,
                                                         const float* __restrict__ B, int64_t ldb, int64_t M,
                                                         int64_t N, int64_t K, EpiArgs ep) {
-  __shared__ float As[SBK][SBM];
-  __shared__ float Bs[SBK][SBN];
+  __shared__ __align__(16) float As[SBK][SBM + SPAD];
+  __shared__ __align__(16) float Bs[SBK][SBN + SPAD];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   const int64_t m0 = (int64_t)blockIdx.y * SBM, n0 = (int64_t)blockIdx.x * SBN;
   float acc[4][8] = {};
@@ -39,14 +44,11 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const float* __restrict_
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < SBK; ++kk) {
-      float a[4], b[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        b[j] = Bs[kk][tx * 4 + j];
-        b[4 + j] = Bs[kk][64 + tx * 4 + j];
-      }
+      const float4 av = *reinterpret_cast<const float4*>(&As[kk][ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][64 + tx * 4]);
+      const float a[4] = {av.x, av.y, av.z, av.w};
+      const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
