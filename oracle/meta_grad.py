@@ -34,6 +34,12 @@ the hand-derived gradient (forward mode over the backward), written out
 step by step; the pages only say that automatic differentiation provides
 it (§4.1, the paragraph after eq. (6)).
 
+``meta_grad_model`` takes eq. (7) over the whole model with fast MLPs in
+every top block (n_u >= 1), where a chunk's loss reaches a lower fast MLP
+through the upper blocks' attention: its Hessian-vector products carry the
+tangent of the attention forward and backward too (see the section comment
+further down for what is held fixed).
+
 All arithmetic is float64.
 """
 from __future__ import annotations
@@ -222,3 +228,272 @@ def adapted_loss_top_mlp(h, r, tgt, W0, gf, head, eta, eps, b):
 
     _, losses = inner_loop(N, W0, eta, loss_grad)
     return float(np.mean(losses))
+
+
+# ----------------------------------------------------------------------------
+# the whole model: fast MLPs in every top block (n_u >= 1)
+#
+# With more than one fast block, a chunk's loss reaches a lower fast MLP
+# through the upper blocks' attention, so H_c v needs the tangent of the
+# attention forward and backward.  Eq. (7) is taken as written: A_c is the
+# chunk loss as a function of W with the chunk's cached keys and values held
+# (they were computed under earlier weights; reading 3 of ttt_oracle), the
+# same A_c whose gradient the inner loop steps along.  With n_u = 1 this is
+# the exact gradient of L (the function above); with n_u > 1 the pages'
+# "main dependency" leaves out the path through the cached keys, and so does
+# this.
+
+
+def _norm_t(x, xt, g, eps):
+    """Tangent of rmsnorm (last axis) along xt: (yt, rt)."""
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    rt = -r ** 3 * np.mean(x * xt, axis=-1, keepdims=True)
+    return g * (xt * r + x * rt), rt
+
+
+def _norm_bwd_t(x, xt, r, rt, g, dy, dyt):
+    """Tangent of rmsnorm_bwd: dx = r u - r^3 x mean(x u), u = g dy."""
+    u, ut = g * dy, g * dyt
+    m = np.mean(x * u, axis=-1, keepdims=True)
+    mt = np.mean(xt * u + x * ut, axis=-1, keepdims=True)
+    return rt * u + r * ut - 3.0 * r * r * rt * x * m - r ** 3 * xt * m - r ** 3 * x * mt
+
+
+def _swiglu_t(h, ht, w, v, G, U):
+    """Forward tangent of swiglu along the input (ht) and the weights (v; None = fixed)."""
+    wg, wu, wd = w
+    sl, d1, _ = _silu_derivs(G)
+    Gt = ht @ wg.T + (h @ v[0].T if v else 0.0)
+    Ut = ht @ wu.T + (h @ v[1].T if v else 0.0)
+    at = d1 * Gt * U + sl * Ut
+    a = sl * U
+    yt = at @ wd.T + (a @ v[2].T if v else 0.0)
+    return Gt, Ut, at, yt
+
+
+def _swiglu_bwd_t(dy, dyt, h, ht, G, U, Gt, Ut, at, w, v):
+    """Primal and tangent of swiglu_bwd: (dh, dht, (grads), (grad tangents))."""
+    wg, wu, wd = w
+    sl, d1, d2 = _silu_derivs(G)
+    a = sl * U
+    da = dy @ wd
+    dat = dyt @ wd + (dy @ v[2] if v else 0.0)
+    dG = da * U * d1
+    dU = da * sl
+    dGt = dat * U * d1 + da * Ut * d1 + da * U * d2 * Gt
+    dUt = dat * sl + da * d1 * Gt
+    grads = (dG.T @ h, dU.T @ h, dy.T @ a)
+    grads_t = (dGt.T @ h + dG.T @ ht, dUt.T @ h + dU.T @ ht, dyt.T @ a + dy.T @ at)
+    dh = dG @ wg + dU @ wu
+    dht = dGt @ wg + dUt @ wu + ((dG @ v[0] + dU @ v[1]) if v else 0.0)
+    return dh, dht, grads, grads_t
+
+
+def model_chunk_grad_hvp(model, W, fwd, weights, V):
+    """(grad, H V) of A = sum_p weights[p] loss_p of one forwarded chunk
+    (ttt_oracle.forward_chunk output) at fast weights W, cached keys held;
+    V is a direction shaped like W.  The primal steps repeat
+    ttt_oracle.backward_chunk; every step also carries its tangent."""
+    from .ttt_oracle import rope, rope_bwd, swa_bwd
+    cfg = model.cfg
+    n, d, H, hd, eps = fwd["n"], cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.norm_eps
+    scale = 1.0 / np.sqrt(hd)
+    cos, sin = fwd["cos"], fwd["sin"]
+    off = fwd["p0"] - fwd["kstart"]
+    top = sorted(W)
+    names = ("w_gate", "w_up", "w_down")
+    # ---- forward tangent, lowest fast block upwards (its input does not depend on W)
+    xt = np.zeros((n, d))
+    T_ = {}
+    for l in top:
+        s = fwd["saved"][l]
+        pre = f"layers.{l}."
+        t = dict(x_in=xt)
+        t["h"], t["r1"] = _norm_t(s["x_in"], xt, model[pre + "attn_norm"], eps)
+        t["q"] = (t["h"] @ model[pre + "wq"].T).reshape(n, H, hd)
+        t["kk"] = (t["h"] @ model[pre + "wk"].T).reshape(n, H, hd)
+        t["v"] = (t["h"] @ model[pre + "wv"].T).reshape(n, H, hd)
+        qnt, t["rq"] = _norm_t(s["q"], t["q"], model[pre + "q_norm"], eps)
+        knt, t["rk"] = _norm_t(s["kk"], t["kk"], model[pre + "k_norm"], eps)
+        t["qr"] = rope(qnt, cos, sin)
+        Kwt = np.zeros_like(s["Kw"])
+        Vwt = np.zeros_like(s["Vw"])
+        Kwt[off:off + n] = rope(knt, cos, sin)
+        Vwt[off:off + n] = t["v"]
+        t["Kw"], t["Vw"] = Kwt, Vwt
+        P = s["P"]
+        St = (np.einsum("nhe,mhe->hnm", t["qr"], s["Kw"]) + np.einsum("nhe,mhe->hnm", s["qr"], Kwt)) * scale
+        t["P"] = P * (St - np.sum(P * St, axis=-1, keepdims=True))
+        ot = np.einsum("hnm,mhe->nhe", t["P"], s["Vw"]) + np.einsum("hnm,mhe->nhe", P, Vwt)
+        t["x_mid"] = xt + ot.reshape(n, d) @ model[pre + "wo"].T
+        t["h2"], t["r2"] = _norm_t(s["x_mid"], t["x_mid"], model[pre + "mlp_norm"], eps)
+        ws = (model[pre + "w_gate"], model[pre + "w_up"], model[pre + "w_down"])
+        wf = tuple(W[l][nm] for nm in names)
+        vf = tuple(V[l][nm] for nm in names)
+        t["ms"] = _swiglu_t(s["h2"], t["h2"], ws, None, s["ms"][0], s["ms"][1])
+        t["mf"] = _swiglu_t(s["h2"], t["h2"], wf, vf, s["mf"][0], s["mf"][1])
+        xt = t["x_mid"] + t["ms"][3] + t["mf"][3]
+        T_[l] = t
+    hft, rft = _norm_t(fwd["x"], xt, model["final_norm"], eps)
+    zt = hft @ model["lm_head"].T
+    # ---- backward and its tangent
+    valid, tgt = fwd["valid"], fwd["tgt"]
+    rows = np.nonzero(valid)[0]
+    Pz = fwd["probs"]
+    dz = np.zeros((n, cfg.vocab))
+    dzt = np.zeros((n, cfg.vocab))
+    wv = weights[valid][:, None]
+    dzv = Pz.copy()
+    dzv[np.arange(len(rows)), tgt[valid]] -= 1.0
+    dz[valid] = dzv * wv
+    ztv = zt[valid]
+    dzt[valid] = wv * Pz * (ztv - np.sum(Pz * ztv, axis=-1, keepdims=True))
+    head = model["lm_head"]
+    dhf, dhft = dz @ head, dzt @ head
+    dx = rmsnorm_bwd(fwd["x"], fwd["rf"], model["final_norm"], dhf)
+    dxt = _norm_bwd_t(fwd["x"], xt, fwd["rf"], rft, model["final_norm"], dhf, dhft)
+    G, HV = {}, {}
+    lowest = top[0]
+    for l in reversed(top):
+        s, t = fwd["saved"][l], T_[l]
+        pre = f"layers.{l}."
+        wf = tuple(W[l][nm] for nm in names)
+        vf = tuple(V[l][nm] for nm in names)
+        Gf, Uf, _ = s["mf"]
+        Gft, Uft, aft, _ = t["mf"]
+        dh2_f, dh2_ft, gr, grt = _swiglu_bwd_t(dx, dxt, s["h2"], t["h2"], Gf, Uf, Gft, Uft, aft, wf, vf)
+        G[l] = dict(zip(names, gr))
+        HV[l] = dict(zip(names, grt))
+        if l == lowest:
+            break  # nothing below the lowest fast block depends on W
+        ws = (model[pre + "w_gate"], model[pre + "w_up"], model[pre + "w_down"])
+        Gs, Us, _ = s["ms"]
+        Gst, Ust, ast, _ = t["ms"]
+        dh2_s, dh2_st, _, _ = _swiglu_bwd_t(dx, dxt, s["h2"], t["h2"], Gs, Us, Gst, Ust, ast, ws, None)
+        g_m = model[pre + "mlp_norm"]
+        dx_mid = dx + rmsnorm_bwd(s["x_mid"], s["r2"], g_m, dh2_s + dh2_f)
+        dx_midt = dxt + _norm_bwd_t(s["x_mid"], t["x_mid"], s["r2"], t["r2"], g_m, dh2_s + dh2_f, dh2_st + dh2_ft)
+        wo = model[pre + "wo"]
+        do = (dx_mid @ wo).reshape(n, H, hd)
+        dot = (dx_midt @ wo).reshape(n, H, hd)
+        # attention backward (primal as ttt_oracle.swa_bwd) and its tangent
+        P, Pt = s["P"], t["P"]
+        dq_r, dK, dV = swa_bwd(do, s["qr"], s["Kw"], s["Vw"], P, hd)
+        dP = np.einsum("nhe,mhe->hnm", do, s["Vw"])
+        dPt = np.einsum("nhe,mhe->hnm", dot, s["Vw"]) + np.einsum("nhe,mhe->hnm", do, t["Vw"])
+        dl = np.sum(dP * P, axis=-1, keepdims=True)
+        dlt = np.sum(dPt * P + dP * Pt, axis=-1, keepdims=True)
+        dS = P * (dP - dl)
+        dSt = Pt * (dP - dl) + P * (dPt - dlt)
+        dq_rt = (np.einsum("hnm,mhe->nhe", dSt, s["Kw"]) + np.einsum("hnm,mhe->nhe", dS, t["Kw"])) * scale
+        dKt = (np.einsum("hnm,nhe->mhe", dSt, s["qr"]) + np.einsum("hnm,nhe->mhe", dS, t["qr"])) * scale
+        dVt = np.einsum("hnm,nhe->mhe", Pt, do) + np.einsum("hnm,nhe->mhe", P, dot)
+        dk_r, dv = dK[off:off + n], dV[off:off + n]
+        dk_rt, dvt = dKt[off:off + n], dVt[off:off + n]
+        dqn, dqnt = rope_bwd(dq_r, cos, sin), rope_bwd(dq_rt, cos, sin)
+        dkn, dknt = rope_bwd(dk_r, cos, sin), rope_bwd(dk_rt, cos, sin)
+        gq, gk = model[pre + "q_norm"], model[pre + "k_norm"]
+        dq = rmsnorm_bwd(s["q"], s["rq"], gq, dqn)
+        dqt = _norm_bwd_t(s["q"], t["q"], s["rq"], t["rq"], gq, dqn, dqnt)
+        dk = rmsnorm_bwd(s["kk"], s["rk"], gk, dkn)
+        dkt = _norm_bwd_t(s["kk"], t["kk"], s["rk"], t["rk"], gk, dkn, dknt)
+        wq, wk, wvv = model[pre + "wq"], model[pre + "wk"], model[pre + "wv"]
+        dh = dq.reshape(n, d) @ wq + dk.reshape(n, d) @ wk + dv.reshape(n, d) @ wvv
+        dht = dqt.reshape(n, d) @ wq + dkt.reshape(n, d) @ wk + dvt.reshape(n, d) @ wvv
+        g_a = model[pre + "attn_norm"]
+        dx = dx_mid + rmsnorm_bwd(s["x_in"], s["r1"], g_a, dh)
+        dxt = dx_midt + _norm_bwd_t(s["x_in"], t["x_in"], s["r1"], t["r1"], g_a, dh, dht)
+    return G, HV
+
+
+def _flat(W):
+    return tuple(W[l][nm] for l in sorted(W) for nm in ("w_gate", "w_up", "w_down"))
+
+
+def _unflat(t, like):
+    out, i = {}, 0
+    for l in sorted(like):
+        out[l] = {}
+        for nm in ("w_gate", "w_up", "w_down"):
+            out[l][nm] = t[i]
+            i += 1
+    return out
+
+
+def _chunk_targets(toks, p0, n):
+    tgt = np.full(n, -1, dtype=np.int64)
+    nt = min(n, len(toks) - 1 - p0)
+    if nt > 0:
+        tgt[:nt] = toks[p0 + 1:p0 + 1 + nt]
+    return tgt
+
+
+def meta_grad_model(model, toks, eta=None):
+    """eq. (7) for every fast MLP of the model over the sequence's full
+    chunks: (grad as {block: {name: array}}, L, per-chunk A_c).  Each chunk's
+    loss is taken with its cached keys and values as the inner loop computed
+    them (see the section comment)."""
+    from .ttt_oracle import State, forward_chunk, init_fast
+    cfg = model.cfg
+    eta = cfg.eta if eta is None else eta
+    toks = np.asarray(toks, dtype=np.int64)
+    b = cfg.b
+    N = len(toks) // b
+    state = State(cfg, len(toks))
+    like = init_fast(model)
+
+    def fwd_of(c, Wt):
+        p0 = c * b
+        tgt = _chunk_targets(toks, p0, b)
+        loss, fwd = forward_chunk(model, _unflat(Wt, like), state, toks[p0:p0 + b], p0, tgt)
+        nc = int((tgt >= 0).sum())
+        wts = np.where(tgt >= 0, 1.0 / nc, 0.0) if nc else np.zeros(b)
+        return loss, fwd, wts, nc
+
+    def loss_grad(c, Wt):
+        loss, fwd, wts, nc = fwd_of(c, Wt)
+        if nc == 0:
+            return 0.0, tuple(np.zeros_like(w) for w in Wt)
+        G, _ = model_chunk_grad_hvp(model, _unflat(Wt, like), fwd, wts, _unflat(tuple(np.zeros_like(w) for w in Wt), like))
+        return float(np.nanmean(loss)), _flat(G)
+
+    def hvp(c, Wt, v):
+        loss, fwd, wts, nc = fwd_of(c, Wt)
+        if nc == 0:
+            return tuple(np.zeros_like(w) for w in Wt)
+        _, HV = model_chunk_grad_hvp(model, _unflat(Wt, like), fwd, wts, _unflat(v, like))
+        return _flat(HV)
+
+    g, L, losses = meta_grad(N, _flat(like), eta, loss_grad, hvp)
+    return _unflat(g, like), L, losses
+
+
+def frozen_adapted_loss(model, toks, W0, cache, eta=None):
+    """L of the inner loop started at W0 (dict like init_fast), every chunk's
+    keys and values of earlier positions taken from ``cache`` (a State of an
+    unperturbed run) instead of this run's: the function whose gradient at
+    the unperturbed W0 is eq. (7) as taken above."""
+    from .ttt_oracle import State, backward_chunk, forward_chunk
+    cfg = model.cfg
+    eta = cfg.eta if eta is None else eta
+    toks = np.asarray(toks, dtype=np.int64)
+    b = cfg.b
+    N = len(toks) // b
+    W = {l: {nm: np.array(a, dtype=F) for nm, a in W0[l].items()} for l in W0}
+    state = State(cfg, len(toks))
+    means = []
+    for c in range(N):
+        p0 = c * b
+        for l in range(cfg.n_layers):
+            state.K[l][:p0] = cache.K[l][:p0]
+            state.V[l][:p0] = cache.V[l][:p0]
+        tgt = _chunk_targets(toks, p0, b)
+        loss, fwd = forward_chunk(model, W, state, toks[p0:p0 + b], p0, tgt)
+        nc = int((tgt >= 0).sum())
+        means.append(float(np.nanmean(loss)) if nc else 0.0)
+        if nc:
+            G = backward_chunk(model, W, fwd, np.where(tgt >= 0, 1.0 / nc, 0.0))
+            for l in G:
+                for nm in G[l]:
+                    W[l][nm] = W[l][nm] - eta * G[l][nm]
+    return float(np.mean(means))

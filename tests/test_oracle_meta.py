@@ -295,3 +295,174 @@ def test_planted_mistakes_are_caught(monkeypatch, target, mutant):
             caught = True
             break
     assert caught, f"no pin caught the mutation of {target}"
+
+
+# --- the whole model: fast MLPs in two blocks (Hessian-vector products through SWA)
+
+MICRO2 = MICRO.with_(n_updated=2, eta=0.8)
+
+
+def _micro2(gains=True):
+    cfg = MICRO2
+    w = synth.make_weights(cfg)
+    arrays = {k: v.astype(np.float64) for k, v in w.arrays.items()}
+    if gains:  # norm gains away from 1, so that a gain on the wrong tensor shows
+        rng = np.random.default_rng(11)
+        for k in arrays:
+            if k.endswith("norm"):
+                arrays[k] = 1.0 + 0.3 * rng.standard_normal(arrays[k].shape)
+    toks = synth.tokens(cfg, cfg.T).astype(np.int64)
+    return cfg, O.Model(cfg, arrays), arrays, toks
+
+
+def _chunk_at(model, toks, c):
+    """State and fast weights when chunk c starts (the inner loop run up to it)."""
+    res = O.prefill(model, toks, n_chunks=c, keep_state=True) if c else None
+    state = res.state if c else O.State(model.cfg, len(toks))
+    W = res.W if c else O.init_fast(model)
+    return state, W
+
+
+def _fwd(model, state, W, toks, c):
+    import copy
+    b = model.cfg.b
+    p0 = c * b
+    tgt = M._chunk_targets(toks, p0, b)
+    _, fwd = O.forward_chunk(model, W, copy.deepcopy(state), toks[p0:p0 + b], p0, tgt)
+    nc = int((tgt >= 0).sum())
+    return fwd, np.where(tgt >= 0, 1.0 / nc, 0.0)
+
+
+def _wdir(W, seed):
+    rng = np.random.default_rng(seed)
+    return {l: {nm: rng.standard_normal(a.shape) for nm, a in W[l].items()} for l in W}
+
+
+def _wax(W, t, V):
+    return {l: {nm: W[l][nm] + t * V[l][nm] for nm in W[l]} for l in W}
+
+
+def test_model_gradient_repeats_the_inner_loop_backward():
+    cfg, model, _, toks = _micro2()
+    state, W = _chunk_at(model, toks, 2)
+    fwd, wts = _fwd(model, state, W, toks, 2)
+    G, _ = M.model_chunk_grad_hvp(model, W, fwd, wts, _wdir(W, 1))
+    want = O.backward_chunk(model, W, fwd, wts)
+    for l in want:
+        for nm in want[l]:
+            assert np.abs(G[l][nm] - want[l][nm]).max() <= 1e-13 * np.abs(want[l][nm]).max()
+
+
+@pytest.mark.parametrize("c", [0, 2])
+def test_model_hvp_matches_finite_differences_of_the_gradient(c):
+    """Through both blocks (the lower fast MLP reaches the loss through the
+    upper block's attention), cached keys held."""
+    cfg, model, _, toks = _micro2()
+    state, W = _chunk_at(model, toks, c)
+    fwd, wts = _fwd(model, state, W, toks, c)
+    V = _wdir(W, 2)
+    _, HV = M.model_chunk_grad_hvp(model, W, fwd, wts, V)
+
+    def grad(Wx):
+        f, w = _fwd(model, state, Wx, toks, c)
+        return O.backward_chunk(model, Wx, f, w)
+
+    e = 1e-4
+    gs = {t: grad(_wax(W, t, V)) for t in (-2 * e, -e, e, 2 * e)}
+    for l in W:
+        for nm in W[l]:
+            fd = (8.0 * (gs[e][l][nm] - gs[-e][l][nm]) - (gs[2 * e][l][nm] - gs[-2 * e][l][nm])) / (12 * e)
+            assert np.abs(HV[l][nm] - fd).max() <= 1e-6 * np.abs(fd).max()
+
+
+def test_model_hvp_is_symmetric():
+    cfg, model, _, toks = _micro2()
+    state, W = _chunk_at(model, toks, 1)
+    fwd, wts = _fwd(model, state, W, toks, 1)
+    U, V = _wdir(W, 3), _wdir(W, 4)
+    _, HU = M.model_chunk_grad_hvp(model, W, fwd, wts, U)
+    _, HV = M.model_chunk_grad_hvp(model, W, fwd, wts, V)
+    a = sum(float(np.sum(V[l][nm] * HU[l][nm])) for l in W for nm in W[l])
+    b = sum(float(np.sum(U[l][nm] * HV[l][nm])) for l in W for nm in W[l])
+    assert abs(a - b) <= 1e-11 * max(1.0, abs(a))
+
+
+def test_model_meta_grad_matches_finite_differences_with_the_cache_held():
+    """eq. (7) over the model's four chunks against central differences of L
+    with every chunk's earlier keys and values held at the unperturbed run's;
+    and L itself against the inner loop's own chunk means."""
+    cfg, model, arrays, toks = _micro2()
+    grad, L, _ = M.meta_grad_model(model, toks)
+    base = O.prefill(model, toks, keep_state=True)
+    assert abs(L - float(np.mean(base.chunk_mean))) <= 1e-12
+    W0 = O.init_fast(model)
+    assert abs(M.frozen_adapted_loss(model, toks, W0, base.state) - L) <= 1e-12
+    for s in range(2):
+        V = _wdir(W0, 40 + s)
+        f = lambda t: M.frozen_adapted_loss(model, toks, _wax(W0, t, V), base.state)
+        e = 1e-4
+        fd = (8.0 * (f(e) - f(-e)) - (f(2 * e) - f(-2 * e))) / (12 * e)
+        dot = sum(float(np.sum(grad[l][nm] * V[l][nm])) for l in W0 for nm in W0[l])
+        assert abs(fd - dot) <= 1e-7 * max(1.0, abs(fd))
+    # neither check is vacuous here: the Hessian term moves the result, and the
+    # path through the cached keys (left out by eq. (7)) moves the full L
+    no_h = M.meta_grad(4, M._flat(W0), cfg.eta, *_model_closures(model, toks, hessian=False))[0]
+    g = M._flat(grad)
+    assert max(np.abs(a - c).max() / np.abs(a).max() for a, c in zip(g, no_h)) > 0.1
+
+    def L_full(Wx):
+        a2 = dict(arrays)
+        for l in Wx:
+            for nm in Wx[l]:
+                a2[f"fast.{l}.{nm}"] = Wx[l][nm]
+        return float(np.mean(O.prefill(O.Model(cfg, a2), toks).chunk_mean))
+
+    V = _wdir(W0, 40)
+    e = 1e-4
+    f = lambda t: L_full(_wax(W0, t, V))
+    fd_full = (8.0 * (f(e) - f(-e)) - (f(2 * e) - f(-2 * e))) / (12 * e)
+    dot = sum(float(np.sum(grad[l][nm] * V[l][nm])) for l in W0 for nm in W0[l])
+    assert abs(fd_full - dot) > 0.05 * abs(fd_full)
+
+
+def _model_closures(model, toks, hessian=True):
+    """loss_grad / hvp of meta_grad_model, with the Hessian term optionally
+    left out (H v = 0)."""
+    b = model.cfg.b
+    like = O.init_fast(model)
+    state = O.State(model.cfg, len(toks))
+
+    def fwd_of(c, Wt):
+        tgt = M._chunk_targets(toks, c * b, b)
+        loss, fwd = O.forward_chunk(model, M._unflat(Wt, like), state, toks[c * b:(c + 1) * b], c * b, tgt)
+        nc = int((tgt >= 0).sum())
+        return loss, fwd, np.where(tgt >= 0, 1.0 / nc, 0.0)
+
+    def lg(c, Wt):
+        loss, fwd, w = fwd_of(c, Wt)
+        return float(np.nanmean(loss)), M._flat(O.backward_chunk(model, M._unflat(Wt, like), fwd, w))
+
+    def hv(c, Wt, v):
+        if not hessian:
+            return tuple(np.zeros_like(x) for x in v)
+        _, fwd, w = fwd_of(c, Wt)
+        return M._flat(M.model_chunk_grad_hvp(model, M._unflat(Wt, like), fwd, w, M._unflat(v, like))[1])
+
+    return lg, hv
+
+
+def test_model_meta_grad_with_one_fast_block_is_the_last_block_case():
+    cfg = MICRO
+    w = synth.make_weights(cfg)
+    arrays = {k: v.astype(np.float64) for k, v in w.arrays.items()}
+    toks = synth.tokens(cfg, cfg.T).astype(np.int64)
+    model = O.Model(cfg, arrays)
+    grad, L, _ = M.meta_grad_model(model, toks)
+    top = cfg.n_layers - 1
+    W0 = tuple(arrays[f"fast.{top}.{nm}"] for nm in ("w_gate", "w_up", "w_down"))
+    h, r, tgt = _inputs_of_the_last_block(model, toks, cfg.b)
+    want, L2, _ = M.meta_grad_top_mlp(h, r, tgt, W0, model["final_norm"], model["lm_head"], cfg.eta,
+                                      cfg.norm_eps, cfg.b)
+    assert abs(L - L2) <= 1e-12
+    for nm, w_ in zip(("w_gate", "w_up", "w_down"), want):
+        assert np.abs(grad[top][nm] - w_).max() <= 1e-12 * np.abs(w_).max()
