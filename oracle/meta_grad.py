@@ -289,6 +289,33 @@ def _swiglu_bwd_t(dy, dyt, h, ht, G, U, Gt, Ut, at, w, v):
     return dh, dht, grads, grads_t
 
 
+def swa_tangent(q, K, V, P, qt, Kt, Vt):
+    """Tangent of swa (ttt_oracle.swa, eq. (1) band) along (qt, Kt, Vt):
+    St = scale (qt K^T + q Kt^T), Pt = P (St - rowsum(P St)), ot = Pt V + P Vt.
+    Masked entries have P = 0, so they carry no tangent.  Returns (Pt, ot)."""
+    scale = 1.0 / np.sqrt(q.shape[-1])
+    St = (np.einsum("nhe,mhe->hnm", qt, K) + np.einsum("nhe,mhe->hnm", q, Kt)) * scale
+    Pt = P * (St - np.sum(P * St, axis=-1, keepdims=True))
+    ot = np.einsum("hnm,mhe->nhe", Pt, V) + np.einsum("hnm,mhe->nhe", P, Vt)
+    return Pt, ot
+
+
+def swa_bwd_tangent(do, dot, q, K, V, P, qt, Kt, Vt, Pt):
+    """Tangent of swa_bwd (dq, dK, dV given dO) along the forward tangents
+    (qt, Kt, Vt, Pt) and dot, the tangent of dO."""
+    scale = 1.0 / np.sqrt(q.shape[-1])
+    dP = np.einsum("nhe,mhe->hnm", do, V)
+    dPt = np.einsum("nhe,mhe->hnm", dot, V) + np.einsum("nhe,mhe->hnm", do, Vt)
+    dl = np.sum(dP * P, axis=-1, keepdims=True)
+    dlt = np.sum(dPt * P + dP * Pt, axis=-1, keepdims=True)
+    dS = P * (dP - dl)
+    dSt = Pt * (dP - dl) + P * (dPt - dlt)
+    dqt = (np.einsum("hnm,mhe->nhe", dSt, K) + np.einsum("hnm,mhe->nhe", dS, Kt)) * scale
+    dKt = (np.einsum("hnm,nhe->mhe", dSt, q) + np.einsum("hnm,nhe->mhe", dS, qt)) * scale
+    dVt = np.einsum("hnm,nhe->mhe", Pt, do) + np.einsum("hnm,nhe->mhe", P, dot)
+    return dqt, dKt, dVt
+
+
 def model_chunk_grad_hvp(model, W, fwd, weights, V):
     """(grad, H V) of A = sum_p weights[p] loss_p of one forwarded chunk
     (ttt_oracle.forward_chunk output) at fast weights W, cached keys held;
@@ -297,7 +324,6 @@ def model_chunk_grad_hvp(model, W, fwd, weights, V):
     from .ttt_oracle import rope, rope_bwd, swa_bwd
     cfg = model.cfg
     n, d, H, hd, eps = fwd["n"], cfg.d_model, cfg.n_heads, cfg.head_dim, cfg.norm_eps
-    scale = 1.0 / np.sqrt(hd)
     cos, sin = fwd["cos"], fwd["sin"]
     off = fwd["p0"] - fwd["kstart"]
     top = sorted(W)
@@ -321,10 +347,7 @@ def model_chunk_grad_hvp(model, W, fwd, weights, V):
         Kwt[off:off + n] = rope(knt, cos, sin)
         Vwt[off:off + n] = t["v"]
         t["Kw"], t["Vw"] = Kwt, Vwt
-        P = s["P"]
-        St = (np.einsum("nhe,mhe->hnm", t["qr"], s["Kw"]) + np.einsum("nhe,mhe->hnm", s["qr"], Kwt)) * scale
-        t["P"] = P * (St - np.sum(P * St, axis=-1, keepdims=True))
-        ot = np.einsum("hnm,mhe->nhe", t["P"], s["Vw"]) + np.einsum("hnm,mhe->nhe", P, Vwt)
+        t["P"], ot = swa_tangent(s["qr"], s["Kw"], s["Vw"], s["P"], t["qr"], Kwt, Vwt)
         t["x_mid"] = xt + ot.reshape(n, d) @ model[pre + "wo"].T
         t["h2"], t["r2"] = _norm_t(s["x_mid"], t["x_mid"], model[pre + "mlp_norm"], eps)
         ws = (model[pre + "w_gate"], model[pre + "w_up"], model[pre + "w_down"])
@@ -379,15 +402,7 @@ def model_chunk_grad_hvp(model, W, fwd, weights, V):
         # attention backward (primal as ttt_oracle.swa_bwd) and its tangent
         P, Pt = s["P"], t["P"]
         dq_r, dK, dV = swa_bwd(do, s["qr"], s["Kw"], s["Vw"], P, hd)
-        dP = np.einsum("nhe,mhe->hnm", do, s["Vw"])
-        dPt = np.einsum("nhe,mhe->hnm", dot, s["Vw"]) + np.einsum("nhe,mhe->hnm", do, t["Vw"])
-        dl = np.sum(dP * P, axis=-1, keepdims=True)
-        dlt = np.sum(dPt * P + dP * Pt, axis=-1, keepdims=True)
-        dS = P * (dP - dl)
-        dSt = Pt * (dP - dl) + P * (dPt - dlt)
-        dq_rt = (np.einsum("hnm,mhe->nhe", dSt, s["Kw"]) + np.einsum("hnm,mhe->nhe", dS, t["Kw"])) * scale
-        dKt = (np.einsum("hnm,nhe->mhe", dSt, s["qr"]) + np.einsum("hnm,nhe->mhe", dS, t["qr"])) * scale
-        dVt = np.einsum("hnm,nhe->mhe", Pt, do) + np.einsum("hnm,nhe->mhe", P, dot)
+        dq_rt, dKt, dVt = swa_bwd_tangent(do, dot, s["qr"], s["Kw"], s["Vw"], P, t["qr"], t["Kw"], t["Vw"], Pt)
         dk_r, dv = dK[off:off + n], dV[off:off + n]
         dk_rt, dvt = dKt[off:off + n], dVt[off:off + n]
         dqn, dqnt = rope_bwd(dq_r, cos, sin), rope_bwd(dq_rt, cos, sin)

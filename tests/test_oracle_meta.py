@@ -466,3 +466,45 @@ def test_model_meta_grad_with_one_fast_block_is_the_last_block_case():
     assert abs(L - L2) <= 1e-12
     for nm, w_ in zip(("w_gate", "w_up", "w_down"), want):
         assert np.abs(grad[top][nm] - w_).max() <= 1e-12 * np.abs(w_).max()
+
+
+# --- op level: the attention tangents a GPU kernel would be checked against
+
+
+def _swa_case(seed=12, n=5, m=9, H=2, hd=8, k=4):
+    rng = np.random.default_rng(seed)
+    q, K, V = (rng.standard_normal(s) for s in ((n, H, hd), (m, H, hd), (m, H, hd)))
+    qt, Kt, Vt = (rng.standard_normal(s) for s in ((n, H, hd), (m, H, hd), (m, H, hd)))
+    do, dot = rng.standard_normal((n, H, hd)), rng.standard_normal((n, H, hd))
+    qpos = np.arange(m - n, m)   # the chunk's queries are the last n key positions
+    kpos = np.arange(m)
+    return q, K, V, qt, Kt, Vt, do, dot, qpos, kpos, k
+
+
+def test_swa_tangent_matches_finite_differences():
+    q, K, V, qt, Kt, Vt, _, _, qpos, kpos, k = _swa_case()
+    o_of = lambda t: O.swa(q + t * qt, K + t * Kt, V + t * Vt, qpos, kpos, k)[0]
+    _, P = O.swa(q, K, V, qpos, kpos, k)
+    _, ot = M.swa_tangent(q, K, V, P, qt, Kt, Vt)
+    e = 1e-4
+    fd = (8.0 * (o_of(e) - o_of(-e)) - (o_of(2 * e) - o_of(-2 * e))) / (12 * e)
+    assert np.abs(ot - fd).max() <= 1e-8 * np.abs(fd).max()
+
+
+def test_swa_bwd_tangent_matches_finite_differences():
+    q, K, V, qt, Kt, Vt, do, dot, qpos, kpos, k = _swa_case(seed=13)
+    hd = q.shape[-1]
+
+    def grads(t):
+        qq, KK, VV = q + t * qt, K + t * Kt, V + t * Vt
+        _, P = O.swa(qq, KK, VV, qpos, kpos, k)
+        return O.swa_bwd(do + t * dot, qq, KK, VV, P, hd)
+
+    _, P = O.swa(q, K, V, qpos, kpos, k)
+    Pt, _ = M.swa_tangent(q, K, V, P, qt, Kt, Vt)
+    tang = M.swa_bwd_tangent(do, dot, q, K, V, P, qt, Kt, Vt, Pt)
+    e = 1e-4
+    gs = {t: grads(t) for t in (-2 * e, -e, e, 2 * e)}
+    for i, a in enumerate(tang):
+        fd = (8.0 * (gs[e][i] - gs[-e][i]) - (gs[2 * e][i] - gs[-2 * e][i])) / (12 * e)
+        assert np.abs(a - fd).max() <= 1e-8 * np.abs(fd).max()
